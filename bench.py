@@ -1,0 +1,414 @@
+"""Benchmark of the ODA decode hot path on B200 (one JSON line on rank 0).
+
+Workload (default): Qwen3-8B-shaped attention, 36 layers, 32 query / 8 KV heads, head_dim 128,
+context 131072, batch 4, flags Bernoulli(0.125) per sequence-step, recall head (D = 4096)
+still run.  A step = local pass (36 layers), recall head, conditional full retry of the
+flagged sequences, commit, for the whole batch.  Inputs: seeded synthetic data (bf16 K/V/q
+~ N(0,1)), the 77 GB cache resident in HBM (larger than L2, no flush needed).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--gpus N > 1 runs under torchrun as N independent replicas (one batch per GPU, no
+collective on the data path); timing is the max over ranks.  --impl reference times the
+CPU oracle (the plain fp64 restatement in oracle/) on the host cores over a bounded sample
+of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ODA decode-attn steps/s + % of HBM peak, 128K ctx, 12.5% recall, 1 B200"
+UNIT = "steps/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling during the timed region (SM clock, max, throttle reasons)."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------ accounting
+def step_bytes(wl, pos_list, flags):
+    """Algorithmic bytes of one step: local KV + flagged full KV + head weights."""
+    from workload import inputs
+    per_tok = wl.Hkv * 128 * 2 * 2
+    b = 0
+    for bi, t in enumerate(pos_list):
+        b += min(t, wl.sinks + wl.window) * per_tok * wl.L
+        if flags[bi]:
+            b += t * per_tok * wl.L
+    return b + inputs.head_param_count(wl.D) * 4
+
+
+def kernel_launches(wl, any_flag: bool) -> int:
+    n = wl.L + (wl.n_layers - wl.L) + 1 + 6 + 1 + 1     # local layers, glue, head, set-cond, commit
+    if wl.hybrid:
+        n += 2
+    if any_flag:
+        n += wl.n_layers + 1 + (2 if wl.hybrid else 0)
+    return n
+
+
+# ------------------------------------------------------------------- multi-rank
+def replica_workload(wl, rank: int, world: int):
+    """Replicas only: every rank decodes its own batch (a distinct seed), no data exchange."""
+    return wl if world <= 1 else wl.replace(seed=wl.seed + 1000 * rank, name=f"{wl.name}_r{rank}")
+
+
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """Device-timed milliseconds, maximised over ranks (all ranks call this in the same order)."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64,
+                     device=device if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------- oracle sample
+class OracleSample:
+    """A bounded sample of one step of the workload for the CPU oracle: sequence 0 of layer 0,
+    the first ``kv_heads`` KV heads (with their query-head groups), local and full attention,
+    plus one recall-head score.  Inputs are generated once, outside the timed region."""
+
+    def __init__(self, wl, kv_heads: int = 1):
+        import numpy as np
+        from workload import inputs
+        self.wl = wl
+        self.kv_heads = kv_heads
+        g = wl.Hq // wl.Hkv
+        self.t = wl.ctx[0] + 1
+        q, kn, vn = inputs.step_qkv(wl, 0, 0, 0)
+        self.q = np.ascontiguousarray(q[0, :kv_heads * g])
+        self.kn = np.ascontiguousarray(kn[0, :kv_heads])
+        self.vn = np.ascontiguousarray(vn[0, :kv_heads])
+        self.kc = np.ascontiguousarray(inputs.cache_tokens(wl, "k", 0, 0, self.t - 1)[:, :kv_heads])
+        self.vc = np.ascontiguousarray(inputs.cache_tokens(wl, "v", 0, 0, self.t - 1)[:, :kv_heads])
+        self.P = inputs.head_weights(wl)
+        self.e = inputs.emb(wl, 0).astype(np.float64)[0]
+        self.hp = inputs.h_prev0(wl).astype(np.float64)[0]
+        per_tok = wl.Hkv * 128 * 2 * 2
+        self.head_bytes = inputs.head_param_count(wl.D) * 4
+        rates = list(wl.rates) if wl.rates else [0.4] * wl.B
+        self.exp_step_bytes = sum(min(self.t, wl.sinks + wl.window) * per_tok * wl.L +
+                                  r * self.t * per_tok * wl.L for r in rates) + self.head_bytes
+
+    def run(self):
+        """Returns (algorithmic bytes processed, seconds)."""
+        import numpy as np
+        from oracle.attention import attend_bits
+        from oracle.head import recall_head
+        from oracle.sets import full_set, local_set
+        wl, t = self.wl, self.t
+        per_head_tok = 128 * 2 * 2
+        t0 = time.perf_counter()
+        o_l = attend_bits(self.q, self.kc, self.vc, self.kn, self.vn, local_set(t, wl.sinks, wl.window))
+        o_f = attend_bits(self.q, self.kc, self.vc, self.kn, self.vn, full_set(t))
+        sc = recall_head(self.P, self.hp, self.e, self.e)
+        dt = time.perf_counter() - t0
+        assert np.isfinite(o_l).all() and np.isfinite(o_f).all() and np.isfinite(sc)
+        nbytes = (min(t, wl.sinks + wl.window) + t) * per_head_tok * self.kv_heads + self.head_bytes
+        return nbytes, dt
+
+    def describe(self, nbytes, dt):
+        return (f"fp64 oracle on sequence 0, layer 0, {self.kv_heads} of {self.wl.Hkv} KV heads: "
+                f"local attention (|S^L|={min(self.t, 2052)}) + full attention (t={self.t}) + one "
+                f"recall-head score = {nbytes / 1e6:.0f} MB of algorithmic bytes in {dt:.2f} s; "
+                f"steps/s = bytes/s / {self.exp_step_bytes / 1e9:.2f} GB (expected bytes per step)")
+
+    def steps_per_s(self, nbytes, dt):
+        return (nbytes / dt) / self.exp_step_bytes
+
+
+def cpu_cores() -> int:
+    return len(os.sched_getaffinity(0))
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return
+    smp = OracleSample(wl, kv_heads=1)
+    vals, desc = [], ""
+    for i in range(args.warmup + args.steps):
+        nb, dt = smp.run()
+        if i >= args.warmup:
+            vals.append(smp.steps_per_s(nb, dt))
+            desc = smp.describe(nb, dt)
+    value = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "layers": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv,
+                       "ctx": wl.ctx[0], "recall_rate": wl.rates[0] if wl.rates else None},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------ GPU arm
+def run_ours(args, wl, rank, world, local_rank):
+    import torch
+    from conditional_sparse_attention_b200 import oda
+    from conditional_sparse_attention_b200.engine import OdaDecoder
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = replica_workload(wl, rank, world)
+    W, K = args.warmup, args.steps
+    n_e2e = K if args.e2e else 0
+    cap = W + K + W + n_e2e + 4
+    t_setup = time.perf_counter()
+    dec = OdaDecoder(wl, device=dev, capacity_steps=cap)
+    n_store = min(cap, W + K)
+    store = [dec.make_step_buffer(s) for s in range(n_store)]
+    torch.cuda.synchronize(dev)
+    setup_s = time.perf_counter() - t_setup
+
+    # first step including graph capture (the pages' "first request" includes capture)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tf = time.perf_counter()
+    dec.capture()
+    dec.stage(store[0])
+    dec.launch()
+    dec.synchronize()
+    first_ms = (time.perf_counter() - tf) * 1000.0
+    step_idx = 1
+    for _ in range(W):
+        dec.step(store[step_idx % n_store])
+        step_idx += 1
+    dec.synchronize()
+
+    # ---------------- timed region: K steps, device-timed with events on the launching stream
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    flags_log, pos_log = [], []
+    pos_before = dec.pos.clone()
+    flag_hist = torch.zeros((K, wl.B), dtype=torch.int32, device=dev)
+    pos_hist = torch.zeros((K, wl.B), dtype=torch.int32, device=dev)
+    with torch.cuda.stream(dec.stream):
+        ev0.record(dec.stream)
+        for i in range(K):
+            pos_hist[i].copy_(dec.pos, non_blocking=True)
+            dec.step(store[step_idx % n_store])
+            flag_hist[i].copy_(dec.flag, non_blocking=True)
+            step_idx += 1
+        ev1.record(dec.stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        torch.distributed.barrier()
+    elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    flags = flag_hist.cpu().numpy()
+    poss = pos_hist.cpu().numpy()
+    total_bytes = sum(step_bytes(wl, poss[i].tolist(), flags[i].tolist()) for i in range(K))
+    realized_rate = float(flags.mean())
+    launches = sum(kernel_launches(wl, bool(flags[i].any())) for i in range(K))
+
+    # ---------------- dominant kernel: the full-set attention, timed per launch with events
+    hbm, peak_src = peaks()
+    full_bytes, full_ms = 0, 0.0
+    loc_bytes, loc_ms = 0, 0.0
+    per_tok = wl.Hkv * 128 * 2 * 2
+    kev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    patterns = [f for f in flags if f.any()] or [torch.ones(wl.B, dtype=torch.int32).numpy()]
+    pos_now = dec.pos.cpu().numpy()
+    for rep, fl in enumerate(patterns[:8]):
+        ft = torch.from_numpy(fl.astype("int32")).to(dev)
+        for a in range(min(wl.L, 6)):
+            with torch.cuda.stream(dec.stream):
+                kev[0].record(dec.stream)
+                oda.oda_attend_full_if(dec.ctx, dec.layers[a], dec.page_table, dec.pos, ft,
+                                       dec.sv["q"][1, a], dec.sv["k"][1, a], dec.sv["v"][1, a],
+                                       dec.o[1, a], dec.stream)
+                kev[1].record(dec.stream)
+            kev[1].synchronize()
+            full_ms += kev[0].elapsed_time(kev[1])
+            full_bytes += sum(int(pos_now[b]) * per_tok for b in range(wl.B) if fl[b])
+            with torch.cuda.stream(dec.stream):
+                kev[0].record(dec.stream)
+                oda.oda_attend_local(dec.ctx, dec.layers[a], dec.page_table, dec.pos,
+                                     dec.sv["q"][0, a], dec.sv["k"][0, a], dec.sv["v"][0, a],
+                                     dec.o[0, a], dec.stream)
+                kev[1].record(dec.stream)
+            kev[1].synchronize()
+            loc_ms += kev[0].elapsed_time(kev[1])
+            loc_bytes += sum(min(int(pos_now[b]), wl.sinks + wl.window) * per_tok for b in range(wl.B))
+    full_gbs = full_bytes / (full_ms * 1e-3) / 1e9
+    loc_gbs = loc_bytes / (loc_ms * 1e-3) / 1e9
+    n_full = min(len(patterns), 8) * min(wl.L, 6)
+
+    # ---------------- end to end: pinned host inputs -> H2D, step, D2H of the results
+    e2e = None
+    if args.e2e:
+        host = [b.cpu().pin_memory() for b in store]
+        out_h = torch.empty((wl.B, wl.D), dtype=torch.float32).pin_memory()
+        out_f = torch.empty(wl.B, dtype=torch.int32).pin_memory()
+        out_s = torch.empty(wl.B, dtype=torch.float32).pin_memory()
+        for i in range(2):
+            dec.step(host[i % n_store])
+        dec.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(dec.stream):
+            e0.record(dec.stream)
+            for i in range(n_e2e):
+                dec.step(host[i % n_store])
+                out_h.copy_(dec.h_prev, non_blocking=True)
+                out_f.copy_(dec.flag, non_blocking=True)
+                out_s.copy_(dec.score, non_blocking=True)
+            e1.record(dec.stream)
+        torch.cuda.synchronize(dev)
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": world * n_e2e / (e_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": dec.layout.nbytes,
+               "d2h_bytes_per_step": out_h.numel() * 4 + out_f.numel() * 4 + out_s.numel() * 4}
+    err = dec.device_error()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        smp = OracleSample(wl, kv_heads=wl.Hkv)
+        nb, dt = smp.run()
+        cpu = {"value": smp.steps_per_s(nb, dt), "unit": UNIT, "cores": cpu_cores(),
+               "kind": "oracle", "sample": smp.describe(nb, dt)}
+
+    if rank == 0:
+        value = world * K / (elapsed_ms * 1e-3)
+        step_gbs = total_bytes / (elapsed_ms * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "layers": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv,
+                       "head_dim": 128, "ctx": wl.ctx[0], "recall_rate": wl.rates[0],
+                       "page_tokens": 16, "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2 (77 GB resident KV cache), no flush"},
+            "roofline": {"bound": "hbm", "achieved": full_gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": full_gbs / hbm, "traffic": None,
+                         "kernel": "attn_kernel (full set, flagged sequences)",
+                         "peak_source": peak_src, "launches_timed": n_full},
+            "step_roofline": {"algorithmic_gb_per_step": total_bytes / K / 1e9,
+                              "achieved_gbs": step_gbs, "frac": step_gbs / hbm},
+            "local_kernel": {"achieved_gbs": loc_gbs, "frac": loc_gbs / hbm},
+            "realized_recall_rate": realized_rate,
+            "first_step_ms_incl_capture": first_ms, "setup_s": setup_s,
+            "gpu_launches": launches, "device_error": err,
+            "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    dec.close()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=32)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="cfg2")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from workload import configs
+    wl = configs.get(args.workload)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        return
+    import torch
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

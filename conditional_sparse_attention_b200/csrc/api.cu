@@ -1,0 +1,356 @@
+// C ABI entry points: argument validation, context scratch, conditional capture, graphs,
+// error reporting.  Every compute step is one of the kernels in attention.cu, head.cu,
+// commit.cu and glue.cu.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+
+#include "internal.h"
+
+namespace oda {
+
+oda_status prepare_attention_kernel();
+oda_status prepare_head_kernel();
+
+static thread_local char g_msg[512] = "";
+
+oda_status set_error(oda_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+oda_status check_cuda(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return ODA_OK;
+  return set_error(ODA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+__global__ void set_condition_kernel(cudaGraphConditionalHandle h, const int32_t* any_flag) {
+  cudaGraphSetConditional(h, *any_flag != 0 ? 1u : 0u);
+}
+
+oda_status launch_set_condition(cudaGraphConditionalHandle h, const int32_t* any_flag,
+                                cudaStream_t stream) {
+  set_condition_kernel<<<1, 1, 0, stream>>>(h, any_flag);
+  return check_cuda(cudaGetLastError(), "set-condition launch");
+}
+
+}  // namespace oda
+
+using oda::check_cuda;
+using oda::set_error;
+
+struct oda_graph {
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+};
+
+namespace {
+
+template <class T>
+oda_status dev_alloc(T** p, size_t n, const char* what) {
+  *p = nullptr;
+  if (n == 0) n = 1;
+  return check_cuda(cudaMalloc(reinterpret_cast<void**>(p), n * sizeof(T)), what);
+}
+
+void free_ctx(oda_ctx* c) {
+  if (!c) return;
+  void* ptrs[] = {c->part_o, c->part_ml, c->attn_cnt, c->err, c->head_part, c->head_ss,
+                  c->head_cnt, c->head_u, c->head_f, c->head_act, c->glue_x, c->glue_ss,
+                  c->glue_cnt};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+  if (c->body_stream) cudaStreamDestroy(c->body_stream);
+  delete c;
+}
+
+bool stream_capturing(cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return false;
+  return cs == cudaStreamCaptureStatusActive;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t oda_version(void) { return ODA_VERSION_MAJOR * 100 + ODA_VERSION_MINOR; }
+
+const char* oda_status_string(oda_status s) {
+  switch (s) {
+    case ODA_OK: return "ODA_OK";
+    case ODA_ERR_INVALID_ARG: return "ODA_ERR_INVALID_ARG";
+    case ODA_ERR_UNSUPPORTED: return "ODA_ERR_UNSUPPORTED";
+    case ODA_ERR_CUDA: return "ODA_ERR_CUDA";
+    case ODA_ERR_DEVICE: return "ODA_ERR_DEVICE";
+    case ODA_ERR_STATE: return "ODA_ERR_STATE";
+  }
+  return "ODA_ERR_UNKNOWN";
+}
+
+const char* oda_last_error(void) { return oda::g_msg; }
+
+oda_status oda_create(const oda_config* cfg, oda_ctx** out) {
+  if (!out) return set_error(ODA_ERR_INVALID_ARG, "create: out is NULL");
+  *out = nullptr;
+  if (!cfg) return set_error(ODA_ERR_INVALID_ARG, "create: cfg is NULL");
+  const oda_config& c = *cfg;
+  if (c.batch < 1 || c.batch > ODA_MAX_BATCH)
+    return set_error(ODA_ERR_UNSUPPORTED, "create: batch must be 1..%d", ODA_MAX_BATCH);
+  if (c.n_q_heads < 1 || c.n_kv_heads < 1 || c.n_q_heads % c.n_kv_heads != 0 ||
+      c.n_q_heads / c.n_kv_heads > 8)
+    return set_error(ODA_ERR_UNSUPPORTED, "create: need Hq %% Hkv == 0 and Hq/Hkv <= 8");
+  if (c.head_dim != 128) return set_error(ODA_ERR_UNSUPPORTED, "create: head_dim must be 128");
+  if (c.page_size != 16) return set_error(ODA_ERR_UNSUPPORTED, "create: page_size must be 16");
+  if (c.max_pages < 1 || (int64_t)c.max_pages * 16 > INT32_MAX - 1)
+    return set_error(ODA_ERR_INVALID_ARG, "create: max_pages out of range");
+  if (c.sinks < 0 || c.sinks > 16) return set_error(ODA_ERR_UNSUPPORTED, "create: sinks must be 0..16");
+  if (c.window < 1) return set_error(ODA_ERR_INVALID_ARG, "create: window must be >= 1");
+  if (c.head_in_dim < 512 || c.head_in_dim > 8192 || c.head_in_dim % 512 != 0)
+    return set_error(ODA_ERR_UNSUPPORTED, "create: head_in_dim must be a multiple of 512 in 512..8192");
+
+  oda_ctx* x = new oda_ctx();
+  x->cfg = c;
+  x->g = c.n_q_heads / c.n_kv_heads;
+  oda_status st = check_cuda(cudaGetDevice(&x->device), "cudaGetDevice");
+  if (st == ODA_OK)
+    st = check_cuda(cudaDeviceGetAttribute(&x->n_sms, cudaDevAttrMultiProcessorCount, x->device),
+                    "cudaDeviceGetAttribute");
+  if (st == ODA_OK) st = oda::prepare_attention_kernel();
+  if (st == ODA_OK) st = oda::prepare_head_kernel();
+  if (st != ODA_OK) {
+    free_ctx(x);
+    return st;
+  }
+  x->attn_ctas = x->n_sms * oda::attention_ctas_per_sm();
+  // split partials: bounded by ~512 MiB and by the combine's shared-memory weight table
+  const int64_t B = c.batch, Hq = c.n_q_heads, Hkv = c.n_kv_heads, D = c.head_in_dim;
+  int64_t ms = (c.max_pages + 7) / 8 + 2;
+  const int64_t budget = (512ll << 20) / (B * Hq * 130 * 4);
+  ms = std::min<int64_t>(ms, std::max<int64_t>(16, budget));
+  ms = std::min<int64_t>(ms, 3072);
+  x->max_splits = (int)ms;
+  const int gch = oda::glue_chunks(c.head_in_dim);
+  st = dev_alloc(&x->part_o, (size_t)B * Hq * ms * 128, "cudaMalloc(partials)");
+  if (st == ODA_OK) st = dev_alloc(&x->part_ml, (size_t)B * Hq * ms * 2, "cudaMalloc(partials)");
+  if (st == ODA_OK) st = dev_alloc(&x->attn_cnt, (size_t)B * Hkv, "cudaMalloc(counters)");
+  if (st == ODA_OK) st = dev_alloc(&x->err, 1, "cudaMalloc(error word)");
+  if (st == ODA_OK) st = dev_alloc(&x->head_part, oda::head_part_floats((int)B, (int)D), "cudaMalloc(head)");
+  if (st == ODA_OK) st = dev_alloc(&x->head_ss, (size_t)96 * (D / 512) * B, "cudaMalloc(head)");
+  if (st == ODA_OK) st = dev_alloc(&x->head_cnt, (size_t)oda::head_counter_count((int)D), "cudaMalloc(head)");
+  if (st == ODA_OK) st = dev_alloc(&x->head_u, (size_t)3 * B * 1024, "cudaMalloc(head)");
+  if (st == ODA_OK) st = dev_alloc(&x->head_f, (size_t)3 * B * 1024, "cudaMalloc(head)");
+  if (st == ODA_OK) st = dev_alloc(&x->head_act, (size_t)B * 2048, "cudaMalloc(head)");
+  if (st == ODA_OK) st = dev_alloc(&x->glue_x, (size_t)B * D, "cudaMalloc(glue)");
+  if (st == ODA_OK) st = dev_alloc(&x->glue_ss, (size_t)B * gch, "cudaMalloc(glue)");
+  if (st == ODA_OK) st = dev_alloc(&x->glue_cnt, (size_t)2 * B, "cudaMalloc(glue)");
+  if (st == ODA_OK) st = check_cuda(cudaMemset(x->attn_cnt, 0, B * Hkv * sizeof(int32_t)), "cudaMemset");
+  if (st == ODA_OK) st = check_cuda(cudaMemset(x->err, 0, sizeof(int32_t)), "cudaMemset");
+  if (st == ODA_OK)
+    st = check_cuda(cudaMemset(x->head_cnt, 0, oda::head_counter_count((int)D) * sizeof(int32_t)),
+                    "cudaMemset");
+  if (st == ODA_OK) st = check_cuda(cudaMemset(x->glue_cnt, 0, 2 * B * sizeof(int32_t)), "cudaMemset");
+  if (st == ODA_OK)
+    st = check_cuda(cudaStreamCreateWithFlags(&x->body_stream, cudaStreamNonBlocking),
+                    "cudaStreamCreate");
+  if (st == ODA_OK) st = check_cuda(cudaDeviceSynchronize(), "cudaDeviceSynchronize");
+  if (st != ODA_OK) {
+    free_ctx(x);
+    return st;
+  }
+  *out = x;
+  return ODA_OK;
+}
+
+oda_status oda_destroy(oda_ctx* ctx) {
+  if (!ctx) return ODA_OK;
+  cudaDeviceSynchronize();
+  free_ctx(ctx);
+  return ODA_OK;
+}
+
+oda_status oda_attend_local(oda_ctx* ctx, const oda_kv_layer* layer, const int32_t* page_table,
+                            const int32_t* pos, const void* q, const void* k_new,
+                            const void* v_new, float* out, cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "attend_local: ctx is NULL");
+  return oda::launch_attention(ctx, layer, page_table, pos, nullptr, q, k_new, v_new, out, 0, stream);
+}
+
+oda_status oda_attend_full_if(oda_ctx* ctx, const oda_kv_layer* layer, const int32_t* page_table,
+                              const int32_t* pos, const int32_t* flag, const void* q,
+                              const void* k_new, const void* v_new, float* out,
+                              cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "attend_full_if: ctx is NULL");
+  return oda::launch_attention(ctx, layer, page_table, pos, flag, q, k_new, v_new, out, 1, stream);
+}
+
+oda_status oda_index_positions(oda_ctx* ctx, int32_t mode, const int32_t* pos, const int32_t* flag,
+                               int32_t* positions, int32_t cap, int32_t* counts,
+                               cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "index_positions: ctx is NULL");
+  return oda::launch_index_positions(ctx, mode, pos, flag, positions, cap, counts, stream);
+}
+
+oda_status oda_recall_score(oda_ctx* ctx, const oda_head_weights* w, const float* h_prev,
+                            const float* emb, const float* h_loc, const int32_t* sched,
+                            float* score, int32_t* flag, int32_t* any_flag, cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "recall_score: ctx is NULL");
+  return oda::launch_recall_head(ctx, w, h_prev, emb, h_loc, sched, score, flag, any_flag, stream);
+}
+
+oda_status oda_commit(oda_ctx* ctx, const oda_kv_layer* layers, int32_t n_layers,
+                      const int32_t* page_table, int32_t* pos, const int32_t* flag,
+                      const void* k_stage_local, const void* v_stage_local,
+                      const void* k_stage_full, const void* v_stage_full,
+                      const float* h_local, const float* h_full, float* h_prev,
+                      cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "commit: ctx is NULL");
+  return oda::launch_commit(ctx, layers, n_layers, page_table, pos, flag, k_stage_local,
+                            v_stage_local, k_stage_full, v_stage_full, h_local, h_full, h_prev,
+                            stream);
+}
+
+oda_status oda_snapshot(oda_ctx* ctx, const oda_state* live, const oda_state* snap,
+                        cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "snapshot: ctx is NULL");
+  return oda::launch_state_copy(live, snap, ctx->cfg.batch, nullptr, stream);
+}
+
+oda_status oda_restore(oda_ctx* ctx, const int32_t* flag, const oda_state* snap,
+                       const oda_state* live, cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "restore: ctx is NULL");
+  if (!flag) return set_error(ODA_ERR_INVALID_ARG, "restore: flag is NULL");
+  return oda::launch_state_copy(snap, live, ctx->cfg.batch, flag, stream);
+}
+
+oda_status oda_glue_hidden(oda_ctx* ctx, const float* emb, const float* terms, int32_t n_terms,
+                           const int32_t* flag, float* h, cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "glue_hidden: ctx is NULL");
+  return oda::launch_glue_hidden(ctx, emb, terms, n_terms, flag, h, stream);
+}
+
+oda_status oda_glue_gdn(oda_ctx* ctx, const oda_state* st, int32_t layer, const float* c,
+                        const float* v, const float* alpha, const float* beta,
+                        const float* taps, const int32_t* flag, float* o, cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "glue_gdn: ctx is NULL");
+  return oda::launch_glue_gdn(ctx, st, layer, c, v, alpha, beta, taps, flag, o, stream);
+}
+
+oda_status oda_cond_begin(oda_ctx* ctx, cudaStream_t stream, const int32_t* any_flag,
+                          cudaStream_t* body_stream) {
+  if (!ctx || !any_flag || !body_stream)
+    return set_error(ODA_ERR_INVALID_ARG, "cond_begin: null argument");
+  if (ctx->cond_open) return set_error(ODA_ERR_STATE, "cond_begin: a conditional is already open");
+  if (!stream_capturing(stream)) {
+    ctx->cond_open = true;
+    ctx->cond_parent = nullptr;
+    *body_stream = stream;
+    return ODA_OK;
+  }
+  cudaStreamCaptureStatus cs;
+  cudaGraph_t graph = nullptr;
+  const cudaGraphNode_t* deps = nullptr;
+  size_t nd = 0;
+  oda_status st = check_cuda(cudaStreamGetCaptureInfo(stream, &cs, nullptr, &graph, &deps, &nd),
+                             "cudaStreamGetCaptureInfo");
+  if (st != ODA_OK) return st;
+  cudaGraphConditionalHandle h;
+  st = check_cuda(cudaGraphConditionalHandleCreate(&h, graph, 0, cudaGraphCondAssignDefault),
+                  "cudaGraphConditionalHandleCreate");
+  if (st != ODA_OK) return st;
+  st = oda::launch_set_condition(h, any_flag, stream);
+  if (st != ODA_OK) return st;
+  st = check_cuda(cudaStreamGetCaptureInfo(stream, &cs, nullptr, &graph, &deps, &nd),
+                  "cudaStreamGetCaptureInfo");
+  if (st != ODA_OK) return st;
+  cudaGraphNodeParams np = {cudaGraphNodeTypeConditional};
+  np.conditional.handle = h;
+  np.conditional.type = cudaGraphCondTypeIf;
+  np.conditional.size = 1;
+  cudaGraphNode_t node;
+  st = check_cuda(cudaGraphAddNode(&node, graph, deps, nd, &np), "cudaGraphAddNode(conditional)");
+  if (st != ODA_OK) return st;
+  cudaGraph_t body = np.conditional.phGraph_out[0];
+  st = check_cuda(cudaStreamUpdateCaptureDependencies(stream, &node, 1,
+                                                      cudaStreamSetCaptureDependencies),
+                  "cudaStreamUpdateCaptureDependencies");
+  if (st != ODA_OK) return st;
+  st = check_cuda(cudaStreamBeginCaptureToGraph(ctx->body_stream, body, nullptr, nullptr, 0,
+                                                cudaStreamCaptureModeRelaxed),
+                  "cudaStreamBeginCaptureToGraph");
+  if (st != ODA_OK) return st;
+  ctx->cond_open = true;
+  ctx->cond_parent = stream;
+  *body_stream = ctx->body_stream;
+  return ODA_OK;
+}
+
+oda_status oda_cond_end(oda_ctx* ctx, cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "cond_end: ctx is NULL");
+  if (!ctx->cond_open) return set_error(ODA_ERR_STATE, "cond_end: no open conditional");
+  ctx->cond_open = false;
+  if (ctx->cond_parent == nullptr) return ODA_OK;
+  if (ctx->cond_parent != stream)
+    return set_error(ODA_ERR_STATE, "cond_end: stream differs from the one given to cond_begin");
+  ctx->cond_parent = nullptr;
+  cudaGraph_t g = nullptr;
+  return check_cuda(cudaStreamEndCapture(ctx->body_stream, &g), "cudaStreamEndCapture(body)");
+}
+
+oda_status oda_graph_begin(cudaStream_t stream) {
+  return check_cuda(cudaStreamBeginCapture(stream, cudaStreamCaptureModeRelaxed),
+                    "cudaStreamBeginCapture");
+}
+
+oda_status oda_graph_end(cudaStream_t stream, oda_graph** out) {
+  if (!out) return set_error(ODA_ERR_INVALID_ARG, "graph_end: out is NULL");
+  *out = nullptr;
+  oda_graph* g = new oda_graph();
+  oda_status st = check_cuda(cudaStreamEndCapture(stream, &g->graph), "cudaStreamEndCapture");
+  if (st == ODA_OK)
+    st = check_cuda(cudaGraphInstantiate(&g->exec, g->graph, 0), "cudaGraphInstantiate");
+  if (st != ODA_OK) {
+    if (g->graph) cudaGraphDestroy(g->graph);
+    delete g;
+    return st;
+  }
+  *out = g;
+  return ODA_OK;
+}
+
+oda_status oda_graph_launch(oda_graph* g, cudaStream_t stream) {
+  if (!g) return set_error(ODA_ERR_INVALID_ARG, "graph_launch: graph is NULL");
+  return check_cuda(cudaGraphLaunch(g->exec, stream), "cudaGraphLaunch");
+}
+
+oda_status oda_graph_destroy(oda_graph* g) {
+  if (!g) return ODA_OK;
+  if (g->exec) cudaGraphExecDestroy(g->exec);
+  if (g->graph) cudaGraphDestroy(g->graph);
+  delete g;
+  return ODA_OK;
+}
+
+oda_status oda_get_error(oda_ctx* ctx, int32_t* device_error) {
+  if (!ctx || !device_error) return set_error(ODA_ERR_INVALID_ARG, "get_error: null argument");
+  oda_status st = check_cuda(cudaDeviceSynchronize(), "cudaDeviceSynchronize");
+  if (st != ODA_OK) return st;
+  st = check_cuda(cudaMemcpy(device_error, ctx->err, sizeof(int32_t), cudaMemcpyDeviceToHost),
+                  "cudaMemcpy(error word)");
+  if (st != ODA_OK) return st;
+  if (*device_error != 0)
+    return set_error(ODA_ERR_DEVICE, "device error word 0x%x", (unsigned)*device_error);
+  return ODA_OK;
+}
+
+oda_status oda_clear_error(oda_ctx* ctx, cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "clear_error: ctx is NULL");
+  return check_cuda(cudaMemsetAsync(ctx->err, 0, sizeof(int32_t), stream), "cudaMemsetAsync");
+}
+
+}  // extern "C"

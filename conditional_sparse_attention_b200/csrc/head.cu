@@ -1,0 +1,424 @@
+// Recall head R(h_{t-1}, E(x_t), h^L_t) -> q_t and the routing gate, fp32.
+//
+// Method: "On-Demand Attention：让语言模型按需读取完整历史" (method notes) §2.2 eq. q_t and the
+// paragraph after it (three inputs, per-input normalise + project + activate to 1024, a 9216-d
+// interaction of the three vectors, their pairwise products and absolute differences, a
+// projection with residual fusion, two residual gated feed-forward blocks, scalar output, fp32);
+// §2.3 (full iff the score exceeds theta or is not finite).  Layer details follow this reading:
+//   u_i = SiLU(W_i (RMSNorm(x_i) * gamma_i) + b_i)
+//   f   = W_f z + b_f + (u_0 + u_1 + u_2) / 3
+//   f  += W_d (SiLU(W_g m) * (W_u m)),  m = RMSNorm(f) * gamma_j      (two blocks)
+//   q   = w_o . (RMSNorm(f) * gamma_o) + b_o
+//
+// Design: at batch sizes of a few sequences the head is a weight-streaming problem (113 MB of
+// fp32 weights for D = 2048, 2*B flops per 4-byte weight), so every phase is a split-K GEMV on
+// CUDA cores: a CTA streams a 32-row x Kc slab of one weight matrix exactly once with 16-byte
+// non-allocating loads and multiplies it against a shared-memory tile of up to 8 sequences'
+// inputs; lanes reduce with a 31-shuffle butterfly.  The input transform of a phase (RMSNorm
+// scale, the interaction vector, the gated activation) is applied while the tile is built, and
+// the output epilogue (bias, SiLU, residual) runs in the last CTA of each row block, which sums
+// the split-K partials in a fixed order (deterministic results).  The last row block of the
+// final phase also computes q and the gate.  Six launches per score.
+#include <cmath>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace oda {
+namespace {
+
+constexpr int kT = 1024;       // tower width
+constexpr int kF = 2048;       // gated FFN width
+constexpr int kHT = 256;       // threads per CTA
+constexpr int kWarps = kHT / 32;
+constexpr int kRowsPerWarp = 4;
+constexpr int kRowsPerCta = kWarps * kRowsPerWarp;   // 32 weight rows
+constexpr int kBT = 8;         // sequences per tile
+constexpr float kEps = 1e-6f;
+
+enum Phase { kTower = 0, kFuse = 1, kUp = 2, kDown = 3 };
+
+struct HeadParams {
+  oda_head_weights w;
+  const float* x[3];      // h_prev, emb, h_loc  [B][D]
+  const int32_t* sched;
+  float* score;
+  int32_t* flag;
+  int32_t* any_flag;
+  float* part;            // split-K partials [nchunks][B][rows_total]
+  float* ss;              // tower sums of squares [row_blocks][nchunks][B]
+  int32_t* cnt;           // [row blocks] + [final]
+  float* u;               // [3][B][T]
+  float* f;               // [3][B][T]  (f0 fusion output, f1 block 0 output, f2 block 1 output)
+  float* act;             // [B][F]
+  int B, D;
+  int phase, block;       // block: FFN block index for kUp / kDown
+  int Kc, nchunks, rows_total, row_blocks;
+  float theta;
+};
+
+__device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
+
+// Weights are read once per score when B <= 8 (streaming hint); larger batches loop over
+// sequence tiles and re-read the CTA's slab, so they keep it cacheable.
+__device__ __forceinline__ float4 ldg_w(const float* p, bool stream) {
+  return stream ? __ldcs(reinterpret_cast<const float4*>(p))
+                : __ldg(reinterpret_cast<const float4*>(p));
+}
+
+// Sum of squares of row x[b][0..n) (whole block cooperates; result in every thread).
+__device__ float block_sum(float v, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < kWarps; ++i) s += red[i];
+  return s;
+}
+
+// The weight row that value slot r (0..3) of warp `warp` in row block `rb` multiplies, and
+// where its partial goes (column of the partial matrix).
+__device__ __forceinline__ const float* weight_row(const HeadParams& p, int rb, int warp, int r,
+                                                   int* col) {
+  const oda_head_weights& w = p.w;
+  if (p.phase == kTower) {
+    const int row = rb * kRowsPerCta + warp * kRowsPerWarp + r;   // 0 .. 3*T-1
+    const int i = row / kT, n = row % kT;
+    *col = row;
+    return w.tower_w[i] + (size_t)n * p.D;
+  }
+  if (p.phase == kFuse) {
+    const int n = rb * kRowsPerCta + warp * kRowsPerWarp + r;
+    *col = n;
+    return w.fuse_w + (size_t)n * (9 * kT);
+  }
+  if (p.phase == kUp) {
+    // 16 FFN units per row block; a warp takes 2 units, gate rows then up rows
+    const int n = rb * (kRowsPerCta / 2) + warp * 2 + (r & 1);
+    const bool up = r >= 2;
+    *col = (up ? kF : 0) + n;
+    return (up ? w.ffn_up[p.block] : w.ffn_gate[p.block]) + (size_t)n * kT;
+  }
+  const int n = rb * kRowsPerCta + warp * kRowsPerWarp + r;
+  *col = n;
+  return w.ffn_down[p.block] + (size_t)n * kF;
+}
+
+// Builds the input tile X[bb][0..Kc) for sequences b0..b0+7 of chunk `chunk` (zeros beyond B).
+__device__ void build_tile(const HeadParams& p, int rb, int chunk, int b0, float* X, float* ss_out,
+                           float* red) {
+  const int k0 = chunk * p.Kc;
+  for (int idx = threadIdx.x; idx < kBT * p.Kc; idx += kHT) {
+    const int bb = idx / p.Kc, k = idx % p.Kc, b = b0 + bb;
+    float v = 0.f;
+    if (b < p.B) {
+      const int kg = k0 + k;
+      if (p.phase == kTower) {
+        const int i = (rb * kRowsPerCta) / kT;
+        v = p.x[i][(size_t)b * p.D + kg];
+      } else if (p.phase == kFuse) {
+        const int blk = kg / kT, e = kg % kT;
+        const float u0 = p.u[((size_t)0 * p.B + b) * kT + e];
+        const float u1 = p.u[((size_t)1 * p.B + b) * kT + e];
+        const float u2 = p.u[((size_t)2 * p.B + b) * kT + e];
+        switch (blk) {
+          case 0: v = u0; break;
+          case 1: v = u1; break;
+          case 2: v = u2; break;
+          case 3: v = u0 * u1; break;
+          case 4: v = u0 * u2; break;
+          case 5: v = u1 * u2; break;
+          case 6: v = fabsf(u0 - u1); break;
+          case 7: v = fabsf(u0 - u2); break;
+          default: v = fabsf(u1 - u2); break;
+        }
+      } else if (p.phase == kUp) {
+        v = p.f[((size_t)p.block * p.B + b) * kT + kg];   // scaled below
+      } else {
+        v = p.act[(size_t)b * kF + kg];
+      }
+    }
+    X[idx] = v;
+  }
+  __syncthreads();
+  if (p.phase == kTower) {
+    // sum of squares of this chunk of x_i per sequence (for the RMSNorm scale), then gamma
+    const int i = (rb * kRowsPerCta) / kT;
+    for (int bb = 0; bb < kBT; ++bb) {
+      float s = 0.f;
+      for (int k = threadIdx.x; k < p.Kc; k += kHT) s += X[bb * p.Kc + k] * X[bb * p.Kc + k];
+      s = block_sum(s, red);
+      if (threadIdx.x == 0 && b0 + bb < p.B)
+        ss_out[((size_t)rb * p.nchunks + chunk) * p.B + b0 + bb] = s;
+    }
+    const float* gam = p.w.tower_norm[i] + k0;
+    for (int idx = threadIdx.x; idx < kBT * p.Kc; idx += kHT) X[idx] *= gam[idx % p.Kc];
+    __syncthreads();
+  } else if (p.phase == kUp) {
+    // m = RMSNorm(f) * gamma over the full 1024-wide f
+    const float* gam = p.w.ffn_norm[p.block] + k0;
+    for (int bb = 0; bb < kBT; ++bb) {
+      const int b = b0 + bb;
+      float s = 0.f;
+      if (b < p.B) {
+        const float* fr = p.f + ((size_t)p.block * p.B + b) * kT;
+        for (int k = threadIdx.x; k < kT; k += kHT) s += fr[k] * fr[k];
+      }
+      s = block_sum(s, red);
+      const float inv = rsqrtf(s / kT + kEps);
+      for (int k = threadIdx.x; k < p.Kc; k += kHT) X[bb * p.Kc + k] *= inv * gam[k];
+    }
+    __syncthreads();
+  }
+}
+
+__global__ void __launch_bounds__(kHT) head_phase_kernel(const HeadParams p) {
+  extern __shared__ float X[];           // [kBT][Kc]
+  __shared__ float red[kWarps];
+  __shared__ int s_last;
+  const int rb = blockIdx.x / p.nchunks, chunk = blockIdx.x % p.nchunks;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k0 = chunk * p.Kc;
+
+  int cols[kRowsPerWarp];
+  const float* wrow[kRowsPerWarp];
+#pragma unroll
+  for (int r = 0; r < kRowsPerWarp; ++r) wrow[r] = weight_row(p, rb, warp, r, &cols[r]) + k0;
+
+  const bool single_pass = p.B <= kBT;
+  for (int b0 = 0; b0 < p.B; b0 += kBT) {
+    build_tile(p, rb, chunk, b0, X, p.ss, red);
+    float acc[kRowsPerWarp][kBT];
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r)
+#pragma unroll
+      for (int bb = 0; bb < kBT; ++bb) acc[r][bb] = 0.f;
+    const int n4 = p.Kc / 4;
+#pragma unroll 2
+    for (int k4 = lane; k4 < n4; k4 += 32) {
+      float4 wv[kRowsPerWarp];
+#pragma unroll
+      for (int r = 0; r < kRowsPerWarp; ++r) wv[r] = ldg_w(wrow[r] + 4 * k4, single_pass);
+#pragma unroll
+      for (int bb = 0; bb < kBT; ++bb) {
+        const float4 xv = *reinterpret_cast<const float4*>(X + bb * p.Kc + 4 * k4);
+#pragma unroll
+        for (int r = 0; r < kRowsPerWarp; ++r)
+          acc[r][bb] += wv[r].x * xv.x + wv[r].y * xv.y + wv[r].z * xv.z + wv[r].w * xv.w;
+      }
+    }
+    // butterfly: after 5 stages lane l holds the lane-sum of value l = (r = l / 8, bb = l % 8)
+    float v[32];
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r)
+#pragma unroll
+      for (int bb = 0; bb < kBT; ++bb) v[r * kBT + bb] = acc[r][bb];
+#pragma unroll
+    for (int half = 16; half >= 1; half >>= 1) {
+      const bool upper = (lane & half) != 0;
+#pragma unroll
+      for (int i = 0; i < half; ++i) {
+        const float send = upper ? v[i] : v[i + half];
+        const float keep = upper ? v[i + half] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+      }
+    }
+    {
+      const int r = lane >> 3, bb = lane & 7, b = b0 + bb;
+      int col = cols[0];
+#pragma unroll
+      for (int rr = 1; rr < kRowsPerWarp; ++rr)
+        if (r == rr) col = cols[rr];
+      if (b < p.B) p.part[((size_t)chunk * p.B + b) * p.rows_total + col] = v[0];
+    }
+    __syncthreads();
+  }
+
+  // ---- last CTA of the row block: reduce partials in chunk order and apply the epilogue
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(&p.cnt[rb], 1) == p.nchunks - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int units = (p.phase == kUp) ? kRowsPerCta / 2 : kRowsPerCta;
+  for (int idx = threadIdx.x; idx < units * p.B; idx += kHT) {
+    const int j = idx % units, b = idx / units;
+    if (p.phase == kTower) {
+      const int row = rb * kRowsPerCta + j, i = row / kT, n = row % kT;
+      float acc = 0.f, ss = 0.f;
+      for (int ch = 0; ch < p.nchunks; ++ch) {
+        acc += __ldcg(p.part + ((size_t)ch * p.B + b) * p.rows_total + row);
+        ss += __ldcg(p.ss + ((size_t)rb * p.nchunks + ch) * p.B + b);
+      }
+      const float inv = rsqrtf(ss / p.D + kEps);
+      p.u[((size_t)i * p.B + b) * kT + n] = silu(acc * inv + p.w.tower_b[i][n]);
+    } else if (p.phase == kFuse) {
+      const int n = rb * kRowsPerCta + j;
+      float acc = 0.f;
+      for (int ch = 0; ch < p.nchunks; ++ch)
+        acc += __ldcg(p.part + ((size_t)ch * p.B + b) * p.rows_total + n);
+      const float mean = (__ldcg(p.u + ((size_t)0 * p.B + b) * kT + n) +
+                          __ldcg(p.u + ((size_t)1 * p.B + b) * kT + n) +
+                          __ldcg(p.u + ((size_t)2 * p.B + b) * kT + n)) / 3.0f;
+      p.f[((size_t)0 * p.B + b) * kT + n] = acc + p.w.fuse_b[n] + mean;
+    } else if (p.phase == kUp) {
+      const int n = rb * (kRowsPerCta / 2) + j;
+      float ga = 0.f, ua = 0.f;
+      for (int ch = 0; ch < p.nchunks; ++ch) {
+        ga += __ldcg(p.part + ((size_t)ch * p.B + b) * p.rows_total + n);
+        ua += __ldcg(p.part + ((size_t)ch * p.B + b) * p.rows_total + kF + n);
+      }
+      p.act[(size_t)b * kF + n] = silu(ga) * ua;
+    } else {
+      const int n = rb * kRowsPerCta + j;
+      float acc = 0.f;
+      for (int ch = 0; ch < p.nchunks; ++ch)
+        acc += __ldcg(p.part + ((size_t)ch * p.B + b) * p.rows_total + n);
+      p.f[((size_t)(p.block + 1) * p.B + b) * kT + n] =
+          __ldcg(p.f + ((size_t)p.block * p.B + b) * kT + n) + acc;
+    }
+  }
+  if (threadIdx.x == 0) p.cnt[rb] = 0;
+  if (!(p.phase == kDown && p.block == 1)) return;
+
+  // ---- final row block done: q = w_o . (RMSNorm(f2) * gamma_o) + b_o and the gate
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(&p.cnt[p.row_blocks], 1) == p.row_blocks - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  __shared__ int s_any;
+  if (threadIdx.x == 0) s_any = 0;
+  __syncthreads();
+  for (int b = warp; b < p.B; b += kWarps) {
+    const float* fr = p.f + ((size_t)2 * p.B + b) * kT;
+    float ss = 0.f, dot = 0.f;
+    for (int k = lane; k < kT; k += 32) {
+      const float fv = __ldcg(fr + k);
+      ss += fv * fv;
+      dot += p.w.out_w[k] * p.w.out_norm[k] * fv;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    }
+    if (lane == 0) {
+      const float q = dot * rsqrtf(ss / kT + kEps) + p.w.out_b[0];
+      p.score[b] = q;
+      int fl;
+      if (p.sched) {
+        fl = p.sched[b] != 0;
+      } else {
+        const bool nonfinite = (__float_as_uint(q) & 0x7f800000u) == 0x7f800000u;
+        fl = (nonfinite || q > p.theta) ? 1 : 0;
+      }
+      p.flag[b] = fl;
+      if (fl) atomicOr(&s_any, 1);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    *p.any_flag = s_any;
+    p.cnt[p.row_blocks] = 0;
+  }
+}
+
+struct PhaseShape {
+  int Kc, nchunks, rows_total, row_blocks;
+};
+
+PhaseShape phase_shape(int phase, int D) {
+  switch (phase) {
+    case kTower: return {512, D / 512, 3 * kT, 3 * kT / kRowsPerCta};
+    case kFuse: return {1024, 9, kT, kT / kRowsPerCta};
+    case kUp: return {512, kT / 512, 2 * kF, kF / (kRowsPerCta / 2)};
+    default: return {256, kF / 256, kT, kT / kRowsPerCta};
+  }
+}
+
+}  // namespace
+
+size_t head_part_floats(int B, int D) {
+  size_t m = 0;
+  for (int ph = 0; ph < 4; ++ph) {
+    const PhaseShape s = phase_shape(ph, D);
+    m = std::max(m, (size_t)s.nchunks * B * s.rows_total);
+  }
+  return m;
+}
+
+int head_counter_count(int D) {
+  int m = 0;
+  for (int ph = 0; ph < 4; ++ph) m = std::max(m, phase_shape(ph, D).row_blocks);
+  return m + 1;
+}
+
+oda_status prepare_head_kernel() {
+  return check_cuda(cudaFuncSetAttribute(head_phase_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kBT * 1024 * (int)sizeof(float)),
+                    "cudaFuncSetAttribute(head)");
+}
+
+oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const float* h_prev,
+                              const float* emb, const float* h_loc, const int32_t* sched,
+                              float* score, int32_t* flag, int32_t* any_flag, cudaStream_t s) {
+  if (!w || !h_prev || !emb || !h_loc || !score || !flag || !any_flag)
+    return set_error(ODA_ERR_INVALID_ARG, "recall_score: null pointer argument");
+  const void* ptrs[] = {w->fuse_w, w->fuse_b, w->out_norm, w->out_w, w->out_b};
+  for (const void* q : ptrs)
+    if (!q) return set_error(ODA_ERR_INVALID_ARG, "recall_score: null weight pointer");
+  for (int i = 0; i < 3; ++i)
+    if (!w->tower_norm[i] || !w->tower_w[i] || !w->tower_b[i])
+      return set_error(ODA_ERR_INVALID_ARG, "recall_score: null tower weight pointer");
+  for (int j = 0; j < 2; ++j)
+    if (!w->ffn_norm[j] || !w->ffn_gate[j] || !w->ffn_up[j] || !w->ffn_down[j])
+      return set_error(ODA_ERR_INVALID_ARG, "recall_score: null FFN weight pointer");
+  const void* mats[] = {w->tower_w[0], w->tower_w[1], w->tower_w[2], w->fuse_w, w->ffn_gate[0],
+                        w->ffn_gate[1], w->ffn_up[0], w->ffn_up[1], w->ffn_down[0], w->ffn_down[1],
+                        h_prev, emb, h_loc};
+  for (const void* q : mats)
+    if (reinterpret_cast<uintptr_t>(q) & 15)
+      return set_error(ODA_ERR_INVALID_ARG, "recall_score: matrices and inputs must be 16-byte aligned");
+  HeadParams p;
+  p.w = *w;
+  p.x[0] = h_prev;
+  p.x[1] = emb;
+  p.x[2] = h_loc;
+  p.sched = sched;
+  p.score = score;
+  p.flag = flag;
+  p.any_flag = any_flag;
+  p.part = ctx->head_part;
+  p.ss = ctx->head_ss;
+  p.cnt = ctx->head_cnt;
+  p.u = ctx->head_u;
+  p.f = ctx->head_f;
+  p.act = ctx->head_act;
+  p.B = ctx->cfg.batch;
+  p.D = ctx->cfg.head_in_dim;
+  p.theta = ctx->cfg.theta;
+  const int seq[6][2] = {{kTower, 0}, {kFuse, 0}, {kUp, 0}, {kDown, 0}, {kUp, 1}, {kDown, 1}};
+  for (int i = 0; i < 6; ++i) {
+    p.phase = seq[i][0];
+    p.block = seq[i][1];
+    const PhaseShape sh = phase_shape(p.phase, p.D);
+    p.Kc = sh.Kc;
+    p.nchunks = sh.nchunks;
+    p.rows_total = sh.rows_total;
+    p.row_blocks = sh.row_blocks;
+    head_phase_kernel<<<sh.row_blocks * sh.nchunks, kHT, kBT * sh.Kc * sizeof(float), s>>>(p);
+    oda_status st = check_cuda(cudaGetLastError(), "recall head launch");
+    if (st != ODA_OK) return st;
+  }
+  return ODA_OK;
+}
+
+}  // namespace oda

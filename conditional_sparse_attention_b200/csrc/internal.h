@@ -1,0 +1,85 @@
+// Internal declarations shared by the library's translation units (not installed).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "oda.h"
+#include "oda_glue.h"
+
+struct oda_ctx {
+  oda_config cfg;
+  int device = 0;
+  int n_sms = 0;
+  int g = 1;
+  // split-KV attention scratch
+  int max_splits = 0;
+  int attn_ctas = 0;          // persistent grid size of the attention kernel
+  float* part_o = nullptr;    // [B*Hq][max_splits][128]
+  float* part_ml = nullptr;   // [B*Hq][max_splits][2]
+  int32_t* attn_cnt = nullptr;  // [B*Hkv] completion counters (self-resetting)
+  int32_t* err = nullptr;       // sticky device error word
+  // recall-head scratch
+  float* head_part = nullptr;   // split-K partial sums, largest phase
+  float* head_ss = nullptr;     // partial sums of squares of the tower inputs
+  int32_t* head_cnt = nullptr;  // per row-block completion counters + final counter
+  float* head_u = nullptr;      // [3][B][1024]
+  float* head_f = nullptr;      // [3][B][1024]: fusion output and the two block outputs
+  float* head_act = nullptr;    // [B][2048]
+  // glue scratch
+  float* glue_x = nullptr;      // [B][D]
+  float* glue_ss = nullptr;     // [B][chunks]
+  int32_t* glue_cnt = nullptr;  // [B]
+  // conditional capture
+  cudaStream_t body_stream = nullptr;
+  cudaStream_t cond_parent = nullptr;
+  bool cond_open = false;
+  void* alloc_base = nullptr;
+};
+
+namespace oda {
+
+oda_status set_error(oda_status s, const char* fmt, ...);
+oda_status check_cuda(cudaError_t e, const char* what);
+
+// attention.cu
+oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32_t* page_table,
+                            const int32_t* pos, const int32_t* flag, const void* q,
+                            const void* k_new, const void* v_new, float* out, int mode,
+                            cudaStream_t stream);
+oda_status launch_index_positions(oda_ctx* ctx, int mode, const int32_t* pos, const int32_t* flag,
+                                  int32_t* positions, int32_t cap, int32_t* counts,
+                                  cudaStream_t stream);
+int attention_smem_bytes();
+int attention_threads();
+int attention_ctas_per_sm();
+
+// head.cu
+oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const float* h_prev,
+                              const float* emb, const float* h_loc, const int32_t* sched,
+                              float* score, int32_t* flag, int32_t* any_flag, cudaStream_t s);
+size_t head_part_floats(int B, int D);
+int head_counter_count(int D);
+
+// commit.cu
+oda_status launch_commit(oda_ctx* ctx, const oda_kv_layer* layers, int32_t n_layers,
+                         const int32_t* page_table, int32_t* pos, const int32_t* flag,
+                         const void* ksl, const void* vsl, const void* ksf, const void* vsf,
+                         const float* h_local, const float* h_full, float* h_prev,
+                         cudaStream_t stream);
+oda_status launch_state_copy(const oda_state* src, const oda_state* dst, int B,
+                             const int32_t* flag, cudaStream_t stream);
+
+// glue.cu
+oda_status launch_glue_hidden(oda_ctx* ctx, const float* emb, const float* terms, int n_terms,
+                              const int32_t* flag, float* h, cudaStream_t stream);
+oda_status launch_glue_gdn(oda_ctx* ctx, const oda_state* st, int layer, const float* c,
+                           const float* v, const float* alpha, const float* beta,
+                           const float* taps, const int32_t* flag, float* o, cudaStream_t s);
+int glue_chunks(int D);
+
+// cond.cu
+oda_status launch_set_condition(cudaGraphConditionalHandle h, const int32_t* any_flag,
+                                cudaStream_t stream);
+
+}  // namespace oda

@@ -1,0 +1,238 @@
+"""Decode-step driver: runs ODA steps of a synthetic workload through the C ABI.
+
+One step, in the order of the method notes ("On-Demand Attention：让语言模型按需读取完整历史")
+§2.3, issued on one stream with no host synchronisation:
+
+  [hybrid] oda_snapshot(live -> snap)
+  local pass : per layer oda_attend_local (S^L) or the recurrent stand-in; oda_glue_hidden -> h^L
+  oda_recall_score(h_{t-1}, E(x_t), h^L) -> score, flag, any_flag
+  oda_cond_begin(any_flag)          # a CUDA-graph IF node when captured
+     [hybrid] oda_restore(flag, snap -> live)
+     full pass: per layer oda_attend_full_if (S^F, flagged sequences only); glue -> h^F
+  oda_cond_end
+  oda_commit(flag): chosen branch's staged K,V -> cache slot of position t, h_{t-1} <- h^b, t += 1
+
+All compute is in liboda.so; this module only allocates buffers (torch), fills the seeded
+inputs (workload/) and issues the calls.  Per-step inputs live in one flat byte buffer
+(``StepLayout``) so that staging a step is a single copy (device-to-device for the kernel
+benchmark, pinned host-to-device for the end-to-end one).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from workload import configs, device as wdev, inputs
+from workload.configs import Workload
+
+from . import oda
+
+LOCAL, FULL = 0, 1
+
+
+class StepLayout:
+    """Offsets of one step's inputs inside a flat, 256-byte aligned byte buffer."""
+
+    def __init__(self, wl: Workload):
+        B, L, Hq, Hkv, D = wl.B, wl.L, wl.Hq, wl.Hkv, wl.D
+        G = len(wl.gdn_layers)
+        ent = [("q", (2, L, B, Hq, 128), torch.bfloat16), ("k", (2, L, B, Hkv, 128), torch.bfloat16),
+               ("v", (2, L, B, Hkv, 128), torch.bfloat16), ("emb", (B, D), torch.float32),
+               ("sched", (B,), torch.int32)]
+        if G:
+            ent += [("gc", (2, G, B, configs.CONV_WIDTH), torch.float32),
+                    ("gv", (2, G, B, configs.GDN_HEADS, configs.GDN_DIM), torch.float32),
+                    ("ga", (2, G, B, configs.GDN_HEADS), torch.float32),
+                    ("gb", (2, G, B, configs.GDN_HEADS), torch.float32)]
+        self.entries = []
+        off = 0
+        for name, shape, dt in ent:
+            nbytes = int(np.prod(shape)) * torch.empty((), dtype=dt).element_size()
+            self.entries.append((name, shape, dt, off, nbytes))
+            off += (nbytes + 255) // 256 * 256
+        self.nbytes = off
+
+    def views(self, buf: torch.Tensor) -> dict:
+        out = {}
+        for name, shape, dt, off, nbytes in self.entries:
+            out[name] = buf[off:off + nbytes].view(dt).view(shape)
+        return out
+
+
+def fill_step_inputs(wl: Workload, step: int, views: dict) -> None:
+    """Writes step ``step``'s seeded inputs into device views (bit-identical to the host
+    generator: q/k/v by the device generator, fp32 inputs generated on the host)."""
+    for br in (LOCAL, FULL):
+        for a, layer in enumerate(wl.attn_layers):
+            kq, kk, kv = inputs.qkv_keys(wl, step, layer, br)
+            wdev.fill_normal_bf16(views["q"][br, a], kq)
+            wdev.fill_normal_bf16(views["k"][br, a], kk)
+            wdev.fill_normal_bf16(views["v"][br, a], kv)
+    views["emb"].copy_(torch.from_numpy(inputs.emb(wl, step)))
+    sched = inputs.schedule(wl, step)
+    views["sched"].copy_(torch.from_numpy(sched if sched is not None else np.zeros(wl.B, np.int32)))
+    for br in (LOCAL, FULL):
+        for j, layer in enumerate(wl.gdn_layers):
+            c, v, a, b = inputs.gdn_step_inputs(wl, step, layer, br)
+            views["gc"][br, j].copy_(torch.from_numpy(c))
+            views["gv"][br, j].copy_(torch.from_numpy(v))
+            views["ga"][br, j].copy_(torch.from_numpy(a))
+            views["gb"][br, j].copy_(torch.from_numpy(b))
+
+
+class OdaDecoder:
+    """Device state of one workload (paged caches, positions, h_{t-1}, head weights, hybrid
+    state) plus the call sequence of one decode step."""
+
+    def __init__(self, wl: Workload, device="cuda", capacity_steps: int = 0,
+                 perturb_head: bool = False, head_params: dict = None, fill_cache: bool = True):
+        if not torch.cuda.is_available():
+            raise RuntimeError("OdaDecoder needs a CUDA device (the CUDA path has no fallback)")
+        self.wl = wl
+        self.device = torch.device(device)
+        torch.cuda.set_device(self.device)
+        B, L, Hkv, D = wl.B, wl.L, wl.Hkv, wl.D
+        self.capacity_steps = max(wl.steps, capacity_steps)
+        self.max_pages = (max(wl.ctx) + self.capacity_steps + 1 + configs.PAGE - 1) // configs.PAGE
+        self.n_pool = B * self.max_pages
+        cfg = oda.make_config(B, wl.Hq, Hkv, self.max_pages, D, wl.sinks, wl.window, wl.theta)
+        self.ctx = oda.oda_create(cfg)
+        dev = self.device
+        self.stream = torch.cuda.Stream(dev)
+        self.page_table = torch.from_numpy(inputs.page_table(wl, self.max_pages)).to(dev)
+        self.k_pool, self.v_pool = [], []
+        for a in range(L):
+            k = torch.empty((self.n_pool, Hkv, configs.PAGE, 128), dtype=torch.bfloat16, device=dev)
+            v = torch.empty_like(k)
+            if fill_cache:
+                wdev.fill_kv(k, self.page_table, wl.ctx,
+                             [inputs.cache_key(wl, "k", a, b) for b in range(B)], Hkv)
+                wdev.fill_kv(v, self.page_table, wl.ctx,
+                             [inputs.cache_key(wl, "v", a, b) for b in range(B)], Hkv)
+            self.k_pool.append(k)
+            self.v_pool.append(v)
+        self.layers = [oda.kv_layer(self.k_pool[a], self.v_pool[a]) for a in range(L)]
+        self.pos = torch.tensor([c + 1 for c in wl.ctx], dtype=torch.int32, device=dev)
+        self.h_prev = torch.from_numpy(inputs.h_prev0(wl)).to(dev)
+        hp = head_params if head_params is not None else inputs.head_weights(wl, perturb_head)
+        self.head_params = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in hp.items()}
+        self.head_w = oda.head_weights(self.head_params)
+        n_layers = wl.n_layers
+        self.o = torch.zeros((2, n_layers, B, D), dtype=torch.float32, device=dev)
+        self.h = torch.zeros((2, B, D), dtype=torch.float32, device=dev)
+        self.score = torch.zeros(B, dtype=torch.float32, device=dev)
+        self.flag = torch.zeros(B, dtype=torch.int32, device=dev)
+        self.any_flag = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.layout = StepLayout(wl)
+        self.staging = torch.zeros(self.layout.nbytes, dtype=torch.uint8, device=dev)
+        self.sv = self.layout.views(self.staging)
+        self.routing_scheduled = wl.routing == "bernoulli"
+        if wl.hybrid:
+            S0, C0 = inputs.gdn_state0(wl)
+            self.rec = torch.from_numpy(S0).to(dev)
+            self.conv = torch.from_numpy(C0).to(dev)
+            self.rec_snap = torch.empty_like(self.rec)
+            self.conv_snap = torch.empty_like(self.conv)
+            self.live = oda.state(self.rec, self.conv)
+            self.snap = oda.state(self.rec_snap, self.conv_snap)
+            self.taps = torch.from_numpy(
+                np.stack([inputs.gdn_taps(wl, layer) for layer in wl.gdn_layers])).to(dev)
+        self.graph = None
+        torch.cuda.synchronize(dev)
+
+    # ---------------------------------------------------------------- inputs
+    def make_step_buffer(self, step: int) -> torch.Tensor:
+        buf = torch.zeros(self.layout.nbytes, dtype=torch.uint8, device=self.device)
+        fill_step_inputs(self.wl, step, self.layout.views(buf))
+        return buf
+
+    def stage(self, src: torch.Tensor) -> None:
+        """Copies one step's input buffer (device or pinned host) into the staging area."""
+        self.stream.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(self.stream):
+            self.staging.copy_(src, non_blocking=True)
+
+    # ------------------------------------------------------------------ step
+    def issue(self) -> None:
+        """Enqueues one decode step on self.stream (eagerly or into a capture)."""
+        wl, s, sv = self.wl, self.stream, self.sv
+        ctx = self.ctx
+        n_layers = wl.n_layers
+        if wl.hybrid:
+            oda.oda_snapshot(ctx, self.live, self.snap, s)
+        a = j = 0
+        for layer in range(n_layers):
+            if layer in wl.attn_layers:
+                oda.oda_attend_local(ctx, self.layers[a], self.page_table, self.pos, sv["q"][LOCAL, a],
+                                     sv["k"][LOCAL, a], sv["v"][LOCAL, a], self.o[LOCAL, layer], s)
+                a += 1
+            else:
+                oda.oda_glue_gdn(ctx, self.live, j, sv["gc"][LOCAL, j], sv["gv"][LOCAL, j],
+                                 sv["ga"][LOCAL, j], sv["gb"][LOCAL, j], self.taps[j], None,
+                                 self.o[LOCAL, layer], s)
+                j += 1
+        oda.oda_glue_hidden(ctx, sv["emb"], self.o[LOCAL], n_layers, None, self.h[LOCAL], s)
+        oda.oda_recall_score(ctx, self.head_w, self.h_prev, sv["emb"], self.h[LOCAL],
+                             sv["sched"] if self.routing_scheduled else None, self.score,
+                             self.flag, self.any_flag, s)
+        body = oda.oda_cond_begin(ctx, s, self.any_flag)
+        if wl.hybrid:
+            oda.oda_restore(ctx, self.flag, self.snap, self.live, body)
+        a = j = 0
+        for layer in range(n_layers):
+            if layer in wl.attn_layers:
+                oda.oda_attend_full_if(ctx, self.layers[a], self.page_table, self.pos, self.flag,
+                                       sv["q"][FULL, a], sv["k"][FULL, a], sv["v"][FULL, a],
+                                       self.o[FULL, layer], body)
+                a += 1
+            else:
+                oda.oda_glue_gdn(ctx, self.live, j, sv["gc"][FULL, j], sv["gv"][FULL, j],
+                                 sv["ga"][FULL, j], sv["gb"][FULL, j], self.taps[j], self.flag,
+                                 self.o[FULL, layer], body)
+                j += 1
+        oda.oda_glue_hidden(ctx, sv["emb"], self.o[FULL], n_layers, self.flag, self.h[FULL], body)
+        oda.oda_cond_end(ctx, s)
+        oda.oda_commit(ctx, self.layers, self.page_table, self.pos, self.flag, sv["k"][LOCAL],
+                       sv["v"][LOCAL], sv["k"][FULL], sv["v"][FULL], self.h[LOCAL], self.h[FULL],
+                       self.h_prev, s)
+
+    def capture(self) -> None:
+        """Records one step (with the retry under a conditional node) as a CUDA graph."""
+        torch.cuda.synchronize(self.device)
+        oda.oda_graph_begin(self.stream)
+        try:
+            self.issue()
+        except Exception:
+            try:
+                oda.oda_graph_end(self.stream).close()
+            except Exception:
+                pass
+            raise
+        self.graph = oda.oda_graph_end(self.stream)
+
+    def launch(self) -> None:
+        if self.graph is not None:
+            self.graph.launch(self.stream)
+        else:
+            self.issue()
+
+    def step(self, src: torch.Tensor = None) -> None:
+        if src is not None:
+            self.stage(src)
+        self.launch()
+
+    def synchronize(self):
+        self.stream.synchronize()
+
+    def device_error(self) -> int:
+        self.synchronize()
+        return oda.oda_get_error(self.ctx)
+
+    def attention_layers_bytes(self) -> int:
+        return sum(k.numel() * 2 * 2 for k in self.k_pool)
+
+    def close(self):
+        if self.graph is not None:
+            self.graph.close()
+            self.graph = None
+        self.ctx.close()

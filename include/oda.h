@@ -1,0 +1,227 @@
+/*
+ * oda.h - C ABI of the On-Demand Attention (ODA) decode hot path for NVIDIA B200 (sm_100a).
+ *
+ * Method (web page "On-Demand Attention：让语言模型按需读取完整历史", the method notes,
+ * cited below as [notes §n]): every decode step first runs a local pass whose restricted
+ * attention layers read the index set S^L_t = {1..min(s,t)} U {max(1,t-w+1)..t} (s = 4 sinks,
+ * w = 2048 window including the current token) of a fully retained KV cache; a recall head
+ * R(h_{t-1}, E(x_t), h^L_t) scores the step; where the score exceeds theta (0) or is not
+ * finite, the full pass is recomputed from the same pre-step state over S^F_t = {1..t};
+ * finally only the chosen branch's hidden state and current K,V are committed.
+ *
+ * Conventions for every entry point
+ *   - Device pointers unless stated otherwise; nothing is retained after the call returns.
+ *     The caller owns all tensors and streams; the context owns only its scratch.
+ *   - Every call is asynchronous on the given stream, allocates nothing after oda_create,
+ *     never synchronises with the host (except oda_get_error / oda_create / oda_destroy) and
+ *     can be captured in a CUDA graph.  Calls on one context must be ordered on one stream
+ *     (they share scratch).
+ *   - Argument and shape errors return synchronously (ODA_ERR_INVALID_ARG /
+ *     ODA_ERR_UNSUPPORTED) and launch nothing.  A failed launch returns ODA_ERR_CUDA.
+ *     Data-dependent violations found on the device (page-table entry outside the pool,
+ *     position beyond capacity, a bounded wait that gave up) set bits in the context's sticky
+ *     device error word, skip the offending access, and are read with oda_get_error.
+ *     Kernels never trap.  oda_last_error() gives a message for the last non-OK status of
+ *     the calling thread.
+ *   - Positions: pos[b] = t, the 1-based position of the token being decoded.  The cache of
+ *     sequence b holds positions 1..t-1 at token indices 0..t-2; position t (the current
+ *     token) is passed as staged k_new / v_new and is never read from the cache.
+ *
+ * Layouts
+ *   KV pool of one layer (K and V separately): bf16 [n_pages][Hkv][16][128]; each
+ *   (page, kv head) block is a contiguous 4 KiB.  page_table: int32 [B][max_pages],
+ *   logical page p of sequence b -> physical page page_table[b*max_pages + p]; the table is
+ *   shared by all layers.  q: bf16 [B][Hq][128].  k_new, v_new: bf16 [B][Hkv][128].
+ *   out: fp32 [B][Hq][128].  Query head h reads KV head h / (Hq/Hkv).
+ */
+#ifndef ODA_H
+#define ODA_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ODA_VERSION_MAJOR 0
+#define ODA_VERSION_MINOR 1
+
+typedef enum {
+  ODA_OK = 0,
+  ODA_ERR_INVALID_ARG = 1,   /* null pointer, bad size or alignment                   */
+  ODA_ERR_UNSUPPORTED = 2,   /* shape outside what the kernels implement               */
+  ODA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed                   */
+  ODA_ERR_DEVICE = 4,        /* oda_get_error found the device error word non-zero     */
+  ODA_ERR_STATE = 5          /* call out of order (e.g. oda_cond_end without begin)    */
+} oda_status;
+
+/* Bits of the sticky device error word. */
+#define ODA_DEVERR_PAGE_RANGE   0x1  /* page-table entry outside [0, n_pages): access skipped  */
+#define ODA_DEVERR_POS_RANGE    0x2  /* pos < 1 or t-1 beyond the table's capacity            */
+#define ODA_DEVERR_WAIT_TIMEOUT 0x4  /* a bounded wait on a copy barrier gave up              */
+
+#define ODA_MAX_BATCH 256
+#define ODA_MAX_LAYERS 64
+
+typedef struct oda_ctx oda_ctx;
+
+typedef struct {
+  int32_t batch;        /* B, 1..ODA_MAX_BATCH                                        */
+  int32_t n_q_heads;    /* Hq                                                          */
+  int32_t n_kv_heads;   /* Hkv; Hq % Hkv == 0 and g = Hq / Hkv in 1..8                  */
+  int32_t head_dim;     /* d_k; must be 128                                            */
+  int32_t page_size;    /* tokens per page; must be 16                                 */
+  int32_t max_pages;    /* pages per sequence = row length of the page table           */
+  int32_t sinks;        /* s (the notes use 4), 0..16                                   */
+  int32_t window;       /* w (the notes use 2048), >= 1, includes the current token    */
+  int32_t head_in_dim;  /* D: width of each recall-head input; multiple of 512, <= 8192 */
+  float theta;          /* routing threshold (the notes use 0)                          */
+} oda_config;
+
+typedef struct {
+  void* k;              /* bf16 [n_pages][Hkv][16][128], 16-byte aligned               */
+  void* v;              /* bf16 [n_pages][Hkv][16][128], 16-byte aligned               */
+  int64_t n_pages;      /* pages in this layer's pool (bounds every page-table entry)   */
+} oda_kv_layer;
+
+/* Recall-head parameters, fp32, row-major [out][in] matrices.  Towers i = 0,1,2 read
+ * h_{t-1}, E(x_t), h^L_t.  D = head_in_dim, T = 1024 (tower width), F = 2048 (FFN width). */
+typedef struct {
+  const float* tower_norm[3];  /* [D]        RMSNorm weight of each input              */
+  const float* tower_w[3];     /* [T][D]                                                */
+  const float* tower_b[3];     /* [T]                                                   */
+  const float* fuse_w;         /* [T][9T]    interaction projection                     */
+  const float* fuse_b;         /* [T]                                                   */
+  const float* ffn_norm[2];    /* [T]                                                   */
+  const float* ffn_gate[2];    /* [F][T]                                                */
+  const float* ffn_up[2];      /* [F][T]                                                */
+  const float* ffn_down[2];    /* [T][F]                                                */
+  const float* out_norm;       /* [T]                                                   */
+  const float* out_w;          /* [T]                                                   */
+  const float* out_b;          /* [1]                                                   */
+} oda_head_weights;
+
+/* Recurrent and conv state of the linear-recurrent layers of a hybrid backbone, fp32.
+ * rec: [B][n_layers][heads][dv][dk]; conv: [B][n_layers][conv_taps][conv_width]. */
+typedef struct {
+  float* rec;
+  float* conv;
+  int32_t n_layers, heads, dk, dv, conv_taps, conv_width;
+} oda_state;
+
+/* ---------------------------------------------------------------- context ---------- */
+
+/* Validates the configuration and allocates the context's scratch on the current device
+ * (split-KV partials, completion counters, recall-head intermediates, the device error
+ * word).  May synchronise.  *out is NULL on failure. */
+oda_status oda_create(const oda_config* cfg, oda_ctx** out);
+
+/* Frees the scratch (synchronises the device).  NULL is accepted. */
+oda_status oda_destroy(oda_ctx* ctx);
+
+/* ----------------------------------------------------------- attention ------------ */
+
+/* Local-branch attention of one layer for all B sequences.  [notes §2.1, eq. o_t with
+ * S_t = S^L_t, eq. S^F/S^L]: o = softmax(q K~[S^L]^T / sqrt(128)) V~[S^L], where K~, V~ are
+ * the cached positions 1..t-1 followed by the staged current (k_new, v_new) at position t.
+ * Writes out[b][h][:] for every b and h; never writes the cache. */
+oda_status oda_attend_local(oda_ctx* ctx, const oda_kv_layer* layer, const int32_t* page_table,
+                            const int32_t* pos, const void* q, const void* k_new,
+                            const void* v_new, float* out, cudaStream_t stream);
+
+/* Full-branch attention of one layer, gated per sequence by the device flag.
+ * [notes §2.3]: the full pass runs only where the recall head fired; here over
+ * S^F_t = {1..t} [notes §2.1].  Sequences with flag[b] == 0 do no work and their rows of out
+ * are left untouched.  The host never reads the flags. */
+oda_status oda_attend_full_if(oda_ctx* ctx, const oda_kv_layer* layer, const int32_t* page_table,
+                              const int32_t* pos, const int32_t* flag, const void* q,
+                              const void* k_new, const void* v_new, float* out,
+                              cudaStream_t stream);
+
+/* The index sets as the attention kernels visit them (same work decomposition): for each
+ * sequence b (mode 0: all, S^L; mode 1: flag[b] != 0, S^F), positions[b*cap + i] receives the
+ * 1-based cache positions read, in page order, followed by t (the staged token);
+ * counts[b] the number written (0 for skipped sequences).  A debug and test entry point:
+ * one thread per sequence.  Writes at most cap entries per sequence. */
+oda_status oda_index_positions(oda_ctx* ctx, int32_t mode, const int32_t* pos, const int32_t* flag,
+                               int32_t* positions, int32_t cap, int32_t* counts,
+                               cudaStream_t stream);
+
+/* ------------------------------------------------------------ recall head ---------- */
+
+/* Recall score and gate for all B sequences.  [notes §2.2, eq. q_t]: q_t = R(h_{t-1},
+ * E(x_t), h^L_t) with inputs h_prev, emb, h_loc (fp32 [B][D]); [notes §2.3]:
+ * flag[b] = (score[b] > theta) || !isfinite(score[b]).  If sched is non-NULL the head still
+ * runs but flag[b] = (sched[b] != 0) (hand-scheduled full calls, [notes §3.3]).
+ * *any_flag = OR of flag[b] (int32, device).  Layer arrangement: see the notes' reading in
+ * the design notes; all arithmetic fp32 with fixed reduction order (deterministic). */
+oda_status oda_recall_score(oda_ctx* ctx, const oda_head_weights* w, const float* h_prev,
+                            const float* emb, const float* h_loc, const int32_t* sched,
+                            float* score, int32_t* flag, int32_t* any_flag, cudaStream_t stream);
+
+/* ------------------------------------------------------------- commit -------------- */
+
+/* Transactional commit.  [notes §2.3, eq. h_t = h^{b_t}_t, C_t = C_{t-1} || dC^{b_t}_t]:
+ * for each sequence b with branch = flag[b] ? full : local and t = pos[b]:
+ *   every layer l: K/V pool slot of position t (page_table[b][(t-1)/16], slot (t-1)%16)
+ *                  <- k_stage_<branch>[l][b], v_stage_<branch>[l][b]  (bit-exact copy);
+ *   h_prev[b] <- h_<branch>[b] (fp32 [B][D]);  pos[b] <- t + 1.
+ * Staging layouts: bf16 [n_layers][B][Hkv][128].  layers: host array of n_layers entries.
+ * The only writer of the cache; writes exactly one position per sequence per layer. */
+oda_status oda_commit(oda_ctx* ctx, const oda_kv_layer* layers, int32_t n_layers,
+                      const int32_t* page_table, int32_t* pos, const int32_t* flag,
+                      const void* k_stage_local, const void* v_stage_local,
+                      const void* k_stage_full, const void* v_stage_full,
+                      const float* h_local, const float* h_full, float* h_prev,
+                      cudaStream_t stream);
+
+/* ----------------------------------------------------- snapshot / restore ---------- */
+
+/* [notes §2.3, third paragraph]: hybrid backbones save the conv and recurrent state before
+ * the local pass and restore the pre-step state before the full retry, so no state is
+ * advanced twice.  oda_snapshot copies live -> snap for all B sequences; oda_restore copies
+ * snap -> live for sequences with flag[b] != 0 only.  Bit-exact copies; both structs (host
+ * pointers) must describe the same shape. */
+oda_status oda_snapshot(oda_ctx* ctx, const oda_state* live, const oda_state* snap,
+                        cudaStream_t stream);
+oda_status oda_restore(oda_ctx* ctx, const int32_t* flag, const oda_state* snap,
+                       const oda_state* live, cudaStream_t stream);
+
+/* --------------------------------------------------- conditional retry ------------- */
+
+/* GPU-side conditional execution of the full retry ([notes §3.3]: conditional execution
+ * and CUDA Graphs keep the branch decision on the device).  If `stream` is being captured,
+ * oda_cond_begin appends a kernel that sets an IF condition from *any_flag (device int32)
+ * and an IF conditional node, and starts capturing the node's body on an internal stream
+ * returned in *body_stream; work issued there until oda_cond_end runs only when
+ * *any_flag != 0 at replay.  If `stream` is not capturing, *body_stream = stream and the
+ * retry's kernels read the per-sequence flags themselves. */
+oda_status oda_cond_begin(oda_ctx* ctx, cudaStream_t stream, const int32_t* any_flag,
+                          cudaStream_t* body_stream);
+oda_status oda_cond_end(oda_ctx* ctx, cudaStream_t stream);
+
+/* --------------------------------------------------------- CUDA graphs ------------- */
+
+typedef struct oda_graph oda_graph;
+/* Begin capturing `stream` (relaxed mode).  Work enqueued until oda_graph_end is recorded. */
+oda_status oda_graph_begin(cudaStream_t stream);
+/* End the capture and instantiate it; *out owns the executable graph. */
+oda_status oda_graph_end(cudaStream_t stream, oda_graph** out);
+oda_status oda_graph_launch(oda_graph* g, cudaStream_t stream);
+oda_status oda_graph_destroy(oda_graph* g);
+
+/* ------------------------------------------------------------- errors -------------- */
+
+/* Waits for all work on the device, then reads (and keeps) the sticky device error word into
+ * *device_error (host int32).  Returns ODA_ERR_DEVICE if it is non-zero. */
+oda_status oda_get_error(oda_ctx* ctx, int32_t* device_error);
+oda_status oda_clear_error(oda_ctx* ctx, cudaStream_t stream);
+const char* oda_status_string(oda_status s);
+const char* oda_last_error(void);
+int32_t oda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ODA_H */

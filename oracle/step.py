@@ -101,10 +101,9 @@ def run_pass(wl: Workload, state: OracleState, step: int, branch: int, active, r
     x = e.copy()
     a = 0
     gdn_j = 0
-    o_rec_by_layer = {}
     for layer in range(wl.n_layers):
         if layer in wl.attn_layers:
-            q, k, v = wi.step_qkv(wl, step, a, branch)
+            q, k, v = wi.step_qkv(wl, step, layer, branch)
             rec.staged_k[(branch, a)] = k
             rec.staged_v[(branch, a)] = v
             o = np.full((B, wl.Hq, wl.d), np.nan)

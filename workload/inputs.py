@@ -53,7 +53,8 @@ def page_table(wl: Workload, max_pages: int) -> np.ndarray:
 
 # ------------------------------------------------------------------------ per-step inputs
 def step_qkv(wl: Workload, step: int, layer: int, branch: int):
-    """(q [B,Hq,128], k [B,Hkv,128], v [B,Hkv,128]) bf16 bits of one attention layer."""
+    """(q [B,Hq,128], k [B,Hkv,128], v [B,Hkv,128]) bf16 bits of the attention layer with
+    backbone index ``layer`` (not its attention ordinal)."""
     br = _branch_id(wl, layer, branch)
     q = gen.normal_bf16(gen.key(wl.seed, Tag.Q, step, layer, br), wl.B * wl.Hq * wl.d)
     k = gen.normal_bf16(gen.key(wl.seed, Tag.K_NEW, step, layer, br), wl.B * wl.Hkv * wl.d)
