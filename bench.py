@@ -220,6 +220,61 @@ def run_reference(args, wl, rank, world):
 
 
 # ------------------------------------------------------------------------ GPU arm
+def time_layer_kernels(dec, mode: int, flag, reps: int = 3) -> float:
+    """Average device milliseconds of one attention launch: a graph holding one launch per
+    layer (local: mode 0, full: mode 1 with the given flags) replayed ``reps`` times."""
+    import torch
+    from conditional_sparse_attention_b200 import oda
+    s = dec.stream
+    wl = dec.wl
+    torch.cuda.synchronize(dec.device)
+    oda.oda_graph_begin(s)
+    for a in range(wl.L):
+        if mode == 0:
+            oda.oda_attend_local(dec.ctx, dec.layers[a], dec.page_table, dec.pos, dec.sv["q"][0, a],
+                                 dec.sv["k"][0, a], dec.sv["v"][0, a], dec.o[0, a], s)
+        else:
+            oda.oda_attend_full_if(dec.ctx, dec.layers[a], dec.page_table, dec.pos, flag,
+                                   dec.sv["q"][1, a], dec.sv["k"][1, a], dec.sv["v"][1, a],
+                                   dec.o[1, a], s)
+    g = oda.oda_graph_end(s)
+    g.launch(s)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(reps):
+        g.launch(s)
+    e1.record(s)
+    e1.synchronize()
+    g.close()
+    return e0.elapsed_time(e1) / (reps * wl.L)
+
+
+def run_kernel_only(args, wl, local_rank):
+    """Profiling mode: set up the workload, stage step 0, launch one attention kernel
+    ``--kernel-reps`` times (full: every sequence flagged) and exit."""
+    import torch
+    from conditional_sparse_attention_b200 import oda
+    from conditional_sparse_attention_b200.engine import OdaDecoder
+    dev = torch.device("cuda", local_rank)
+    dec = OdaDecoder(wl, device=dev, capacity_steps=4)
+    dec.stage(dec.make_step_buffer(0))
+    dec.synchronize()
+    ones = torch.ones(wl.B, dtype=torch.int32, device=dev)
+    for r in range(args.kernel_reps):
+        a = r % wl.L
+        if args.kernel_only == "full":
+            oda.oda_attend_full_if(dec.ctx, dec.layers[a], dec.page_table, dec.pos, ones,
+                                   dec.sv["q"][1, a], dec.sv["k"][1, a], dec.sv["v"][1, a],
+                                   dec.o[1, a], dec.stream)
+        else:
+            oda.oda_attend_local(dec.ctx, dec.layers[a], dec.page_table, dec.pos, dec.sv["q"][0, a],
+                                 dec.sv["k"][0, a], dec.sv["v"][0, a], dec.o[0, a], dec.stream)
+    dec.synchronize()
+    err = dec.device_error()
+    print(json.dumps({"kernel_only": args.kernel_only, "workload": wl.name,
+                      "launches": args.kernel_reps, "device_error": err}), flush=True)
+    dec.close()
+
 def run_ours(args, wl, rank, world, local_rank):
     import torch
     from conditional_sparse_attention_b200 import oda
@@ -283,38 +338,30 @@ def run_ours(args, wl, rank, world, local_rank):
     realized_rate = float(flags.mean())
     launches = sum(kernel_launches(wl, bool(flags[i].any())) for i in range(K))
 
-    # ---------------- dominant kernel: the full-set attention, timed per launch with events
+    # ---------------- per-kernel timing: each attention kernel replayed as a graph of one launch
+    # per layer (no host gaps), CUDA events on the launching stream
     hbm, peak_src = peaks()
-    full_bytes, full_ms = 0, 0.0
-    loc_bytes, loc_ms = 0, 0.0
     per_tok = wl.Hkv * 128 * 2 * 2
-    kev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    patterns = [f for f in flags if f.any()] or [torch.ones(wl.B, dtype=torch.int32).numpy()]
     pos_now = dec.pos.cpu().numpy()
-    for rep, fl in enumerate(patterns[:8]):
-        ft = torch.from_numpy(fl.astype("int32")).to(dev)
-        for a in range(min(wl.L, 6)):
-            with torch.cuda.stream(dec.stream):
-                kev[0].record(dec.stream)
-                oda.oda_attend_full_if(dec.ctx, dec.layers[a], dec.page_table, dec.pos, ft,
-                                       dec.sv["q"][1, a], dec.sv["k"][1, a], dec.sv["v"][1, a],
-                                       dec.o[1, a], dec.stream)
-                kev[1].record(dec.stream)
-            kev[1].synchronize()
-            full_ms += kev[0].elapsed_time(kev[1])
-            full_bytes += sum(int(pos_now[b]) * per_tok for b in range(wl.B) if fl[b])
-            with torch.cuda.stream(dec.stream):
-                kev[0].record(dec.stream)
-                oda.oda_attend_local(dec.ctx, dec.layers[a], dec.page_table, dec.pos,
-                                     dec.sv["q"][0, a], dec.sv["k"][0, a], dec.sv["v"][0, a],
-                                     dec.o[0, a], dec.stream)
-                kev[1].record(dec.stream)
-            kev[1].synchronize()
-            loc_ms += kev[0].elapsed_time(kev[1])
-            loc_bytes += sum(min(int(pos_now[b]), wl.sinks + wl.window) * per_tok for b in range(wl.B))
+    pats = {}
+    for f in flags:
+        if f.any():
+            key = tuple(int(x) for x in f)
+            pats[key] = pats.get(key, 0) + 1
+    if not pats:
+        pats = {tuple([1] + [0] * (wl.B - 1)): 1}
+    full_bytes = full_ms = 0.0
+    n_full = 0
+    for pat, count in pats.items():
+        ft = torch.tensor(pat, dtype=torch.int32, device=dev)
+        ms = time_layer_kernels(dec, 1, ft, reps=2)
+        full_ms += count * ms
+        full_bytes += count * sum(int(pos_now[b]) * per_tok for b in range(wl.B) if pat[b])
+        n_full += 2 * wl.L
     full_gbs = full_bytes / (full_ms * 1e-3) / 1e9
+    loc_ms = time_layer_kernels(dec, 0, None, reps=3)
+    loc_bytes = sum(min(int(pos_now[b]), wl.sinks + wl.window) * per_tok for b in range(wl.B))
     loc_gbs = loc_bytes / (loc_ms * 1e-3) / 1e9
-    n_full = min(len(patterns), 8) * min(wl.L, 6)
 
     # ---------------- end to end: pinned host inputs -> H2D, step, D2H of the results
     e2e = None
@@ -365,10 +412,13 @@ def run_ours(args, wl, rank, world, local_rank):
             "roofline": {"bound": "hbm", "achieved": full_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": full_gbs / hbm, "traffic": None,
                          "kernel": "attn_kernel (full set, flagged sequences)",
-                         "peak_source": peak_src, "launches_timed": n_full},
+                         "peak_source": peak_src, "launches_timed": n_full,
+                         "us_per_launch": full_ms * 1000.0 / sum(pats.values()),
+                         "flag_patterns": {"".join(map(str, k)): v for k, v in pats.items()}},
             "step_roofline": {"algorithmic_gb_per_step": total_bytes / K / 1e9,
                               "achieved_gbs": step_gbs, "frac": step_gbs / hbm},
-            "local_kernel": {"achieved_gbs": loc_gbs, "frac": loc_gbs / hbm},
+            "local_kernel": {"achieved_gbs": loc_gbs, "frac": loc_gbs / hbm,
+                             "us_per_launch": loc_ms * 1000.0},
             "realized_recall_rate": realized_rate,
             "first_step_ms_incl_capture": first_ms, "setup_s": setup_s,
             "gpu_launches": launches, "device_error": err,
@@ -387,6 +437,9 @@ def main():
     ap.add_argument("--workload", default="cfg2")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-only", choices=["full", "local"], default=None,
+                    help="profiling mode: launch one attention kernel --kernel-reps times and exit")
+    ap.add_argument("--kernel-reps", type=int, default=3)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -397,6 +450,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, wl, rank, world)
+        return
+    if args.kernel_only:
+        run_kernel_only(args, wl, local_rank)
         return
     import torch
     if world > 1:

@@ -11,7 +11,6 @@
 
 namespace oda {
 
-oda_status prepare_attention_kernel();
 oda_status prepare_head_kernel();
 
 static thread_local char g_msg[512] = "";
@@ -121,23 +120,18 @@ oda_status oda_create(const oda_config* cfg, oda_ctx** out) {
   if (st == ODA_OK)
     st = check_cuda(cudaDeviceGetAttribute(&x->n_sms, cudaDevAttrMultiProcessorCount, x->device),
                     "cudaDeviceGetAttribute");
-  if (st == ODA_OK) st = oda::prepare_attention_kernel();
+  if (st == ODA_OK) st = oda::prepare_attention_kernel(x->g, x->n_sms, &x->attn_ctas);
   if (st == ODA_OK) st = oda::prepare_head_kernel();
   if (st != ODA_OK) {
     free_ctx(x);
     return st;
   }
-  x->attn_ctas = x->n_sms * oda::attention_ctas_per_sm();
-  // split partials: bounded by ~512 MiB and by the combine's shared-memory weight table
-  const int64_t B = c.batch, Hq = c.n_q_heads, Hkv = c.n_kv_heads, D = c.head_in_dim;
-  int64_t ms = (c.max_pages + 7) / 8 + 2;
-  const int64_t budget = (512ll << 20) / (B * Hq * 130 * 4);
-  ms = std::min<int64_t>(ms, std::max<int64_t>(16, budget));
-  ms = std::min<int64_t>(ms, 3072);
-  x->max_splits = (int)ms;
+  const int64_t B = c.batch, Hkv = c.n_kv_heads, D = c.head_in_dim;
+  x->n_slots = (int)(x->attn_ctas + B * Hkv);
+  const int64_t ms = x->n_slots;
   const int gch = oda::glue_chunks(c.head_in_dim);
-  st = dev_alloc(&x->part_o, (size_t)B * Hq * ms * 128, "cudaMalloc(partials)");
-  if (st == ODA_OK) st = dev_alloc(&x->part_ml, (size_t)B * Hq * ms * 2, "cudaMalloc(partials)");
+  st = dev_alloc(&x->part_o, (size_t)ms * x->g * 128, "cudaMalloc(partials)");
+  if (st == ODA_OK) st = dev_alloc(&x->part_ml, (size_t)ms * x->g * 2, "cudaMalloc(partials)");
   if (st == ODA_OK) st = dev_alloc(&x->attn_cnt, (size_t)B * Hkv, "cudaMalloc(counters)");
   if (st == ODA_OK) st = dev_alloc(&x->err, 1, "cudaMalloc(error word)");
   if (st == ODA_OK) st = dev_alloc(&x->head_part, oda::head_part_floats((int)B, (int)D), "cudaMalloc(head)");
@@ -200,6 +194,7 @@ oda_status oda_recall_score(oda_ctx* ctx, const oda_head_weights* w, const float
                             const float* emb, const float* h_loc, const int32_t* sched,
                             float* score, int32_t* flag, int32_t* any_flag, cudaStream_t stream) {
   if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "recall_score: ctx is NULL");
+  ctx->prev_attention = false;
   return oda::launch_recall_head(ctx, w, h_prev, emb, h_loc, sched, score, flag, any_flag, stream);
 }
 
@@ -210,6 +205,7 @@ oda_status oda_commit(oda_ctx* ctx, const oda_kv_layer* layers, int32_t n_layers
                       const float* h_local, const float* h_full, float* h_prev,
                       cudaStream_t stream) {
   if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "commit: ctx is NULL");
+  ctx->prev_attention = false;
   return oda::launch_commit(ctx, layers, n_layers, page_table, pos, flag, k_stage_local,
                             v_stage_local, k_stage_full, v_stage_full, h_local, h_full, h_prev,
                             stream);
@@ -218,6 +214,7 @@ oda_status oda_commit(oda_ctx* ctx, const oda_kv_layer* layers, int32_t n_layers
 oda_status oda_snapshot(oda_ctx* ctx, const oda_state* live, const oda_state* snap,
                         cudaStream_t stream) {
   if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "snapshot: ctx is NULL");
+  ctx->prev_attention = false;
   return oda::launch_state_copy(live, snap, ctx->cfg.batch, nullptr, stream);
 }
 
@@ -225,12 +222,14 @@ oda_status oda_restore(oda_ctx* ctx, const int32_t* flag, const oda_state* snap,
                        const oda_state* live, cudaStream_t stream) {
   if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "restore: ctx is NULL");
   if (!flag) return set_error(ODA_ERR_INVALID_ARG, "restore: flag is NULL");
+  ctx->prev_attention = false;
   return oda::launch_state_copy(snap, live, ctx->cfg.batch, flag, stream);
 }
 
 oda_status oda_glue_hidden(oda_ctx* ctx, const float* emb, const float* terms, int32_t n_terms,
                            const int32_t* flag, float* h, cudaStream_t stream) {
   if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "glue_hidden: ctx is NULL");
+  ctx->prev_attention = false;
   return oda::launch_glue_hidden(ctx, emb, terms, n_terms, flag, h, stream);
 }
 
@@ -238,6 +237,7 @@ oda_status oda_glue_gdn(oda_ctx* ctx, const oda_state* st, int32_t layer, const 
                         const float* v, const float* alpha, const float* beta,
                         const float* taps, const int32_t* flag, float* o, cudaStream_t stream) {
   if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "glue_gdn: ctx is NULL");
+  ctx->prev_attention = false;
   return oda::launch_glue_gdn(ctx, st, layer, c, v, alpha, beta, taps, flag, o, stream);
 }
 
@@ -246,6 +246,7 @@ oda_status oda_cond_begin(oda_ctx* ctx, cudaStream_t stream, const int32_t* any_
   if (!ctx || !any_flag || !body_stream)
     return set_error(ODA_ERR_INVALID_ARG, "cond_begin: null argument");
   if (ctx->cond_open) return set_error(ODA_ERR_STATE, "cond_begin: a conditional is already open");
+  ctx->prev_attention = false;
   if (!stream_capturing(stream)) {
     ctx->cond_open = true;
     ctx->cond_parent = nullptr;
@@ -294,6 +295,7 @@ oda_status oda_cond_end(oda_ctx* ctx, cudaStream_t stream) {
   if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "cond_end: ctx is NULL");
   if (!ctx->cond_open) return set_error(ODA_ERR_STATE, "cond_end: no open conditional");
   ctx->cond_open = false;
+  ctx->prev_attention = false;
   if (ctx->cond_parent == nullptr) return ODA_OK;
   if (ctx->cond_parent != stream)
     return set_error(ODA_ERR_STATE, "cond_end: stream differs from the one given to cond_begin");
@@ -350,6 +352,7 @@ oda_status oda_get_error(oda_ctx* ctx, int32_t* device_error) {
 
 oda_status oda_clear_error(oda_ctx* ctx, cudaStream_t stream) {
   if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "clear_error: ctx is NULL");
+  ctx->prev_attention = false;
   return check_cuda(cudaMemsetAsync(ctx->err, 0, sizeof(int32_t), stream), "cudaMemsetAsync");
 }
 

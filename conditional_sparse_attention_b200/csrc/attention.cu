@@ -5,25 +5,34 @@
 // S^L_t = {1..min(s,t)} U {max(1,t-w+1)..t} or the full set S^F_t = {1..t} of one retained
 // cache; the current token's K,V (position t) come from the branch's staging, not the cache.
 //
-// Kernel design (sm_100a):
-//   * persistent grid (2 CTAs per SM); a work item is (sequence b, KV head h, split of
-//     pages); items are enumerated on the device from pos[] (and flag[] for the full set),
-//     so the full retry of unflagged sequences costs nothing and the host never syncs;
-//   * each of the 4 warps of a CTA streams every 4th page of its item through a private
-//     3-stage ring: one 2-D TMA tile load per 64-dim half of K and V (4 x 2 KiB per page,
-//     128-byte swizzle), completion on an mbarrier (bounded waits, no spin without limit);
+// Shared per-page arithmetic (sm_100a):
+//   * every warp streams its pages through a private 3-stage ring: one 2-D TMA tile load per
+//     64-dim half of K and V (4 x 2 KiB per page, 128-byte swizzle), completion on an mbarrier
+//     (bounded waits, no spin without limit);
 //   * scores S = K Q^T with tokens as the M dimension and the g query heads of the GQA group
 //     as N (mma.sync m16n8k16 bf16 -> fp32); online softmax in the exp2 domain with
 //     warp-shuffle column maxima; P^T reaches the PV product through movmatrix.trans; P is
-//     split into bf16 hi + lo parts so the PV product keeps ~fp32 accuracy;
-//   * per item, the 4 warp states are merged in shared memory into one (m, l, acc[128])
-//     partial per query head; the last CTA to finish a (b, h) (completion counter, no
-//     spin-wait) merges all splits plus the staged current token and writes o.
+//     split into bf16 hi + lo parts so the PV product keeps ~fp32 accuracy.
+// Two kernels:
+//   * local set (at most s + w positions per sequence): one thread-block cluster per
+//     (sequence, KV head); its CTAs split the pages and merge their partials through
+//     distributed shared memory, no global scratch;
+//   * full set (flag-gated, up to the whole history): a persistent grid whose CTAs own equal
+//     contiguous ranges of (sequence, KV head, page) units enumerated on the device from pos[]
+//     and flag[] (unflagged sequences cost nothing, the host never syncs); each range's piece
+//     of a (b, h) leaves one partial in global scratch, and the CTA that completes a (b, h)
+//     (completion counter, no waiting) merges them with the staged current token.
+// Consecutive attention launches of one context may overlap (programmatic dependent launch):
+// a launch prefetches its first pages before waiting for the previous one.
 #include <cmath>
 #include <cstdio>
 
+#include <cooperative_groups.h>
+
 #include "internal.h"
 #include "ptx.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace oda {
 namespace {
@@ -34,12 +43,9 @@ constexpr int kThreads = kW * 32;
 constexpr int kPageTok = 16;
 constexpr int kStageBytes = 8192;     // K (4 KiB) + V (4 KiB) of one (page, KV head)
 constexpr int kStagesBytes = kW * kR * kStageBytes;
-constexpr int kSmemBytes = kStagesBytes + 1024;
 constexpr int kMergeStride = 132;     // floats per (warp, head) row of the merge area
 constexpr uint64_t kWaitNs = 2000000000ull;
-constexpr int kMinSplitPages = 8;
-constexpr int kItemsPerCta = 4;       // target work items per CTA when sizing splits
-constexpr int kCtasPerSm = 2;
+constexpr int kMaxCluster = 8;
 
 struct AttnParams {
   const int32_t* page_table;
@@ -49,12 +55,13 @@ struct AttnParams {
   const uint32_t* k_new;  // bf16 pairs [B][Hkv][64]
   const uint32_t* v_new;
   float* out;             // [B][Hq][128]
-  float* part_o;          // [B*Hq][max_splits][128]
-  float* part_ml;         // [B*Hq][max_splits][2]
-  int32_t* counters;      // [B*Hkv]
+  float* part_o;          // full set: [slot][g][128]   slot = CTA index + b*Hkv + h
+  float* part_ml;         // full set: [slot][g][2]
+  int32_t* counters;      // full set: [B*Hkv]
   int32_t* err;
   int64_t n_pool_pages;
-  int32_t B, Hq, Hkv, g, max_pages, max_splits, sinks, window, mode;
+  int32_t B, Hq, Hkv, g, max_pages, sinks, window, mode;
+  int32_t cluster;        // local set: CTAs per (b, h)
   float scale_log2;       // log2(e) / sqrt(128)
 };
 
@@ -114,33 +121,410 @@ __device__ __forceinline__ bool geom_has(const Geom& g, int j) {
   return j < g.n_cache && (j < g.sink_hi || j >= g.win_lo);
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
-attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-            const AttnParams p) {
+// Online-softmax state of one warp for the g (<= 8) query heads of one KV head.  Lane
+// (r = lane/4, c = lane%4) holds heads 2c and 2c+1; o holds O^T fragments (dims x heads).
+struct WarpAcc {
+  float m0, m1, l0, l1;
+  float o[8][4];
+};
+
+__device__ __forceinline__ void acc_init(WarpAcc& A) {
+  A.m0 = A.m1 = -INFINITY;
+  A.l0 = A.l1 = 0.f;
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) A.o[mt][0] = A.o[mt][1] = A.o[mt][2] = A.o[mt][3] = 0.f;
+}
+
+// Query fragments (B operand of S = K Q^T): head n = lane/4 of the group, dims 2c, 2c+1.
+__device__ __forceinline__ void load_qf(uint32_t (&qf)[8][2], const AttnParams& p, int b, int h,
+                                        int lane) {
+  const int n = lane >> 2, c = lane & 3;
+  if (n < p.g) {
+    const uint32_t* qrow = p.q + ((size_t)b * p.Hq + h * p.g + n) * 64;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      qf[kk][0] = qrow[kk * 8 + c];
+      qf[kk][1] = qrow[kk * 8 + 4 + c];
+    }
+  } else {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) qf[kk][0] = qf[kk][1] = 0u;
+  }
+}
+
+// Issues the four tile loads of one (page, KV head) into a stage (K at +0, V at +4096).
+__device__ __forceinline__ void issue_page(uint8_t* dst, uint64_t* bar, const CUtensorMap* tmK,
+                                           const CUtensorMap* tmV, int phys, int Hkv, int h) {
+  fence_proxy_async_smem();
+  mbar_arrive_expect_tx(bar, kStageBytes);
+  const int y = (phys * Hkv + h) * kPageTok;
+  tma_load_2d(dst, tmK, 0, y, bar);
+  tma_load_2d(dst + 2048, tmK, 64, y, bar);
+  tma_load_2d(dst + 4096, tmV, 0, y, bar);
+  tma_load_2d(dst + 6144, tmV, 64, y, bar);
+}
+
+// One 16-token page in a stage: scores, online softmax, PV.  in0 / in1: whether this lane's
+// token rows r and r + 8 belong to the set.  Warp-uniform; no-op if no token belongs.
+__device__ __forceinline__ void page_compute(WarpAcc& A, const uint32_t (&qf)[8][2],
+                                             uint8_t* stage, bool in0, bool in1,
+                                             float scale_log2, int lane) {
+  if (!__any_sync(0xffffffffu, in0 || in1)) return;
+  const int r = lane >> 2, c = lane & 3;
+  const int mi = lane >> 3, rr = lane & 7;     // ldmatrix: matrix index, row in matrix
+  const int krow = ((mi & 1) << 3) + rr;       // K tile row (token) this lane addresses
+  const int vrow = ((mi >> 1) << 3) + rr;      // V tile row (token) this lane addresses
+  const uint32_t sb = smem_u32(stage);
+  // S[token][head] = K[token] . Q[head]; two independent accumulation chains
+  float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int kk = 0; kk < 8; kk += 2) {
+    uint32_t a0[4], a1[4];
+    const int ch0 = 2 * kk + (mi >> 1), ch1 = ch0 + 2;
+    ldsm_x4(a0, sb + (ch0 >> 3) * 2048 + krow * 128 + (((ch0 & 7) ^ rr) << 4));
+    ldsm_x4(a1, sb + (ch1 >> 3) * 2048 + krow * 128 + (((ch1 & 7) ^ rr) << 4));
+    mma_bf16_16816(sa, a0, qf[kk][0], qf[kk][1]);
+    mma_bf16_16816(sb2, a1, qf[kk + 1][0], qf[kk + 1][1]);
+  }
+  const float x0 = in0 ? (sa[0] + sb2[0]) * scale_log2 : -INFINITY;
+  const float x1 = in0 ? (sa[1] + sb2[1]) * scale_log2 : -INFINITY;
+  const float x2 = in1 ? (sa[2] + sb2[2]) * scale_log2 : -INFINITY;
+  const float x3 = in1 ? (sa[3] + sb2[3]) * scale_log2 : -INFINITY;
+  float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+  }
+  const float mn0 = fmaxf(A.m0, mx0), mn1 = fmaxf(A.m1, mx1);
+  if (mn0 > A.m0 || mn1 > A.m1) {
+    const float al0 = exp2f(A.m0 - mn0), al1 = exp2f(A.m1 - mn1);
+    A.l0 *= al0;
+    A.l1 *= al1;
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      A.o[mt][0] *= al0;
+      A.o[mt][1] *= al1;
+      A.o[mt][2] *= al0;
+      A.o[mt][3] *= al1;
+    }
+    A.m0 = mn0;
+    A.m1 = mn1;
+  }
+  const float p0 = exp2f(x0 - A.m0), p1 = exp2f(x1 - A.m1);
+  const float p2 = exp2f(x2 - A.m0), p3 = exp2f(x3 - A.m1);
+  A.l0 += p0 + p2;
+  A.l1 += p1 + p3;
+  const __nv_bfloat16 h0 = __float2bfloat16_rn(p0), h1 = __float2bfloat16_rn(p1);
+  const __nv_bfloat16 h2 = __float2bfloat16_rn(p2), h3 = __float2bfloat16_rn(p3);
+  const uint32_t hi01 = pack_bf16x2(h0, h1), hi23 = pack_bf16x2(h2, h3);
+  const uint32_t lo01 = pack_bf16x2(__float2bfloat16_rn(p0 - __bfloat162float(h0)),
+                                    __float2bfloat16_rn(p1 - __bfloat162float(h1)));
+  const uint32_t lo23 = pack_bf16x2(__float2bfloat16_rn(p2 - __bfloat162float(h2)),
+                                    __float2bfloat16_rn(p3 - __bfloat162float(h3)));
+  // P^T fragments (k = token, n = head) for the PV product
+  const uint32_t bh0 = movmatrix_trans(hi01), bh1 = movmatrix_trans(hi23);
+  const uint32_t bl0 = movmatrix_trans(lo01), bl1 = movmatrix_trans(lo23);
+  // Tokens outside the set have P = 0, but their V rows may hold stale bytes (slots not yet
+  // committed, or a partly filled page): 0 * NaN would poison the sum, so zero them.
+  if (__any_sync(0xffffffffu, !(in0 && in1))) {
+    uint4* vbase = reinterpret_cast<uint4*>(stage + 4096);
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    if (!in0) {   // token row r: 8 x 16 bytes in each 64-dim half
+      vbase[r * 8 + 2 * c] = z;
+      vbase[r * 8 + 2 * c + 1] = z;
+      vbase[128 + r * 8 + 2 * c] = z;
+      vbase[128 + r * 8 + 2 * c + 1] = z;
+    }
+    if (!in1) {   // token row r + 8
+      vbase[(r + 8) * 8 + 2 * c] = z;
+      vbase[(r + 8) * 8 + 2 * c + 1] = z;
+      vbase[128 + (r + 8) * 8 + 2 * c] = z;
+      vbase[128 + (r + 8) * 8 + 2 * c + 1] = z;
+    }
+    __syncwarp();
+  }
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    const int chunk = 2 * mt + (mi & 1);
+    uint32_t a[4];
+    ldsm_x4_trans(a, sb + 4096 + (chunk >> 3) * 2048 + vrow * 128 + (((chunk & 7) ^ rr) << 4));
+    mma_bf16_16816(A.o[mt], a, bh0, bh1);
+    mma_bf16_16816(A.o[mt], a, bl0, bl1);
+  }
+}
+
+// Reduces l over the token rows and writes the warp's state to its merge slot:
+// mo [g][kMergeStride] (O^T columns), ml [8][2] (m, l).
+__device__ __forceinline__ void warp_flush(WarpAcc& A, float* mo, float* ml, int g, int lane) {
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    A.l0 += __shfl_xor_sync(0xffffffffu, A.l0, off);
+    A.l1 += __shfl_xor_sync(0xffffffffu, A.l1, off);
+  }
+  const int r = lane >> 2, c = lane & 3;
+  const int n0 = 2 * c, n1 = 2 * c + 1;
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    const int d = 16 * mt + r;
+    if (n0 < g) {
+      mo[n0 * kMergeStride + d] = A.o[mt][0];
+      mo[n0 * kMergeStride + d + 8] = A.o[mt][2];
+    }
+    if (n1 < g) {
+      mo[n1 * kMergeStride + d] = A.o[mt][1];
+      mo[n1 * kMergeStride + d + 8] = A.o[mt][3];
+    }
+  }
+  if (r == 0) {
+    ml[n0 * 2] = A.m0;
+    ml[n0 * 2 + 1] = A.l0;
+    ml[n1 * 2] = A.m1;
+    ml[n1 * 2 + 1] = A.l1;
+  }
+}
+
+// Merge of the kW warp states for head n, dim d: (M, L, O) relative to exp2(M).
+__device__ __forceinline__ void cta_merge(const float* merge_o, const float* merge_ml, int g,
+                                          int n, int d, float& M, float& L, float& O) {
+  M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kW; ++w) M = fmaxf(M, merge_ml[w * 16 + n * 2]);
+  O = 0.f;
+  L = 0.f;
+  if (M == -INFINITY) return;
+#pragma unroll
+  for (int w = 0; w < kW; ++w) {
+    const float mw = merge_ml[w * 16 + n * 2];
+    if (mw != -INFINITY) {
+      const float sc = exp2f(mw - M);
+      O += sc * merge_o[(w * g + n) * kMergeStride + d];
+      L += sc * merge_ml[w * 16 + n * 2 + 1];
+    }
+  }
+}
+
+// q . k_new of head n of the group, in the exp2 domain (whole warp; result in every lane).
+__device__ __forceinline__ float staged_score(const AttnParams& p, int b, int h, int n, int lane) {
+  const uint32_t* qrow = p.q + ((size_t)b * p.Hq + h * p.g + n) * 64;
+  const uint32_t* krow = p.k_new + ((size_t)b * p.Hkv + h) * 64;
+  const uint32_t qa0 = qrow[lane], qa1 = qrow[lane + 32];
+  const uint32_t ka0 = krow[lane], ka1 = krow[lane + 32];
+  const float acc = bf16_lo_to_f32(qa0) * bf16_lo_to_f32(ka0) +
+                    bf16_hi_to_f32(qa0) * bf16_hi_to_f32(ka0) +
+                    bf16_lo_to_f32(qa1) * bf16_lo_to_f32(ka1) +
+                    bf16_hi_to_f32(qa1) * bf16_hi_to_f32(ka1);
+  return warp_sum(acc) * p.scale_log2;
+}
+
+__device__ __forceinline__ float staged_value(const AttnParams& p, int b, int h, int d) {
+  const uint32_t vv = p.v_new[((size_t)b * p.Hkv + h) * 64 + (d >> 1)];
+  return (d & 1) ? bf16_hi_to_f32(vv) : bf16_lo_to_f32(vv);
+}
+
+// Work units are (sequence b, KV head h, visited page v) in (b, h, v) order; every active
+// sequence has max(1, pages) units per KV head (an empty cache keeps one unit that loads
+// nothing, so the staged token still produces the output).  CTA c owns the contiguous unit
+// range [c*U/G, (c+1)*U/G) with G = min(grid size, U): equal work per CTA.  The part of that range inside one (b, h)
+// is a segment; each segment yields one partial in slot c + b*Hkv + h (unique, since the
+// CTAs walk the (b, h) pairs in order).
+struct Seg {
+  int b, h, v0, n;   // first visited page of the segment, units in this CTA's segment
+  int s0, nv;        // first unit of (b, h) and units per KV head of sequence b
+};
+
+__device__ __forceinline__ Seg decode_seg(int u, int u1, const int* s_us, const int* s_nv, int B,
+                                          int Hkv) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_us[mid] <= u) lo = mid; else hi = mid - 1;
+  }
+  Seg s;
+  s.b = lo;
+  s.nv = s_nv[lo];
+  const int r = u - s_us[lo];
+  s.h = r / s.nv;
+  s.v0 = r - s.h * s.nv;
+  s.s0 = s_us[lo] + s.h * s.nv;
+  s.n = min(u1, s.s0 + s.nv) - u;
+  return s;
+}
+
+// CTA owning unit u when G CTAs split U units.
+__device__ __forceinline__ int cta_of(long long u, long long U, long long G) {
+  return (int)(((u + 1) * G - 1) / U);
+}
+
+// ---------------------------------------------------------------- local set: clusters
+// Cluster of p.cluster CTAs per (b, h); CTA `rank` takes the contiguous share
+// [rank*nv/C, (rank+1)*nv/C) of the visited pages; warps take every kW-th page of it.
+__global__ void __launch_bounds__(kThreads, 2)
+attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int g = p.g;
+  float* merge_o = reinterpret_cast<float*>(stages + kStagesBytes);   // [W][g][132]
+  float* merge_ml = merge_o + kW * g * kMergeStride;                  // [W][8][2]
+  float* cpart_o = merge_ml + kW * 16;                                // [g][128] CTA partial
+  float* cpart_ml = cpart_o + g * 128;                                // [g][2]
+  __shared__ __align__(8) uint64_t bars[kW * kR];
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = p.cluster;
+  const int rank = (int)cluster.block_rank();
+  const int bh = blockIdx.x / C;
+  const int b = bh / p.Hkv, h = bh - (bh / p.Hkv) * p.Hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < kW * kR; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+  }
+  const int t = __ldcg(p.pos + b);
+  const Geom ge = make_geom(t, 0, p.sinks, p.window, p.max_pages, true);
+  if (!ge.active && rank == 0 && tid == 0) atomicOr(p.err, ODA_DEVERR_POS_RANGE);
+  const int nv = ge.active ? geom_pages(ge) : 0;
+  const int v_lo = (int)((long long)rank * nv / C), v_hi = (int)((long long)(rank + 1) * nv / C);
+  const int cw = (v_hi - v_lo - warp > 0) ? (v_hi - v_lo - warp + kW - 1) / kW : 0;
+  const int* ptab = p.page_table + (size_t)b * p.max_pages;
+  uint8_t* my_stages = stages + warp * kR * kStageBytes;
+  uint64_t* my_bars = bars + warp * kR;
+  __syncthreads();
+
+  // lane k holds the physical page of this warp's (pt_base + k)-th page
+  int pt_phys = -1, pt_base = -64;
+  auto refill = [&](int base) {
+    const int k = base + lane;
+    pt_phys = -1;
+    if (k < cw && ge.n_cache > 0) {
+      const int phys = __ldcg(ptab + geom_page(ge, v_lo + warp + k * kW));
+      pt_phys = (phys >= 0 && (int64_t)phys < p.n_pool_pages) ? phys : -2;
+      if (pt_phys == -2) atomicOr(p.err, ODA_DEVERR_PAGE_RANGE);
+    }
+    pt_base = base;
+  };
+  uint32_t vbits = 0;
+  auto issue = [&](int k) {
+    if (k - pt_base >= 32) refill(k & ~31);
+    const uint32_t st = (uint32_t)k % kR;
+    const int phys = __shfl_sync(0xffffffffu, pt_phys, k - pt_base);
+    if (lane == k - pt_base) {
+      if (phys >= 0)
+        issue_page(my_stages + st * kStageBytes, my_bars + st, &tmK, &tmV, phys, p.Hkv, h);
+      else
+        mbar_arrive(my_bars + st);
+    }
+    vbits = phys >= 0 ? (vbits | (1u << st)) : (vbits & ~(1u << st));
+  };
+  for (int k = 0; k < kR && k < cw; ++k) issue(k);
+  // the previous launch on the stream may still run: wait before reading q or writing
+  grid_dependency_wait();
+  grid_dependents_launch();
+
+  uint32_t qf[8][2];
+  load_qf(qf, p, b, h, lane);
+  WarpAcc A;
+  acc_init(A);
+  const int r = lane >> 2;
+  int k = 0;
+  bool dead = false;
+  for (; k < cw; ++k) {
+    const uint32_t st = (uint32_t)k % kR;
+    if (!mbar_wait_bounded(my_bars + st, ((uint32_t)k / kR) & 1u, kWaitNs)) {
+      if (lane == 0) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
+      dead = true;
+      break;
+    }
+    const int lp = geom_page(ge, v_lo + warp + k * kW);
+    const bool ok = (vbits >> st) & 1u;
+    const int j0 = lp * kPageTok + r;
+    page_compute(A, qf, my_stages + st * kStageBytes, ok && geom_has(ge, j0),
+                 ok && geom_has(ge, j0 + 8), p.scale_log2, lane);
+    __syncwarp();
+    if (k + kR < cw) issue(k + kR);
+  }
+  warp_flush(A, merge_o + warp * g * kMergeStride, merge_ml + warp * 16, g, lane);
+  __syncthreads();
+  for (int idx = tid; idx < g * 128; idx += kThreads) {
+    const int n = idx >> 7, d = idx & 127;
+    float M, L, O;
+    cta_merge(merge_o, merge_ml, g, n, d, M, L, O);
+    cpart_o[n * 128 + d] = O;
+    if (d == 0) {
+      cpart_ml[n * 2] = M;
+      cpart_ml[n * 2 + 1] = L;
+    }
+  }
+  cluster.sync();
+  if (rank == 0 && ge.active) {
+    // merge the cluster's partials (distributed shared memory) and the staged token
+    const int d = tid;  // kThreads == 128 == head_dim
+    const float vd = staged_value(p, b, h, d);
+    for (int n = 0; n < g; ++n) {
+      const float snew = staged_score(p, b, h, n, lane);
+      float Mr[kMaxCluster], Lr[kMaxCluster], Or[kMaxCluster];
+      float M = snew;
+#pragma unroll
+      for (int q = 0; q < kMaxCluster; ++q) {
+        if (q < C) {
+          const float* rml = cluster.map_shared_rank(cpart_ml, q);
+          const float* ro = cluster.map_shared_rank(cpart_o, q);
+          Mr[q] = rml[n * 2];
+          Lr[q] = rml[n * 2 + 1];
+          Or[q] = ro[n * 128 + d];
+          M = fmaxf(M, Mr[q]);
+        }
+      }
+      const float wn = exp2f(snew - M);
+      float L = wn, O = wn * vd;
+#pragma unroll
+      for (int q = 0; q < kMaxCluster; ++q) {
+        if (q < C && Mr[q] != -INFINITY) {
+          const float w = exp2f(Mr[q] - M);
+          L += w * Lr[q];
+          O += w * Or[q];
+        }
+      }
+      p.out[((size_t)b * p.Hq + h * g + n) * 128 + d] = O / L;
+    }
+  }
+  // keep every CTA's shared memory alive until rank 0 has read it
+  cluster.sync();
+  if (dead) {
+    for (int kk = k; kk < cw && kk < k + kR; ++kk)
+      (void)mbar_wait_bounded(my_bars + (kk % kR), ((uint32_t)kk / kR) & 1u, kWaitNs);
+  }
+}
+
+// ------------------------------------------------------------ full set: persistent grid
+__global__ void __launch_bounds__(kThreads, 2)
+attn_full_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* stages = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int g = p.g;
+  float* merge_o = reinterpret_cast<float*>(stages + kStagesBytes);   // [W][g][132]
+  float* merge_ml = merge_o + kW * g * kMergeStride;                  // [W][8][2]
   __shared__ __align__(8) uint64_t bars[kW * kR];
   __shared__ int s_t[ODA_MAX_BATCH];
   __shared__ int s_nv[ODA_MAX_BATCH];
-  __shared__ int s_start[ODA_MAX_BATCH + 1];
-  __shared__ int s_sp;
+  __shared__ int s_us[ODA_MAX_BATCH + 1];
   __shared__ int s_last;
-  __shared__ float s_L[8], s_wnew[8];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int B = p.B, Hkv = p.Hkv, g = p.g;
+  const int B = p.B, Hkv = p.Hkv;
 
   if (tid == 0) {
 #pragma unroll
@@ -149,337 +533,238 @@ attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
   }
-  // ---- per-sequence geometry, split size and item prefix sums (identical in every CTA)
+  // ---- per-sequence geometry and unit prefix sums (identical in every CTA)
   for (int b = tid; b < B; b += kThreads) {
-    const int t = p.pos[b];
-    const bool wanted = (p.mode == 0) || (p.flag[b] != 0);
-    const Geom ge = make_geom(t, p.mode, p.sinks, p.window, p.max_pages, wanted);
+    const int t = __ldcg(p.pos + b);
+    const bool wanted = __ldcg(p.flag + b) != 0;
+    const Geom ge = make_geom(t, 1, p.sinks, p.window, p.max_pages, wanted);
     s_t[b] = t;
-    s_nv[b] = ge.active ? geom_pages(ge) : -1;
+    s_nv[b] = ge.active ? max(1, geom_pages(ge)) : 0;
     if (wanted && !ge.active && blockIdx.x == 0) atomicOr(p.err, ODA_DEVERR_POS_RANGE);
   }
   __syncthreads();
   if (warp == 0) {
-    long long sum = 0;
-    int mx = 0;
-    for (int b = lane; b < B; b += 32) {
-      const int nv = s_nv[b];
-      if (nv > 0) {
-        sum += nv;
-        mx = max(mx, nv);
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    }
-    const long long target = (long long)kItemsPerCta * gridDim.x;
-    int sp = (int)((sum * Hkv + target - 1) / target);
-    sp = max(sp, kMinSplitPages);
-    sp = max(sp, (mx + p.max_splits - 1) / p.max_splits);
     int running = 0;
     for (int base = 0; base < B; base += 32) {
       const int b = base + lane;
-      int cnt = 0;
-      if (b < B && s_nv[b] >= 0) cnt = Hkv * max(1, (s_nv[b] + sp - 1) / sp);
+      const int cnt = (b < B) ? Hkv * s_nv[b] : 0;
       int incl = cnt;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
-      if (b < B) s_start[b] = running + incl - cnt;
+      if (b < B) s_us[b] = running + incl - cnt;
       running += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) {
-      s_start[B] = running;
-      s_sp = sp;
-    }
+    if (lane == 0) s_us[B] = running;
   }
   __syncthreads();
-  const int total = s_start[B];
-  const int SP = s_sp;
-
-  uint32_t issued = 0, consumed = 0;
-  bool dead = false;
-  const int r = lane >> 2, c = lane & 3;       // mma fragment row / column group
-  const int mi = lane >> 3, rr = lane & 7;     // ldmatrix: matrix index, row in matrix
-  const int krow = ((mi & 1) << 3) + rr;       // K tile row (token) this lane addresses
-  const int vrow = ((mi >> 1) << 3) + rr;      // V tile row (token) this lane addresses
+  // G = min(grid, U) CTAs share the units, so that every one of them owns at least one unit
+  // and the CTAs covering a (b, h) are exactly the consecutive range found by cta_of.
+  const long long U = s_us[B];
+  const long long G = U < (long long)gridDim.x ? U : (long long)gridDim.x;
+  int u0 = 0, u1 = 0;
+  if ((long long)blockIdx.x < G) {
+    u0 = (int)(blockIdx.x * U / G);
+    u1 = (int)((blockIdx.x + 1) * U / G);
+  }
   uint8_t* my_stages = stages + warp * kR * kStageBytes;
   uint64_t* my_bars = bars + warp * kR;
 
-  for (int item = blockIdx.x; item < total; item += gridDim.x) {
-    // ---- decode the item
-    int lo = 0, hi = B - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_start[mid] <= item) lo = mid; else hi = mid - 1;
+  // ---- this warp's copy stream: its units (every kW-th of each segment), kR ahead.  Lane k
+  // of the warp holds the physical page and KV head of the warp's (pt_base + k)-th unit,
+  // refilled 32 units at a time with parallel loads, and issues that unit's copy itself.
+  uint32_t issued = 0, consumed = 0, vbits = 0, pt_base = 0;
+  int pt_phys = -1, pt_head = 0;
+  bool pt_live = false;
+  bool dead = false;
+  int is_u = u0, is_i = warp;
+  Seg is{0, 0, 0, 0, 0, 1};
+  if (is_u < u1) is = decode_seg(is_u, u1, s_us, s_nv, B, Hkv);
+  auto normalize = [&](int& cu, int& ci, Seg& cs_) {
+    while (cu < u1 && ci >= cs_.n) {
+      cu += cs_.n;
+      ci = warp;
+      if (cu < u1) cs_ = decode_seg(cu, u1, s_us, s_nv, B, Hkv);
     }
-    const int b = lo;
-    const int rel = item - s_start[b];
-    const int split = rel / Hkv, h = rel - split * Hkv;
-    const int nv = s_nv[b];
-    const int nsplit = max(1, (nv + SP - 1) / SP);
-    const Geom ge = make_geom(s_t[b], p.mode, p.sinks, p.window, p.max_pages, true);
-    const int v0 = split * SP, v1 = min(v0 + SP, nv);
-    const int cw = (v1 - v0 - warp > 0) ? (v1 - v0 - warp + kW - 1) / kW : 0;
-    const int* ptab = p.page_table + (size_t)b * p.max_pages;
+  };
+  normalize(is_u, is_i, is);
+  auto refill = [&]() {
+    // each lane walks `lane` units ahead of the issue cursor and looks up its page
+    int cu = is_u, ci = is_i;
+    Seg cs_ = is;
+    for (int k = 0; k < lane && cu < u1; ++k) {
+      ci += kW;
+      normalize(cu, ci, cs_);
+    }
+    pt_phys = -1;
+    pt_head = cs_.h;
+    if (cu < u1) {
+      const Geom ge = make_geom(s_t[cs_.b], 1, p.sinks, p.window, p.max_pages, true);
+      if (ge.n_cache > 0) {
+        const int lp = geom_page(ge, cs_.v0 + ci);
+        const int phys = __ldcg(p.page_table + (size_t)cs_.b * p.max_pages + lp);
+        pt_phys = (phys >= 0 && (int64_t)phys < p.n_pool_pages) ? phys : -2;
+        if (pt_phys == -2) atomicOr(p.err, ODA_DEVERR_PAGE_RANGE);
+      }
+    }
+    pt_base = issued;
+    pt_live = true;
+  };
+  auto issue_next = [&]() {
+    if (dead || is_u >= u1) return;
+    if (!pt_live || issued - pt_base >= 32u) refill();
+    const uint32_t st = issued % kR;
+    const int src = (int)(issued - pt_base);
+    const int phys = __shfl_sync(0xffffffffu, pt_phys, src);
+    const int head = __shfl_sync(0xffffffffu, pt_head, src);
+    if (lane == src) {
+      if (phys >= 0)
+        issue_page(my_stages + st * kStageBytes, my_bars + st, &tmK, &tmV, phys, Hkv, head);
+      else
+        mbar_arrive(my_bars + st);
+    }
+    vbits = phys >= 0 ? (vbits | (1u << st)) : (vbits & ~(1u << st));
+    ++issued;
+    is_i += kW;
+    normalize(is_u, is_i, is);
+  };
+  for (int k = 0; k < kR; ++k) issue_next();
+  // Everything above reads only the cache, the page table and positions/flags, which an
+  // attention launch never writes; the previous launch of the stream may still be running
+  // (programmatic dependent launch).  Wait for it before reading q or writing anything.
+  grid_dependency_wait();
+  grid_dependents_launch();
 
-    // ---- query fragments (B operand of S = K Q^T): head n = r of the group, dims 2c, 2c+1
+  // ---- segments of this CTA, in order
+  for (int seg_u = u0; seg_u < u1;) {
+    const Seg cs = decode_seg(seg_u, u1, s_us, s_nv, B, Hkv);
+    const Geom ge = make_geom(s_t[cs.b], 1, p.sinks, p.window, p.max_pages, true);
+    const int b = cs.b, h = cs.h;
     uint32_t qf[8][2];
-    {
-      const int n = r;
-      if (n < g) {
-        const uint32_t* qrow = p.q + ((size_t)b * p.Hq + h * g + n) * 64;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          qf[kk][0] = qrow[kk * 8 + c];
-          qf[kk][1] = qrow[kk * 8 + 4 + c];
-        }
-      } else {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) qf[kk][0] = qf[kk][1] = 0u;
+    load_qf(qf, p, b, h, lane);
+    WarpAcc A;
+    acc_init(A);
+    const int r = lane >> 2;
+    for (int i = warp; i < cs.n && !dead; i += kW) {
+      const uint32_t st = consumed % kR;
+      if (!mbar_wait_bounded(my_bars + st, (consumed / kR) & 1u, kWaitNs)) {
+        if (lane == 0) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
+        dead = true;
+        break;
       }
-    }
-
-    auto issue = [&](int k) {
-      const int v = v0 + warp + k * kW;
-      const int lp = geom_page(ge, v);
-      const uint32_t st = issued % kR;
-      if (lane == 0) {
-        const int phys = ptab[lp];
-        uint64_t* bar = my_bars + st;
-        if (phys >= 0 && (int64_t)phys < p.n_pool_pages) {
-          uint8_t* dst = my_stages + st * kStageBytes;
-          fence_proxy_async_smem();
-          mbar_arrive_expect_tx(bar, kStageBytes);
-          const int y = (phys * Hkv + h) * kPageTok;
-          tma_load_2d(dst, &tmK, 0, y, bar);
-          tma_load_2d(dst + 2048, &tmK, 64, y, bar);
-          tma_load_2d(dst + 4096, &tmV, 0, y, bar);
-          tma_load_2d(dst + 6144, &tmV, 64, y, bar);
-        } else {
-          atomicOr(p.err, ODA_DEVERR_PAGE_RANGE);
-          mbar_arrive(bar);
-        }
-      }
-      ++issued;
-    };
-
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    float o[8][4];
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-
-    if (!dead) {
+      const bool ok = (vbits >> st) & 1u;
+      const int lp = geom_page(ge, cs.v0 + i);
+      const int j0 = lp * kPageTok + r;
+      page_compute(A, qf, my_stages + st * kStageBytes, ok && geom_has(ge, j0),
+                   ok && geom_has(ge, j0 + 8), p.scale_log2, lane);
+      ++consumed;
       __syncwarp();
-      const int pre = min(cw, kR);
-      for (int k = 0; k < pre; ++k) issue(k);
-      for (int k = 0; k < cw; ++k) {
-        const uint32_t st = consumed % kR;
-        if (!mbar_wait_bounded(my_bars + st, (consumed / kR) & 1u, kWaitNs)) {
-          if (lane == 0) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
-          dead = true;
-          break;
-        }
-        const int v = v0 + warp + k * kW;
-        const int lp = geom_page(ge, v);
-        const int phys = ptab[lp];
-        const bool page_ok = phys >= 0 && (int64_t)phys < p.n_pool_pages;
-        const int j0 = lp * kPageTok + r, j1 = j0 + 8;
-        const bool in0 = page_ok && geom_has(ge, j0);
-        const bool in1 = page_ok && geom_has(ge, j1);
-        if (__any_sync(0xffffffffu, in0 || in1)) {
-          const uint32_t sb = smem_u32(my_stages + st * kStageBytes);
-          // S[token][head] = K[token] . Q[head]
-          float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const int chunk = 2 * kk + (mi >> 1);
-            uint32_t a[4];
-            ldsm_x4(a, sb + (chunk >> 3) * 2048 + krow * 128 + (((chunk & 7) ^ rr) << 4));
-            mma_bf16_16816(sacc, a, qf[kk][0], qf[kk][1]);
-          }
-          const float x0 = in0 ? sacc[0] * p.scale_log2 : -INFINITY;
-          const float x1 = in0 ? sacc[1] * p.scale_log2 : -INFINITY;
-          const float x2 = in1 ? sacc[2] * p.scale_log2 : -INFINITY;
-          const float x3 = in1 ? sacc[3] * p.scale_log2 : -INFINITY;
-          float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-          for (int off = 4; off < 32; off <<= 1) {
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-          }
-          const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-          const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
-          m0 = mn0;
-          m1 = mn1;
-          l0 *= al0;
-          l1 *= al1;
-#pragma unroll
-          for (int mt = 0; mt < 8; ++mt) {
-            o[mt][0] *= al0;
-            o[mt][1] *= al1;
-            o[mt][2] *= al0;
-            o[mt][3] *= al1;
-          }
-          const float p0 = exp2f(x0 - mn0), p1 = exp2f(x1 - mn1);
-          const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
-          l0 += p0 + p2;
-          l1 += p1 + p3;
-          const __nv_bfloat16 h0 = __float2bfloat16_rn(p0), h1 = __float2bfloat16_rn(p1);
-          const __nv_bfloat16 h2 = __float2bfloat16_rn(p2), h3 = __float2bfloat16_rn(p3);
-          const uint32_t hi01 = pack_bf16x2(h0, h1), hi23 = pack_bf16x2(h2, h3);
-          const uint32_t lo01 = pack_bf16x2(__float2bfloat16_rn(p0 - __bfloat162float(h0)),
-                                            __float2bfloat16_rn(p1 - __bfloat162float(h1)));
-          const uint32_t lo23 = pack_bf16x2(__float2bfloat16_rn(p2 - __bfloat162float(h2)),
-                                            __float2bfloat16_rn(p3 - __bfloat162float(h3)));
-          // P^T fragments (k = token, n = head) for the PV product
-          const uint32_t bh0 = movmatrix_trans(hi01), bh1 = movmatrix_trans(hi23);
-          const uint32_t bl0 = movmatrix_trans(lo01), bl1 = movmatrix_trans(lo23);
-#pragma unroll
-          for (int mt = 0; mt < 8; ++mt) {
-            const int chunk = 2 * mt + (mi & 1);
-            uint32_t a[4];
-            ldsm_x4_trans(a, sb + 4096 + (chunk >> 3) * 2048 + vrow * 128 +
-                                 (((chunk & 7) ^ rr) << 4));
-            mma_bf16_16816(o[mt], a, bh0, bh1);
-            mma_bf16_16816(o[mt], a, bl0, bl1);
-          }
-        }
-        ++consumed;
-        __syncwarp();
-        if (k + kR < cw) issue(k + kR);
-      }
+      issue_next();
     }
-
-    // ---- column sums of l across the 8 token rows held by lanes with the same c
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-    }
-    // ---- this warp's state -> its own (now idle) stage memory
-    {
-      float* mo = reinterpret_cast<float*>(my_stages);
-      float* ml = mo + 8 * kMergeStride;
-      const int n0 = 2 * c, n1 = 2 * c + 1;
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        const int d = 16 * mt + r;
-        if (n0 < g) {
-          mo[n0 * kMergeStride + d] = o[mt][0];
-          mo[n0 * kMergeStride + d + 8] = o[mt][2];
-        }
-        if (n1 < g) {
-          mo[n1 * kMergeStride + d] = o[mt][1];
-          mo[n1 * kMergeStride + d + 8] = o[mt][3];
-        }
-      }
-      if (r == 0) {
-        ml[n0 * 2] = m0;
-        ml[n0 * 2 + 1] = l0;
-        ml[n1 * 2] = m1;
-        ml[n1 * 2 + 1] = l1;
-      }
-    }
+    warp_flush(A, merge_o + warp * g * kMergeStride, merge_ml + warp * 16, g, lane);
     __syncthreads();
-    // ---- merge the warps into one partial per query head of the group
+    // ---- merge the warps into this segment's partial (one per query head of the group)
+    const int bh = b * Hkv + h;
+    const int slot = (int)blockIdx.x + bh;
     for (int idx = tid; idx < g * 128; idx += kThreads) {
       const int n = idx >> 7, d = idx & 127;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kW; ++w) {
-        const float* ml = reinterpret_cast<const float*>(stages + w * kR * kStageBytes) +
-                          8 * kMergeStride;
-        M = fmaxf(M, ml[n * 2]);
-      }
-      float O = 0.f, L = 0.f;
-      if (M != -INFINITY) {
-#pragma unroll
-        for (int w = 0; w < kW; ++w) {
-          const float* mo = reinterpret_cast<const float*>(stages + w * kR * kStageBytes);
-          const float* ml = mo + 8 * kMergeStride;
-          const float mw = ml[n * 2];
-          if (mw != -INFINITY) {
-            const float s = exp2f(mw - M);
-            O += s * mo[n * kMergeStride + d];
-            L += s * ml[n * 2 + 1];
-          }
-        }
-      }
-      const size_t pi = (size_t)(b * p.Hq + h * g + n) * p.max_splits + split;
-      p.part_o[pi * 128 + d] = O;
+      float M, L, O;
+      cta_merge(merge_o, merge_ml, g, n, d, M, L, O);
+      p.part_o[((size_t)slot * g + n) * 128 + d] = O;
       if (d == 0) {
-        p.part_ml[pi * 2] = M;
-        p.part_ml[pi * 2 + 1] = L;
+        p.part_ml[((size_t)slot * g + n) * 2] = M;
+        p.part_ml[((size_t)slot * g + n) * 2 + 1] = L;
       }
     }
-    __threadfence();
+    // publish: the CTA barrier orders every thread's partial writes before thread 0's
+    // gpu-scope fence and count; the CTA that completes the count reads all partials
     __syncthreads();
+    const int c_first = cta_of(cs.s0, U, G), c_last = cta_of(cs.s0 + cs.nv - 1, U, G);
+    const int nparts = c_last - c_first + 1;
     if (tid == 0) {
-      const int old = atomicAdd(&p.counters[b * Hkv + h], 1);
-      s_last = (old == nsplit - 1);
+      __threadfence();
+      s_last = (atomicAdd(&p.counters[bh], 1) == nparts - 1);
+      if (s_last) __threadfence();
     }
     __syncthreads();
     if (s_last) {
-      // ---- last CTA of (b, h): merge all splits and the staged current token
-      __threadfence();
-      float* s_w = reinterpret_cast<float*>(stages);  // [g][nsplit] split weights
+      // ---- last CTA of (b, h): merge the partials and the staged current token.  Loads are
+      // issued together: warps find each head's maximum and weights with lanes over partials,
+      // then every thread sums its dim over the partials with independent loads.
+      const int slot0 = c_first + bh;
+      float* s_w = merge_o;                  // [g][nparts] weights; nparts <= grid size
+      float* s_fin = merge_ml;               // [g][2]: 1 / L, weight of the staged token
       for (int n = warp; n < g; n += kW) {
-        const uint32_t* qrow = p.q + ((size_t)b * p.Hq + h * g + n) * 64;
-        const uint32_t* krow_new = p.k_new + ((size_t)b * Hkv + h) * 64;
-        float acc = 0.f;
-        for (int i = lane; i < 64; i += 32) {
-          const uint32_t qa = qrow[i], ka = krow_new[i];
-          acc += bf16_lo_to_f32(qa) * bf16_lo_to_f32(ka) + bf16_hi_to_f32(qa) * bf16_hi_to_f32(ka);
-        }
-        const float snew = warp_sum(acc) * p.scale_log2;
-        const float* pml = p.part_ml + (size_t)(b * p.Hq + h * g + n) * p.max_splits * 2;
+        const float snew = staged_score(p, b, h, n, lane);
+        float ms[2], ls[2];
         float M = snew;
-        for (int s = lane; s < nsplit; s += 32) M = fmaxf(M, __ldcg(pml + 2 * s));
-        M = warp_max(M);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int s = lane + 32 * q;
+          ms[q] = -INFINITY;
+          ls[q] = 0.f;
+          if (s < nparts) {
+            const size_t pi = (size_t)(slot0 + s) * g + n;
+            ms[q] = __ldcg(p.part_ml + pi * 2);
+            ls[q] = __ldcg(p.part_ml + pi * 2 + 1);
+          }
+          M = fmaxf(M, ms[q]);
+        }
+        for (int s = lane + 64; s < nparts; s += 32)
+          M = fmaxf(M, __ldcg(p.part_ml + ((size_t)(slot0 + s) * g + n) * 2));
+#pragma unroll
+        for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
         float L = 0.f;
-        for (int s = lane; s < nsplit; s += 32) {
-          const float ms = __ldcg(pml + 2 * s);
-          const float w = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
-          s_w[n * nsplit + s] = w;
-          L += w * __ldcg(pml + 2 * s + 1);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int s = lane + 32 * q;
+          if (s < nparts) {
+            const float w = (ms[q] == -INFINITY) ? 0.f : exp2f(ms[q] - M);
+            s_w[n * nparts + s] = w;
+            L += w * ls[q];
+          }
+        }
+        for (int s = lane + 64; s < nparts; s += 32) {
+          const size_t pi = (size_t)(slot0 + s) * g + n;
+          const float m2 = __ldcg(p.part_ml + pi * 2);
+          const float w = (m2 == -INFINITY) ? 0.f : exp2f(m2 - M);
+          s_w[n * nparts + s] = w;
+          L += w * __ldcg(p.part_ml + pi * 2 + 1);
         }
         L = warp_sum(L);
         const float wnew = exp2f(snew - M);
         if (lane == 0) {
-          s_L[n] = L + wnew;
-          s_wnew[n] = wnew;
+          s_fin[n * 2] = 1.0f / (L + wnew);
+          s_fin[n * 2 + 1] = wnew;
         }
       }
       __syncthreads();
-      for (int idx = tid; idx < g * 128; idx += kThreads) {
-        const int n = idx >> 7, d = idx & 127;
-        const float* po = p.part_o + (size_t)(b * p.Hq + h * g + n) * p.max_splits * 128 + d;
-        const float* wn = s_w + n * nsplit;
+      const int d = tid;  // kThreads == 128 == head_dim
+      const float vd = staged_value(p, b, h, d);
+      for (int n = 0; n < g; ++n) {
+        const float* wn = s_w + n * nparts;
+        const float* po = p.part_o + ((size_t)slot0 * g + n) * 128 + d;
+        const size_t stride = (size_t)g * 128;
         float O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
         int s = 0;
-        for (; s + 4 <= nsplit; s += 4) {
-          O0 += wn[s] * __ldcg(po + (size_t)s * 128);
-          O1 += wn[s + 1] * __ldcg(po + (size_t)(s + 1) * 128);
-          O2 += wn[s + 2] * __ldcg(po + (size_t)(s + 2) * 128);
-          O3 += wn[s + 3] * __ldcg(po + (size_t)(s + 3) * 128);
+        for (; s + 4 <= nparts; s += 4) {
+          const float a0 = __ldcg(po + (size_t)s * stride), a1 = __ldcg(po + (size_t)(s + 1) * stride);
+          const float a2 = __ldcg(po + (size_t)(s + 2) * stride), a3 = __ldcg(po + (size_t)(s + 3) * stride);
+          O0 += wn[s] * a0;
+          O1 += wn[s + 1] * a1;
+          O2 += wn[s + 2] * a2;
+          O3 += wn[s + 3] * a3;
         }
-        for (; s < nsplit; ++s) O0 += wn[s] * __ldcg(po + (size_t)s * 128);
-        const uint32_t vv = p.v_new[((size_t)b * Hkv + h) * 64 + (d >> 1)];
-        const float vd = (d & 1) ? bf16_hi_to_f32(vv) : bf16_lo_to_f32(vv);
-        const float O = (O0 + O1) + (O2 + O3) + s_wnew[n] * vd;
-        p.out[((size_t)b * p.Hq + h * g + n) * 128 + d] = O / s_L[n];
+        for (; s < nparts; ++s) O0 += wn[s] * __ldcg(po + (size_t)s * stride);
+        p.out[((size_t)b * p.Hq + h * g + n) * 128 + d] =
+            ((O0 + O1) + (O2 + O3) + s_fin[n * 2 + 1] * vd) * s_fin[n * 2];
       }
-      if (tid == 0) p.counters[b * Hkv + h] = 0;
+      if (tid == 0) p.counters[bh] = 0;
     }
-    // the stage memory was used through the generic proxy above; the next item's TMA writes
-    // it through the async proxy
-    fence_proxy_async_smem();
     __syncthreads();
+    seg_u += cs.n;
   }
   // a warp that gave up on a barrier waits (bounded) for the copies it still has in flight
   if (dead) {
@@ -555,9 +840,31 @@ oda_status encode_pool(CUtensorMap* m, void* base, int64_t n_pages, int Hkv) {
 
 }  // namespace
 
-int attention_smem_bytes() { return kSmemBytes; }
-int attention_threads() { return kThreads; }
-int attention_ctas_per_sm() { return kCtasPerSm; }
+int attention_smem_bytes(int g) {
+  return 1024 + kStagesBytes + (kW * g * kMergeStride + kW * 16 + g * 130) * (int)sizeof(float);
+}
+
+// Sets the shared-memory limits and returns the persistent grid size for group size g.
+oda_status prepare_attention_kernel(int g, int n_sms, int* ctas) {
+  const int smem = attention_smem_bytes(g);
+  oda_status st = check_cuda(
+      cudaFuncSetAttribute(attn_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+      "cudaFuncSetAttribute(full attention)");
+  if (st == ODA_OK)
+    st = check_cuda(
+        cudaFuncSetAttribute(attn_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+        "cudaFuncSetAttribute(local attention)");
+  if (st != ODA_OK) return st;
+  int occ = 0;
+  st = check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, attn_full_kernel, kThreads, smem),
+                  "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+  if (st != ODA_OK) return st;
+  occ = std::max(1, std::min(occ, 2));
+  *ctas = n_sms * occ;
+  // the combine keeps one weight per partial and head in the merge area
+  if (*ctas > kW * kMergeStride) return set_error(ODA_ERR_UNSUPPORTED, "too many CTAs for the merge area");
+  return ODA_OK;
+}
 
 oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32_t* page_table,
                             const int32_t* pos, const int32_t* flag, const void* q,
@@ -598,19 +905,45 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
   p.Hkv = cf.n_kv_heads;
   p.g = ctx->g;
   p.max_pages = cf.max_pages;
-  p.max_splits = ctx->max_splits;
   p.sinks = cf.sinks;
   p.window = cf.window;
   p.mode = mode;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(128.0));
-  attn_kernel<<<ctx->attn_ctas, kThreads, kSmemBytes, stream>>>(tmK, tmV, p);
-  return check_cuda(cudaGetLastError(), "attention launch");
-}
+  // cluster size of the local kernel: enough CTAs per (b, h) to cover the GPU, at most 8
+  const int pairs = cf.batch * cf.n_kv_heads;
+  p.cluster = std::max(1, std::min(kMaxCluster, (ctx->attn_ctas + pairs / 2) / pairs));
 
-oda_status prepare_attention_kernel() {
-  return check_cuda(cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes),
-                    "cudaFuncSetAttribute(attention)");
+  // Consecutive attention launches of one context overlap when the context allows it: the
+  // later one may start (and prefetch its pages) while the earlier one finishes; it waits
+  // before reading q or writing.
+  cudaLaunchConfig_t lc = {};
+  lc.blockDim = dim3(kThreads);
+  lc.dynamicSmemBytes = attention_smem_bytes(ctx->g);
+  lc.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (cf.overlap_layers && ctx->prev_attention) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (mode == 0) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = p.cluster;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+    lc.gridDim = dim3(pairs * p.cluster);
+  } else {
+    lc.gridDim = dim3(ctx->attn_ctas);
+  }
+  lc.attrs = attr;
+  lc.numAttrs = na;
+  st = (mode == 0)
+           ? check_cuda(cudaLaunchKernelEx(&lc, attn_local_kernel, tmK, tmV, p), "local attention launch")
+           : check_cuda(cudaLaunchKernelEx(&lc, attn_full_kernel, tmK, tmV, p), "full attention launch");
+  ctx->prev_attention = (st == ODA_OK);
+  return st;
 }
 
 oda_status launch_index_positions(oda_ctx* ctx, int mode, const int32_t* pos, const int32_t* flag,
@@ -619,6 +952,7 @@ oda_status launch_index_positions(oda_ctx* ctx, int mode, const int32_t* pos, co
   if (!pos || !positions || !counts || cap <= 0 || (mode == 1 && !flag) || (mode != 0 && mode != 1))
     return set_error(ODA_ERR_INVALID_ARG, "index_positions: bad argument");
   const oda_config& cf = ctx->cfg;
+  ctx->prev_attention = false;
   index_positions_kernel<<<(cf.batch + 31) / 32, 32, 0, stream>>>(
       pos, flag, cf.batch, mode, cf.sinks, cf.window, cf.max_pages, positions, cap, counts);
   return check_cuda(cudaGetLastError(), "index_positions launch");

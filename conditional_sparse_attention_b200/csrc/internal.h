@@ -13,10 +13,10 @@ struct oda_ctx {
   int n_sms = 0;
   int g = 1;
   // split-KV attention scratch
-  int max_splits = 0;
   int attn_ctas = 0;          // persistent grid size of the attention kernel
-  float* part_o = nullptr;    // [B*Hq][max_splits][128]
-  float* part_ml = nullptr;   // [B*Hq][max_splits][2]
+  int n_slots = 0;            // partial slots: attn_ctas + B*Hkv
+  float* part_o = nullptr;    // [n_slots][g][128]
+  float* part_ml = nullptr;   // [n_slots][g][2]
   int32_t* attn_cnt = nullptr;  // [B*Hkv] completion counters (self-resetting)
   int32_t* err = nullptr;       // sticky device error word
   // recall-head scratch
@@ -34,6 +34,9 @@ struct oda_ctx {
   cudaStream_t body_stream = nullptr;
   cudaStream_t cond_parent = nullptr;
   bool cond_open = false;
+  // true when the last kernel this context launched was an attention kernel: the next
+  // attention launch may then overlap it (programmatic dependent launch)
+  bool prev_attention = false;
   void* alloc_base = nullptr;
 };
 
@@ -50,9 +53,8 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
 oda_status launch_index_positions(oda_ctx* ctx, int mode, const int32_t* pos, const int32_t* flag,
                                   int32_t* positions, int32_t cap, int32_t* counts,
                                   cudaStream_t stream);
-int attention_smem_bytes();
-int attention_threads();
-int attention_ctas_per_sm();
+int attention_smem_bytes(int g);
+oda_status prepare_attention_kernel(int g, int n_sms, int* ctas);
 
 // head.cu
 oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const float* h_prev,

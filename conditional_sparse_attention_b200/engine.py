@@ -85,17 +85,22 @@ class OdaDecoder:
     state) plus the call sequence of one decode step."""
 
     def __init__(self, wl: Workload, device="cuda", capacity_steps: int = 0,
-                 perturb_head: bool = False, head_params: dict = None, fill_cache: bool = True):
+                 perturb_head: bool = False, head_params: dict = None, fill_cache: bool = True,
+                 overlap_layers: bool = True):
         if not torch.cuda.is_available():
             raise RuntimeError("OdaDecoder needs a CUDA device (the CUDA path has no fallback)")
         self.wl = wl
-        self.device = torch.device(device)
+        dev = torch.device(device)
+        if dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        self.device = dev
         torch.cuda.set_device(self.device)
         B, L, Hkv, D = wl.B, wl.L, wl.Hkv, wl.D
         self.capacity_steps = max(wl.steps, capacity_steps)
         self.max_pages = (max(wl.ctx) + self.capacity_steps + 1 + configs.PAGE - 1) // configs.PAGE
         self.n_pool = B * self.max_pages
-        cfg = oda.make_config(B, wl.Hq, Hkv, self.max_pages, D, wl.sinks, wl.window, wl.theta)
+        cfg = oda.make_config(B, wl.Hq, Hkv, self.max_pages, D, wl.sinks, wl.window, wl.theta,
+                              overlap_layers=overlap_layers)
         self.ctx = oda.oda_create(cfg)
         dev = self.device
         self.stream = torch.cuda.Stream(dev)

@@ -77,6 +77,12 @@ typedef struct {
   int32_t window;       /* w (the notes use 2048), >= 1, includes the current token    */
   int32_t head_in_dim;  /* D: width of each recall-head input; multiple of 512, <= 8192 */
   float theta;          /* routing threshold (the notes use 0)                          */
+  int32_t overlap_layers; /* 1: two consecutive attention calls of this context overlap
+                           * (programmatic dependent launch): the later call prefetches its
+                           * pages while the earlier one finishes.  The caller then must not
+                           * write pos, flag, the page table or the KV pools on the stream
+                           * between two consecutive attention calls.  0: every call starts
+                           * after all prior work on the stream.                          */
 } oda_config;
 
 typedef struct {

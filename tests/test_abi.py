@@ -38,9 +38,10 @@ def test_struct_layouts_match_header(lib, tmp_path):
 #include <stddef.h>
 #include "oda.h"
 int main(void) {
-  printf("%zu %zu %zu %zu %zu %zu %zu\\n", sizeof(oda_config), sizeof(oda_kv_layer),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(oda_config), sizeof(oda_kv_layer),
          sizeof(oda_head_weights), sizeof(oda_state), offsetof(oda_config, theta),
-         offsetof(oda_head_weights, out_b), offsetof(oda_state, conv_width));
+         offsetof(oda_config, overlap_layers), offsetof(oda_head_weights, out_b),
+         offsetof(oda_state, conv_width));
   printf("%d %d\\n", ODA_MAX_BATCH, ODA_MAX_LAYERS);
   return 0;
 }
@@ -53,7 +54,8 @@ int main(void) {
     got = [int(x) for x in out]
     C = _lib
     want = [ctypes.sizeof(C.OdaConfig), ctypes.sizeof(C.OdaKVLayer), ctypes.sizeof(C.OdaHeadWeights),
-            ctypes.sizeof(C.OdaState), C.OdaConfig.theta.offset, C.OdaHeadWeights.out_b.offset,
+            ctypes.sizeof(C.OdaState), C.OdaConfig.theta.offset, C.OdaConfig.overlap_layers.offset,
+            C.OdaHeadWeights.out_b.offset,
             C.OdaState.conv_width.offset, C.MAX_BATCH, C.MAX_LAYERS]
     assert got == want
 
@@ -62,12 +64,12 @@ def test_host_validation_without_gpu(lib):
     assert lib.oda_version() == 1
     assert lib.oda_status_string(1) == b"ODA_ERR_INVALID_ARG"
     out = ctypes.c_void_p()
-    bad = _lib.OdaConfig(1, 16, 5, 128, 16, 10, 4, 2048, 2048, 0.0)
+    bad = _lib.OdaConfig(1, 16, 5, 128, 16, 10, 4, 2048, 2048, 0.0, 0)
     assert lib.oda_create(ctypes.byref(bad), ctypes.byref(out)) == 2
     assert b"Hkv" in lib.oda_last_error() and not out.value
-    bad = _lib.OdaConfig(1, 16, 8, 64, 16, 10, 4, 2048, 2048, 0.0)
+    bad = _lib.OdaConfig(1, 16, 8, 64, 16, 10, 4, 2048, 2048, 0.0, 0)
     assert lib.oda_create(ctypes.byref(bad), ctypes.byref(out)) == 2
-    bad = _lib.OdaConfig(1, 16, 8, 128, 16, 10, 4, 2048, 1000, 0.0)
+    bad = _lib.OdaConfig(1, 16, 8, 128, 16, 10, 4, 2048, 1000, 0.0, 0)
     assert lib.oda_create(ctypes.byref(bad), ctypes.byref(out)) == 2
     assert lib.oda_create(None, ctypes.byref(out)) == 1
     assert lib.oda_attend_local(None, None, None, None, None, None, None, None, None) == 1

@@ -40,8 +40,9 @@ class Setup:
         self.pt_np = inputs.page_table(wl, self.max_pages)
         self.pt = torch.from_numpy(self.pt_np).to(dev)
         n_pool = wl.B * self.max_pages + extra_pool_pages
-        self.k = torch.zeros((n_pool, wl.Hkv, 16, 128), dtype=torch.bfloat16, device=dev)
-        self.v = torch.zeros_like(self.k)
+        # slots outside every sequence's cache hold NaN: they must never reach an output
+        self.k = torch.full((n_pool, wl.Hkv, 16, 128), float("nan"), dtype=torch.bfloat16, device=dev)
+        self.v = torch.full_like(self.k, float("inf"))
         wdev.fill_kv(self.k, self.pt, wl.ctx, [inputs.cache_key(wl, "k", 0, b) for b in range(wl.B)], wl.Hkv)
         wdev.fill_kv(self.v, self.pt, wl.ctx, [inputs.cache_key(wl, "v", 0, b) for b in range(wl.B)], wl.Hkv)
         self.layer = oda.kv_layer(self.k, self.v)

@@ -140,7 +140,15 @@ def cfg4() -> Workload:
                     note="hybrid: 6 attention + 18 gated-delta layers, snapshot/restore, recall 0.4")
 
 
-ALL = {"cfg0": cfg0, "cfg1": cfg1, "cfg2": cfg2, "cfg3": cfg3, "cfg4": cfg4}
+def cfg2_ctx32k_l2() -> Workload:
+    """Profiling case of the 128K workload's kernels: same heads and batch, 2 layers, context
+    32768 (1 GiB of cache: larger than L2, small enough for a many-pass profiler capture)."""
+    return cfg2().replace(name="cfg2_profile_ctx32k_l2", n_layers=2, attn_layers=(0, 1),
+                          ctx=(32768,) * 4, steps=8)
+
+
+ALL = {"cfg0": cfg0, "cfg1": cfg1, "cfg2": cfg2, "cfg3": cfg3, "cfg4": cfg4,
+       "cfg2_ctx32k_l2": cfg2_ctx32k_l2}
 
 
 def get(name: str) -> Workload:
