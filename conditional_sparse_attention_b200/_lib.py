@@ -55,6 +55,9 @@ _SIGS = {
                           c_void_p, c_void_p, c_void_p], c_int32),
     "oda_attend_full_if": ([c_void_p, _P(OdaKVLayer), c_void_p, c_void_p, c_void_p, c_void_p,
                             c_void_p, c_void_p, c_void_p, c_void_p], c_int32),
+    "oda_attend_full_if_noalloc": ([_P(OdaConfig), _P(OdaKVLayer), c_void_p, c_void_p, c_void_p,
+                                    c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p],
+                                   c_int32),
     "oda_index_positions": ([c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_int32, c_void_p,
                              c_void_p], c_int32),
     "oda_recall_score": ([c_void_p, _P(OdaHeadWeights), c_void_p, c_void_p, c_void_p, c_void_p,

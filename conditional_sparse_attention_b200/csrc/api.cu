@@ -183,6 +183,15 @@ oda_status oda_attend_full_if(oda_ctx* ctx, const oda_kv_layer* layer, const int
   return oda::launch_attention(ctx, layer, page_table, pos, flag, q, k_new, v_new, out, 1, stream);
 }
 
+oda_status oda_attend_full_if_noalloc(const oda_config* cfg, const oda_kv_layer* layer,
+                                      const int32_t* page_table, const int32_t* pos,
+                                      const int32_t* flag, const void* q, const void* k_new,
+                                      const void* v_new, float* out, int32_t* device_error,
+                                      cudaStream_t stream) {
+  return oda::launch_attention_noalloc(cfg, layer, page_table, pos, flag, q, k_new, v_new, out,
+                                       device_error, stream);
+}
+
 oda_status oda_index_positions(oda_ctx* ctx, int32_t mode, const int32_t* pos, const int32_t* flag,
                                int32_t* positions, int32_t cap, int32_t* counts,
                                cudaStream_t stream) {

@@ -26,6 +26,7 @@
 // a launch prefetches its first pages before waiting for the previous one.
 #include <cmath>
 #include <cstdio>
+#include <mutex>
 
 #include <cooperative_groups.h>
 
@@ -956,6 +957,142 @@ oda_status launch_index_positions(oda_ctx* ctx, int mode, const int32_t* pos, co
   index_positions_kernel<<<(cf.batch + 31) / 32, 32, 0, stream>>>(
       pos, flag, cf.batch, mode, cf.sinks, cf.window, cf.max_pages, positions, cap, counts);
   return check_cuda(cudaGetLastError(), "index_positions launch");
+}
+
+
+// ------------------------------------------------------------- allocation-free variant
+// Callers that must not allocate device memory (a plugin that may only use the buffers its
+// host framework hands it, code that runs where a cudaMalloc/cudaFree would synchronise the
+// device in a latency-critical loop, or a process whose memory is reserved up front) get
+// the full-set attention with its scratch in this file-scope device array instead of a
+// context.  Every GPU that loads the library holds the array until the process exits.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;   // 4 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+struct NoAllocDevice {
+  unsigned char* scratch = nullptr;   // device address of g_noalloc_scratch on this device
+  int ctas = 0;                       // persistent grid size of the full-set kernel
+  bool ready = false;
+};
+constexpr int kNoAllocMaxDevices = 64;
+NoAllocDevice g_noalloc[kNoAllocMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Once per device, with that device current: the array's device address (host code only
+// sees a stand-in symbol) and the grid size.
+oda_status noalloc_setup(int g, NoAllocDevice** out) {
+  int dev = 0;
+  oda_status st = check_cuda(cudaGetDevice(&dev), "cudaGetDevice");
+  if (st != ODA_OK) return st;
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return set_error(ODA_ERR_UNSUPPORTED, "noalloc: device %d beyond the supported %d", dev,
+                     kNoAllocMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoAllocDevice& d = g_noalloc[dev];
+  if (!d.ready) {
+    void* ptr = nullptr;
+    st = check_cuda(cudaGetSymbolAddress(&ptr, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
+    if (st != ODA_OK) return st;
+    int n_sms = 0;
+    st = check_cuda(cudaDeviceGetAttribute(&n_sms, cudaDevAttrMultiProcessorCount, dev),
+                    "cudaDeviceGetAttribute");
+    if (st != ODA_OK) return st;
+    d.scratch = static_cast<unsigned char*>(ptr);
+    d.ctas = n_sms;   // one CTA per SM: fits the shared memory of every g
+    d.ready = true;
+  }
+  (void)g;
+  *out = &d;
+  return ODA_OK;
+}
+
+}  // namespace
+
+size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* layer,
+                                    const int32_t* page_table, const int32_t* pos,
+                                    const int32_t* flag, const void* q, const void* k_new,
+                                    const void* v_new, float* out, int32_t* device_error,
+                                    cudaStream_t stream) {
+  if (!cfg) return set_error(ODA_ERR_INVALID_ARG, "noalloc: cfg is NULL");
+  const oda_config& cf = *cfg;
+  if (cf.batch < 1 || cf.batch > ODA_MAX_BATCH || cf.n_q_heads < 1 || cf.n_kv_heads < 1 ||
+      cf.n_q_heads % cf.n_kv_heads != 0 || cf.n_q_heads / cf.n_kv_heads > 8 || cf.head_dim != 128 ||
+      cf.page_size != 16 || cf.max_pages < 1 || (int64_t)cf.max_pages * 16 > INT32_MAX - 1)
+    return set_error(ODA_ERR_UNSUPPORTED, "noalloc: configuration outside what the kernel supports");
+  if (!layer || !layer->k || !layer->v || !page_table || !pos || !flag || !q || !k_new || !v_new ||
+      !out)
+    return set_error(ODA_ERR_INVALID_ARG, "noalloc: null pointer argument");
+  if (layer->n_pages <= 0 || layer->n_pages * (int64_t)cf.n_kv_heads * kPageTok > INT32_MAX)
+    return set_error(ODA_ERR_INVALID_ARG, "noalloc: n_pages out of range");
+  if ((reinterpret_cast<uintptr_t>(layer->k) | reinterpret_cast<uintptr_t>(layer->v)) & 15)
+    return set_error(ODA_ERR_INVALID_ARG, "noalloc: K/V pools must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k_new) |
+       reinterpret_cast<uintptr_t>(v_new) | reinterpret_cast<uintptr_t>(out)) & 3)
+    return set_error(ODA_ERR_INVALID_ARG, "noalloc: q/k_new/v_new/out must be 4-byte aligned");
+  const int g = cf.n_q_heads / cf.n_kv_heads;
+  NoAllocDevice* d = nullptr;
+  oda_status st = noalloc_setup(g, &d);
+  if (st != ODA_OK) return st;
+  // the shared-memory limit is a per-function setting that a context created later may have
+  // lowered: raise it to this call's need (host-side, no allocation)
+  st = check_cuda(cudaFuncSetAttribute(attn_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       attention_smem_bytes(8)),
+                  "cudaFuncSetAttribute(full attention)");
+  if (st != ODA_OK) return st;
+  // scratch layout: counters [B*Hkv] | error word | partial (m, l) | partial O
+  const size_t pairs = (size_t)cf.batch * cf.n_kv_heads;
+  const size_t slots = (size_t)d->ctas + pairs;
+  const size_t cnt_bytes = ((pairs + 1) * sizeof(int32_t) + 255) / 256 * 256;
+  const size_t ml_bytes = (slots * g * 2 * sizeof(float) + 255) / 256 * 256;
+  const size_t o_bytes = slots * g * 128 * sizeof(float);
+  if (cnt_bytes + ml_bytes + o_bytes > kNoAllocScratchBytes)
+    return set_error(ODA_ERR_UNSUPPORTED,
+                     "noalloc: needs %zu bytes of scratch for B=%d, Hkv=%d, g=%d; the static "
+                     "scratch holds %zu",
+                     cnt_bytes + ml_bytes + o_bytes, cf.batch, cf.n_kv_heads, g,
+                     kNoAllocScratchBytes);
+  int32_t* counters = reinterpret_cast<int32_t*>(d->scratch);
+  int32_t* err_word = counters + pairs;
+  float* part_ml = reinterpret_cast<float*>(d->scratch + cnt_bytes);
+  float* part_o = reinterpret_cast<float*>(d->scratch + cnt_bytes + ml_bytes);
+  // the completion counters (and the scratch error word) must start at zero on every call
+  st = check_cuda(cudaMemsetAsync(counters, 0, (pairs + 1) * sizeof(int32_t), stream),
+                  "cudaMemsetAsync(noalloc counters)");
+  if (st != ODA_OK) return st;
+  CUtensorMap tmK, tmV;
+  st = encode_pool(&tmK, layer->k, layer->n_pages, cf.n_kv_heads);
+  if (st != ODA_OK) return st;
+  st = encode_pool(&tmV, layer->v, layer->n_pages, cf.n_kv_heads);
+  if (st != ODA_OK) return st;
+  AttnParams p;
+  p.page_table = page_table;
+  p.pos = pos;
+  p.flag = flag;
+  p.q = static_cast<const uint32_t*>(q);
+  p.k_new = static_cast<const uint32_t*>(k_new);
+  p.v_new = static_cast<const uint32_t*>(v_new);
+  p.out = out;
+  p.part_o = part_o;
+  p.part_ml = part_ml;
+  p.counters = counters;
+  p.err = device_error ? device_error : err_word;
+  p.n_pool_pages = layer->n_pages;
+  p.B = cf.batch;
+  p.Hq = cf.n_q_heads;
+  p.Hkv = cf.n_kv_heads;
+  p.g = g;
+  p.max_pages = cf.max_pages;
+  p.sinks = cf.sinks;
+  p.window = cf.window;
+  p.mode = 1;
+  p.cluster = 1;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(128.0));
+  attn_full_kernel<<<d->ctas, kThreads, attention_smem_bytes(g), stream>>>(tmK, tmV, p);
+  return check_cuda(cudaGetLastError(), "noalloc full attention launch");
 }
 
 }  // namespace oda

@@ -55,6 +55,11 @@ oda_status launch_index_positions(oda_ctx* ctx, int mode, const int32_t* pos, co
                                   cudaStream_t stream);
 int attention_smem_bytes(int g);
 oda_status prepare_attention_kernel(int g, int n_sms, int* ctas);
+oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* layer,
+                                    const int32_t* page_table, const int32_t* pos,
+                                    const int32_t* flag, const void* q, const void* k_new,
+                                    const void* v_new, float* out, int32_t* device_error,
+                                    cudaStream_t stream);
 
 // head.cu
 oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const float* h_prev,

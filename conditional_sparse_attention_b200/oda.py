@@ -112,6 +112,15 @@ def oda_attend_full_if(ctx, layer: OdaKVLayer, page_table, pos, flag, q, k_new, 
                                          _p(flag), _p(q), _p(k_new), _p(v_new), _p(out), _s(stream)))
 
 
+def oda_attend_full_if_noalloc(cfg: OdaConfig, layer: OdaKVLayer, page_table, pos, flag, q, k_new,
+                               v_new, out, device_error=None, stream=None):
+    """Full-set attention without a context: scratch in the library's static device array."""
+    check(_lib.load().oda_attend_full_if_noalloc(ctypes.byref(cfg), ctypes.byref(layer),
+                                                 _p(page_table), _p(pos), _p(flag), _p(q),
+                                                 _p(k_new), _p(v_new), _p(out), _p(device_error),
+                                                 _s(stream)))
+
+
 def oda_index_positions(ctx, mode: int, pos, flag, positions, cap: int, counts, stream=None):
     check(_lib.load().oda_index_positions(ctx.handle, mode, _p(pos), _p(flag), _p(positions), cap,
                                           _p(counts), _s(stream)))

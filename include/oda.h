@@ -145,6 +145,29 @@ oda_status oda_attend_full_if(oda_ctx* ctx, const oda_kv_layer* layer, const int
                               const void* k_new, const void* v_new, float* out,
                               cudaStream_t stream);
 
+/* Allocation-free variant of oda_attend_full_if (the method notes have no counterpart: this
+ * is a deployment convenience).  Same computation, arguments and layouts, without a context:
+ * its scratch (split partials and completion counters) lives in a static device array of
+ * 4 MiB that every GPU loading the library holds until exit, so the call allocates nothing.
+ * It is meant for callers that cannot allocate device memory: code running inside a host
+ * framework that only lends it buffers, or a latency-critical loop where cudaMalloc's
+ * implicit device synchronisation is not acceptable.
+ *   - cfg: the shape (same rules as oda_create; overlap_layers and head_in_dim are ignored).
+ *   - device_error: optional device int32 that receives sticky ODA_DEVERR_* bits (OR-ed in,
+ *     never cleared by the call); NULL keeps them in the static scratch, unread.
+ *   - Returns ODA_ERR_UNSUPPORTED, launching nothing, when the shape needs more scratch than
+ *     the array holds (about (SMs + B*Hkv) * g * 520 bytes plus 4 * B*Hkv).
+ *   - The first call on a device looks up the array's device address and sets the kernel's
+ *     shared-memory limit (with that device current); make that first call before any stream
+ *     capture.  Each call clears the counters it needs with cudaMemsetAsync on `stream`.
+ *   - All calls share the one array: calls that may overlap on the GPU (other streams, other
+ *     host threads) race and must be serialised by the caller. */
+oda_status oda_attend_full_if_noalloc(const oda_config* cfg, const oda_kv_layer* layer,
+                                      const int32_t* page_table, const int32_t* pos,
+                                      const int32_t* flag, const void* q, const void* k_new,
+                                      const void* v_new, float* out, int32_t* device_error,
+                                      cudaStream_t stream);
+
 /* The index sets as the attention kernels visit them (same work decomposition): for each
  * sequence b (mode 0: all, S^L; mode 1: flag[b] != 0, S^F), positions[b*cap + i] receives the
  * 1-based cache positions read, in page order, followed by t (the staged token);
