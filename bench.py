@@ -28,8 +28,27 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "ODA decode-attn steps/s + % of HBM peak, 128K ctx, 12.5% recall, 1 B200"
+
+# DRAM bytes (read + write) of one full-set attention launch from the ncu capture summarised in
+# profiles/attn_full_kernel_cfg2_ctx32k_l2.md (4 flagged sequences x 32768 cached tokens); the
+# bench scales it to its own launches by cached tokens processed.  Valid only for the kernel
+# source it was taken from (first 16 hex digits of the file's SHA-256).
+NCU_FULL_KERNEL_TRAFFIC = {"attention_cu_sha256": "0f1765d626426219", "bytes": 541386496,
+                           "cached_tokens": 4 * 32768}
 UNIT = "steps/s"
 FALLBACK_HBM_GBS = 6650.0
+
+
+def traffic_per_token():
+    """ncu DRAM bytes per cached token of one full-set launch, or None if the kernel changed."""
+    import hashlib
+    path = os.path.join(ROOT, "conditional_sparse_attention_b200", "csrc", "attention.cu")
+    try:
+        sha = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    t = NCU_FULL_KERNEL_TRAFFIC
+    return t["bytes"] / t["cached_tokens"] if sha == t["attention_cu_sha256"] else None
 
 
 def peaks():
@@ -249,6 +268,28 @@ def time_layer_kernels(dec, mode: int, flag, reps: int = 3) -> float:
     return e0.elapsed_time(e1) / (reps * wl.L)
 
 
+def time_head(dec, reps: int = 5) -> float:
+    """Average device milliseconds of one recall-head score (its six launches as a graph)."""
+    import torch
+    from conditional_sparse_attention_b200 import oda
+    s = dec.stream
+    torch.cuda.synchronize(dec.device)
+    oda.oda_graph_begin(s)
+    oda.oda_recall_score(dec.ctx, dec.head_w, dec.h_prev, dec.sv["emb"], dec.h[0],
+                         dec.sv["sched"] if dec.routing_scheduled else None, dec.score, dec.flag,
+                         dec.any_flag, s)
+    g = oda.oda_graph_end(s)
+    g.launch(s)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(reps):
+        g.launch(s)
+    e1.record(s)
+    e1.synchronize()
+    g.close()
+    return e0.elapsed_time(e1) / reps
+
+
 def run_kernel_only(args, wl, local_rank):
     """Profiling mode: set up the workload, stage step 0, launch one attention kernel
     ``--kernel-reps`` times (full: every sequence flagged) and exit."""
@@ -279,6 +320,7 @@ def run_ours(args, wl, rank, world, local_rank):
     import torch
     from conditional_sparse_attention_b200 import oda
     from conditional_sparse_attention_b200.engine import OdaDecoder
+    from workload import inputs as inputs_mod
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -296,7 +338,8 @@ def run_ours(args, wl, rank, world, local_rank):
     # first step including graph capture (the pages' "first request" includes capture)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     tf = time.perf_counter()
-    dec.capture()
+    if not args.eager:
+        dec.capture()
     dec.stage(store[0])
     dec.launch()
     dec.synchronize()
@@ -359,7 +402,12 @@ def run_ours(args, wl, rank, world, local_rank):
         full_bytes += count * sum(int(pos_now[b]) * per_tok for b in range(wl.B) if pat[b])
         n_full += 2 * wl.L
     full_gbs = full_bytes / (full_ms * 1e-3) / 1e9
+    tpt = traffic_per_token()
+    n_pat_launches = sum(pats.values())
+    full_traffic = (tpt * (full_bytes / per_tok) / n_pat_launches) if tpt else None
     loc_ms = time_layer_kernels(dec, 0, None, reps=3)
+    head_ms = time_head(dec, reps=5)
+    head_bytes = inputs_mod.head_param_count(wl.D) * 4
     loc_bytes = sum(min(int(pos_now[b]), wl.sinks + wl.window) * per_tok for b in range(wl.B))
     loc_gbs = loc_bytes / (loc_ms * 1e-3) / 1e9
 
@@ -408,10 +456,12 @@ def run_ours(args, wl, rank, world, local_rank):
             "config": {"workload": wl.name, "B": wl.B, "layers": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv,
                        "head_dim": 128, "ctx": wl.ctx[0], "recall_rate": wl.rates[0],
                        "page_tokens": 16, "parallelism": f"replicas{world}",
-                       "l2": "inputs larger than L2 (77 GB resident KV cache), no flush"},
+                       "l2": "inputs larger than L2 (77 GB resident KV cache), no flush",
+                       "launch": "eager" if args.eager else "cuda-graph with conditional IF node"},
             "roofline": {"bound": "hbm", "achieved": full_gbs, "peak": hbm, "unit": "GB/s",
-                         "frac": full_gbs / hbm, "traffic": None,
-                         "kernel": "attn_kernel (full set, flagged sequences)",
+                         "frac": full_gbs / hbm, "traffic": full_traffic,
+                         "algorithmic_bytes_per_launch": full_bytes / n_pat_launches,
+                         "kernel": "attn_full_kernel (full set, flagged sequences)",
                          "peak_source": peak_src, "launches_timed": n_full,
                          "us_per_launch": full_ms * 1000.0 / sum(pats.values()),
                          "flag_patterns": {"".join(map(str, k)): v for k, v in pats.items()}},
@@ -419,6 +469,9 @@ def run_ours(args, wl, rank, world, local_rank):
                               "achieved_gbs": step_gbs, "frac": step_gbs / hbm},
             "local_kernel": {"achieved_gbs": loc_gbs, "frac": loc_gbs / hbm,
                              "us_per_launch": loc_ms * 1000.0},
+            "recall_head": {"us_per_score": head_ms * 1000.0,
+                            "achieved_gbs": head_bytes / (head_ms * 1e-3) / 1e9,
+                            "frac": head_bytes / (head_ms * 1e-3) / 1e9 / hbm},
             "realized_recall_rate": realized_rate,
             "first_step_ms_incl_capture": first_ms, "setup_s": setup_s,
             "gpu_launches": launches, "device_error": err,
@@ -437,6 +490,9 @@ def main():
     ap.add_argument("--workload", default="cfg2")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="issue every step's kernels directly instead of replaying a CUDA graph "
+                         "(profilers cannot see kernel nodes of graphs with conditional nodes)")
     ap.add_argument("--kernel-only", choices=["full", "local"], default=None,
                     help="profiling mode: launch one attention kernel --kernel-reps times and exit")
     ap.add_argument("--kernel-reps", type=int, default=3)

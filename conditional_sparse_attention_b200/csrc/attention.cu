@@ -365,7 +365,9 @@ __device__ __forceinline__ int cta_of(long long u, long long U, long long G) {
 
 // ---------------------------------------------------------------- local set: clusters
 // Cluster of p.cluster CTAs per (b, h); CTA `rank` takes the contiguous share
-// [rank*nv/C, (rank+1)*nv/C) of the visited pages; warps take every kW-th page of it.
+// [rank*nv/C, (rank+1)*nv/C) of the visited pages; warps take every kW-th page of it.  After a
+// cluster barrier each rank finishes its share of the g*128 outputs from all ranks' partials
+// (read through distributed shared memory).
 __global__ void __launch_bounds__(kThreads, 2)
 attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const AttnParams p) {
@@ -435,6 +437,12 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
 
   uint32_t qf[8][2];
   load_qf(qf, p, b, h, lane);
+  // staged current token: its score per head and its value, fetched while pages arrive
+  __shared__ float s_snew[8];
+  for (int n = warp; n < g; n += kW) {
+    const float sn = staged_score(p, b, h, n, lane);
+    if (lane == 0) s_snew[n] = sn;
+  }
   WarpAcc A;
   acc_init(A);
   const int r = lane >> 2;
@@ -468,12 +476,14 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     }
   }
   cluster.sync();
-  if (rank == 0 && ge.active) {
-    // merge the cluster's partials (distributed shared memory) and the staged token
-    const int d = tid;  // kThreads == 128 == head_dim
-    const float vd = staged_value(p, b, h, d);
-    for (int n = 0; n < g; ++n) {
-      const float snew = staged_score(p, b, h, n, lane);
+  if (ge.active) {
+    // merge the cluster's partials through distributed shared memory plus the staged token;
+    // the g*128 outputs are shared out among the ranks, one output per thread
+    const int n_out = g * 128;
+    const int o_lo = (int)((long long)rank * n_out / C), o_hi = (int)((long long)(rank + 1) * n_out / C);
+    for (int idx = o_lo + tid; idx < o_hi; idx += kThreads) {
+      const int n = idx >> 7, d = idx & 127;
+      const float snew = s_snew[n];
       float Mr[kMaxCluster], Lr[kMaxCluster], Or[kMaxCluster];
       float M = snew;
 #pragma unroll
@@ -488,7 +498,7 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         }
       }
       const float wn = exp2f(snew - M);
-      float L = wn, O = wn * vd;
+      float L = wn, O = wn * staged_value(p, b, h, d);
 #pragma unroll
       for (int q = 0; q < kMaxCluster; ++q) {
         if (q < C && Mr[q] != -INFINITY) {
@@ -500,7 +510,7 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       p.out[((size_t)b * p.Hq + h * g + n) * 128 + d] = O / L;
     }
   }
-  // keep every CTA's shared memory alive until rank 0 has read it
+  // keep every CTA's shared memory alive until the other ranks have read it
   cluster.sync();
   if (dead) {
     for (int kk = k; kk < cw && kk < k + kR; ++kk)
@@ -910,7 +920,7 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
   p.window = cf.window;
   p.mode = mode;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(128.0));
-  // cluster size of the local kernel: enough CTAs per (b, h) to cover the GPU, at most 8
+  // cluster size of the local kernel: enough CTAs per (b, h) to fill the GPU (at most 8)
   const int pairs = cf.batch * cf.n_kv_heads;
   p.cluster = std::max(1, std::min(kMaxCluster, (ctx->attn_ctas + pairs / 2) / pairs));
 

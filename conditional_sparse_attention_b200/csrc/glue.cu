@@ -36,8 +36,19 @@ hidden_kernel(const float* emb, const float* terms, int n_terms, const int32_t* 
   const int d = chunk * kGlueChunk + threadIdx.x;
   float x = 0.f;
   if (d < D) {
-    x = emb[(size_t)b * D + d];
-    for (int i = 0; i < n_terms; ++i) x += terms[((size_t)i * B + b) * D + d];
+    // independent partial sums so the loads of all terms are in flight together
+    const float* tp = terms + (size_t)b * D + d;
+    const size_t stride = (size_t)B * D;
+    float a0 = emb[(size_t)b * D + d], a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int i = 0;
+    for (; i + 4 <= n_terms; i += 4) {
+      a0 += tp[(size_t)i * stride];
+      a1 += tp[(size_t)(i + 1) * stride];
+      a2 += tp[(size_t)(i + 2) * stride];
+      a3 += tp[(size_t)(i + 3) * stride];
+    }
+    for (; i < n_terms; ++i) a0 += tp[(size_t)i * stride];
+    x = (a0 + a1) + (a2 + a3);
     xbuf[(size_t)b * D + d] = x;
   }
   const float ss = block_sum256(x * x, red);

@@ -18,7 +18,9 @@
 // scale, the interaction vector, the gated activation) is applied while the tile is built, and
 // the output epilogue (bias, SiLU, residual) runs in the last CTA of each row block, which sums
 // the split-K partials in a fixed order (deterministic results).  The last row block of the
-// final phase also computes q and the gate.  Six launches per score.
+// final phase also computes q and the gate.  Six launches per score; each may start while the
+// previous one finishes (programmatic dependent launch) and pulls its weight slab toward L2
+// before waiting for the previous phase's outputs.
 #include <cmath>
 
 #include "internal.h"
@@ -66,18 +68,25 @@ __device__ __forceinline__ float4 ldg_w(const float* p, bool stream) {
                 : __ldg(reinterpret_cast<const float4*>(p));
 }
 
-// Sum of squares of row x[b][0..n) (whole block cooperates; result in every thread).
-__device__ float block_sum(float v, float* red) {
+// Block-wide sums of 8 per-thread values; on return red[0..7] hold the totals (all threads
+// may read them).  red must hold kWarps * 8 floats.
+__device__ void block_sum8(float (&v)[kBT], float* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  float s = 0.f;
+  for (int bb = 0; bb < kBT; ++bb)
 #pragma unroll
-  for (int i = 0; i < kWarps; ++i) s += red[i];
-  return s;
+    for (int o = 16; o > 0; o >>= 1) v[bb] += __shfl_xor_sync(0xffffffffu, v[bb], o);
+  __syncthreads();
+  if (lane == 0)
+#pragma unroll
+    for (int bb = 0; bb < kBT; ++bb) red[kBT + warp * kBT + bb] = v[bb];
+  __syncthreads();
+  if (threadIdx.x < kBT) {
+    float t = 0.f;
+    for (int w = 0; w < kWarps; ++w) t += red[kBT + w * kBT + threadIdx.x];
+    red[threadIdx.x] = t;
+  }
+  __syncthreads();
 }
 
 // The weight row that value slot r (0..3) of warp `warp` in row block `rb` multiplies, and
@@ -108,77 +117,111 @@ __device__ __forceinline__ const float* weight_row(const HeadParams& p, int rb, 
   return w.ffn_down[p.block] + (size_t)n * kF;
 }
 
+// Four consecutive input values X[b][kg..kg+3] of a phase (kg a multiple of 4), before any
+// per-sequence scaling: the tower input, the interaction vector z, f, or the gated activation.
+__device__ __forceinline__ float4 tile_value4(const HeadParams& p, int rb, int b, int kg) {
+  if (p.phase == kTower) {
+    const int i = (rb * kRowsPerCta) / kT;
+    return *reinterpret_cast<const float4*>(p.x[i] + (size_t)b * p.D + kg);
+  }
+  if (p.phase == kFuse) {
+    const int blk = kg / kT, e = kg % kT;
+    const float4 u0 = *reinterpret_cast<const float4*>(p.u + ((size_t)0 * p.B + b) * kT + e);
+    const float4 u1 = *reinterpret_cast<const float4*>(p.u + ((size_t)1 * p.B + b) * kT + e);
+    const float4 u2 = *reinterpret_cast<const float4*>(p.u + ((size_t)2 * p.B + b) * kT + e);
+    switch (blk) {
+      case 0: return u0;
+      case 1: return u1;
+      case 2: return u2;
+      case 3: return make_float4(u0.x * u1.x, u0.y * u1.y, u0.z * u1.z, u0.w * u1.w);
+      case 4: return make_float4(u0.x * u2.x, u0.y * u2.y, u0.z * u2.z, u0.w * u2.w);
+      case 5: return make_float4(u1.x * u2.x, u1.y * u2.y, u1.z * u2.z, u1.w * u2.w);
+      case 6: return make_float4(fabsf(u0.x - u1.x), fabsf(u0.y - u1.y), fabsf(u0.z - u1.z), fabsf(u0.w - u1.w));
+      case 7: return make_float4(fabsf(u0.x - u2.x), fabsf(u0.y - u2.y), fabsf(u0.z - u2.z), fabsf(u0.w - u2.w));
+      default: return make_float4(fabsf(u1.x - u2.x), fabsf(u1.y - u2.y), fabsf(u1.z - u2.z), fabsf(u1.w - u2.w));
+    }
+  }
+  if (p.phase == kUp)   // scaled by the RMSNorm below
+    return *reinterpret_cast<const float4*>(p.f + ((size_t)p.block * p.B + b) * kT + kg);
+  return *reinterpret_cast<const float4*>(p.act + (size_t)b * kF + kg);
+}
+
 // Builds the input tile X[bb][0..Kc) for sequences b0..b0+7 of chunk `chunk` (zeros beyond B).
+// 16-byte loads, four per thread in flight before any is stored.
 __device__ void build_tile(const HeadParams& p, int rb, int chunk, int b0, float* X, float* ss_out,
                            float* red) {
   const int k0 = chunk * p.Kc;
-  for (int idx = threadIdx.x; idx < kBT * p.Kc; idx += kHT) {
-    const int bb = idx / p.Kc, k = idx % p.Kc, b = b0 + bb;
-    float v = 0.f;
-    if (b < p.B) {
-      const int kg = k0 + k;
-      if (p.phase == kTower) {
-        const int i = (rb * kRowsPerCta) / kT;
-        v = p.x[i][(size_t)b * p.D + kg];
-      } else if (p.phase == kFuse) {
-        const int blk = kg / kT, e = kg % kT;
-        const float u0 = p.u[((size_t)0 * p.B + b) * kT + e];
-        const float u1 = p.u[((size_t)1 * p.B + b) * kT + e];
-        const float u2 = p.u[((size_t)2 * p.B + b) * kT + e];
-        switch (blk) {
-          case 0: v = u0; break;
-          case 1: v = u1; break;
-          case 2: v = u2; break;
-          case 3: v = u0 * u1; break;
-          case 4: v = u0 * u2; break;
-          case 5: v = u1 * u2; break;
-          case 6: v = fabsf(u0 - u1); break;
-          case 7: v = fabsf(u0 - u2); break;
-          default: v = fabsf(u1 - u2); break;
-        }
-      } else if (p.phase == kUp) {
-        v = p.f[((size_t)p.block * p.B + b) * kT + kg];   // scaled below
-      } else {
-        v = p.act[(size_t)b * kF + kg];
+  const int kc4 = p.Kc / 4, n4 = kBT * kc4;
+  float4* X4 = reinterpret_cast<float4*>(X);
+  for (int base = threadIdx.x; base < n4; base += 4 * kHT) {
+    float4 v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int idx = base + j * kHT;
+      v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (idx < n4) {
+        const int bb = idx / kc4, k4 = idx - bb * kc4;
+        if (b0 + bb < p.B) v[j] = tile_value4(p, rb, b0 + bb, k0 + 4 * k4);
       }
     }
-    X[idx] = v;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (base + j * kHT < n4) X4[base + j * kHT] = v[j];
   }
   __syncthreads();
   if (p.phase == kTower) {
-    // sum of squares of this chunk of x_i per sequence (for the RMSNorm scale), then gamma
+    // sums of squares of this chunk of x_i for the 8 sequences of the tile, one pass
     const int i = (rb * kRowsPerCta) / kT;
+    float ssq[kBT];
+#pragma unroll
     for (int bb = 0; bb < kBT; ++bb) {
-      float s = 0.f;
-      for (int k = threadIdx.x; k < p.Kc; k += kHT) s += X[bb * p.Kc + k] * X[bb * p.Kc + k];
-      s = block_sum(s, red);
-      if (threadIdx.x == 0 && b0 + bb < p.B)
-        ss_out[((size_t)rb * p.nchunks + chunk) * p.B + b0 + bb] = s;
+      ssq[bb] = 0.f;
+      for (int k = threadIdx.x; k < p.Kc; k += kHT) ssq[bb] += X[bb * p.Kc + k] * X[bb * p.Kc + k];
     }
+    block_sum8(ssq, red);
+    if (threadIdx.x < kBT && b0 + threadIdx.x < p.B)
+      ss_out[((size_t)rb * p.nchunks + chunk) * p.B + b0 + threadIdx.x] = red[threadIdx.x];
     const float* gam = p.w.tower_norm[i] + k0;
     for (int idx = threadIdx.x; idx < kBT * p.Kc; idx += kHT) X[idx] *= gam[idx % p.Kc];
     __syncthreads();
   } else if (p.phase == kUp) {
-    // m = RMSNorm(f) * gamma over the full 1024-wide f
+    // m = RMSNorm(f) * gamma over the full 1024-wide f, one pass for the 8 sequences
     const float* gam = p.w.ffn_norm[p.block] + k0;
+    float ssq[kBT];
+#pragma unroll
     for (int bb = 0; bb < kBT; ++bb) {
-      const int b = b0 + bb;
-      float s = 0.f;
-      if (b < p.B) {
-        const float* fr = p.f + ((size_t)p.block * p.B + b) * kT;
-        for (int k = threadIdx.x; k < kT; k += kHT) s += fr[k] * fr[k];
+      ssq[bb] = 0.f;
+      if (b0 + bb < p.B) {
+        const float* fr = p.f + ((size_t)p.block * p.B + b0 + bb) * kT;
+        for (int k = threadIdx.x; k < kT; k += kHT) ssq[bb] += fr[k] * fr[k];
       }
-      s = block_sum(s, red);
-      const float inv = rsqrtf(s / kT + kEps);
-      for (int k = threadIdx.x; k < p.Kc; k += kHT) X[bb * p.Kc + k] *= inv * gam[k];
+    }
+    block_sum8(ssq, red);
+    for (int idx = threadIdx.x; idx < kBT * p.Kc; idx += kHT) {
+      const int bb = idx / p.Kc, k = idx % p.Kc;
+      X[idx] *= rsqrtf(red[bb] / kT + kEps) * gam[k];
     }
     __syncthreads();
   }
 }
 
+// Split-K partials of output column `col` for sequence b, summed in chunk order; all loads are
+// issued before the first add (at most kMaxChunks chunks).
+constexpr int kMaxChunks = 16;
+__device__ __forceinline__ float sum_chunks(const HeadParams& p, int b, int col) {
+  float v[kMaxChunks];
+#pragma unroll
+  for (int ch = 0; ch < kMaxChunks; ++ch)
+    v[ch] = ch < p.nchunks ? __ldcg(p.part + ((size_t)ch * p.B + b) * p.rows_total + col) : 0.f;
+  float acc = 0.f;
+#pragma unroll
+  for (int ch = 0; ch < kMaxChunks; ++ch) acc += v[ch];
+  return acc;
+}
+
 __global__ void __launch_bounds__(kHT) head_phase_kernel(const HeadParams p) {
   extern __shared__ float X[];           // [kBT][Kc]
-  __shared__ float red[kWarps];
+  __shared__ float red[kBT + kWarps * kBT];
   __shared__ int s_last;
   const int rb = blockIdx.x / p.nchunks, chunk = blockIdx.x % p.nchunks;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -188,6 +231,13 @@ __global__ void __launch_bounds__(kHT) head_phase_kernel(const HeadParams p) {
   const float* wrow[kRowsPerWarp];
 #pragma unroll
   for (int r = 0; r < kRowsPerWarp; ++r) wrow[r] = weight_row(p, rb, warp, r, &cols[r]) + k0;
+  // The weights never change: pull this CTA's slab toward L2 while the previous phase may
+  // still be running (programmatic dependent launch), then wait for its outputs.
+  for (int r = 0; r < kRowsPerWarp; ++r)
+    for (int k = lane * 32; k < p.Kc; k += 32 * 32)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(wrow[r] + k));
+  grid_dependency_wait();
+  grid_dependents_launch();
 
   const bool single_pass = p.B <= kBT;
   for (int b0 = 0; b0 < p.B; b0 += kBT) {
@@ -250,35 +300,25 @@ __global__ void __launch_bounds__(kHT) head_phase_kernel(const HeadParams p) {
     const int j = idx % units, b = idx / units;
     if (p.phase == kTower) {
       const int row = rb * kRowsPerCta + j, i = row / kT, n = row % kT;
-      float acc = 0.f, ss = 0.f;
-      for (int ch = 0; ch < p.nchunks; ++ch) {
-        acc += __ldcg(p.part + ((size_t)ch * p.B + b) * p.rows_total + row);
-        ss += __ldcg(p.ss + ((size_t)rb * p.nchunks + ch) * p.B + b);
-      }
+      const float acc = sum_chunks(p, b, row);
+      float ss = 0.f;
+      for (int ch = 0; ch < p.nchunks; ++ch) ss += __ldcg(p.ss + ((size_t)rb * p.nchunks + ch) * p.B + b);
       const float inv = rsqrtf(ss / p.D + kEps);
       p.u[((size_t)i * p.B + b) * kT + n] = silu(acc * inv + p.w.tower_b[i][n]);
     } else if (p.phase == kFuse) {
       const int n = rb * kRowsPerCta + j;
-      float acc = 0.f;
-      for (int ch = 0; ch < p.nchunks; ++ch)
-        acc += __ldcg(p.part + ((size_t)ch * p.B + b) * p.rows_total + n);
+      const float acc = sum_chunks(p, b, n);
       const float mean = (__ldcg(p.u + ((size_t)0 * p.B + b) * kT + n) +
                           __ldcg(p.u + ((size_t)1 * p.B + b) * kT + n) +
                           __ldcg(p.u + ((size_t)2 * p.B + b) * kT + n)) / 3.0f;
       p.f[((size_t)0 * p.B + b) * kT + n] = acc + p.w.fuse_b[n] + mean;
     } else if (p.phase == kUp) {
       const int n = rb * (kRowsPerCta / 2) + j;
-      float ga = 0.f, ua = 0.f;
-      for (int ch = 0; ch < p.nchunks; ++ch) {
-        ga += __ldcg(p.part + ((size_t)ch * p.B + b) * p.rows_total + n);
-        ua += __ldcg(p.part + ((size_t)ch * p.B + b) * p.rows_total + kF + n);
-      }
+      const float ga = sum_chunks(p, b, n), ua = sum_chunks(p, b, kF + n);
       p.act[(size_t)b * kF + n] = silu(ga) * ua;
     } else {
       const int n = rb * kRowsPerCta + j;
-      float acc = 0.f;
-      for (int ch = 0; ch < p.nchunks; ++ch)
-        acc += __ldcg(p.part + ((size_t)ch * p.B + b) * p.rows_total + n);
+      const float acc = sum_chunks(p, b, n);
       p.f[((size_t)(p.block + 1) * p.B + b) * kT + n] =
           __ldcg(p.f + ((size_t)p.block * p.B + b) * kT + n) + acc;
     }
@@ -336,7 +376,7 @@ struct PhaseShape {
 
 PhaseShape phase_shape(int phase, int D) {
   switch (phase) {
-    case kTower: return {512, D / 512, 3 * kT, 3 * kT / kRowsPerCta};
+    case kTower: return {D / 2, 2, 3 * kT, 3 * kT / kRowsPerCta};
     case kFuse: return {1024, 9, kT, kT / kRowsPerCta};
     case kUp: return {512, kT / 512, 2 * kF, kF / (kRowsPerCta / 2)};
     default: return {256, kF / 256, kT, kT / kRowsPerCta};
@@ -361,9 +401,10 @@ int head_counter_count(int D) {
 }
 
 oda_status prepare_head_kernel() {
+  // largest input tile: the tower phase with D = 8192 (Kc = 4096)
   return check_cuda(cudaFuncSetAttribute(head_phase_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kBT * 1024 * (int)sizeof(float)),
+                                         kBT * 4096 * (int)sizeof(float)),
                     "cudaFuncSetAttribute(head)");
 }
 
@@ -414,8 +455,17 @@ oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const flo
     p.nchunks = sh.nchunks;
     p.rows_total = sh.rows_total;
     p.row_blocks = sh.row_blocks;
-    head_phase_kernel<<<sh.row_blocks * sh.nchunks, kHT, kBT * sh.Kc * sizeof(float), s>>>(p);
-    oda_status st = check_cuda(cudaGetLastError(), "recall head launch");
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(sh.row_blocks * sh.nchunks);
+    lc.blockDim = dim3(kHT);
+    lc.dynamicSmemBytes = kBT * sh.Kc * sizeof(float);
+    lc.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    oda_status st = check_cuda(cudaLaunchKernelEx(&lc, head_phase_kernel, p), "recall head launch");
     if (st != ODA_OK) return st;
   }
   return ODA_OK;
