@@ -47,6 +47,9 @@ constexpr int kStagesBytes = kW * kR * kStageBytes;
 constexpr int kMergeStride = 132;     // floats per (warp, head) row of the merge area
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kMaxCluster = 8;
+constexpr int kL2Ahead = 8;           // local set: pages per warp past the ring pulled into L2
+constexpr int kCombineQ = 10;         // partials per lane whose (m, l) loads issue together
+constexpr int kCombineRows = 16;      // partial rows per lane in flight in the output merge
 
 struct AttnParams {
   const int32_t* page_table;
@@ -55,6 +58,8 @@ struct AttnParams {
   const uint32_t* q;      // bf16 pairs [B][Hq][64]
   const uint32_t* k_new;  // bf16 pairs [B][Hkv][64]
   const uint32_t* v_new;
+  const uint8_t* k_pool;  // layer pools (L2 prefetch addresses): [n_pages][Hkv][16][128] bf16
+  const uint8_t* v_pool;
   float* out;             // [B][Hq][128]
   float* part_o;          // full set: [slot][g][128]   slot = CTA index + b*Hkv + h
   float* part_ml;         // full set: [slot][g][2]
@@ -431,18 +436,39 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     vbits = phys >= 0 ? (vbits | (1u << st)) : (vbits & ~(1u << st));
   };
   for (int k = 0; k < kR && k < cw; ++k) issue(k);
+  // pages past the ring's first fill: pull them toward L2 now (their copies are issued as
+  // stages free up, after the dependency wait, and then read L2 instead of DRAM)
+  {
+    const int k = pt_base + lane;
+    if (k >= kR && k < cw && k < kR + kL2Ahead && pt_phys >= 0) {
+      const size_t blk = ((size_t)pt_phys * p.Hkv + h) * (kStageBytes / 2);
+      prefetch_l2_bulk(p.k_pool + blk, kStageBytes / 2);
+      prefetch_l2_bulk(p.v_pool + blk, kStageBytes / 2);
+    }
+  }
   // the previous launch on the stream may still run: wait before reading q or writing
   grid_dependency_wait();
   grid_dependents_launch();
 
   uint32_t qf[8][2];
   load_qf(qf, p, b, h, lane);
-  // staged current token: its score per head and its value, fetched while pages arrive
+  // staged current token: its q . k words (heads warp, warp + kW) and the value this thread
+  // combines first are loaded now and used after the page loop, off the critical path
   __shared__ float s_snew[8];
-  for (int n = warp; n < g; n += kW) {
-    const float sn = staged_score(p, b, h, n, lane);
-    if (lane == 0) s_snew[n] = sn;
+  uint32_t sq[2][2] = {{0u, 0u}, {0u, 0u}};
+  const uint32_t* krow_new = p.k_new + ((size_t)b * p.Hkv + h) * 64;
+  const uint32_t sk0 = krow_new[lane], sk1 = krow_new[lane + 32];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int n = warp + i * kW;
+    if (n < g) {
+      const uint32_t* qrow = p.q + ((size_t)b * p.Hq + h * g + n) * 64;
+      sq[i][0] = qrow[lane];
+      sq[i][1] = qrow[lane + 32];
+    }
   }
+  const int o_lo0 = (int)((long long)rank * (g * 128) / C);
+  const float v_first = staged_value(p, b, h, (o_lo0 + tid) & 127);
   WarpAcc A;
   acc_init(A);
   const int r = lane >> 2;
@@ -462,6 +488,18 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
                  ok && geom_has(ge, j0 + 8), p.scale_log2, lane);
     __syncwarp();
     if (k + kR < cw) issue(k + kR);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int n = warp + i * kW;
+    if (n < g) {
+      const float acc = bf16_lo_to_f32(sq[i][0]) * bf16_lo_to_f32(sk0) +
+                        bf16_hi_to_f32(sq[i][0]) * bf16_hi_to_f32(sk0) +
+                        bf16_lo_to_f32(sq[i][1]) * bf16_lo_to_f32(sk1) +
+                        bf16_hi_to_f32(sq[i][1]) * bf16_hi_to_f32(sk1);
+      const float sn = warp_sum(acc) * p.scale_log2;
+      if (lane == 0) s_snew[n] = sn;
+    }
   }
   warp_flush(A, merge_o + warp * g * kMergeStride, merge_ml + warp * 16, g, lane);
   __syncthreads();
@@ -498,7 +536,8 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
         }
       }
       const float wn = exp2f(snew - M);
-      float L = wn, O = wn * staged_value(p, b, h, d);
+      const float vd = (idx == o_lo + tid) ? v_first : staged_value(p, b, h, d);
+      float L = wn, O = wn * vd;
 #pragma unroll
       for (int q = 0; q < kMaxCluster; ++q) {
         if (q < C && Mr[q] != -INFINITY) {
@@ -528,6 +567,7 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   const int g = p.g;
   float* merge_o = reinterpret_cast<float*>(stages + kStagesBytes);   // [W][g][132]
   float* merge_ml = merge_o + kW * g * kMergeStride;                  // [W][8][2]
+  float* cpart_o = merge_ml + kW * 16;                                // combine scratch
   __shared__ __align__(8) uint64_t bars[kW * kR];
   __shared__ int s_t[ODA_MAX_BATCH];
   __shared__ int s_nv[ODA_MAX_BATCH];
@@ -701,18 +741,17 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     }
     __syncthreads();
     if (s_last) {
-      // ---- last CTA of (b, h): merge the partials and the staged current token.  Loads are
-      // issued together: warps find each head's maximum and weights with lanes over partials,
-      // then every thread sums its dim over the partials with independent loads.
+      // ---- last CTA of (b, h): merge the partials and the staged current token.  The merge
+      // reads nparts x g partials from L2; every load of a phase is issued before its first
+      // use, so the phase costs a few L2 round trips whatever nparts is.
       const int slot0 = c_first + bh;
       float* s_w = merge_o;                  // [g][nparts] weights; nparts <= grid size
       float* s_fin = merge_ml;               // [g][2]: 1 / L, weight of the staged token
+      float* s_red = cpart_o;                // [kW][128] per-warp sums (g < kW)
       for (int n = warp; n < g; n += kW) {
-        const float snew = staged_score(p, b, h, n, lane);
-        float ms[2], ls[2];
-        float M = snew;
+        float ms[kCombineQ], ls[kCombineQ];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
+        for (int q = 0; q < kCombineQ; ++q) {
           const int s = lane + 32 * q;
           ms[q] = -INFINITY;
           ls[q] = 0.f;
@@ -721,15 +760,18 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             ms[q] = __ldcg(p.part_ml + pi * 2);
             ls[q] = __ldcg(p.part_ml + pi * 2 + 1);
           }
-          M = fmaxf(M, ms[q]);
         }
-        for (int s = lane + 64; s < nparts; s += 32)
+        const float snew = staged_score(p, b, h, n, lane);
+        float M = snew;
+#pragma unroll
+        for (int q = 0; q < kCombineQ; ++q) M = fmaxf(M, ms[q]);
+        for (int s = lane + 32 * kCombineQ; s < nparts; s += 32)
           M = fmaxf(M, __ldcg(p.part_ml + ((size_t)(slot0 + s) * g + n) * 2));
 #pragma unroll
         for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
         float L = 0.f;
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
+        for (int q = 0; q < kCombineQ; ++q) {
           const int s = lane + 32 * q;
           if (s < nparts) {
             const float w = (ms[q] == -INFINITY) ? 0.f : exp2f(ms[q] - M);
@@ -737,7 +779,7 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
             L += w * ls[q];
           }
         }
-        for (int s = lane + 64; s < nparts; s += 32) {
+        for (int s = lane + 32 * kCombineQ; s < nparts; s += 32) {
           const size_t pi = (size_t)(slot0 + s) * g + n;
           const float m2 = __ldcg(p.part_ml + pi * 2);
           const float w = (m2 == -INFINITY) ? 0.f : exp2f(m2 - M);
@@ -752,25 +794,71 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         }
       }
       __syncthreads();
-      const int d = tid;  // kThreads == 128 == head_dim
-      const float vd = staged_value(p, b, h, d);
-      for (int n = 0; n < g; ++n) {
+      // O: a warp per head (heads n, n + kW, ... when g > kW; kW / g warps share a head's
+      // partials when g < kW); lane l holds dims 4l..4l+3; kCombineRows rows in flight.
+      // (g = 3: warps 0..2 take one head each, warp 3 idles)
+      const int wph = g >= kW ? 1 : kW / g;
+      const int n_first = g >= kW ? warp : warp % g;
+      const int sub = g >= kW ? 0 : warp / g;
+      const size_t rs = (size_t)g * 32;       // float4 stride between consecutive partials
+      for (int n = n_first; n < g && sub < wph; n += kW) {
         const float* wn = s_w + n * nparts;
-        const float* po = p.part_o + ((size_t)slot0 * g + n) * 128 + d;
-        const size_t stride = (size_t)g * 128;
-        float O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
-        int s = 0;
-        for (; s + 4 <= nparts; s += 4) {
-          const float a0 = __ldcg(po + (size_t)s * stride), a1 = __ldcg(po + (size_t)(s + 1) * stride);
-          const float a2 = __ldcg(po + (size_t)(s + 2) * stride), a3 = __ldcg(po + (size_t)(s + 3) * stride);
-          O0 += wn[s] * a0;
-          O1 += wn[s + 1] * a1;
-          O2 += wn[s + 2] * a2;
-          O3 += wn[s + 3] * a3;
+        const float4* base =
+            reinterpret_cast<const float4*>(p.part_o + ((size_t)slot0 * g + n) * 128) + lane;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s0 = sub; s0 < nparts; s0 += kCombineRows * wph) {
+          float4 v[kCombineRows];
+#pragma unroll
+          for (int j = 0; j < kCombineRows; ++j) {
+            const int s = s0 + j * wph;
+            v[j] = s < nparts ? __ldcg(base + (size_t)s * rs) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int j = 0; j < kCombineRows; ++j) {
+            const int s = s0 + j * wph;
+            const float w = s < nparts ? wn[s] : 0.f;
+            acc.x += w * v[j].x;
+            acc.y += w * v[j].y;
+            acc.z += w * v[j].z;
+            acc.w += w * v[j].w;
+          }
         }
-        for (; s < nparts; ++s) O0 += wn[s] * __ldcg(po + (size_t)s * stride);
-        p.out[((size_t)b * p.Hq + h * g + n) * 128 + d] =
-            ((O0 + O1) + (O2 + O3) + s_fin[n * 2 + 1] * vd) * s_fin[n * 2];
+        if (wph > 1) reinterpret_cast<float4*>(s_red + warp * 128)[lane] = acc;
+        if (wph == 1) {
+          const float wnew = s_fin[n * 2 + 1], inv = s_fin[n * 2];
+          const uint32_t* vp = p.v_new + ((size_t)b * p.Hkv + h) * 64 + 2 * lane;
+          const uint32_t v01 = vp[0], v23 = vp[1];
+          float4 o;
+          o.x = (acc.x + wnew * bf16_lo_to_f32(v01)) * inv;
+          o.y = (acc.y + wnew * bf16_hi_to_f32(v01)) * inv;
+          o.z = (acc.z + wnew * bf16_lo_to_f32(v23)) * inv;
+          o.w = (acc.w + wnew * bf16_hi_to_f32(v23)) * inv;
+          reinterpret_cast<float4*>(p.out + ((size_t)b * p.Hq + h * g + n) * 128)[lane] = o;
+        }
+      }
+      if (wph > 1) {
+        __syncthreads();
+        // warps w < g sum the kW / g rows of head w (rows w, w + g, ...)
+        if (warp < g) {
+          const int n = warp;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int k = 0; k < wph; ++k) {
+            const float4 r = reinterpret_cast<const float4*>(s_red + (k * g + n) * 128)[lane];
+            acc.x += r.x;
+            acc.y += r.y;
+            acc.z += r.z;
+            acc.w += r.w;
+          }
+          const float wnew = s_fin[n * 2 + 1], inv = s_fin[n * 2];
+          const uint32_t* vp = p.v_new + ((size_t)b * p.Hkv + h) * 64 + 2 * lane;
+          const uint32_t v01 = vp[0], v23 = vp[1];
+          float4 o;
+          o.x = (acc.x + wnew * bf16_lo_to_f32(v01)) * inv;
+          o.y = (acc.y + wnew * bf16_hi_to_f32(v01)) * inv;
+          o.z = (acc.z + wnew * bf16_lo_to_f32(v23)) * inv;
+          o.w = (acc.w + wnew * bf16_hi_to_f32(v23)) * inv;
+          reinterpret_cast<float4*>(p.out + ((size_t)b * p.Hq + h * g + n) * 128)[lane] = o;
+        }
       }
       if (tid == 0) p.counters[bh] = 0;
     }
@@ -851,8 +939,10 @@ oda_status encode_pool(CUtensorMap* m, void* base, int64_t n_pages, int Hkv) {
 
 }  // namespace
 
+// stages | merge_o [kW][g][132] | merge_ml [kW][16] | CTA partial / combine scratch
 int attention_smem_bytes(int g) {
-  return 1024 + kStagesBytes + (kW * g * kMergeStride + kW * 16 + g * 130) * (int)sizeof(float);
+  const int tail = g * 130 > kW * 128 ? g * 130 : kW * 128;
+  return 1024 + kStagesBytes + (kW * g * kMergeStride + kW * 16 + tail) * (int)sizeof(float);
 }
 
 // Sets the shared-memory limits and returns the persistent grid size for group size g.
@@ -905,6 +995,8 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
   p.q = static_cast<const uint32_t*>(q);
   p.k_new = static_cast<const uint32_t*>(k_new);
   p.v_new = static_cast<const uint32_t*>(v_new);
+  p.k_pool = static_cast<const uint8_t*>(layer->k);
+  p.v_pool = static_cast<const uint8_t*>(layer->v);
   p.out = out;
   p.part_o = ctx->part_o;
   p.part_ml = ctx->part_ml;
@@ -920,9 +1012,10 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
   p.window = cf.window;
   p.mode = mode;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(128.0));
-  // cluster size of the local kernel: enough CTAs per (b, h) to fill the GPU (at most 8)
+  // cluster size of the local kernel: about one CTA per SM (at most 8 per (b, h)), so that
+  // the CTAs of the next layer's launch fit beside this one's and prefetch while it finishes
   const int pairs = cf.batch * cf.n_kv_heads;
-  p.cluster = std::max(1, std::min(kMaxCluster, (ctx->attn_ctas + pairs / 2) / pairs));
+  p.cluster = std::max(1, std::min(kMaxCluster, ctx->n_sms / pairs));
 
   // Consecutive attention launches of one context overlap when the context allows it: the
   // later one may start (and prefetch its pages) while the earlier one finishes; it waits
@@ -1085,6 +1178,8 @@ oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* l
   p.q = static_cast<const uint32_t*>(q);
   p.k_new = static_cast<const uint32_t*>(k_new);
   p.v_new = static_cast<const uint32_t*>(v_new);
+  p.k_pool = static_cast<const uint8_t*>(layer->k);
+  p.v_pool = static_cast<const uint8_t*>(layer->v);
   p.out = out;
   p.part_o = part_o;
   p.part_ml = part_ml;

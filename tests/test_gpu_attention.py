@@ -64,7 +64,7 @@ class Setup:
         return attend_bits(self.q_np[b], kc, vc, self.kn_np[b], self.vn_np[b], S)
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(16, 8), (32, 8), (8, 1), (4, 4)])
+@pytest.mark.parametrize("Hq,Hkv", [(16, 8), (32, 8), (8, 1), (4, 4), (24, 8)])
 def test_local_matches_oracle(Hq, Hkv):
     s = Setup(_wl(EDGE_CTX, Hq, Hkv))
     out = torch.full((s.wl.B, Hq, 128), 7.0, device="cuda")
@@ -77,7 +77,7 @@ def test_local_matches_oracle(Hq, Hkv):
         assert ok, f"b={b} ctx={s.wl.ctx[b]} max_abs={ma:.3g} rel_l2={rel:.3g}"
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(16, 8), (32, 8)])
+@pytest.mark.parametrize("Hq,Hkv", [(16, 8), (32, 8), (8, 1), (4, 4), (24, 8)])
 def test_full_if_matches_oracle_and_skips_unflagged(Hq, Hkv):
     ctx = [0, 17, 2052, 2053, 2064, 4096, 5000, 9000, 16, 3333]
     s = Setup(_wl(ctx, Hq, Hkv, seed=78))
