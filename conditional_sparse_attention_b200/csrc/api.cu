@@ -132,7 +132,7 @@ oda_status oda_create(const oda_config* cfg, oda_ctx** out) {
   const int gch = oda::glue_chunks(c.head_in_dim);
   st = dev_alloc(&x->part_o, (size_t)ms * x->g * 128, "cudaMalloc(partials)");
   if (st == ODA_OK) st = dev_alloc(&x->part_ml, (size_t)ms * x->g * 2, "cudaMalloc(partials)");
-  if (st == ODA_OK) st = dev_alloc(&x->attn_cnt, (size_t)B * Hkv, "cudaMalloc(counters)");
+  if (st == ODA_OK) st = dev_alloc(&x->attn_cnt, (size_t)2 * B * Hkv, "cudaMalloc(counters)");
   if (st == ODA_OK) st = dev_alloc(&x->err, 1, "cudaMalloc(error word)");
   if (st == ODA_OK) st = dev_alloc(&x->head_part, oda::head_part_floats((int)B, (int)D), "cudaMalloc(head)");
   if (st == ODA_OK) st = dev_alloc(&x->head_ss, (size_t)96 * (D / 512) * B, "cudaMalloc(head)");
@@ -143,7 +143,7 @@ oda_status oda_create(const oda_config* cfg, oda_ctx** out) {
   if (st == ODA_OK) st = dev_alloc(&x->glue_x, (size_t)B * D, "cudaMalloc(glue)");
   if (st == ODA_OK) st = dev_alloc(&x->glue_ss, (size_t)B * gch, "cudaMalloc(glue)");
   if (st == ODA_OK) st = dev_alloc(&x->glue_cnt, (size_t)2 * B, "cudaMalloc(glue)");
-  if (st == ODA_OK) st = check_cuda(cudaMemset(x->attn_cnt, 0, B * Hkv * sizeof(int32_t)), "cudaMemset");
+  if (st == ODA_OK) st = check_cuda(cudaMemset(x->attn_cnt, 0, 2 * B * Hkv * sizeof(int32_t)), "cudaMemset");
   if (st == ODA_OK) st = check_cuda(cudaMemset(x->err, 0, sizeof(int32_t)), "cudaMemset");
   if (st == ODA_OK)
     st = check_cuda(cudaMemset(x->head_cnt, 0, oda::head_counter_count((int)D) * sizeof(int32_t)),

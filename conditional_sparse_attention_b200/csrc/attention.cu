@@ -47,7 +47,8 @@ constexpr int kStagesBytes = kW * kR * kStageBytes;
 constexpr int kMergeStride = 132;     // floats per (warp, head) row of the merge area
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kMaxCluster = 8;
-constexpr int kL2Ahead = 8;           // local set: pages per warp past the ring pulled into L2
+constexpr int kChunk = 4;             // full set: pages per claimed chunk
+constexpr int kQueueLow = kR + kChunk;   // full set: queue length that triggers the next claim
 constexpr int kCombineQ = 10;         // partials per lane whose (m, l) loads issue together
 constexpr int kCombineRows = 16;      // partial rows per lane in flight in the output merge
 
@@ -58,12 +59,11 @@ struct AttnParams {
   const uint32_t* q;      // bf16 pairs [B][Hq][64]
   const uint32_t* k_new;  // bf16 pairs [B][Hkv][64]
   const uint32_t* v_new;
-  const uint8_t* k_pool;  // layer pools (L2 prefetch addresses): [n_pages][Hkv][16][128] bf16
-  const uint8_t* v_pool;
   float* out;             // [B][Hq][128]
   float* part_o;          // full set: [slot][g][128]   slot = CTA index + b*Hkv + h
   float* part_ml;         // full set: [slot][g][2]
-  int32_t* counters;      // full set: [B*Hkv]
+  int32_t* counters;      // full set: [B*Hkv] completion counts of the (b, h) partials
+  int32_t* claims;        // full set: [B*Hkv] chunk claim counters
   int32_t* err;
   int64_t n_pool_pages;
   int32_t B, Hq, Hkv, g, max_pages, sinks, window, mode;
@@ -436,16 +436,6 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     vbits = phys >= 0 ? (vbits | (1u << st)) : (vbits & ~(1u << st));
   };
   for (int k = 0; k < kR && k < cw; ++k) issue(k);
-  // pages past the ring's first fill: pull them toward L2 now (their copies are issued as
-  // stages free up, after the dependency wait, and then read L2 instead of DRAM)
-  {
-    const int k = pt_base + lane;
-    if (k >= kR && k < cw && k < kR + kL2Ahead && pt_phys >= 0) {
-      const size_t blk = ((size_t)pt_phys * p.Hkv + h) * (kStageBytes / 2);
-      prefetch_l2_bulk(p.k_pool + blk, kStageBytes / 2);
-      prefetch_l2_bulk(p.v_pool + blk, kStageBytes / 2);
-    }
-  }
   // the previous launch on the stream may still run: wait before reading q or writing
   grid_dependency_wait();
   grid_dependents_launch();
@@ -623,96 +613,171 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   uint8_t* my_stages = stages + warp * kR * kStageBytes;
   uint64_t* my_bars = bars + warp * kR;
 
-  // ---- this warp's copy stream: its units (every kW-th of each segment), kR ahead.  Lane k
-  // of the warp holds the physical page and KV head of the warp's (pt_base + k)-th unit,
-  // refilled 32 units at a time with parallel loads, and issues that unit's copy itself.
-  uint32_t issued = 0, consumed = 0, vbits = 0, pt_base = 0;
-  int pt_phys = -1, pt_head = 0;
-  bool pt_live = false;
+  // ---- this warp's copy stream.  The pages of a (b, h) are split into chunks of kChunk
+  // pages.  Every warp of a CTA whose range starts in (b, h) owns one fixed chunk (rank-major,
+  // so it can be fetched before the dependency wait); the remaining chunks are claimed from the
+  // (b, h)'s counter by the warps of all CTAs covering it, so that CTAs on faster SMs take more
+  // of them.  Claimed pages wait in a per-warp queue held one entry per lane (entry i in lane
+  // i % 32); copies run kR pages ahead of the arithmetic and may cross into the next segment.
+  uint32_t issued = 0, consumed = 0, vbits = 0;
+  uint32_t f_head = 0, f_tail = 0;            // queue entries [f_head, f_tail)
+  int f_phys = -1, f_h = 0, f_lp = 0, f_seg = 0;
+  int st_lp = 0, st_seg = 0;                  // lane st: logical page and segment of stage st
   bool dead = false;
-  int is_u = u0, is_i = warp;
-  Seg is{0, 0, 0, 0, 0, 1};
-  if (is_u < u1) is = decode_seg(is_u, u1, s_us, s_nv, B, Hkv);
-  auto normalize = [&](int& cu, int& ci, Seg& cs_) {
-    while (cu < u1 && ci >= cs_.n) {
-      cu += cs_.n;
-      ci = warp;
-      if (cu < u1) cs_ = decode_seg(cu, u1, s_us, s_nv, B, Hkv);
+  // claim side (warp-uniform; `pend` lives in lane 0)
+  int is_seg = 0, is_u = u0, is_b = 0, is_h = 0, is_bh = 0, is_nv = 0, is_ncache = 0;
+  int is_nch = 0, is_base = 0, is_fixed = -1, pend = 0;
+  bool is_done = u0 >= u1, claims_ok = false, has_pend = false;
+  auto enter_seg = [&](bool first) {
+    const Seg cs_ = decode_seg(is_u, u1, s_us, s_nv, B, Hkv);
+    is_b = cs_.b;
+    is_h = cs_.h;
+    is_bh = cs_.b * Hkv + cs_.h;
+    is_nv = cs_.nv;
+    is_ncache = s_t[cs_.b] - 1;
+    is_nch = (is_nv + kChunk - 1) / kChunk;
+    // CTAs whose range starts inside this (b, h): [cfs, cfe); their warps own chunks
+    // 0 .. (cfe - cfs) * kW - 1, one each; claims hand out the chunks after those
+    const long long s0 = cs_.s0, s1 = (long long)cs_.s0 + cs_.nv;
+    const long long cfs = (s0 * G + U - 1) / U;
+    const long long cfe = min(G, (s1 * G + U - 1) / U);
+    is_base = (int)(cfe - cfs) * kW;
+    is_fixed = first ? (int)((long long)blockIdx.x - cfs) * kW + warp : -1;
+    has_pend = false;
+    if (claims_ok) {
+      if (lane == 0) pend = atomicAdd(p.claims + is_bh, 1);
+      has_pend = true;
     }
   };
-  normalize(is_u, is_i, is);
-  auto refill = [&]() {
-    // each lane walks `lane` units ahead of the issue cursor and looks up its page
-    int cu = is_u, ci = is_i;
-    Seg cs_ = is;
-    for (int k = 0; k < lane && cu < u1; ++k) {
-      ci += kW;
-      normalize(cu, ci, cs_);
+  // lanes look up the physical pages of chunk c of the claim segment into queue entries
+  auto push_chunk = [&](int c) {
+    const int first = c * kChunk;
+    const int np = min(kChunk, is_nv - first);
+    const int j = (int)(((uint32_t)lane - f_tail) & 31u);
+    if (j < np) {
+      const int lp = first + j;
+      int phys = -1;   // an empty cache keeps one unit that loads nothing
+      if (is_ncache > 0) {
+        const int e = __ldcg(p.page_table + (size_t)is_b * p.max_pages + lp);
+        phys = (e >= 0 && (int64_t)e < p.n_pool_pages) ? e : -2;
+        if (phys == -2) atomicOr(p.err, ODA_DEVERR_PAGE_RANGE);
+      }
+      f_phys = phys;
+      f_h = is_h;
+      f_lp = lp;
+      f_seg = is_seg;
     }
-    pt_phys = -1;
-    pt_head = cs_.h;
-    if (cu < u1) {
-      const Geom ge = make_geom(s_t[cs_.b], 1, p.sinks, p.window, p.max_pages, true);
-      if (ge.n_cache > 0) {
-        const int lp = geom_page(ge, cs_.v0 + ci);
-        const int phys = __ldcg(p.page_table + (size_t)cs_.b * p.max_pages + lp);
-        pt_phys = (phys >= 0 && (int64_t)phys < p.n_pool_pages) ? phys : -2;
-        if (pt_phys == -2) atomicOr(p.err, ODA_DEVERR_PAGE_RANGE);
+    f_tail += (uint32_t)np;
+  };
+  // queue one more chunk, or move the claim side to the next segment
+  auto top_up = [&]() {
+    if (is_done || dead || f_tail - f_head >= (uint32_t)kQueueLow) return;
+    if (is_fixed >= 0) {
+      const int c = is_fixed;
+      is_fixed = -1;
+      if (c < is_nch) {
+        push_chunk(c);
+        return;
       }
     }
-    pt_base = issued;
-    pt_live = true;
+    if (!claims_ok) return;
+    if (!has_pend) {
+      if (lane == 0) pend = atomicAdd(p.claims + is_bh, 1);
+      has_pend = true;
+    }
+    const int c = is_base + __shfl_sync(0xffffffffu, pend, 0);
+    has_pend = false;
+    if (c < is_nch) {
+      push_chunk(c);
+      if (lane == 0) pend = atomicAdd(p.claims + is_bh, 1);
+      has_pend = true;
+    } else {
+      is_u += decode_seg(is_u, u1, s_us, s_nv, B, Hkv).n;
+      ++is_seg;
+      if (is_u >= u1) is_done = true;
+      else enter_seg(false);
+    }
   };
-  auto issue_next = [&]() {
-    if (dead || is_u >= u1) return;
-    if (!pt_live || issued - pt_base >= 32u) refill();
+  // copy the queue head into the next stage
+  auto issue_one = [&]() {
+    const int src = (int)(f_head & 31u);
+    const int phys = __shfl_sync(0xffffffffu, f_phys, src);
+    const int hh = __shfl_sync(0xffffffffu, f_h, src);
+    const int lp = __shfl_sync(0xffffffffu, f_lp, src);
+    const int sg = __shfl_sync(0xffffffffu, f_seg, src);
     const uint32_t st = issued % kR;
-    const int src = (int)(issued - pt_base);
-    const int phys = __shfl_sync(0xffffffffu, pt_phys, src);
-    const int head = __shfl_sync(0xffffffffu, pt_head, src);
     if (lane == src) {
       if (phys >= 0)
-        issue_page(my_stages + st * kStageBytes, my_bars + st, &tmK, &tmV, phys, Hkv, head);
+        issue_page(my_stages + st * kStageBytes, my_bars + st, &tmK, &tmV, phys, Hkv, hh);
       else
         mbar_arrive(my_bars + st);
     }
+    if (lane == (int)st) {
+      st_lp = lp;
+      st_seg = sg;
+    }
     vbits = phys >= 0 ? (vbits | (1u << st)) : (vbits & ~(1u << st));
     ++issued;
-    is_i += kW;
-    normalize(is_u, is_i, is);
+    ++f_head;
   };
-  for (int k = 0; k < kR; ++k) issue_next();
+  // keep kR copies in flight while pages remain
+  auto pump = [&]() {
+    while (!dead && issued - consumed < (uint32_t)kR) {
+      if (f_head == f_tail) {
+        top_up();
+        if (f_head == f_tail) {
+          if (is_done || !claims_ok) break;
+          continue;
+        }
+      }
+      issue_one();
+    }
+  };
+  if (!is_done) enter_seg(true);
+  pump();
   // Everything above reads only the cache, the page table and positions/flags, which an
   // attention launch never writes; the previous launch of the stream may still be running
-  // (programmatic dependent launch).  Wait for it before reading q or writing anything.
+  // (programmatic dependent launch).  Wait for it before claiming, reading q or writing.
   grid_dependency_wait();
   grid_dependents_launch();
+  claims_ok = true;
+  if (!is_done && is_fixed < 0) {
+    if (lane == 0) pend = atomicAdd(p.claims + is_bh, 1);
+    has_pend = true;
+  }
 
   // ---- segments of this CTA, in order
-  for (int seg_u = u0; seg_u < u1;) {
+  int cseg = 0;
+  for (int seg_u = u0; seg_u < u1; ++cseg) {
     const Seg cs = decode_seg(seg_u, u1, s_us, s_nv, B, Hkv);
-    const Geom ge = make_geom(s_t[cs.b], 1, p.sinks, p.window, p.max_pages, true);
     const int b = cs.b, h = cs.h;
+    const int n_cache = s_t[b] - 1;
     uint32_t qf[8][2];
     load_qf(qf, p, b, h, lane);
     WarpAcc A;
     acc_init(A);
     const int r = lane >> 2;
-    for (int i = warp; i < cs.n && !dead; i += kW) {
+    while (!dead) {
+      if (consumed == issued) {
+        pump();
+        if (consumed == issued) break;
+      }
       const uint32_t st = consumed % kR;
+      if (__shfl_sync(0xffffffffu, st_seg, (int)st) != cseg) break;  // a later segment's page
       if (!mbar_wait_bounded(my_bars + st, (consumed / kR) & 1u, kWaitNs)) {
         if (lane == 0) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
         dead = true;
         break;
       }
       const bool ok = (vbits >> st) & 1u;
-      const int lp = geom_page(ge, cs.v0 + i);
+      const int lp = __shfl_sync(0xffffffffu, st_lp, (int)st);
       const int j0 = lp * kPageTok + r;
-      page_compute(A, qf, my_stages + st * kStageBytes, ok && geom_has(ge, j0),
-                   ok && geom_has(ge, j0 + 8), p.scale_log2, lane);
+      page_compute(A, qf, my_stages + st * kStageBytes, ok && j0 < n_cache, ok && j0 + 8 < n_cache,
+                   p.scale_log2, lane);
       ++consumed;
       __syncwarp();
-      issue_next();
+      top_up();
+      pump();
     }
     warp_flush(A, merge_o + warp * g * kMergeStride, merge_ml + warp * 16, g, lane);
     __syncthreads();
@@ -860,7 +925,10 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
           reinterpret_cast<float4*>(p.out + ((size_t)b * p.Hq + h * g + n) * 128)[lane] = o;
         }
       }
-      if (tid == 0) p.counters[bh] = 0;
+      if (tid == 0) {
+        p.counters[bh] = 0;
+        p.claims[bh] = 0;
+      }
     }
     __syncthreads();
     seg_u += cs.n;
@@ -995,12 +1063,11 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
   p.q = static_cast<const uint32_t*>(q);
   p.k_new = static_cast<const uint32_t*>(k_new);
   p.v_new = static_cast<const uint32_t*>(v_new);
-  p.k_pool = static_cast<const uint8_t*>(layer->k);
-  p.v_pool = static_cast<const uint8_t*>(layer->v);
   p.out = out;
   p.part_o = ctx->part_o;
   p.part_ml = ctx->part_ml;
   p.counters = ctx->attn_cnt;
+  p.claims = ctx->attn_cnt + (size_t)cf.batch * cf.n_kv_heads;
   p.err = ctx->err;
   p.n_pool_pages = layer->n_pages;
   p.B = cf.batch;
@@ -1146,10 +1213,11 @@ oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* l
                                        attention_smem_bytes(8)),
                   "cudaFuncSetAttribute(full attention)");
   if (st != ODA_OK) return st;
-  // scratch layout: counters [B*Hkv] | error word | partial (m, l) | partial O
+  // scratch layout: completion counters [B*Hkv] | claim counters [B*Hkv] | error word |
+  // partial (m, l) | partial O
   const size_t pairs = (size_t)cf.batch * cf.n_kv_heads;
   const size_t slots = (size_t)d->ctas + pairs;
-  const size_t cnt_bytes = ((pairs + 1) * sizeof(int32_t) + 255) / 256 * 256;
+  const size_t cnt_bytes = ((2 * pairs + 1) * sizeof(int32_t) + 255) / 256 * 256;
   const size_t ml_bytes = (slots * g * 2 * sizeof(float) + 255) / 256 * 256;
   const size_t o_bytes = slots * g * 128 * sizeof(float);
   if (cnt_bytes + ml_bytes + o_bytes > kNoAllocScratchBytes)
@@ -1159,11 +1227,11 @@ oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* l
                      cnt_bytes + ml_bytes + o_bytes, cf.batch, cf.n_kv_heads, g,
                      kNoAllocScratchBytes);
   int32_t* counters = reinterpret_cast<int32_t*>(d->scratch);
-  int32_t* err_word = counters + pairs;
+  int32_t* err_word = counters + 2 * pairs;
   float* part_ml = reinterpret_cast<float*>(d->scratch + cnt_bytes);
   float* part_o = reinterpret_cast<float*>(d->scratch + cnt_bytes + ml_bytes);
-  // the completion counters (and the scratch error word) must start at zero on every call
-  st = check_cuda(cudaMemsetAsync(counters, 0, (pairs + 1) * sizeof(int32_t), stream),
+  // the counters (and the scratch error word) must start at zero on every call
+  st = check_cuda(cudaMemsetAsync(counters, 0, (2 * pairs + 1) * sizeof(int32_t), stream),
                   "cudaMemsetAsync(noalloc counters)");
   if (st != ODA_OK) return st;
   CUtensorMap tmK, tmV;
@@ -1178,12 +1246,11 @@ oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* l
   p.q = static_cast<const uint32_t*>(q);
   p.k_new = static_cast<const uint32_t*>(k_new);
   p.v_new = static_cast<const uint32_t*>(v_new);
-  p.k_pool = static_cast<const uint8_t*>(layer->k);
-  p.v_pool = static_cast<const uint8_t*>(layer->v);
   p.out = out;
   p.part_o = part_o;
   p.part_ml = part_ml;
   p.counters = counters;
+  p.claims = counters + pairs;
   p.err = device_error ? device_error : err_word;
   p.n_pool_pages = layer->n_pages;
   p.B = cf.batch;

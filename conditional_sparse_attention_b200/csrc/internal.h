@@ -17,7 +17,7 @@ struct oda_ctx {
   int n_slots = 0;            // partial slots: attn_ctas + B*Hkv
   float* part_o = nullptr;    // [n_slots][g][128]
   float* part_ml = nullptr;   // [n_slots][g][2]
-  int32_t* attn_cnt = nullptr;  // [B*Hkv] completion counters (self-resetting)
+  int32_t* attn_cnt = nullptr;  // [2][B*Hkv] completion and chunk-claim counters (self-resetting)
   int32_t* err = nullptr;       // sticky device error word
   // recall-head scratch
   float* head_part = nullptr;   // split-K partial sums, largest phase

@@ -173,3 +173,25 @@ def test_invalid_arguments_rejected_on_host():
     s = Setup(_wl([10], seed=82))
     with pytest.raises(OdaError):
         s.oda.oda_attend_local(s.ctx, s.layer, s.pt, s.pos, s.q, s.kn, s.vn, None)
+
+
+@pytest.mark.parametrize("ctx,Hq,Hkv", [
+    # many short sequences: fewer units than CTAs, CTAs spanning several (sequence, head) pairs
+    ([int(x) for x in np.random.default_rng(5).integers(0, 300, 40)], 16, 8),
+    # one long sequence and one KV head: every CTA claims chunks of the same (b, h)
+    ([50000], 8, 1),
+    # lengths spread over two orders of magnitude with every sequence flagged
+    ([70000, 900, 33, 20000, 4097, 1, 131072 - 3000], 32, 8),
+])
+def test_full_set_chunk_claims_cover_every_page(ctx, Hq, Hkv):
+    s = Setup(_wl(ctx, Hq, Hkv, seed=83))
+    flag = torch.ones(len(ctx), dtype=torch.int32, device="cuda")
+    out = torch.full((s.wl.B, Hq, 128), 7.0, device="cuda")
+    for rep in range(2):   # the second launch runs on counters reset by the first
+        s.oda.oda_attend_full_if(s.ctx, s.layer, s.pt, s.pos, flag, s.q, s.kn, s.vn, out)
+        torch.cuda.synchronize()
+        assert s.oda.oda_get_error(s.ctx) == 0
+        got = out.cpu().numpy()
+        for b in range(s.wl.B):
+            ok, ma, rel = attn_close(got[b], s.oracle(b, 1))
+            assert ok, f"rep={rep} b={b} ctx={ctx[b]} max_abs={ma:.3g} rel_l2={rel:.3g}"
