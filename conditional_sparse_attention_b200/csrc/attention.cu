@@ -38,12 +38,18 @@ namespace cg = cooperative_groups;
 namespace oda {
 namespace {
 
-constexpr int kW = 4;                 // warps per CTA (each streams its own pages)
+// full set: 4 warps per CTA, two CTAs per SM; local set: 8 warps, one CTA per SM (its
+// launch is latency-bound, so more warps in flight beat the room for a second CTA)
+constexpr int kW = 4;                 // full set: warps per CTA (each streams its own pages)
 constexpr int kR = 3;                 // pages in flight per warp
 constexpr int kThreads = kW * 32;
+constexpr int kWL = 8;                // local set: warps per CTA
+constexpr int kRL = 3;                // local set: pages in flight per warp
+constexpr int kThreadsL = kWL * 32;
 constexpr int kPageTok = 16;
 constexpr int kStageBytes = 8192;     // K (4 KiB) + V (4 KiB) of one (page, KV head)
 constexpr int kStagesBytes = kW * kR * kStageBytes;
+constexpr int kStagesBytesL = kWL * kRL * kStageBytes;
 constexpr int kMergeStride = 132;     // floats per (warp, head) row of the merge area
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kMaxCluster = 8;
@@ -68,6 +74,7 @@ struct AttnParams {
   int64_t n_pool_pages;
   int32_t B, Hq, Hkv, g, max_pages, sinks, window, mode;
   int32_t cluster;        // local set: CTAs per (b, h)
+  int32_t kv_single;      // 1: tmA spans both pools (one copy per page); 0: tmA = K, tmB = V
   float scale_log2;       // log2(e) / sqrt(128)
 };
 
@@ -164,16 +171,21 @@ __device__ __forceinline__ void load_qf(uint32_t (&qf)[8][2], const AttnParams& 
   }
 }
 
-// Issues the four tile loads of one (page, KV head) into a stage (K at +0, V at +4096).
-__device__ __forceinline__ void issue_page(uint8_t* dst, uint64_t* bar, const CUtensorMap* tmK,
-                                           const CUtensorMap* tmV, int phys, int Hkv, int h) {
+// Issues the copy of one (page, KV head) into a stage (K at +0, V at +4096; each as two
+// 64-column halves of 16 rows, 128-byte swizzle): one 4-D copy when a single map spans both
+// pools, else one 3-D copy per pool.
+__device__ __forceinline__ void issue_page(uint8_t* dst, uint64_t* bar, const CUtensorMap* tmA,
+                                           const CUtensorMap* tmB, bool single, int phys, int Hkv,
+                                           int h) {
   fence_proxy_async_smem();
   mbar_arrive_expect_tx(bar, kStageBytes);
   const int y = (phys * Hkv + h) * kPageTok;
-  tma_load_2d(dst, tmK, 0, y, bar);
-  tma_load_2d(dst + 2048, tmK, 64, y, bar);
-  tma_load_2d(dst + 4096, tmV, 0, y, bar);
-  tma_load_2d(dst + 6144, tmV, 64, y, bar);
+  if (single) {
+    tma_load_4d(dst, tmA, 0, y, 0, 0, bar);
+  } else {
+    tma_load_3d(dst, tmA, 0, y, 0, bar);
+    tma_load_3d(dst + 4096, tmB, 0, y, 0, bar);
+  }
 }
 
 // One 16-token page in a stage: scores, online softmax, PV.  in0 / in1: whether this lane's
@@ -266,6 +278,147 @@ __device__ __forceinline__ void page_compute(WarpAcc& A, const uint32_t (&qf)[8]
   }
 }
 
+// Scores S = K Q^T of one 16-token page (tokens as M, the group's heads as N), in the exp2
+// domain; tokens outside the set get -inf.
+__device__ __forceinline__ void page_scores(float (&x)[4], const uint32_t (&qf)[8][2], uint32_t sb,
+                                            bool in0, bool in1, float scale_log2, int lane) {
+  const int mi = lane >> 3, rr = lane & 7;
+  const int krow = ((mi & 1) << 3) + rr;
+  float sa[4] = {0.f, 0.f, 0.f, 0.f}, sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int kk = 0; kk < 8; kk += 2) {
+    uint32_t a0[4], a1[4];
+    const int ch0 = 2 * kk + (mi >> 1), ch1 = ch0 + 2;
+    ldsm_x4(a0, sb + (ch0 >> 3) * 2048 + krow * 128 + (((ch0 & 7) ^ rr) << 4));
+    ldsm_x4(a1, sb + (ch1 >> 3) * 2048 + krow * 128 + (((ch1 & 7) ^ rr) << 4));
+    mma_bf16_16816(sa, a0, qf[kk][0], qf[kk][1]);
+    mma_bf16_16816(sc, a1, qf[kk + 1][0], qf[kk + 1][1]);
+  }
+  x[0] = in0 ? (sa[0] + sc[0]) * scale_log2 : -INFINITY;
+  x[1] = in0 ? (sa[1] + sc[1]) * scale_log2 : -INFINITY;
+  x[2] = in1 ? (sa[2] + sc[2]) * scale_log2 : -INFINITY;
+  x[3] = in1 ? (sa[3] + sc[3]) * scale_log2 : -INFINITY;
+}
+
+// P (fp32, this lane's rows r / r + 8 and heads 2c / 2c + 1) as P^T fragments for the PV
+// product, split into bf16 hi + lo parts.
+__device__ __forceinline__ void p_fragments(const float (&pv)[4], uint32_t& bh0, uint32_t& bh1,
+                                            uint32_t& bl0, uint32_t& bl1) {
+  const __nv_bfloat16 h0 = __float2bfloat16_rn(pv[0]), h1 = __float2bfloat16_rn(pv[1]);
+  const __nv_bfloat16 h2 = __float2bfloat16_rn(pv[2]), h3 = __float2bfloat16_rn(pv[3]);
+  bh0 = movmatrix_trans(pack_bf16x2(h0, h1));
+  bh1 = movmatrix_trans(pack_bf16x2(h2, h3));
+  bl0 = movmatrix_trans(pack_bf16x2(__float2bfloat16_rn(pv[0] - __bfloat162float(h0)),
+                                    __float2bfloat16_rn(pv[1] - __bfloat162float(h1))));
+  bl1 = movmatrix_trans(pack_bf16x2(__float2bfloat16_rn(pv[2] - __bfloat162float(h2)),
+                                    __float2bfloat16_rn(pv[3] - __bfloat162float(h3))));
+}
+
+// Zeroes the V rows of tokens outside the set (their P is 0, but stale bytes could be NaN).
+// Returns true if it wrote to the stage.
+__device__ __forceinline__ bool zero_masked_v(uint8_t* stage, bool in0, bool in1, int lane) {
+  if (!__any_sync(0xffffffffu, !(in0 && in1))) return false;
+  const int r = lane >> 2, c = lane & 3;
+  uint4* vbase = reinterpret_cast<uint4*>(stage + 4096);
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  if (!in0) {
+    vbase[r * 8 + 2 * c] = z;
+    vbase[r * 8 + 2 * c + 1] = z;
+    vbase[128 + r * 8 + 2 * c] = z;
+    vbase[128 + r * 8 + 2 * c + 1] = z;
+  }
+  if (!in1) {
+    vbase[(r + 8) * 8 + 2 * c] = z;
+    vbase[(r + 8) * 8 + 2 * c + 1] = z;
+    vbase[128 + (r + 8) * 8 + 2 * c] = z;
+    vbase[128 + (r + 8) * 8 + 2 * c + 1] = z;
+  }
+  __syncwarp();
+  return true;
+}
+
+// Two pages (32 tokens) in one online-softmax step: both score blocks are independent, the
+// running maximum and the rescale are taken once for the pair, and the PV products of the two
+// pages accumulate into separate hi / lo chains.  Same result as two page_compute calls up to
+// fp32 rounding.
+__device__ __forceinline__ void page_compute2(WarpAcc& A, const uint32_t (&qf)[8][2],
+                                              uint8_t* stA, bool a0, bool a1,
+                                              uint8_t* stB, bool b0, bool b1,
+                                              float scale_log2, int lane) {
+  const bool anyA = __any_sync(0xffffffffu, a0 || a1), anyB = __any_sync(0xffffffffu, b0 || b1);
+  if (!anyA || !anyB) {   // a page without tokens in the set: the other one alone
+    if (anyA) page_compute(A, qf, stA, a0, a1, scale_log2, lane);
+    if (anyB) page_compute(A, qf, stB, b0, b1, scale_log2, lane);
+    return;
+  }
+  const int mi = lane >> 3, rr = lane & 7;
+  const int vrow = ((mi >> 1) << 3) + rr;
+  const uint32_t sA = smem_u32(stA), sB = smem_u32(stB);
+  float xa[4], xb[4];
+  page_scores(xa, qf, sA, a0, a1, scale_log2, lane);
+  page_scores(xb, qf, sB, b0, b1, scale_log2, lane);
+  float mx0 = fmaxf(fmaxf(xa[0], xa[2]), fmaxf(xb[0], xb[2]));
+  float mx1 = fmaxf(fmaxf(xa[1], xa[3]), fmaxf(xb[1], xb[3]));
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+  }
+  const float mn0 = fmaxf(A.m0, mx0), mn1 = fmaxf(A.m1, mx1);
+  if (mn0 > A.m0 || mn1 > A.m1) {
+    const float al0 = exp2f(A.m0 - mn0), al1 = exp2f(A.m1 - mn1);
+    A.l0 *= al0;
+    A.l1 *= al1;
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      A.o[mt][0] *= al0;
+      A.o[mt][1] *= al1;
+      A.o[mt][2] *= al0;
+      A.o[mt][3] *= al1;
+    }
+    A.m0 = mn0;
+    A.m1 = mn1;
+  }
+  float pa[4], pb[4];
+  pa[0] = exp2f(xa[0] - A.m0);
+  pa[1] = exp2f(xa[1] - A.m1);
+  pa[2] = exp2f(xa[2] - A.m0);
+  pa[3] = exp2f(xa[3] - A.m1);
+  pb[0] = exp2f(xb[0] - A.m0);
+  pb[1] = exp2f(xb[1] - A.m1);
+  pb[2] = exp2f(xb[2] - A.m0);
+  pb[3] = exp2f(xb[3] - A.m1);
+  A.l0 += (pa[0] + pa[2]) + (pb[0] + pb[2]);
+  A.l1 += (pa[1] + pa[3]) + (pb[1] + pb[3]);
+  uint32_t ah0, ah1, al0, al1, bh0, bh1, bl0, bl1;
+  p_fragments(pa, ah0, ah1, al0, al1);
+  p_fragments(pb, bh0, bh1, bl0, bl1);
+  zero_masked_v(stA, a0, a1, lane);
+  zero_masked_v(stB, b0, b1, lane);
+  float lo[8][4];
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) lo[mt][0] = lo[mt][1] = lo[mt][2] = lo[mt][3] = 0.f;
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    const int chunk = 2 * mt + (mi & 1);
+    const uint32_t off = 4096 + (chunk >> 3) * 2048 + vrow * 128 + (((chunk & 7) ^ rr) << 4);
+    uint32_t va[4], vb[4];
+    ldsm_x4_trans(va, sA + off);
+    ldsm_x4_trans(vb, sB + off);
+    mma_bf16_16816(A.o[mt], va, ah0, ah1);
+    mma_bf16_16816(lo[mt], va, al0, al1);
+    mma_bf16_16816(A.o[mt], vb, bh0, bh1);
+    mma_bf16_16816(lo[mt], vb, bl0, bl1);
+  }
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    A.o[mt][0] += lo[mt][0];
+    A.o[mt][1] += lo[mt][1];
+    A.o[mt][2] += lo[mt][2];
+    A.o[mt][3] += lo[mt][3];
+  }
+}
+
 // Reduces l over the token rows and writes the warp's state to its merge slot:
 // mo [g][kMergeStride] (O^T columns), ml [8][2] (m, l).
 __device__ __forceinline__ void warp_flush(WarpAcc& A, float* mo, float* ml, int g, int lane) {
@@ -296,17 +449,18 @@ __device__ __forceinline__ void warp_flush(WarpAcc& A, float* mo, float* ml, int
   }
 }
 
-// Merge of the kW warp states for head n, dim d: (M, L, O) relative to exp2(M).
+// Merge of the W warp states for head n, dim d: (M, L, O) relative to exp2(M).
+template <int W>
 __device__ __forceinline__ void cta_merge(const float* merge_o, const float* merge_ml, int g,
                                           int n, int d, float& M, float& L, float& O) {
   M = -INFINITY;
 #pragma unroll
-  for (int w = 0; w < kW; ++w) M = fmaxf(M, merge_ml[w * 16 + n * 2]);
+  for (int w = 0; w < W; ++w) M = fmaxf(M, merge_ml[w * 16 + n * 2]);
   O = 0.f;
   L = 0.f;
   if (M == -INFINITY) return;
 #pragma unroll
-  for (int w = 0; w < kW; ++w) {
+  for (int w = 0; w < W; ++w) {
     const float mw = merge_ml[w * 16 + n * 2];
     if (mw != -INFINITY) {
       const float sc = exp2f(mw - M);
@@ -370,21 +524,22 @@ __device__ __forceinline__ int cta_of(long long u, long long U, long long G) {
 
 // ---------------------------------------------------------------- local set: clusters
 // Cluster of p.cluster CTAs per (b, h); CTA `rank` takes the contiguous share
-// [rank*nv/C, (rank+1)*nv/C) of the visited pages; warps take every kW-th page of it.  After a
+// [rank*nv/C, (rank+1)*nv/C) of the visited pages; warps take every kWL-th page of it.  After a
 // cluster barrier each rank finishes its share of the g*128 outputs from all ranks' partials
 // (read through distributed shared memory).
-__global__ void __launch_bounds__(kThreads, 2)
-attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+__global__ void __launch_bounds__(kThreadsL, 1)
+attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int g = p.g;
-  float* merge_o = reinterpret_cast<float*>(stages + kStagesBytes);   // [W][g][132]
-  float* merge_ml = merge_o + kW * g * kMergeStride;                  // [W][8][2]
-  float* cpart_o = merge_ml + kW * 16;                                // [g][128] CTA partial
+  // the merge areas reuse the stages: they are written only after every copy has landed
+  float* merge_o = reinterpret_cast<float*>(stages);                   // [W][g][132]
+  float* merge_ml = merge_o + kWL * g * kMergeStride;                  // [W][8][2]
+  float* cpart_o = merge_ml + kWL * 16;                                // [g][128] CTA partial
   float* cpart_ml = cpart_o + g * 128;                                // [g][2]
-  __shared__ __align__(8) uint64_t bars[kW * kR];
+  __shared__ __align__(8) uint64_t bars[kWL * kRL];
 
   cg::cluster_group cluster = cg::this_cluster();
   const int C = p.cluster;
@@ -394,20 +549,20 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
 #pragma unroll
-    for (int i = 0; i < kW * kR; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < kWL * kRL; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
-    prefetch_tensormap(&tmK);
-    prefetch_tensormap(&tmV);
+    prefetch_tensormap(&tmA);
+    if (!p.kv_single) prefetch_tensormap(&tmB);
   }
   const int t = __ldcg(p.pos + b);
   const Geom ge = make_geom(t, 0, p.sinks, p.window, p.max_pages, true);
   if (!ge.active && rank == 0 && tid == 0) atomicOr(p.err, ODA_DEVERR_POS_RANGE);
   const int nv = ge.active ? geom_pages(ge) : 0;
   const int v_lo = (int)((long long)rank * nv / C), v_hi = (int)((long long)(rank + 1) * nv / C);
-  const int cw = (v_hi - v_lo - warp > 0) ? (v_hi - v_lo - warp + kW - 1) / kW : 0;
+  const int cw = (v_hi - v_lo - warp > 0) ? (v_hi - v_lo - warp + kWL - 1) / kWL : 0;
   const int* ptab = p.page_table + (size_t)b * p.max_pages;
-  uint8_t* my_stages = stages + warp * kR * kStageBytes;
-  uint64_t* my_bars = bars + warp * kR;
+  uint8_t* my_stages = stages + warp * kRL * kStageBytes;
+  uint64_t* my_bars = bars + warp * kRL;
   __syncthreads();
 
   // lane k holds the physical page of this warp's (pt_base + k)-th page
@@ -416,7 +571,7 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     const int k = base + lane;
     pt_phys = -1;
     if (k < cw && ge.n_cache > 0) {
-      const int phys = __ldcg(ptab + geom_page(ge, v_lo + warp + k * kW));
+      const int phys = __ldcg(ptab + geom_page(ge, v_lo + warp + k * kWL));
       pt_phys = (phys >= 0 && (int64_t)phys < p.n_pool_pages) ? phys : -2;
       if (pt_phys == -2) atomicOr(p.err, ODA_DEVERR_PAGE_RANGE);
     }
@@ -425,24 +580,24 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   uint32_t vbits = 0;
   auto issue = [&](int k) {
     if (k - pt_base >= 32) refill(k & ~31);
-    const uint32_t st = (uint32_t)k % kR;
+    const uint32_t st = (uint32_t)k % kRL;
     const int phys = __shfl_sync(0xffffffffu, pt_phys, k - pt_base);
     if (lane == k - pt_base) {
       if (phys >= 0)
-        issue_page(my_stages + st * kStageBytes, my_bars + st, &tmK, &tmV, phys, p.Hkv, h);
+        issue_page(my_stages + st * kStageBytes, my_bars + st, &tmA, &tmB, p.kv_single, phys, p.Hkv, h);
       else
         mbar_arrive(my_bars + st);
     }
     vbits = phys >= 0 ? (vbits | (1u << st)) : (vbits & ~(1u << st));
   };
-  for (int k = 0; k < kR && k < cw; ++k) issue(k);
+  for (int k = 0; k < kRL && k < cw; ++k) issue(k);
   // the previous launch on the stream may still run: wait before reading q or writing
   grid_dependency_wait();
   grid_dependents_launch();
 
   uint32_t qf[8][2];
   load_qf(qf, p, b, h, lane);
-  // staged current token: its q . k words (heads warp, warp + kW) and the value this thread
+  // staged current token: its q . k words (heads warp, warp + kWL) and the value this thread
   // combines first are loaded now and used after the page loop, off the critical path
   __shared__ float s_snew[8];
   uint32_t sq[2][2] = {{0u, 0u}, {0u, 0u}};
@@ -450,7 +605,7 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   const uint32_t sk0 = krow_new[lane], sk1 = krow_new[lane + 32];
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const int n = warp + i * kW;
+    const int n = warp + i * kWL;
     if (n < g) {
       const uint32_t* qrow = p.q + ((size_t)b * p.Hq + h * g + n) * 64;
       sq[i][0] = qrow[lane];
@@ -464,24 +619,43 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   const int r = lane >> 2;
   int k = 0;
   bool dead = false;
-  for (; k < cw; ++k) {
-    const uint32_t st = (uint32_t)k % kR;
-    if (!mbar_wait_bounded(my_bars + st, ((uint32_t)k / kR) & 1u, kWaitNs)) {
+  // pages are taken two at a time (one softmax step for 32 tokens) whenever the second one has
+  // already arrived, else one at a time
+  while (k < cw) {
+    const uint32_t st = (uint32_t)k % kRL;
+    if (!mbar_wait_bounded(my_bars + st, ((uint32_t)k / kRL) & 1u, kWaitNs)) {
       if (lane == 0) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
       dead = true;
       break;
     }
-    const int lp = geom_page(ge, v_lo + warp + k * kW);
+    const int lp = geom_page(ge, v_lo + warp + k * kWL);
     const bool ok = (vbits >> st) & 1u;
     const int j0 = lp * kPageTok + r;
-    page_compute(A, qf, my_stages + st * kStageBytes, ok && geom_has(ge, j0),
-                 ok && geom_has(ge, j0 + 8), p.scale_log2, lane);
-    __syncwarp();
-    if (k + kR < cw) issue(k + kR);
+    const uint32_t st1 = (uint32_t)(k + 1) % kRL;
+    const bool pair = __all_sync(0xffffffffu, k + 1 < cw &&
+                                 mbar_try_wait(my_bars + st1, ((uint32_t)(k + 1) / kRL) & 1u));
+    if (pair) {
+      const int lp1 = geom_page(ge, v_lo + warp + (k + 1) * kWL);
+      const bool ok1 = (vbits >> st1) & 1u;
+      const int j1 = lp1 * kPageTok + r;
+      page_compute2(A, qf, my_stages + st * kStageBytes, ok && geom_has(ge, j0),
+                    ok && geom_has(ge, j0 + 8), my_stages + st1 * kStageBytes,
+                    ok1 && geom_has(ge, j1), ok1 && geom_has(ge, j1 + 8), p.scale_log2, lane);
+      __syncwarp();
+      if (k + kRL < cw) issue(k + kRL);
+      if (k + 1 + kRL < cw) issue(k + 1 + kRL);
+      k += 2;
+    } else {
+      page_compute(A, qf, my_stages + st * kStageBytes, ok && geom_has(ge, j0),
+                   ok && geom_has(ge, j0 + 8), p.scale_log2, lane);
+      __syncwarp();
+      if (k + kRL < cw) issue(k + kRL);
+      k += 1;
+    }
   }
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const int n = warp + i * kW;
+    const int n = warp + i * kWL;
     if (n < g) {
       const float acc = bf16_lo_to_f32(sq[i][0]) * bf16_lo_to_f32(sk0) +
                         bf16_hi_to_f32(sq[i][0]) * bf16_hi_to_f32(sk0) +
@@ -491,12 +665,19 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
       if (lane == 0) s_snew[n] = sn;
     }
   }
+  // a warp that gave up on a barrier first waits (bounded) for the copies it still has in
+  // flight; then every warp is done with the stages, which become the merge area
+  if (dead) {
+    for (int kk = k; kk < cw && kk < k + kRL; ++kk)
+      (void)mbar_wait_bounded(my_bars + (kk % kRL), ((uint32_t)kk / kRL) & 1u, kWaitNs);
+  }
+  __syncthreads();
   warp_flush(A, merge_o + warp * g * kMergeStride, merge_ml + warp * 16, g, lane);
   __syncthreads();
-  for (int idx = tid; idx < g * 128; idx += kThreads) {
+  for (int idx = tid; idx < g * 128; idx += kThreadsL) {
     const int n = idx >> 7, d = idx & 127;
     float M, L, O;
-    cta_merge(merge_o, merge_ml, g, n, d, M, L, O);
+    cta_merge<kWL>(merge_o, merge_ml, g, n, d, M, L, O);
     cpart_o[n * 128 + d] = O;
     if (d == 0) {
       cpart_ml[n * 2] = M;
@@ -509,7 +690,7 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
     // the g*128 outputs are shared out among the ranks, one output per thread
     const int n_out = g * 128;
     const int o_lo = (int)((long long)rank * n_out / C), o_hi = (int)((long long)(rank + 1) * n_out / C);
-    for (int idx = o_lo + tid; idx < o_hi; idx += kThreads) {
+    for (int idx = o_lo + tid; idx < o_hi; idx += kThreadsL) {
       const int n = idx >> 7, d = idx & 127;
       const float snew = s_snew[n];
       float Mr[kMaxCluster], Lr[kMaxCluster], Or[kMaxCluster];
@@ -541,15 +722,11 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant
   }
   // keep every CTA's shared memory alive until the other ranks have read it
   cluster.sync();
-  if (dead) {
-    for (int kk = k; kk < cw && kk < k + kR; ++kk)
-      (void)mbar_wait_bounded(my_bars + (kk % kR), ((uint32_t)kk / kR) & 1u, kWaitNs);
-  }
 }
 
 // ------------------------------------------------------------ full set: persistent grid
 __global__ void __launch_bounds__(kThreads, 2)
-attn_full_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = reinterpret_cast<uint8_t*>(
@@ -571,8 +748,8 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
 #pragma unroll
     for (int i = 0; i < kW * kR; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
-    prefetch_tensormap(&tmK);
-    prefetch_tensormap(&tmV);
+    prefetch_tensormap(&tmA);
+    if (!p.kv_single) prefetch_tensormap(&tmB);
   }
   // ---- per-sequence geometry and unit prefix sums (identical in every CTA)
   for (int b = tid; b < B; b += kThreads) {
@@ -708,7 +885,7 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     const uint32_t st = issued % kR;
     if (lane == src) {
       if (phys >= 0)
-        issue_page(my_stages + st * kStageBytes, my_bars + st, &tmK, &tmV, phys, Hkv, hh);
+        issue_page(my_stages + st * kStageBytes, my_bars + st, &tmA, &tmB, p.kv_single, phys, Hkv, hh);
       else
         mbar_arrive(my_bars + st);
     }
@@ -787,7 +964,7 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     for (int idx = tid; idx < g * 128; idx += kThreads) {
       const int n = idx >> 7, d = idx & 127;
       float M, L, O;
-      cta_merge(merge_o, merge_ml, g, n, d, M, L, O);
+      cta_merge<kW>(merge_o, merge_ml, g, n, d, M, L, O);
       p.part_o[((size_t)slot * g + n) * 128 + d] = O;
       if (d == 0) {
         p.part_ml[((size_t)slot * g + n) * 2] = M;
@@ -989,29 +1166,57 @@ EncodeFn get_encode() {
   return fn;
 }
 
-// Tensor map over one layer's pool seen as a 2-D array [n_pages*Hkv*16 rows][128 bf16],
-// boxes of 16 rows x 64 columns (128 bytes) with the 128-byte swizzle.
-oda_status encode_pool(CUtensorMap* m, void* base, int64_t n_pages, int Hkv) {
+// Tensor maps of one layer's pools [n_pages][Hkv][16][128] bf16, seen as rows of 128 values
+// split into two 64-value (128-byte) halves: dims {64, rows, 2} with byte strides {256, 128},
+// box {64, 16, 2}, 128-byte swizzle, so a box lands in shared memory as [half][row][64].
+// When V lies above K a fourth dimension of stride v - k selects the pool, and one
+// {64, 16, 2, 2} box brings K and V of a page together.
+oda_status encode_kv(CUtensorMap* a, CUtensorMap* b, int* single, const void* k, const void* v,
+                     int64_t n_pages, int Hkv) {
   EncodeFn enc = get_encode();
   if (!enc) return set_error(ODA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-  cuuint64_t dims[2] = {128, (cuuint64_t)n_pages * Hkv * kPageTok};
-  cuuint64_t strides[1] = {256};
-  cuuint32_t box[2] = {64, kPageTok};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return set_error(ODA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  const cuuint64_t rows = (cuuint64_t)n_pages * Hkv * kPageTok;
+  const uintptr_t ka = reinterpret_cast<uintptr_t>(k), va = reinterpret_cast<uintptr_t>(v);
+  const uint64_t kv_stride = va > ka ? (uint64_t)(va - ka) : 0;
+  cuuint32_t box[4] = {64, kPageTok, 2, 2};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  if (kv_stride > 0 && kv_stride % 16 == 0 && kv_stride < (uint64_t(1) << 40)) {
+    cuuint64_t dims[4] = {64, rows, 2, 2};
+    cuuint64_t strides[3] = {256, 128, kv_stride};
+    CUresult r = enc(a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(k), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r == CUDA_SUCCESS) {
+      *b = *a;
+      *single = 1;
+      return ODA_OK;
+    }
+  }
+  cuuint64_t dims[3] = {64, rows, 2};
+  cuuint64_t strides[2] = {256, 128};
+  const void* base[2] = {k, v};
+  CUtensorMap* m[2] = {a, b};
+  for (int i = 0; i < 2; ++i) {
+    CUresult r = enc(m[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base[i]), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+      return set_error(ODA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  }
+  *single = 0;
   return ODA_OK;
 }
 
 }  // namespace
 
-// stages | merge_o [kW][g][132] | merge_ml [kW][16] | CTA partial / combine scratch
+// stages | merge_o [W][g][132] | merge_ml [W][16] | CTA partial / combine scratch
 int attention_smem_bytes(int g) {
   const int tail = g * 130 > kW * 128 ? g * 130 : kW * 128;
   return 1024 + kStagesBytes + (kW * g * kMergeStride + kW * 16 + tail) * (int)sizeof(float);
 }
+// local set: the merge areas live in the stages (kWL * g * 132 + kWL * 16 + g * 130 floats,
+// 38 KB at g = 8, within the 192 KB of stages)
+int local_smem_bytes(int) { return 1024 + kStagesBytesL; }
 
 // Sets the shared-memory limits and returns the persistent grid size for group size g.
 oda_status prepare_attention_kernel(int g, int n_sms, int* ctas) {
@@ -1020,9 +1225,9 @@ oda_status prepare_attention_kernel(int g, int n_sms, int* ctas) {
       cudaFuncSetAttribute(attn_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
       "cudaFuncSetAttribute(full attention)");
   if (st == ODA_OK)
-    st = check_cuda(
-        cudaFuncSetAttribute(attn_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
-        "cudaFuncSetAttribute(local attention)");
+    st = check_cuda(cudaFuncSetAttribute(attn_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         local_smem_bytes(g)),
+                    "cudaFuncSetAttribute(local attention)");
   if (st != ODA_OK) return st;
   int occ = 0;
   st = check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, attn_full_kernel, kThreads, smem),
@@ -1051,12 +1256,13 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
   if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k_new) |
        reinterpret_cast<uintptr_t>(v_new) | reinterpret_cast<uintptr_t>(out)) & 3)
     return set_error(ODA_ERR_INVALID_ARG, "attention: q/k_new/v_new/out must be 4-byte aligned");
-  CUtensorMap tmK, tmV;
-  oda_status st = encode_pool(&tmK, layer->k, layer->n_pages, cf.n_kv_heads);
-  if (st != ODA_OK) return st;
-  st = encode_pool(&tmV, layer->v, layer->n_pages, cf.n_kv_heads);
+  CUtensorMap tmA, tmB;
+  int kv_single = 0;
+  oda_status st = encode_kv(&tmA, &tmB, &kv_single, layer->k, layer->v, layer->n_pages,
+                            cf.n_kv_heads);
   if (st != ODA_OK) return st;
   AttnParams p;
+  p.kv_single = kv_single;
   p.page_table = page_table;
   p.pos = pos;
   p.flag = flag;
@@ -1088,8 +1294,8 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
   // later one may start (and prefetch its pages) while the earlier one finishes; it waits
   // before reading q or writing.
   cudaLaunchConfig_t lc = {};
-  lc.blockDim = dim3(kThreads);
-  lc.dynamicSmemBytes = attention_smem_bytes(ctx->g);
+  lc.blockDim = dim3(mode == 0 ? kThreadsL : kThreads);
+  lc.dynamicSmemBytes = mode == 0 ? local_smem_bytes(ctx->g) : attention_smem_bytes(ctx->g);
   lc.stream = stream;
   cudaLaunchAttribute attr[2];
   int na = 0;
@@ -1111,8 +1317,8 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
   lc.attrs = attr;
   lc.numAttrs = na;
   st = (mode == 0)
-           ? check_cuda(cudaLaunchKernelEx(&lc, attn_local_kernel, tmK, tmV, p), "local attention launch")
-           : check_cuda(cudaLaunchKernelEx(&lc, attn_full_kernel, tmK, tmV, p), "full attention launch");
+           ? check_cuda(cudaLaunchKernelEx(&lc, attn_local_kernel, tmA, tmB, p), "local attention launch")
+           : check_cuda(cudaLaunchKernelEx(&lc, attn_full_kernel, tmA, tmB, p), "full attention launch");
   ctx->prev_attention = (st == ODA_OK);
   return st;
 }
@@ -1234,12 +1440,12 @@ oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* l
   st = check_cuda(cudaMemsetAsync(counters, 0, (2 * pairs + 1) * sizeof(int32_t), stream),
                   "cudaMemsetAsync(noalloc counters)");
   if (st != ODA_OK) return st;
-  CUtensorMap tmK, tmV;
-  st = encode_pool(&tmK, layer->k, layer->n_pages, cf.n_kv_heads);
-  if (st != ODA_OK) return st;
-  st = encode_pool(&tmV, layer->v, layer->n_pages, cf.n_kv_heads);
+  CUtensorMap tmA, tmB;
+  int kv_single = 0;
+  st = encode_kv(&tmA, &tmB, &kv_single, layer->k, layer->v, layer->n_pages, cf.n_kv_heads);
   if (st != ODA_OK) return st;
   AttnParams p;
+  p.kv_single = kv_single;
   p.page_table = page_table;
   p.pos = pos;
   p.flag = flag;
@@ -1263,7 +1469,7 @@ oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* l
   p.mode = 1;
   p.cluster = 1;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(128.0));
-  attn_full_kernel<<<d->ctas, kThreads, attention_smem_bytes(g), stream>>>(tmK, tmV, p);
+  attn_full_kernel<<<d->ctas, kThreads, attention_smem_bytes(g), stream>>>(tmA, tmB, p);
   return check_cuda(cudaGetLastError(), "noalloc full attention launch");
 }
 
