@@ -55,8 +55,7 @@ constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kMaxCluster = 8;
 constexpr int kChunk = 4;             // full set: pages per claimed chunk
 constexpr int kQueueLow = kR + kChunk;   // full set: queue length that triggers the next claim
-constexpr int kCombineQ = 10;         // partials per lane whose (m, l) loads issue together
-constexpr int kCombineRows = 16;      // partial rows per lane in flight in the output merge
+constexpr int kMergeRows = 20;        // full set: partial rows folded per round of the merge
 
 struct AttnParams {
   const int32_t* page_table;
@@ -75,6 +74,7 @@ struct AttnParams {
   int32_t B, Hq, Hkv, g, max_pages, sinks, window, mode;
   int32_t cluster;        // local set: CTAs per (b, h)
   int32_t kv_single;      // 1: tmA spans both pools (one copy per page); 0: tmA = K, tmB = V
+  int32_t cta_perm;       // full set: stride of the CTA -> range permutation (coprime to grid)
   float scale_log2;       // log2(e) / sqrt(128)
 };
 
@@ -783,9 +783,13 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   const long long U = s_us[B];
   const long long G = U < (long long)gridDim.x ? U : (long long)gridDim.x;
   int u0 = 0, u1 = 0;
-  if ((long long)blockIdx.x < G) {
-    u0 = (int)(blockIdx.x * U / G);
-    u1 = (int)((blockIdx.x + 1) * U / G);
+  // Ranges go to CTAs through the stride permutation v = c * perm mod grid (perm coprime to
+  // the grid): the CTAs covering one (b, h) are then spread over the dispatch order instead of
+  // being dispatched together, so no (b, h) is left to the CTAs that start last.
+  const int vc = (int)(((long long)blockIdx.x * p.cta_perm) % gridDim.x);
+  if ((long long)vc < G) {
+    u0 = (int)(vc * U / G);
+    u1 = (int)((vc + 1) * U / G);
   }
   uint8_t* my_stages = stages + warp * kR * kStageBytes;
   uint64_t* my_bars = bars + warp * kR;
@@ -819,7 +823,7 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const long long cfs = (s0 * G + U - 1) / U;
     const long long cfe = min(G, (s1 * G + U - 1) / U);
     is_base = (int)(cfe - cfs) * kW;
-    is_fixed = first ? (int)((long long)blockIdx.x - cfs) * kW + warp : -1;
+    is_fixed = first ? (int)((long long)vc - cfs) * kW + warp : -1;
     has_pend = false;
     if (claims_ok) {
       if (lane == 0) pend = atomicAdd(p.claims + is_bh, 1);
@@ -960,7 +964,7 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     __syncthreads();
     // ---- merge the warps into this segment's partial (one per query head of the group)
     const int bh = b * Hkv + h;
-    const int slot = (int)blockIdx.x + bh;
+    const int slot = vc + bh;
     for (int idx = tid; idx < g * 128; idx += kThreads) {
       const int n = idx >> 7, d = idx & 127;
       float M, L, O;
@@ -983,123 +987,125 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
     __syncthreads();
     if (s_last) {
-      // ---- last CTA of (b, h): merge the partials and the staged current token.  The merge
-      // reads nparts x g partials from L2; every load of a phase is issued before its first
-      // use, so the phase costs a few L2 round trips whatever nparts is.
+      // ---- last CTA of (b, h): merge the nparts partials and the staged current token in one
+      // online pass.  Each round loads kMergeRows partial rows of a head together with their
+      // (m, l) and folds them into a running (M, L, O), so nparts = 37 costs two L2 round trips.
       const int slot0 = c_first + bh;
-      float* s_w = merge_o;                  // [g][nparts] weights; nparts <= grid size
-      float* s_fin = merge_ml;               // [g][2]: 1 / L, weight of the staged token
-      float* s_red = cpart_o;                // [kW][128] per-warp sums (g < kW)
-      for (int n = warp; n < g; n += kW) {
-        float ms[kCombineQ], ls[kCombineQ];
-#pragma unroll
-        for (int q = 0; q < kCombineQ; ++q) {
-          const int s = lane + 32 * q;
-          ms[q] = -INFINITY;
-          ls[q] = 0.f;
-          if (s < nparts) {
-            const size_t pi = (size_t)(slot0 + s) * g + n;
-            ms[q] = __ldcg(p.part_ml + pi * 2);
-            ls[q] = __ldcg(p.part_ml + pi * 2 + 1);
-          }
-        }
-        const float snew = staged_score(p, b, h, n, lane);
-        float M = snew;
-#pragma unroll
-        for (int q = 0; q < kCombineQ; ++q) M = fmaxf(M, ms[q]);
-        for (int s = lane + 32 * kCombineQ; s < nparts; s += 32)
-          M = fmaxf(M, __ldcg(p.part_ml + ((size_t)(slot0 + s) * g + n) * 2));
-#pragma unroll
-        for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
-        float L = 0.f;
-#pragma unroll
-        for (int q = 0; q < kCombineQ; ++q) {
-          const int s = lane + 32 * q;
-          if (s < nparts) {
-            const float w = (ms[q] == -INFINITY) ? 0.f : exp2f(ms[q] - M);
-            s_w[n * nparts + s] = w;
-            L += w * ls[q];
-          }
-        }
-        for (int s = lane + 32 * kCombineQ; s < nparts; s += 32) {
-          const size_t pi = (size_t)(slot0 + s) * g + n;
-          const float m2 = __ldcg(p.part_ml + pi * 2);
-          const float w = (m2 == -INFINITY) ? 0.f : exp2f(m2 - M);
-          s_w[n * nparts + s] = w;
-          L += w * __ldcg(p.part_ml + pi * 2 + 1);
-        }
-        L = warp_sum(L);
-        const float wnew = exp2f(snew - M);
-        if (lane == 0) {
-          s_fin[n * 2] = 1.0f / (L + wnew);
-          s_fin[n * 2 + 1] = wnew;
-        }
-      }
-      __syncthreads();
-      // O: a warp per head (heads n, n + kW, ... when g > kW; kW / g warps share a head's
-      // partials when g < kW); lane l holds dims 4l..4l+3; kCombineRows rows in flight.
-      // (g = 3: warps 0..2 take one head each, warp 3 idles)
-      const int wph = g >= kW ? 1 : kW / g;
-      const int n_first = g >= kW ? warp : warp % g;
-      const int sub = g >= kW ? 0 : warp / g;
-      const size_t rs = (size_t)g * 32;       // float4 stride between consecutive partials
-      for (int n = n_first; n < g && sub < wph; n += kW) {
-        const float* wn = s_w + n * nparts;
+      const size_t rs = (size_t)g * 32;   // float4 stride between partial rows
+      // (M, L, O) of head n over the partials s = sub, sub + step, ... (lane l: dims 4l..4l+3)
+      auto fold = [&](int n, int sub, int step, float& M, float& L, float4& acc) {
         const float4* base =
             reinterpret_cast<const float4*>(p.part_o + ((size_t)slot0 * g + n) * 128) + lane;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s0 = sub; s0 < nparts; s0 += kCombineRows * wph) {
-          float4 v[kCombineRows];
-#pragma unroll
-          for (int j = 0; j < kCombineRows; ++j) {
-            const int s = s0 + j * wph;
-            v[j] = s < nparts ? __ldcg(base + (size_t)s * rs) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float* mlb = p.part_ml + ((size_t)slot0 * g + n) * 2;
+        M = -INFINITY;
+        L = 0.f;
+        acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s0 = sub; s0 < nparts; s0 += kMergeRows * step) {
+          float4 v[kMergeRows];
+          const int sj = s0 + lane * step;   // lane j < kMergeRows holds (m, l) of row j
+          float mj = -INFINITY, lj = 0.f;
+          if (lane < kMergeRows && sj < nparts) {
+            mj = __ldcg(mlb + (size_t)sj * g * 2);
+            lj = __ldcg(mlb + (size_t)sj * g * 2 + 1);
           }
 #pragma unroll
-          for (int j = 0; j < kCombineRows; ++j) {
-            const int s = s0 + j * wph;
-            const float w = s < nparts ? wn[s] : 0.f;
+          for (int j = 0; j < kMergeRows; ++j) {
+            const int sr = s0 + j * step;
+            v[j] = sr < nparts ? __ldcg(base + (size_t)sr * rs) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          float mb = mj;
+#pragma unroll
+          for (int o2 = 16; o2 > 0; o2 >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o2));
+          const float Mn = fmaxf(M, mb);
+          if (Mn == -INFINITY) continue;   // no tokens so far (empty partials)
+          const float sc = (M == -INFINITY) ? 0.f : exp2f(M - Mn);
+          const float wj = (mj == -INFINITY) ? 0.f : exp2f(mj - Mn);
+          acc.x *= sc;
+          acc.y *= sc;
+          acc.z *= sc;
+          acc.w *= sc;
+          L = L * sc + warp_sum(wj * lj);
+#pragma unroll
+          for (int j = 0; j < kMergeRows; ++j) {
+            const float w = __shfl_sync(0xffffffffu, wj, j);
             acc.x += w * v[j].x;
             acc.y += w * v[j].y;
             acc.z += w * v[j].z;
             acc.w += w * v[j].w;
           }
+          M = Mn;
         }
-        if (wph > 1) reinterpret_cast<float4*>(s_red + warp * 128)[lane] = acc;
-        if (wph == 1) {
-          const float wnew = s_fin[n * 2 + 1], inv = s_fin[n * 2];
-          const uint32_t* vp = p.v_new + ((size_t)b * p.Hkv + h) * 64 + 2 * lane;
-          const uint32_t v01 = vp[0], v23 = vp[1];
-          float4 o;
-          o.x = (acc.x + wnew * bf16_lo_to_f32(v01)) * inv;
-          o.y = (acc.y + wnew * bf16_hi_to_f32(v01)) * inv;
-          o.z = (acc.z + wnew * bf16_lo_to_f32(v23)) * inv;
-          o.w = (acc.w + wnew * bf16_hi_to_f32(v23)) * inv;
-          reinterpret_cast<float4*>(p.out + ((size_t)b * p.Hq + h * g + n) * 128)[lane] = o;
+      };
+      // the staged current token of head n: its words are loaded before the partial rounds
+      struct Staged { uint32_t qa0, qa1, ka0, ka1, v01, v23; };
+      auto staged_words = [&](int n) {
+        const uint32_t* qrow = p.q + ((size_t)b * p.Hq + h * g + n) * 64;
+        const uint32_t* krow = p.k_new + ((size_t)b * p.Hkv + h) * 64;
+        const uint32_t* vp = p.v_new + ((size_t)b * p.Hkv + h) * 64 + 2 * lane;
+        return Staged{qrow[lane], qrow[lane + 32], krow[lane], krow[lane + 32], vp[0], vp[1]};
+      };
+      // adds the staged current token of head n and writes the output row
+      auto finish = [&](int n, const Staged& sw, float M, float L, float4 acc) {
+        const uint32_t qa0 = sw.qa0, qa1 = sw.qa1, ka0 = sw.ka0, ka1 = sw.ka1;
+        const uint32_t v01 = sw.v01, v23 = sw.v23;
+        const float snew = warp_sum(bf16_lo_to_f32(qa0) * bf16_lo_to_f32(ka0) +
+                                    bf16_hi_to_f32(qa0) * bf16_hi_to_f32(ka0) +
+                                    bf16_lo_to_f32(qa1) * bf16_lo_to_f32(ka1) +
+                                    bf16_hi_to_f32(qa1) * bf16_hi_to_f32(ka1)) * p.scale_log2;
+        const float Mf = fmaxf(M, snew);
+        const float wa = (M == -INFINITY) ? 0.f : exp2f(M - Mf), wn = exp2f(snew - Mf);
+        const float inv = 1.0f / (L * wa + wn);
+        float4 o;
+        o.x = (acc.x * wa + wn * bf16_lo_to_f32(v01)) * inv;
+        o.y = (acc.y * wa + wn * bf16_hi_to_f32(v01)) * inv;
+        o.z = (acc.z * wa + wn * bf16_lo_to_f32(v23)) * inv;
+        o.w = (acc.w * wa + wn * bf16_hi_to_f32(v23)) * inv;
+        reinterpret_cast<float4*>(p.out + ((size_t)b * p.Hq + h * g + n) * 128)[lane] = o;
+      };
+      if (g >= kW) {
+        // a warp per head: heads warp, warp + kW, ...
+        for (int n = warp; n < g; n += kW) {
+          const Staged sw = staged_words(n);
+          float M, L;
+          float4 acc;
+          fold(n, 0, 1, M, L, acc);
+          finish(n, sw, M, L, acc);
         }
-      }
-      if (wph > 1) {
+      } else {
+        // kW / g warps share a head's partials, then warp n (< g) combines them
+        // (g = 3: warps 0..2 take one head each, warp 3 idles)
+        const int wph = kW / g, n = warp % g, sub = warp / g;
+        const Staged sw = staged_words(n);
+        float* s_red = cpart_o;   // [kW][132]: O (128), M, L
+        float M = -INFINITY, L = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (sub < wph) fold(n, sub, wph, M, L, acc);
+        reinterpret_cast<float4*>(s_red + warp * 132)[lane] = acc;
+        if (lane == 0) {
+          s_red[warp * 132 + 128] = M;
+          s_red[warp * 132 + 129] = L;
+        }
         __syncthreads();
-        // warps w < g sum the kW / g rows of head w (rows w, w + g, ...)
         if (warp < g) {
-          const int n = warp;
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int k = 0; k < wph; ++k) {
-            const float4 r = reinterpret_cast<const float4*>(s_red + (k * g + n) * 128)[lane];
-            acc.x += r.x;
-            acc.y += r.y;
-            acc.z += r.z;
-            acc.w += r.w;
+          float Mt = -INFINITY;
+          for (int k2 = 0; k2 < wph; ++k2) Mt = fmaxf(Mt, s_red[(k2 * g + warp) * 132 + 128]);
+          float Lt = 0.f;
+          float4 at = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (Mt != -INFINITY) {
+            for (int k2 = 0; k2 < wph; ++k2) {
+              const float* r = s_red + (k2 * g + warp) * 132;
+              const float mk = r[128];
+              if (mk == -INFINITY) continue;
+              const float w = exp2f(mk - Mt);
+              const float4 rv = reinterpret_cast<const float4*>(r)[lane];
+              at.x += w * rv.x;
+              at.y += w * rv.y;
+              at.z += w * rv.z;
+              at.w += w * rv.w;
+              Lt += w * r[129];
+            }
           }
-          const float wnew = s_fin[n * 2 + 1], inv = s_fin[n * 2];
-          const uint32_t* vp = p.v_new + ((size_t)b * p.Hkv + h) * 64 + 2 * lane;
-          const uint32_t v01 = vp[0], v23 = vp[1];
-          float4 o;
-          o.x = (acc.x + wnew * bf16_lo_to_f32(v01)) * inv;
-          o.y = (acc.y + wnew * bf16_hi_to_f32(v01)) * inv;
-          o.z = (acc.z + wnew * bf16_lo_to_f32(v23)) * inv;
-          o.w = (acc.w + wnew * bf16_hi_to_f32(v23)) * inv;
-          reinterpret_cast<float4*>(p.out + ((size_t)b * p.Hq + h * g + n) * 128)[lane] = o;
+          finish(warp, sw, Mt, Lt, at);
         }
       }
       if (tid == 0) {
@@ -1209,9 +1215,24 @@ oda_status encode_kv(CUtensorMap* a, CUtensorMap* b, int* single, const void* k,
 
 }  // namespace
 
+// Stride of the full-set CTA -> range permutation: near a quarter of the grid, coprime to it.
+int cta_stride(int grid) {
+  if (grid <= 2) return 1;
+  for (int k = grid / 4 + 1; k < grid; ++k) {
+    int a = k, b = grid;
+    while (b) {
+      const int t = a % b;
+      a = b;
+      b = t;
+    }
+    if (a == 1) return k;
+  }
+  return 1;
+}
+
 // stages | merge_o [W][g][132] | merge_ml [W][16] | CTA partial / combine scratch
 int attention_smem_bytes(int g) {
-  const int tail = g * 130 > kW * 128 ? g * 130 : kW * 128;
+  const int tail = g * 130 > kW * 132 ? g * 130 : kW * 132;
   return 1024 + kStagesBytes + (kW * g * kMergeStride + kW * 16 + tail) * (int)sizeof(float);
 }
 // local set: the merge areas live in the stages (kWL * g * 132 + kWL * 16 + g * 130 floats,
@@ -1263,6 +1284,7 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
   if (st != ODA_OK) return st;
   AttnParams p;
   p.kv_single = kv_single;
+  p.cta_perm = 1;
   p.page_table = page_table;
   p.pos = pos;
   p.flag = flag;
@@ -1285,8 +1307,8 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
   p.window = cf.window;
   p.mode = mode;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(128.0));
-  // cluster size of the local kernel: about one CTA per SM (at most 8 per (b, h)), so that
-  // the CTAs of the next layer's launch fit beside this one's and prefetch while it finishes
+  // cluster size of the local kernel: about one CTA per SM (each CTA's page rings take most of
+  // an SM's shared memory), at most 8 per (b, h)
   const int pairs = cf.batch * cf.n_kv_heads;
   p.cluster = std::max(1, std::min(kMaxCluster, ctx->n_sms / pairs));
 
@@ -1313,6 +1335,7 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
     lc.gridDim = dim3(pairs * p.cluster);
   } else {
     lc.gridDim = dim3(ctx->attn_ctas);
+    p.cta_perm = cta_stride(ctx->attn_ctas);
   }
   lc.attrs = attr;
   lc.numAttrs = na;
@@ -1446,6 +1469,7 @@ oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* l
   if (st != ODA_OK) return st;
   AttnParams p;
   p.kv_single = kv_single;
+  p.cta_perm = 1;
   p.page_table = page_table;
   p.pos = pos;
   p.flag = flag;
@@ -1469,6 +1493,7 @@ oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* l
   p.mode = 1;
   p.cluster = 1;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(128.0));
+  p.cta_perm = cta_stride(d->ctas);
   attn_full_kernel<<<d->ctas, kThreads, attention_smem_bytes(g), stream>>>(tmA, tmB, p);
   return check_cuda(cudaGetLastError(), "noalloc full attention launch");
 }
