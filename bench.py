@@ -33,7 +33,7 @@ METRIC = "ODA decode-attn steps/s + % of HBM peak, 128K ctx, 12.5% recall, 1 B20
 # profiles/attn_full_kernel_cfg2_ctx32k_l2.md (4 flagged sequences x 32768 cached tokens); the
 # bench scales it to its own launches by cached tokens processed.  Valid only for the kernel
 # source it was taken from (first 16 hex digits of the file's SHA-256).
-NCU_FULL_KERNEL_TRAFFIC = {"attention_cu_sha256": "0f1765d626426219", "bytes": 541386496,
+NCU_FULL_KERNEL_TRAFFIC = {"attention_cu_sha256": "2fef1cc4a049eebe", "bytes": 541111040,
                            "cached_tokens": 4 * 32768}
 UNIT = "steps/s"
 FALLBACK_HBM_GBS = 6650.0

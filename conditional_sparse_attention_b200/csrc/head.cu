@@ -231,34 +231,51 @@ __global__ void __launch_bounds__(kHT) head_phase_kernel(const HeadParams p) {
   const float* wrow[kRowsPerWarp];
 #pragma unroll
   for (int r = 0; r < kRowsPerWarp; ++r) wrow[r] = weight_row(p, rb, warp, r, &cols[r]) + k0;
-  // The weights never change: pull this CTA's slab toward L2 while the previous phase may
-  // still be running (programmatic dependent launch), then wait for its outputs.
+  // The weights never change: pull this CTA's slab toward L2 and load the first two rounds of
+  // it into registers while the previous phase may still be running (programmatic dependent
+  // launch), then wait for its outputs.
+  const bool single_pass = p.B <= kBT;
+  const int n4 = p.Kc / 4;   // >= 64 in every phase: two rounds of 32 lanes
+  float4 wa[kRowsPerWarp], wb[kRowsPerWarp];
+  auto load_w = [&](float4 (&w)[kRowsPerWarp], int k4) {
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r) w[r] = ldg_w(wrow[r] + 4 * k4, single_pass);
+  };
   for (int r = 0; r < kRowsPerWarp; ++r)
-    for (int k = lane * 32; k < p.Kc; k += 32 * 32)
+    for (int k = lane * 32 + 256; k < p.Kc; k += 32 * 32)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(wrow[r] + k));
+  load_w(wa, lane);
+  load_w(wb, lane + 32);
   grid_dependency_wait();
   grid_dependents_launch();
 
-  const bool single_pass = p.B <= kBT;
   for (int b0 = 0; b0 < p.B; b0 += kBT) {
+    if (b0 > 0) {   // later sequence tiles read the slab again
+      load_w(wa, lane);
+      load_w(wb, lane + 32);
+    }
     build_tile(p, rb, chunk, b0, X, p.ss, red);
     float acc[kRowsPerWarp][kBT];
 #pragma unroll
     for (int r = 0; r < kRowsPerWarp; ++r)
 #pragma unroll
       for (int bb = 0; bb < kBT; ++bb) acc[r][bb] = 0.f;
-    const int n4 = p.Kc / 4;
-#pragma unroll 2
-    for (int k4 = lane; k4 < n4; k4 += 32) {
-      float4 wv[kRowsPerWarp];
-#pragma unroll
-      for (int r = 0; r < kRowsPerWarp; ++r) wv[r] = ldg_w(wrow[r] + 4 * k4, single_pass);
+    auto fma_w = [&](const float4 (&w)[kRowsPerWarp], int k4) {
 #pragma unroll
       for (int bb = 0; bb < kBT; ++bb) {
         const float4 xv = *reinterpret_cast<const float4*>(X + bb * p.Kc + 4 * k4);
 #pragma unroll
         for (int r = 0; r < kRowsPerWarp; ++r)
-          acc[r][bb] += wv[r].x * xv.x + wv[r].y * xv.y + wv[r].z * xv.z + wv[r].w * xv.w;
+          acc[r][bb] += w[r].x * xv.x + w[r].y * xv.y + w[r].z * xv.z + w[r].w * xv.w;
+      }
+    };
+    // two register buffers, each refilled two rounds ahead of its use
+    for (int k4 = lane; k4 < n4; k4 += 64) {
+      fma_w(wa, k4);
+      if (k4 + 64 < n4) load_w(wa, k4 + 64);
+      if (k4 + 32 < n4) {
+        fma_w(wb, k4 + 32);
+        if (k4 + 96 < n4) load_w(wb, k4 + 96);
       }
     }
     // butterfly: after 5 stages lane l holds the lane-sum of value l = (r = l / 8, bb = l % 8)
