@@ -215,6 +215,15 @@ def cpu_cores() -> int:
     return len(os.sched_getaffinity(0))
 
 
+def workload_config(wl, world: int, eager: bool) -> dict:
+    """The `config` object of both arms' JSON lines (the workload and how the GPU arm runs it)."""
+    return {"workload": wl.name, "B": wl.B, "layers": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv,
+            "head_dim": 128, "ctx": wl.ctx[0], "recall_rate": wl.rates[0] if wl.rates else None,
+            "page_tokens": 16, "parallelism": f"replicas{world}",
+            "l2": "inputs larger than L2 (77 GB resident KV cache), no flush",
+            "launch": "eager" if eager else "cuda-graph with conditional IF node"}
+
+
 def run_reference(args, wl, rank, world):
     if rank != 0:
         return
@@ -230,8 +239,7 @@ def run_reference(args, wl, rank, world):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000.0 / value, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "B": wl.B, "layers": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv,
-                       "ctx": wl.ctx[0], "recall_rate": wl.rates[0] if wl.rates else None},
+            "config": workload_config(wl, world, args.eager),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -426,6 +434,7 @@ def run_ours(args, wl, rank, world, local_rank):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(dec.stream):
             e0.record(dec.stream)
+            dec.copy_stream.wait_event(e0)   # every upload of the timed steps starts after e0
             for i in range(n_e2e):
                 dec.step(host[i % n_store])
                 out_h.copy_(dec.h_prev, non_blocking=True)
@@ -453,11 +462,7 @@ def run_ours(args, wl, rank, world, local_rank):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": wl.name, "B": wl.B, "layers": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv,
-                       "head_dim": 128, "ctx": wl.ctx[0], "recall_rate": wl.rates[0],
-                       "page_tokens": 16, "parallelism": f"replicas{world}",
-                       "l2": "inputs larger than L2 (77 GB resident KV cache), no flush",
-                       "launch": "eager" if args.eager else "cuda-graph with conditional IF node"},
+            "config": workload_config(wl, world, args.eager),
             "roofline": {"bound": "hbm", "achieved": full_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": full_gbs / hbm, "traffic": full_traffic,
                          "algorithmic_bytes_per_launch": full_bytes / n_pat_launches,

@@ -129,8 +129,17 @@ class OdaDecoder:
         self.flag = torch.zeros(B, dtype=torch.int32, device=dev)
         self.any_flag = torch.zeros(1, dtype=torch.int32, device=dev)
         self.layout = StepLayout(wl)
-        self.staging = torch.zeros(self.layout.nbytes, dtype=torch.uint8, device=dev)
-        self.sv = self.layout.views(self.staging)
+        # Two staging buffers, used by alternate steps (and one captured graph each): host inputs
+        # of step i + 1 are uploaded on a copy stream into the buffer step i does not read, so
+        # the upload overlaps step i's kernels.
+        self.staging = [torch.zeros(self.layout.nbytes, dtype=torch.uint8, device=dev)
+                        for _ in range(2)]
+        self.svs = [self.layout.views(b) for b in self.staging]
+        self.slot = 0
+        self._n_staged = 0
+        self.copy_stream = torch.cuda.Stream(dev)
+        self.staged = [torch.cuda.Event() for _ in range(2)]
+        self.released = [torch.cuda.Event() for _ in range(2)]
         self.routing_scheduled = wl.routing == "bernoulli"
         if wl.hybrid:
             S0, C0 = inputs.gdn_state0(wl)
@@ -151,11 +160,29 @@ class OdaDecoder:
         fill_step_inputs(self.wl, step, self.layout.views(buf))
         return buf
 
+    @property
+    def sv(self) -> dict:
+        """Views of the staging buffer of the most recently staged step."""
+        return self.svs[self.slot]
+
     def stage(self, src: torch.Tensor) -> None:
-        """Copies one step's input buffer (device or pinned host) into the staging area."""
+        """Copies one step's input buffer into the next staging buffer.  A device buffer is
+        copied in the step stream's order; a (pinned) host buffer is uploaded on the copy stream
+        once the step that last read that staging buffer has run, so the upload overlaps the
+        previous step.  The caller keeps a host buffer unchanged until its step has run."""
+        self.slot = self._n_staged % 2
+        self._n_staged += 1
+        i, dst = self.slot, self.staging[self.slot]
         self.stream.wait_stream(torch.cuda.current_stream(self.device))
-        with torch.cuda.stream(self.stream):
-            self.staging.copy_(src, non_blocking=True)
+        if src.is_cuda:
+            with torch.cuda.stream(self.stream):
+                dst.copy_(src, non_blocking=True)
+            return
+        self.copy_stream.wait_event(self.released[i])
+        with torch.cuda.stream(self.copy_stream):
+            dst.copy_(src, non_blocking=True)
+            self.staged[i].record(self.copy_stream)
+        self.stream.wait_event(self.staged[i])
 
     # ------------------------------------------------------------------ step
     def issue(self) -> None:
@@ -202,24 +229,35 @@ class OdaDecoder:
                        self.h_prev, s)
 
     def capture(self) -> None:
-        """Records one step (with the retry under a conditional node) as a CUDA graph."""
+        """Records one step (with the retry under a conditional node) as a CUDA graph, once per
+        staging buffer."""
         torch.cuda.synchronize(self.device)
-        oda.oda_graph_begin(self.stream)
-        try:
-            self.issue()
-        except Exception:
+        graphs, slot = [], self.slot
+        for i in range(2):
+            self.slot = i
+            oda.oda_graph_begin(self.stream)
             try:
-                oda.oda_graph_end(self.stream).close()
+                self.issue()
             except Exception:
-                pass
-            raise
-        self.graph = oda.oda_graph_end(self.stream)
+                try:
+                    oda.oda_graph_end(self.stream).close()
+                except Exception:
+                    pass
+                for g in graphs:
+                    g.close()
+                self.slot = slot
+                raise
+            graphs.append(oda.oda_graph_end(self.stream))
+        self.slot = slot
+        self.graph = graphs
 
     def launch(self) -> None:
+        """Runs one step on the most recently staged inputs."""
         if self.graph is not None:
-            self.graph.launch(self.stream)
+            self.graph[self.slot].launch(self.stream)
         else:
             self.issue()
+        self.released[self.slot].record(self.stream)
 
     def step(self, src: torch.Tensor = None) -> None:
         if src is not None:
@@ -238,6 +276,7 @@ class OdaDecoder:
 
     def close(self):
         if self.graph is not None:
-            self.graph.close()
+            for g in self.graph:
+                g.close()
             self.graph = None
         self.ctx.close()
