@@ -420,7 +420,7 @@ def run_ours(args, wl, rank, world, local_rank):
     loc_gbs = loc_bytes / (loc_ms * 1e-3) / 1e9
 
     # ---------------- end to end: pinned host inputs -> H2D, step, D2H of the results
-    e2e = None
+    e2e = e2e_detail = None
     if args.e2e:
         host = [b.cpu().pin_memory() for b in store]
         out_h = torch.empty((wl.B, wl.D), dtype=torch.float32).pin_memory()
@@ -435,17 +435,61 @@ def run_ours(args, wl, rank, world, local_rank):
         with torch.cuda.stream(dec.stream):
             e0.record(dec.stream)
             dec.copy_stream.wait_event(e0)   # every upload of the timed steps starts after e0
+            h0 = time.perf_counter()
             for i in range(n_e2e):
                 dec.step(host[i % n_store])
                 out_h.copy_(dec.h_prev, non_blocking=True)
                 out_f.copy_(dec.flag, non_blocking=True)
                 out_s.copy_(dec.score, non_blocking=True)
+            host_issue_s = time.perf_counter() - h0
             e1.record(dec.stream)
         torch.cuda.synchronize(dev)
         e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         e2e = {"value": world * n_e2e / (e_ms * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": dec.layout.nbytes,
                "d2h_bytes_per_step": out_h.numel() * 4 + out_f.numel() * 4 + out_s.numel() * 4}
+        # the copies alone, for reading the end-to-end number: uploads back to back on the copy
+        # stream, and the read-backs on the step stream
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(dec.copy_stream):
+            c0.record(dec.copy_stream)
+            for i in range(n_e2e):
+                dec.staging[i % 2].copy_(host[i % n_store], non_blocking=True)
+            c1.record(dec.copy_stream)
+        c1.synchronize()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(dec.stream):
+            d0.record(dec.stream)
+            for i in range(n_e2e):
+                out_h.copy_(dec.h_prev, non_blocking=True)
+                out_f.copy_(dec.flag, non_blocking=True)
+                out_s.copy_(dec.score, non_blocking=True)
+            d1.record(dec.stream)
+        d1.synchronize()
+        e2e_detail = {"upload_us_per_step": c0.elapsed_time(c1) * 1e3 / n_e2e,
+                      "upload_gbs": dec.layout.nbytes * n_e2e / (c0.elapsed_time(c1) * 1e-3) / 1e9,
+                      "readback_us_per_step": d0.elapsed_time(d1) * 1e3 / n_e2e,
+                      "host_issue_us_per_step": host_issue_s * 1e6 / n_e2e,
+                      "step_us": e_ms * 1e3 / n_e2e}
+    # ---------------- a step with no flagged sequence (the IF node skips the retry): what the
+    # local pass and the head leave to the glue (hidden-state sums, commit, condition node)
+    quiet = dec.make_step_buffer(0)
+    dec.layout.views(quiet)["sched"].zero_()
+    if dec.routing_scheduled:
+        dec.step(quiet)
+        dec.synchronize()
+        q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        q0.record(dec.stream)
+        for _ in range(2):
+            dec.step(quiet)
+        q1.record(dec.stream)
+        q1.synchronize()
+        quiet_us = q0.elapsed_time(q1) * 1e3 / 2
+        step_detail = {"unflagged_step_us": quiet_us, "local_pass_us": loc_ms * 1e3 * wl.L,
+                       "head_us": head_ms * 1e3,
+                       "glue_us": quiet_us - loc_ms * 1e3 * wl.L - head_ms * 1e3}
+    else:
+        step_detail = None
     err = dec.device_error()
 
     cpu = None
@@ -480,7 +524,8 @@ def run_ours(args, wl, rank, world, local_rank):
             "realized_recall_rate": realized_rate,
             "first_step_ms_incl_capture": first_ms, "setup_s": setup_s,
             "gpu_launches": launches, "device_error": err,
-            "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
+            "clocks": clocks, "e2e": e2e, "e2e_detail": e2e_detail, "step_detail": step_detail,
+            "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
     dec.close()

@@ -28,7 +28,7 @@ class OdaConfig(ctypes.Structure):
     _fields_ = [("batch", c_int32), ("n_q_heads", c_int32), ("n_kv_heads", c_int32),
                 ("head_dim", c_int32), ("page_size", c_int32), ("max_pages", c_int32),
                 ("sinks", c_int32), ("window", c_int32), ("head_in_dim", c_int32),
-                ("theta", c_float), ("overlap_layers", c_int32)]
+                ("theta", c_float), ("overlap_layers", c_int32), ("deterministic", c_int32)]
 
 
 class OdaKVLayer(ctypes.Structure):

@@ -112,6 +112,8 @@ oda_status oda_create(const oda_config* cfg, oda_ctx** out) {
   if (c.window < 1) return set_error(ODA_ERR_INVALID_ARG, "create: window must be >= 1");
   if (c.head_in_dim < 512 || c.head_in_dim > 8192 || c.head_in_dim % 512 != 0)
     return set_error(ODA_ERR_UNSUPPORTED, "create: head_in_dim must be a multiple of 512 in 512..8192");
+  if ((c.overlap_layers != 0 && c.overlap_layers != 1) || (c.deterministic != 0 && c.deterministic != 1))
+    return set_error(ODA_ERR_INVALID_ARG, "create: overlap_layers and deterministic must be 0 or 1");
 
   oda_ctx* x = new oda_ctx();
   x->cfg = c;

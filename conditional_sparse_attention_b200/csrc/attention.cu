@@ -75,6 +75,7 @@ struct AttnParams {
   int32_t cluster;        // local set: CTAs per (b, h)
   int32_t kv_single;      // 1: tmA spans both pools (one copy per page); 0: tmA = K, tmB = V
   int32_t cta_perm;       // full set: stride of the CTA -> range permutation (coprime to grid)
+  int32_t deterministic;  // full set: chunks in a fixed pattern instead of run-time claims
   float scale_log2;       // log2(e) / sqrt(128)
 };
 
@@ -619,11 +620,14 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   const int r = lane >> 2;
   int k = 0;
   bool dead = false;
-  // pages are taken two at a time (one softmax step for 32 tokens) whenever the second one has
-  // already arrived, else one at a time
+  // pages are taken two at a time (one softmax step for 32 tokens), in fixed pairs so that the
+  // rounding never depends on when a copy lands; an odd last page goes alone
   while (k < cw) {
     const uint32_t st = (uint32_t)k % kRL;
-    if (!mbar_wait_bounded(my_bars + st, ((uint32_t)k / kRL) & 1u, kWaitNs)) {
+    const bool pair = k + 1 < cw;
+    const uint32_t st1 = (uint32_t)(k + 1) % kRL;
+    if (!mbar_wait_bounded(my_bars + st, ((uint32_t)k / kRL) & 1u, kWaitNs) ||
+        (pair && !mbar_wait_bounded(my_bars + st1, ((uint32_t)(k + 1) / kRL) & 1u, kWaitNs))) {
       if (lane == 0) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
       dead = true;
       break;
@@ -631,9 +635,6 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     const int lp = geom_page(ge, v_lo + warp + k * kWL);
     const bool ok = (vbits >> st) & 1u;
     const int j0 = lp * kPageTok + r;
-    const uint32_t st1 = (uint32_t)(k + 1) % kRL;
-    const bool pair = __all_sync(0xffffffffu, k + 1 < cw &&
-                                 mbar_try_wait(my_bars + st1, ((uint32_t)(k + 1) / kRL) & 1u));
     if (pair) {
       const int lp1 = geom_page(ge, v_lo + warp + (k + 1) * kWL);
       const bool ok1 = (vbits >> st1) & 1u;
@@ -808,6 +809,7 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   // claim side (warp-uniform; `pend` lives in lane 0)
   int is_seg = 0, is_u = u0, is_b = 0, is_h = 0, is_bh = 0, is_nv = 0, is_ncache = 0;
   int is_nch = 0, is_base = 0, is_fixed = -1, pend = 0;
+  int is_rank = 0, is_nc = 1, is_next = 0;   // fixed pattern: rank among covering CTAs, count, cursor
   bool is_done = u0 >= u1, claims_ok = false, has_pend = false;
   auto enter_seg = [&](bool first) {
     const Seg cs_ = decode_seg(is_u, u1, s_us, s_nv, B, Hkv);
@@ -825,6 +827,15 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     is_base = (int)(cfe - cfs) * kW;
     is_fixed = first ? (int)((long long)vc - cfs) * kW + warp : -1;
     has_pend = false;
+    if (p.deterministic) {
+      // fixed pattern: chunk j goes to covering CTA j % nc, and within it to warp (j / nc) % kW
+      const int c0 = cta_of(cs_.s0, U, G), c1 = cta_of(s1 - 1, U, G);
+      is_nc = c1 - c0 + 1;
+      is_rank = vc - c0;
+      is_next = 0;
+      is_fixed = -1;
+      return;
+    }
     if (claims_ok) {
       if (lane == 0) pend = atomicAdd(p.claims + is_bh, 1);
       has_pend = true;
@@ -850,9 +861,25 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
     f_tail += (uint32_t)np;
   };
+  auto next_segment = [&]() {
+    is_u += decode_seg(is_u, u1, s_us, s_nv, B, Hkv).n;
+    ++is_seg;
+    if (is_u >= u1) is_done = true;
+    else enter_seg(false);
+  };
   // queue one more chunk, or move the claim side to the next segment
   auto top_up = [&]() {
     if (is_done || dead || f_tail - f_head >= (uint32_t)kQueueLow) return;
+    if (p.deterministic) {   // this warp's i-th chunk is rank + nc * (warp + kW * i)
+      const int c = is_rank + is_nc * (warp + kW * is_next);
+      if (c < is_nch) {
+        ++is_next;
+        push_chunk(c);
+      } else {
+        next_segment();
+      }
+      return;
+    }
     if (is_fixed >= 0) {
       const int c = is_fixed;
       is_fixed = -1;
@@ -873,10 +900,7 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       if (lane == 0) pend = atomicAdd(p.claims + is_bh, 1);
       has_pend = true;
     } else {
-      is_u += decode_seg(is_u, u1, s_us, s_nv, B, Hkv).n;
-      ++is_seg;
-      if (is_u >= u1) is_done = true;
-      else enter_seg(false);
+      next_segment();
     }
   };
   // copy the queue head into the next stage
@@ -907,7 +931,7 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       if (f_head == f_tail) {
         top_up();
         if (f_head == f_tail) {
-          if (is_done || !claims_ok) break;
+          if (is_done || (!claims_ok && !p.deterministic)) break;
           continue;
         }
       }
@@ -922,7 +946,7 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   grid_dependency_wait();
   grid_dependents_launch();
   claims_ok = true;
-  if (!is_done && is_fixed < 0) {
+  if (!is_done && is_fixed < 0 && !p.deterministic) {
     if (lane == 0) pend = atomicAdd(p.claims + is_bh, 1);
     has_pend = true;
   }
@@ -1285,6 +1309,7 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
   AttnParams p;
   p.kv_single = kv_single;
   p.cta_perm = 1;
+  p.deterministic = cf.deterministic;
   p.page_table = page_table;
   p.pos = pos;
   p.flag = flag;
@@ -1470,6 +1495,7 @@ oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* l
   AttnParams p;
   p.kv_single = kv_single;
   p.cta_perm = 1;
+  p.deterministic = cf.deterministic;
   p.page_table = page_table;
   p.pos = pos;
   p.flag = flag;

@@ -35,7 +35,7 @@ constexpr int kHT = 256;       // threads per CTA
 constexpr int kWarps = kHT / 32;
 constexpr int kRowsPerWarp = 4;
 constexpr int kRowsPerCta = kWarps * kRowsPerWarp;   // 32 weight rows
-constexpr int kBT = 8;         // sequences per tile
+constexpr int kBTMax = 8;      // sequences per tile (4 when the batch has at most 4)
 constexpr float kEps = 1e-6f;
 
 enum Phase { kTower = 0, kFuse = 1, kUp = 2, kDown = 3 };
@@ -68,22 +68,23 @@ __device__ __forceinline__ float4 ldg_w(const float* p, bool stream) {
                 : __ldg(reinterpret_cast<const float4*>(p));
 }
 
-// Block-wide sums of 8 per-thread values; on return red[0..7] hold the totals (all threads
-// may read them).  red must hold kWarps * 8 floats.
-__device__ void block_sum8(float (&v)[kBT], float* red) {
+// Block-wide sums of BT per-thread values; on return red[0..BT) hold the totals (all threads
+// may read them).  red must hold (kWarps + 1) * BT floats.
+template <int BT>
+__device__ void block_sum(float (&v)[BT], float* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-  for (int bb = 0; bb < kBT; ++bb)
+  for (int bb = 0; bb < BT; ++bb)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v[bb] += __shfl_xor_sync(0xffffffffu, v[bb], o);
   __syncthreads();
   if (lane == 0)
 #pragma unroll
-    for (int bb = 0; bb < kBT; ++bb) red[kBT + warp * kBT + bb] = v[bb];
+    for (int bb = 0; bb < BT; ++bb) red[BT + warp * BT + bb] = v[bb];
   __syncthreads();
-  if (threadIdx.x < kBT) {
+  if (threadIdx.x < BT) {
     float t = 0.f;
-    for (int w = 0; w < kWarps; ++w) t += red[kBT + w * kBT + threadIdx.x];
+    for (int w = 0; w < kWarps; ++w) t += red[BT + w * BT + threadIdx.x];
     red[threadIdx.x] = t;
   }
   __syncthreads();
@@ -146,12 +147,13 @@ __device__ __forceinline__ float4 tile_value4(const HeadParams& p, int rb, int b
   return *reinterpret_cast<const float4*>(p.act + (size_t)b * kF + kg);
 }
 
-// Builds the input tile X[bb][0..Kc) for sequences b0..b0+7 of chunk `chunk` (zeros beyond B).
+// Builds the input tile X[bb][0..Kc) for sequences b0..b0+BT-1 of chunk `chunk` (zeros beyond B).
 // 16-byte loads, four per thread in flight before any is stored.
+template <int BT>
 __device__ void build_tile(const HeadParams& p, int rb, int chunk, int b0, float* X, float* ss_out,
                            float* red) {
   const int k0 = chunk * p.Kc;
-  const int kc4 = p.Kc / 4, n4 = kBT * kc4;
+  const int kc4 = p.Kc / 4, n4 = BT * kc4;
   float4* X4 = reinterpret_cast<float4*>(X);
   for (int base = threadIdx.x; base < n4; base += 4 * kHT) {
     float4 v[4];
@@ -170,34 +172,34 @@ __device__ void build_tile(const HeadParams& p, int rb, int chunk, int b0, float
   }
   __syncthreads();
   if (p.phase == kTower) {
-    // sums of squares of this chunk of x_i for the 8 sequences of the tile, one pass
+    // sums of squares of this chunk of x_i for the BT sequences of the tile, one pass
     const int i = (rb * kRowsPerCta) / kT;
-    float ssq[kBT];
+    float ssq[BT];
 #pragma unroll
-    for (int bb = 0; bb < kBT; ++bb) {
+    for (int bb = 0; bb < BT; ++bb) {
       ssq[bb] = 0.f;
       for (int k = threadIdx.x; k < p.Kc; k += kHT) ssq[bb] += X[bb * p.Kc + k] * X[bb * p.Kc + k];
     }
-    block_sum8(ssq, red);
-    if (threadIdx.x < kBT && b0 + threadIdx.x < p.B)
+    block_sum<BT>(ssq, red);
+    if (threadIdx.x < BT && b0 + threadIdx.x < p.B)
       ss_out[((size_t)rb * p.nchunks + chunk) * p.B + b0 + threadIdx.x] = red[threadIdx.x];
     const float* gam = p.w.tower_norm[i] + k0;
-    for (int idx = threadIdx.x; idx < kBT * p.Kc; idx += kHT) X[idx] *= gam[idx % p.Kc];
+    for (int idx = threadIdx.x; idx < BT * p.Kc; idx += kHT) X[idx] *= gam[idx % p.Kc];
     __syncthreads();
   } else if (p.phase == kUp) {
-    // m = RMSNorm(f) * gamma over the full 1024-wide f, one pass for the 8 sequences
+    // m = RMSNorm(f) * gamma over the full 1024-wide f, one pass for the BT sequences
     const float* gam = p.w.ffn_norm[p.block] + k0;
-    float ssq[kBT];
+    float ssq[BT];
 #pragma unroll
-    for (int bb = 0; bb < kBT; ++bb) {
+    for (int bb = 0; bb < BT; ++bb) {
       ssq[bb] = 0.f;
       if (b0 + bb < p.B) {
         const float* fr = p.f + ((size_t)p.block * p.B + b0 + bb) * kT;
         for (int k = threadIdx.x; k < kT; k += kHT) ssq[bb] += fr[k] * fr[k];
       }
     }
-    block_sum8(ssq, red);
-    for (int idx = threadIdx.x; idx < kBT * p.Kc; idx += kHT) {
+    block_sum<BT>(ssq, red);
+    for (int idx = threadIdx.x; idx < BT * p.Kc; idx += kHT) {
       const int bb = idx / p.Kc, k = idx % p.Kc;
       X[idx] *= rsqrtf(red[bb] / kT + kEps) * gam[k];
     }
@@ -219,9 +221,13 @@ __device__ __forceinline__ float sum_chunks(const HeadParams& p, int b, int col)
   return acc;
 }
 
+// BT: sequences per tile (4 or 8); NB: register buffers of weights (NB rounds of 32 lanes x 4
+// rows x 16 bytes in flight per warp), 4 with 4-wide tiles and 2 with 8-wide ones, so both fit
+// the same 128 registers.
+template <int BT, int NB>
 __global__ void __launch_bounds__(kHT) head_phase_kernel(const HeadParams p) {
-  extern __shared__ float X[];           // [kBT][Kc]
-  __shared__ float red[kBT + kWarps * kBT];
+  extern __shared__ float X[];           // [BT][Kc]
+  __shared__ float red[BT + kWarps * BT];
   __shared__ int s_last;
   const int rb = blockIdx.x / p.nchunks, chunk = blockIdx.x % p.nchunks;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -231,61 +237,66 @@ __global__ void __launch_bounds__(kHT) head_phase_kernel(const HeadParams p) {
   const float* wrow[kRowsPerWarp];
 #pragma unroll
   for (int r = 0; r < kRowsPerWarp; ++r) wrow[r] = weight_row(p, rb, warp, r, &cols[r]) + k0;
-  // The weights never change: pull this CTA's slab toward L2 and load the first two rounds of
-  // it into registers while the previous phase may still be running (programmatic dependent
-  // launch), then wait for its outputs.
-  const bool single_pass = p.B <= kBT;
-  const int n4 = p.Kc / 4;   // >= 64 in every phase: two rounds of 32 lanes
-  float4 wa[kRowsPerWarp], wb[kRowsPerWarp];
+  // The weights never change: pull this CTA's slab toward L2 and load its first NB rounds into
+  // registers while the previous phase may still be running (programmatic dependent launch),
+  // then wait for its outputs.
+  const bool single_pass = p.B <= BT;
+  const int n4 = p.Kc / 4;   // >= 64 in every phase
+  float4 wbuf[NB][kRowsPerWarp];
   auto load_w = [&](float4 (&w)[kRowsPerWarp], int k4) {
 #pragma unroll
     for (int r = 0; r < kRowsPerWarp; ++r) w[r] = ldg_w(wrow[r] + 4 * k4, single_pass);
   };
+  auto load_first = [&]() {
+#pragma unroll
+    for (int j = 0; j < NB; ++j)
+      if (lane + 32 * j < n4) load_w(wbuf[j], lane + 32 * j);
+  };
   for (int r = 0; r < kRowsPerWarp; ++r)
-    for (int k = lane * 32 + 256; k < p.Kc; k += 32 * 32)
+    for (int k = lane * 32 + 128 * NB; k < p.Kc; k += 32 * 32)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(wrow[r] + k));
-  load_w(wa, lane);
-  load_w(wb, lane + 32);
+  load_first();
   grid_dependency_wait();
   grid_dependents_launch();
 
-  for (int b0 = 0; b0 < p.B; b0 += kBT) {
-    if (b0 > 0) {   // later sequence tiles read the slab again
-      load_w(wa, lane);
-      load_w(wb, lane + 32);
-    }
-    build_tile(p, rb, chunk, b0, X, p.ss, red);
-    float acc[kRowsPerWarp][kBT];
+  for (int b0 = 0; b0 < p.B; b0 += BT) {
+    if (b0 > 0) load_first();   // later sequence tiles read the slab again
+    build_tile<BT>(p, rb, chunk, b0, X, p.ss, red);
+    float acc[kRowsPerWarp][BT];
 #pragma unroll
     for (int r = 0; r < kRowsPerWarp; ++r)
 #pragma unroll
-      for (int bb = 0; bb < kBT; ++bb) acc[r][bb] = 0.f;
+      for (int bb = 0; bb < BT; ++bb) acc[r][bb] = 0.f;
     auto fma_w = [&](const float4 (&w)[kRowsPerWarp], int k4) {
 #pragma unroll
-      for (int bb = 0; bb < kBT; ++bb) {
+      for (int bb = 0; bb < BT; ++bb) {
         const float4 xv = *reinterpret_cast<const float4*>(X + bb * p.Kc + 4 * k4);
 #pragma unroll
         for (int r = 0; r < kRowsPerWarp; ++r)
           acc[r][bb] += w[r].x * xv.x + w[r].y * xv.y + w[r].z * xv.z + w[r].w * xv.w;
       }
     };
-    // two register buffers, each refilled two rounds ahead of its use
-    for (int k4 = lane; k4 < n4; k4 += 64) {
-      fma_w(wa, k4);
-      if (k4 + 64 < n4) load_w(wa, k4 + 64);
-      if (k4 + 32 < n4) {
-        fma_w(wb, k4 + 32);
-        if (k4 + 96 < n4) load_w(wb, k4 + 96);
+    // NB register buffers, each refilled NB rounds ahead of its use
+    for (int k4 = lane; k4 < n4; k4 += 32 * NB) {
+#pragma unroll
+      for (int j = 0; j < NB; ++j) {
+        const int kk = k4 + 32 * j;
+        if (kk < n4) {
+          fma_w(wbuf[j], kk);
+          if (kk + 32 * NB < n4) load_w(wbuf[j], kk + 32 * NB);
+        }
       }
     }
-    // butterfly: after 5 stages lane l holds the lane-sum of value l = (r = l / 8, bb = l % 8)
-    float v[32];
+    // butterfly over the kRowsPerWarp * BT values (32 or 16): afterwards lane l holds the
+    // lane-sum of value l % NV (r = (l % NV) / BT, bb = l % BT)
+    constexpr int NV = kRowsPerWarp * BT;
+    float v[NV];
 #pragma unroll
     for (int r = 0; r < kRowsPerWarp; ++r)
 #pragma unroll
-      for (int bb = 0; bb < kBT; ++bb) v[r * kBT + bb] = acc[r][bb];
+      for (int bb = 0; bb < BT; ++bb) v[r * BT + bb] = acc[r][bb];
 #pragma unroll
-    for (int half = 16; half >= 1; half >>= 1) {
+    for (int half = NV / 2; half >= 1; half >>= 1) {
       const bool upper = (lane & half) != 0;
 #pragma unroll
       for (int i = 0; i < half; ++i) {
@@ -294,8 +305,10 @@ __global__ void __launch_bounds__(kHT) head_phase_kernel(const HeadParams p) {
         v[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
       }
     }
-    {
-      const int r = lane >> 3, bb = lane & 7, b = b0 + bb;
+#pragma unroll
+    for (int o = NV; o < 32; o <<= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+    if (lane < NV) {
+      const int r = lane / BT, bb = lane % BT, b = b0 + bb;
       int col = cols[0];
 #pragma unroll
       for (int rr = 1; rr < kRowsPerWarp; ++rr)
@@ -419,9 +432,14 @@ int head_counter_count(int D) {
 
 oda_status prepare_head_kernel() {
   // largest input tile: the tower phase with D = 8192 (Kc = 4096)
-  return check_cuda(cudaFuncSetAttribute(head_phase_kernel,
+  oda_status st = check_cuda(cudaFuncSetAttribute(head_phase_kernel<8, 2>,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  8 * 4096 * (int)sizeof(float)),
+                             "cudaFuncSetAttribute(head)");
+  if (st != ODA_OK) return st;
+  return check_cuda(cudaFuncSetAttribute(head_phase_kernel<4, 4>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kBT * 4096 * (int)sizeof(float)),
+                                         4 * 4096 * (int)sizeof(float)),
                     "cudaFuncSetAttribute(head)");
 }
 
@@ -475,14 +493,17 @@ oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const flo
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(sh.row_blocks * sh.nchunks);
     lc.blockDim = dim3(kHT);
-    lc.dynamicSmemBytes = kBT * sh.Kc * sizeof(float);
+    const int bt = p.B <= 4 ? 4 : kBTMax;
+    lc.dynamicSmemBytes = bt * sh.Kc * sizeof(float);
     lc.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
     lc.numAttrs = 1;
-    oda_status st = check_cuda(cudaLaunchKernelEx(&lc, head_phase_kernel, p), "recall head launch");
+    oda_status st = check_cuda(bt == 4 ? cudaLaunchKernelEx(&lc, head_phase_kernel<4, 4>, p)
+                                       : cudaLaunchKernelEx(&lc, head_phase_kernel<8, 2>, p),
+                               "recall head launch");
     if (st != ODA_OK) return st;
   }
   return ODA_OK;

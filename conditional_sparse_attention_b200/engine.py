@@ -86,7 +86,7 @@ class OdaDecoder:
 
     def __init__(self, wl: Workload, device="cuda", capacity_steps: int = 0,
                  perturb_head: bool = False, head_params: dict = None, fill_cache: bool = True,
-                 overlap_layers: bool = True):
+                 overlap_layers: bool = True, deterministic: bool = False):
         if not torch.cuda.is_available():
             raise RuntimeError("OdaDecoder needs a CUDA device (the CUDA path has no fallback)")
         self.wl = wl
@@ -100,7 +100,7 @@ class OdaDecoder:
         self.max_pages = (max(wl.ctx) + self.capacity_steps + 1 + configs.PAGE - 1) // configs.PAGE
         self.n_pool = B * self.max_pages
         cfg = oda.make_config(B, wl.Hq, Hkv, self.max_pages, D, wl.sinks, wl.window, wl.theta,
-                              overlap_layers=overlap_layers)
+                              overlap_layers=overlap_layers, deterministic=deterministic)
         self.ctx = oda.oda_create(cfg)
         dev = self.device
         self.stream = torch.cuda.Stream(dev)

@@ -55,9 +55,10 @@ class Context:
 
 
 def make_config(batch, n_q_heads, n_kv_heads, max_pages, head_in_dim, sinks=4, window=2048,
-                theta=0.0, head_dim=128, page_size=16, overlap_layers=False) -> OdaConfig:
+                theta=0.0, head_dim=128, page_size=16, overlap_layers=False,
+                deterministic=False) -> OdaConfig:
     return OdaConfig(batch, n_q_heads, n_kv_heads, head_dim, page_size, max_pages, sinks, window,
-                     head_in_dim, theta, 1 if overlap_layers else 0)
+                     head_in_dim, theta, 1 if overlap_layers else 0, 1 if deterministic else 0)
 
 
 def kv_layer(k: torch.Tensor, v: torch.Tensor) -> OdaKVLayer:

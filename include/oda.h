@@ -83,6 +83,12 @@ typedef struct {
                            * write pos, flag, the page table or the KV pools on the stream
                            * between two consecutive attention calls.  0: every call starts
                            * after all prior work on the stream.                          */
+  int32_t deterministic;  /* 1: the full-set attention gives the pages of each (sequence, KV
+                           * head) to its CTAs in a fixed pattern, so every launch rounds the
+                           * same way (bit-identical replays).  0: pages are claimed at run time
+                           * by whichever CTA is free (faster on an unevenly loaded GPU; the
+                           * fp32 rounding of the output may differ from run to run within the
+                           * attention tolerance).                                          */
 } oda_config;
 
 typedef struct {

@@ -40,7 +40,7 @@ def test_struct_layouts_match_header(lib, tmp_path):
 int main(void) {
   printf("%zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(oda_config), sizeof(oda_kv_layer),
          sizeof(oda_head_weights), sizeof(oda_state), offsetof(oda_config, theta),
-         offsetof(oda_config, overlap_layers), offsetof(oda_head_weights, out_b),
+         offsetof(oda_config, deterministic), offsetof(oda_head_weights, out_b),
          offsetof(oda_state, conv_width));
   printf("%d %d\\n", ODA_MAX_BATCH, ODA_MAX_LAYERS);
   return 0;
@@ -54,7 +54,7 @@ int main(void) {
     got = [int(x) for x in out]
     C = _lib
     want = [ctypes.sizeof(C.OdaConfig), ctypes.sizeof(C.OdaKVLayer), ctypes.sizeof(C.OdaHeadWeights),
-            ctypes.sizeof(C.OdaState), C.OdaConfig.theta.offset, C.OdaConfig.overlap_layers.offset,
+            ctypes.sizeof(C.OdaState), C.OdaConfig.theta.offset, C.OdaConfig.deterministic.offset,
             C.OdaHeadWeights.out_b.offset,
             C.OdaState.conv_width.offset, C.MAX_BATCH, C.MAX_LAYERS]
     assert got == want

@@ -31,7 +31,7 @@ def _wl(ctx, Hq=16, Hkv=8, seed=77, shuffle=True, steps=2):
 
 
 class Setup:
-    def __init__(self, wl, extra_pool_pages=0):
+    def __init__(self, wl, extra_pool_pages=0, deterministic=False):
         from conditional_sparse_attention_b200 import oda
         self.oda = oda
         self.wl = wl
@@ -52,7 +52,8 @@ class Setup:
         self.kn = torch.from_numpy(kn.view(np.int16)).to(dev)
         self.vn = torch.from_numpy(vn.view(np.int16)).to(dev)
         self.pos = torch.tensor([c + 1 for c in wl.ctx], dtype=torch.int32, device=dev)
-        cfg = oda.make_config(wl.B, wl.Hq, wl.Hkv, self.max_pages, max(512, wl.D), wl.sinks, wl.window)
+        cfg = oda.make_config(wl.B, wl.Hq, wl.Hkv, self.max_pages, max(512, wl.D), wl.sinks, wl.window,
+                              deterministic=deterministic)
         self.ctx = oda.oda_create(cfg)
 
     def oracle(self, b, mode):
@@ -195,3 +196,22 @@ def test_full_set_chunk_claims_cover_every_page(ctx, Hq, Hkv):
         for b in range(s.wl.B):
             ok, ma, rel = attn_close(got[b], s.oracle(b, 1))
             assert ok, f"rep={rep} b={b} ctx={ctx[b]} max_abs={ma:.3g} rel_l2={rel:.3g}"
+
+
+def test_full_set_fixed_pattern_is_bitwise_repeatable():
+    """deterministic = 1: the pages of each (sequence, head) go to the CTAs in a fixed pattern,
+    so repeated launches give identical bits (and match the oracle within tolerance)."""
+    ctx = [60000, 900, 20000, 4097, 33, 131072 - 3000]
+    s = Setup(_wl(ctx, 32, 8, seed=84), deterministic=True)
+    flag = torch.ones(len(ctx), dtype=torch.int32, device="cuda")
+    outs = []
+    for rep in range(3):
+        out = torch.full((s.wl.B, 32, 128), 7.0, device="cuda")
+        s.oda.oda_attend_full_if(s.ctx, s.layer, s.pt, s.pos, flag, s.q, s.kn, s.vn, out)
+        torch.cuda.synchronize()
+        assert s.oda.oda_get_error(s.ctx) == 0
+        outs.append(out.cpu().numpy())
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
+    for b in range(s.wl.B):
+        ok, ma, rel = attn_close(outs[0][b], s.oracle(b, 1))
+        assert ok, f"b={b} ctx={ctx[b]} max_abs={ma:.3g} rel_l2={rel:.3g}"
