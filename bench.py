@@ -426,8 +426,9 @@ def run_ours(args, wl, rank, world, local_rank):
         out_h = torch.empty((wl.B, wl.D), dtype=torch.float32).pin_memory()
         out_f = torch.empty(wl.B, dtype=torch.int32).pin_memory()
         out_s = torch.empty(wl.B, dtype=torch.float32).pin_memory()
+        # the same step inputs (and so the same scheduled flags) as the device-timed loop
         for i in range(2):
-            dec.step(host[i % n_store])
+            dec.step(host[(W - 1 + i) % n_store])
         dec.synchronize()
         if world > 1:
             torch.distributed.barrier()
@@ -437,7 +438,7 @@ def run_ours(args, wl, rank, world, local_rank):
             dec.copy_stream.wait_event(e0)   # every upload of the timed steps starts after e0
             h0 = time.perf_counter()
             for i in range(n_e2e):
-                dec.step(host[i % n_store])
+                dec.step(host[(1 + W + i) % n_store])
                 out_h.copy_(dec.h_prev, non_blocking=True)
                 out_f.copy_(dec.flag, non_blocking=True)
                 out_s.copy_(dec.score, non_blocking=True)
@@ -454,7 +455,7 @@ def run_ours(args, wl, rank, world, local_rank):
         with torch.cuda.stream(dec.copy_stream):
             c0.record(dec.copy_stream)
             for i in range(n_e2e):
-                dec.staging[i % 2].copy_(host[i % n_store], non_blocking=True)
+                dec.staging[i % 2].copy_(host[(1 + W + i) % n_store], non_blocking=True)
             c1.record(dec.copy_stream)
         c1.synchronize()
         d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -187,14 +187,15 @@ __device__ void build_tile(const HeadParams& p, int rb, int chunk, int b0, float
     for (int idx = threadIdx.x; idx < BT * p.Kc; idx += kHT) X[idx] *= gam[idx % p.Kc];
     __syncthreads();
   } else if (p.phase == kUp) {
-    // m = RMSNorm(f) * gamma over the full 1024-wide f, one pass for the BT sequences
+    // m = RMSNorm(f) * gamma over the full 1024-wide f, one pass for the BT sequences (from the
+    // tile itself when it holds the whole of f)
     const float* gam = p.w.ffn_norm[p.block] + k0;
     float ssq[BT];
 #pragma unroll
     for (int bb = 0; bb < BT; ++bb) {
       ssq[bb] = 0.f;
       if (b0 + bb < p.B) {
-        const float* fr = p.f + ((size_t)p.block * p.B + b0 + bb) * kT;
+        const float* fr = p.Kc == kT ? X + bb * kT : p.f + ((size_t)p.block * p.B + b0 + bb) * kT;
         for (int k = threadIdx.x; k < kT; k += kHT) ssq[bb] += fr[k] * fr[k];
       }
     }
@@ -307,7 +308,16 @@ __global__ void __launch_bounds__(kHT) head_phase_kernel(const HeadParams p) {
     }
 #pragma unroll
     for (int o = NV; o < 32; o <<= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
-    if (lane < NV) {
+    if (p.phase == kUp && p.nchunks == 1) {
+      // whole rows: lanes [0, 2 BT) hold the gate sums of the warp's two units, lanes
+      // [2 BT, 4 BT) the up sums of the same units; act = SiLU(gate) * up
+      const float up = __shfl_down_sync(0xffffffffu, v[0], 2 * BT);
+      const int r = lane / BT, bb = lane % BT, b = b0 + bb;
+      if (lane < 2 * BT && b < p.B) {
+        const int n = rb * (kRowsPerCta / 2) + warp * 2 + r;
+        p.act[(size_t)b * kF + n] = silu(v[0]) * up;
+      }
+    } else if (lane < NV) {
       const int r = lane / BT, bb = lane % BT, b = b0 + bb;
       int col = cols[0];
 #pragma unroll
@@ -319,6 +329,8 @@ __global__ void __launch_bounds__(kHT) head_phase_kernel(const HeadParams p) {
   }
 
   // ---- last CTA of the row block: reduce partials in chunk order and apply the epilogue
+  // (the up projection over whole rows has written its output already)
+  if (p.phase == kUp && p.nchunks == 1) return;
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) s_last = (atomicAdd(&p.cnt[rb], 1) == p.nchunks - 1);
@@ -408,7 +420,7 @@ PhaseShape phase_shape(int phase, int D) {
   switch (phase) {
     case kTower: return {D / 2, 2, 3 * kT, 3 * kT / kRowsPerCta};
     case kFuse: return {1024, 9, kT, kT / kRowsPerCta};
-    case kUp: return {512, kT / 512, 2 * kF, kF / (kRowsPerCta / 2)};
+    case kUp: return {kT, 1, 2 * kF, kF / (kRowsPerCta / 2)};   // whole rows: epilogue in registers
     default: return {256, kF / 256, kT, kT / kRowsPerCta};
   }
 }
