@@ -486,9 +486,18 @@ def run_ours(args, wl, rank, world, local_rank):
         q1.record(dec.stream)
         q1.synchronize()
         quiet_us = q0.elapsed_time(q1) * 1e3 / 2
+        # the step-input staging copy alone (device to device, in the step stream)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(dec.stream):
+            s0.record(dec.stream)
+            for i in range(8):
+                dec.staging[i % 2].copy_(store[i % n_store], non_blocking=True)
+            s1.record(dec.stream)
+        s1.synchronize()
+        stage_us = s0.elapsed_time(s1) * 1e3 / 8
         step_detail = {"unflagged_step_us": quiet_us, "local_pass_us": loc_ms * 1e3 * wl.L,
-                       "head_us": head_ms * 1e3,
-                       "glue_us": quiet_us - loc_ms * 1e3 * wl.L - head_ms * 1e3}
+                       "head_us": head_ms * 1e3, "staging_copy_us": stage_us,
+                       "glue_us": quiet_us - loc_ms * 1e3 * wl.L - head_ms * 1e3 - stage_us}
     else:
         step_detail = None
     err = dec.device_error()

@@ -8,6 +8,7 @@
 #include <cstring>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace oda {
 
@@ -29,13 +30,23 @@ oda_status check_cuda(cudaError_t e, const char* what) {
 }
 
 __global__ void set_condition_kernel(cudaGraphConditionalHandle h, const int32_t* any_flag) {
+  grid_dependency_wait();   // any_flag comes from the kernel before (programmatic launch)
   cudaGraphSetConditional(h, *any_flag != 0 ? 1u : 0u);
 }
 
 oda_status launch_set_condition(cudaGraphConditionalHandle h, const int32_t* any_flag,
-                                cudaStream_t stream) {
-  set_condition_kernel<<<1, 1, 0, stream>>>(h, any_flag);
-  return check_cuda(cudaGetLastError(), "set-condition launch");
+                                bool overlap, cudaStream_t stream) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(1);
+  lc.blockDim = dim3(1);
+  lc.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = overlap ? 1 : 0;
+  return check_cuda(cudaLaunchKernelEx(&lc, set_condition_kernel, h, any_flag),
+                    "set-condition launch");
 }
 
 }  // namespace oda
@@ -275,7 +286,7 @@ oda_status oda_cond_begin(oda_ctx* ctx, cudaStream_t stream, const int32_t* any_
   st = check_cuda(cudaGraphConditionalHandleCreate(&h, graph, 0, cudaGraphCondAssignDefault),
                   "cudaGraphConditionalHandleCreate");
   if (st != ODA_OK) return st;
-  st = oda::launch_set_condition(h, any_flag, stream);
+  st = oda::launch_set_condition(h, any_flag, ctx->cfg.overlap_layers != 0, stream);
   if (st != ODA_OK) return st;
   st = check_cuda(cudaStreamGetCaptureInfo(stream, &cs, nullptr, &graph, &deps, &nd),
                   "cudaStreamGetCaptureInfo");

@@ -6,6 +6,7 @@
 // of §2.2).  The hybrid workload's 18 linear-recurrent layers (§3.1: Gated DeltaNet) are
 // stood in for by a 4-tap causal conv plus the gated delta rule on a 16 x 128 x 128 state.
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace oda {
 namespace {
@@ -30,6 +31,10 @@ __global__ void __launch_bounds__(kGlueChunk)
 hidden_kernel(const float* emb, const float* terms, int n_terms, const int32_t* flag, float* h,
               float* xbuf, float* ssbuf, int32_t* cnt, int B, int D) {
   const int b = blockIdx.y, chunk = blockIdx.x, nch = gridDim.x;
+  // launched with programmatic dependent launch: wait for the kernels that wrote the layer
+  // outputs (and the flags) before reading anything, and let the recall head start early
+  grid_dependency_wait();
+  grid_dependents_launch();
   if (flag && flag[b] == 0) return;
   __shared__ float red[kGlueChunk / 32];
   __shared__ int s_last;
@@ -133,9 +138,18 @@ oda_status launch_glue_hidden(oda_ctx* ctx, const float* emb, const float* terms
   if (!emb || !h || n_terms < 0 || (n_terms > 0 && !terms))
     return set_error(ODA_ERR_INVALID_ARG, "glue_hidden: bad argument");
   const int B = ctx->cfg.batch, D = ctx->cfg.head_in_dim;
-  hidden_kernel<<<dim3(glue_chunks(D), B), kGlueChunk, 0, stream>>>(
-      emb, terms, n_terms, flag, h, ctx->glue_x, ctx->glue_ss, ctx->glue_cnt, B, D);
-  return check_cuda(cudaGetLastError(), "glue_hidden launch");
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(glue_chunks(D), B);
+  lc.blockDim = dim3(kGlueChunk);
+  lc.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = ctx->cfg.overlap_layers ? 1 : 0;
+  return check_cuda(cudaLaunchKernelEx(&lc, hidden_kernel, emb, terms, n_terms, flag, h,
+                                       ctx->glue_x, ctx->glue_ss, ctx->glue_cnt, B, D),
+                    "glue_hidden launch");
 }
 
 oda_status launch_glue_gdn(oda_ctx* ctx, const oda_state* st, int layer, const float* c,

@@ -87,6 +87,6 @@ int glue_chunks(int D);
 
 // cond.cu
 oda_status launch_set_condition(cudaGraphConditionalHandle h, const int32_t* any_flag,
-                                cudaStream_t stream);
+                                bool overlap, cudaStream_t stream);
 
 }  // namespace oda
