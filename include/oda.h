@@ -81,8 +81,10 @@ typedef struct {
                            * (programmatic dependent launch): the later call prefetches its
                            * pages while the earlier one finishes.  The caller then must not
                            * write pos, flag, the page table or the KV pools on the stream
-                           * between two consecutive attention calls.  0: every call starts
-                           * after all prior work on the stream.                          */
+                           * between two consecutive attention calls.  The hidden-state glue
+                           * and the conditional's set-condition kernel are then launched the
+                           * same way; they read nothing before the previous kernel completes.
+                           * 0: every call starts after all prior work on the stream.      */
   int32_t deterministic;  /* 1: the full-set attention gives the pages of each (sequence, KV
                            * head) to its CTAs in a fixed pattern, so every launch rounds the
                            * same way (bit-identical replays).  0: pages are claimed at run time
