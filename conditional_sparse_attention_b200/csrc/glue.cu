@@ -41,11 +41,24 @@ hidden_kernel(const float* emb, const float* terms, int n_terms, const int32_t* 
   const int d = chunk * kGlueChunk + threadIdx.x;
   float x = 0.f;
   if (d < D) {
-    // independent partial sums so the loads of all terms are in flight together
+    // four partial sums (term i goes to sum i mod 4, in increasing i); the loads of twelve
+    // terms are issued before any of them is added, so they are in flight together
     const float* tp = terms + (size_t)b * D + d;
     const size_t stride = (size_t)B * D;
     float a0 = emb[(size_t)b * D + d], a1 = 0.f, a2 = 0.f, a3 = 0.f;
     int i = 0;
+    for (; i + 12 <= n_terms; i += 12) {
+      float v[12];
+#pragma unroll
+      for (int j = 0; j < 12; ++j) v[j] = tp[(size_t)(i + j) * stride];
+#pragma unroll
+      for (int j = 0; j < 12; j += 4) {
+        a0 += v[j];
+        a1 += v[j + 1];
+        a2 += v[j + 2];
+        a3 += v[j + 3];
+      }
+    }
     for (; i + 4 <= n_terms; i += 4) {
       a0 += tp[(size_t)i * stride];
       a1 += tp[(size_t)(i + 1) * stride];

@@ -11,16 +11,18 @@
 //   q   = w_o . (RMSNorm(f) * gamma_o) + b_o
 //
 // Design: at batch sizes of a few sequences the head is a weight-streaming problem (113 MB of
-// fp32 weights for D = 2048, 2*B flops per 4-byte weight), so every phase is a split-K GEMV on
-// CUDA cores: a CTA streams a 32-row x Kc slab of one weight matrix exactly once with 16-byte
-// non-allocating loads and multiplies it against a shared-memory tile of up to 8 sequences'
-// inputs; lanes reduce with a 31-shuffle butterfly.  The input transform of a phase (RMSNorm
+// fp32 weights for D = 2048, 2*B flops per 4-byte weight) on CUDA cores.  Up to 8 sequences run
+// in one cooperative launch of all six phases (head_fused_kernel, further down).  Larger batches
+// run six phase launches, each a split-K GEMV: a CTA streams a 32-row x Kc slab of one weight
+// matrix exactly once with 16-byte non-allocating loads and multiplies it against a
+// shared-memory tile of up to 8 sequences' inputs; lanes reduce with a 31-shuffle butterfly.  The input transform of a phase (RMSNorm
 // scale, the interaction vector, the gated activation) is applied while the tile is built, and
 // the output epilogue (bias, SiLU, residual) runs in the last CTA of each row block, which sums
 // the split-K partials in a fixed order (deterministic results).  The last row block of the
 // final phase also computes q and the gate.  Six launches per score; each may start while the
 // previous one finishes (programmatic dependent launch) and pulls its weight slab toward L2
 // before waiting for the previous phase's outputs.
+#include <algorithm>
 #include <cmath>
 
 #include "internal.h"
@@ -208,6 +210,38 @@ __device__ void build_tile(const HeadParams& p, int rb, int chunk, int b0, float
   }
 }
 
+// q = w_o . (RMSNorm(f2) * gamma_o) + b_o for sequence b (whole warp; f2 row written by other
+// CTAs of this launch or an earlier one) and its gate: full iff q > theta or q is not finite,
+// or the scheduled flag where a schedule is given.
+__device__ __forceinline__ void score_and_gate(const oda_head_weights& w, const float* fr, int b,
+                                               const int32_t* sched, float theta, float* score,
+                                               int32_t* flag, int* s_any, int lane) {
+  float ss = 0.f, dot = 0.f;
+  for (int k = lane; k < kT; k += 32) {
+    const float fv = __ldcg(fr + k);
+    ss += fv * fv;
+    dot += w.out_w[k] * w.out_norm[k] * fv;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  }
+  if (lane == 0) {
+    const float q = dot * rsqrtf(ss / kT + kEps) + w.out_b[0];
+    score[b] = q;
+    int fl;
+    if (sched) {
+      fl = sched[b] != 0;
+    } else {
+      const bool nonfinite = (__float_as_uint(q) & 0x7f800000u) == 0x7f800000u;
+      fl = (nonfinite || q > theta) ? 1 : 0;
+    }
+    flag[b] = fl;
+    if (fl) atomicOr(s_any, 1);
+  }
+}
+
 // Split-K partials of output column `col` for sequence b, summed in chunk order; all loads are
 // issued before the first add (at most kMaxChunks chunks).
 constexpr int kMaxChunks = 16;
@@ -378,37 +412,426 @@ __global__ void __launch_bounds__(kHT) head_phase_kernel(const HeadParams p) {
   __shared__ int s_any;
   if (threadIdx.x == 0) s_any = 0;
   __syncthreads();
-  for (int b = warp; b < p.B; b += kWarps) {
-    const float* fr = p.f + ((size_t)2 * p.B + b) * kT;
-    float ss = 0.f, dot = 0.f;
-    for (int k = lane; k < kT; k += 32) {
-      const float fv = __ldcg(fr + k);
-      ss += fv * fv;
-      dot += p.w.out_w[k] * p.w.out_norm[k] * fv;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      dot += __shfl_xor_sync(0xffffffffu, dot, o);
-    }
-    if (lane == 0) {
-      const float q = dot * rsqrtf(ss / kT + kEps) + p.w.out_b[0];
-      p.score[b] = q;
-      int fl;
-      if (p.sched) {
-        fl = p.sched[b] != 0;
-      } else {
-        const bool nonfinite = (__float_as_uint(q) & 0x7f800000u) == 0x7f800000u;
-        fl = (nonfinite || q > p.theta) ? 1 : 0;
-      }
-      p.flag[b] = fl;
-      if (fl) atomicOr(&s_any, 1);
-    }
-  }
+  for (int b = warp; b < p.B; b += kWarps)
+    score_and_gate(p.w, p.f + ((size_t)2 * p.B + b) * kT, b, p.sched, p.theta, p.score, p.flag,
+                   &s_any, lane);
   __syncthreads();
   if (threadIdx.x == 0) {
     *p.any_flag = s_any;
     p.cnt[p.row_blocks] = 0;
+  }
+}
+
+// ------------------------------------------------------------ fused head (batch <= 8)
+// One cooperative launch, one CTA per SM, runs all six phases.  Warp 8 streams every weight row
+// segment (1024 floats, 4 KiB) the CTA owns through a ring of 32 KiB stages with bulk copies,
+// phase after phase: the weights never depend on a phase's inputs, so HBM keeps streaming while
+// the grid waits between phases.  Warps 0-7 take one segment each per stage and dot it against
+// the phase's input, held whole in shared memory for the sequence tile.  Each CTA owns whole
+// output rows of every phase (all of their K-chunks), so it finishes them itself (norm scale,
+// bias, activation, residual) and no split-K partial leaves the SM; a grid-wide barrier (a
+// counter with a bounded spin) separates the phases.  The last CTA to finish computes q and the
+// gate.
+constexpr int kFC = 8;                              // consumer warps
+constexpr int kFThreads = (kFC + 1) * 32;           // + one producer warp
+constexpr int kSeg = 1024;                          // floats per weight segment
+constexpr int kSegBytes = kSeg * 4;
+constexpr int kFStageBytes = kFC * kSegBytes;       // one segment per consumer warp
+constexpr int kMaxRing = 5;
+constexpr int kMaxOwnSegs = 32;                     // segments per chunk a CTA may own in a phase
+constexpr uint64_t kFWaitNs = 2000000000ull;
+constexpr uint64_t kGridWaitNs = 1000000000ull;
+
+struct FusedParams {
+  oda_head_weights w;
+  const float* x[3];      // h_prev, emb, h_loc  [B][D]
+  const int32_t* sched;
+  float* score;
+  int32_t* flag;
+  int32_t* any_flag;
+  float* u;               // [3][B][T]
+  float* f;               // [3][B][T]
+  float* act;             // [B][F]
+  int32_t* cnt;           // [0] grid-barrier arrivals, [1] finished CTAs; both back to 0 at exit
+  int32_t* err;
+  int B, D, ring;
+  float theta;
+};
+
+// The rows of phase ph (0 tower, 1 fuse, 2 up 0, 3 down 0, 4 up 1, 5 down 1) that CTA c of G
+// owns: [lo, lo + n) (gate/up row pairs for the up projections); the tower phase splits the
+// grid into three groups, one per tower.  nseg: weight segments per K-chunk.
+struct Own {
+  int kind, blk, tower, lo, n, nchunk, nseg;
+};
+
+__device__ __forceinline__ Own own_rows(int ph, int c, int G, int D) {
+  Own o;
+  o.kind = ph == 0 ? kTower : ph == 1 ? kFuse : ((ph & 1) == 0 ? kUp : kDown);
+  o.blk = ph >= 4 ? 1 : 0;
+  o.tower = 0;
+  int rows = kT, cc = c, gg = G;
+  if (o.kind == kTower) {
+    int i = 0;
+    while (i < 2 && (long long)G * (i + 1) / 3 <= c) ++i;
+    const int g0 = (int)((long long)G * i / 3), g1 = (int)((long long)G * (i + 1) / 3);
+    o.tower = i;
+    cc = c - g0;
+    gg = g1 - g0;
+  } else if (o.kind == kUp) {
+    rows = kF;
+  }
+  o.lo = (int)((long long)rows * cc / gg);
+  o.n = (int)((long long)rows * (cc + 1) / gg) - o.lo;
+  o.nchunk = o.kind == kTower ? D / kSeg : o.kind == kFuse ? 9 : o.kind == kUp ? 1 : kF / kSeg;
+  o.nseg = o.kind == kUp ? 2 * o.n : o.n;
+  return o;
+}
+
+// Segment r of K-chunk ch of the CTA's rows (for the up projections r < n are gate rows and
+// r >= n the up rows of the same units).
+__device__ __forceinline__ const float* seg_ptr(const FusedParams& p, const Own& o, int ch, int r) {
+  const oda_head_weights& w = p.w;
+  switch (o.kind) {
+    case kTower: return w.tower_w[o.tower] + (size_t)(o.lo + r) * p.D + ch * kSeg;
+    case kFuse: return w.fuse_w + (size_t)(o.lo + r) * (9 * kT) + ch * kSeg;
+    case kUp:
+      return r < o.n ? w.ffn_gate[o.blk] + (size_t)(o.lo + r) * kT
+                     : w.ffn_up[o.blk] + (size_t)(o.lo + r - o.n) * kT;
+    default: return w.ffn_down[o.blk] + (size_t)(o.lo + r) * kF + ch * kSeg;
+  }
+}
+
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kFC * 32) : "memory");
+}
+
+// Butterfly over 32 values: afterwards lane l holds the sum over the warp of value l.
+__device__ __forceinline__ float butterfly32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int half = 16; half >= 1; half >>= 1) {
+    const bool upper = (lane & half) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? v[i] : v[i + half];
+      const float keep = upper ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+    }
+  }
+  return v[0];
+}
+
+// Pulls every weight segment of the CTA's part of a phase toward L2 (lanes share the work).
+__device__ __forceinline__ void prefetch_phase(const FusedParams& p, const Own& o, int lane) {
+  const int total = o.nchunk * o.nseg;
+  for (int i = lane; i < total; i += 32) {
+    const int ch = i / o.nseg, r = i - ch * o.nseg;
+    prefetch_l2_bulk(seg_ptr(p, o, ch, r), kSegBytes);
+  }
+}
+
+// This warp's 128-column slice of K-chunk ch of the phase input, lane l holding columns
+// 4*col4 .. 4*col4+3 of the chunk, for the BT sequences of the tile (zeros beyond B).  Tower:
+// the raw x_i rows are in `src` ([B][D]); the slice is x*gamma and ssl collects x^2.  Fuse: z is
+// formed from u_0, u_1, u_2 ([3][BT][T]): chunk 0-2 is u_c, 3-5 the products u0u1, u0u2, u1u2,
+// 6-8 the absolute differences in the same order.
+template <int BT>
+__device__ __forceinline__ void input_slice(const Own& o, int B, int D, const float* src, int ch,
+                                            int col4, float4 gam, float (&ssl)[BT], float4 (&xs)[BT]) {
+  const float4* s4 = reinterpret_cast<const float4*>(src);
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (o.kind == kTower) {
+#pragma unroll
+    for (int bb = 0; bb < BT; ++bb) {
+      const float4 x = bb < B ? s4[(size_t)bb * (D / 4) + ch * (kSeg / 4) + col4] : zero;
+      ssl[bb] += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+      xs[bb] = make_float4(x.x * gam.x, x.y * gam.y, x.z * gam.z, x.w * gam.w);
+    }
+  } else if (o.kind == kFuse) {
+    const int m = (ch + 6) % 3;   // 0, 1, 2 for chunks 3|6, 4|7, 5|8
+    const int ia = ch < 3 ? ch : (m == 2 ? 1 : 0), ib = ch < 3 ? ch : (m == 0 ? 1 : 2);
+#pragma unroll
+    for (int bb = 0; bb < BT; ++bb) {
+      const float4 a = s4[(ia * BT + bb) * (kT / 4) + col4];
+      if (ch < 3) {
+        xs[bb] = a;
+      } else {
+        const float4 b = s4[(ib * BT + bb) * (kT / 4) + col4];
+        xs[bb] = ch < 6 ? make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w)
+                        : make_float4(fabsf(a.x - b.x), fabsf(a.y - b.y), fabsf(a.z - b.z),
+                                      fabsf(a.w - b.w));
+      }
+    }
+  } else if (o.kind == kUp) {
+#pragma unroll
+    for (int bb = 0; bb < BT; ++bb) xs[bb] = s4[bb * (kT / 4) + col4];
+  } else {
+#pragma unroll
+    for (int bb = 0; bb < BT; ++bb) xs[bb] = s4[bb * (kF / 4) + ch * (kSeg / 4) + col4];
+  }
+}
+
+// The warp's share of one stage: its 128 columns of each of the n (<= 8) segments, dotted with
+// the input slice; 32 values per butterfly (segments x sequences), and the lane holding value
+// (segment i, sequence bb) adds it to the warp's row sum acc[(8g + i)][bb].
+template <int BT>
+__device__ __forceinline__ void stage_dot(const uint8_t* stage, int n, int col4, const float4 (&xs)[BT],
+                                          float* acc, int g, int lane) {
+  constexpr int NS = 32 / BT;   // segments per butterfly
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int hf = 0; hf < kFC / NS; ++hf) {
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < NS; ++i) {
+      const int si = hf * NS + i;
+      const float4 w = si < n ? reinterpret_cast<const float4*>(stage + si * kSegBytes)[col4] : zero;
+#pragma unroll
+      for (int bb = 0; bb < BT; ++bb)
+        v[i * BT + bb] = w.x * xs[bb].x + w.y * xs[bb].y + w.z * xs[bb].z + w.w * xs[bb].w;
+    }
+    const float t = butterfly32(v, lane);
+    const int si = hf * NS + lane / BT;
+    if (si < n) acc[(g * kFC + si) * BT + lane % BT] += t;
+  }
+}
+
+// The input of the fuse, up and down phases for the sequence tile, into shared memory (zeros
+// beyond B): fuse u_0, u_1, u_2 [3][BT][T]; up f_j * gamma_j [BT][T] (inv[bb] receives 1 / rms(f_j),
+// applied to the dot products); down act [BT][F].  These rows were written by other CTAs of
+// this launch (L2 loads).  Ends with a consumer barrier.
+template <int BT>
+__device__ void load_source(const FusedParams& p, const Own& o, float* src, float* red, float* inv,
+                            int tid) {
+  const int B = p.B, lane = tid & 31, warp = tid >> 5;
+  float4* s4 = reinterpret_cast<float4*>(src);
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (o.kind == kUp) {
+    float ss[BT];
+    const float4* g4 = reinterpret_cast<const float4*>(p.w.ffn_norm[o.blk]);
+#pragma unroll
+    for (int bb = 0; bb < BT; ++bb) {
+      const float4* x4 = reinterpret_cast<const float4*>(p.f + ((size_t)o.blk * B + bb) * kT);
+      const int k4 = tid;   // kT / 4 == 256 == consumer threads
+      const float4 v = bb < B ? __ldcg(x4 + k4) : zero;
+      const float4 g = g4[k4];
+      ss[bb] = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+      s4[bb * (kT / 4) + k4] = make_float4(v.x * g.x, v.y * g.y, v.z * g.z, v.w * g.w);
+    }
+#pragma unroll
+    for (int bb = 0; bb < BT; ++bb)
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ss[bb] += __shfl_xor_sync(0xffffffffu, ss[bb], off);
+    if (lane == 0)
+#pragma unroll
+      for (int bb = 0; bb < BT; ++bb) red[warp * BT + bb] = ss[bb];
+    consumer_sync();
+    if (tid < BT) {
+      float t = 0.f;
+      for (int w = 0; w < kFC; ++w) t += red[w * BT + tid];
+      inv[tid] = rsqrtf(t / kT + kEps);
+    }
+  } else if (o.kind == kFuse) {
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+#pragma unroll
+      for (int bb = 0; bb < BT; ++bb) {
+        const float4* u4 = reinterpret_cast<const float4*>(p.u + ((size_t)i * B + bb) * kT);
+        s4[(i * BT + bb) * (kT / 4) + tid] = bb < B ? __ldcg(u4 + tid) : zero;
+      }
+  } else {
+#pragma unroll
+    for (int bb = 0; bb < BT; ++bb) {
+      const float4* a4 = reinterpret_cast<const float4*>(p.act + (size_t)bb * kF);
+#pragma unroll
+      for (int k4 = tid; k4 < kF / 4; k4 += kFC * 32)
+        s4[bb * (kF / 4) + k4] = bb < B ? __ldcg(a4 + k4) : zero;
+    }
+  }
+  consumer_sync();
+}
+
+// Finishes the CTA's rows of the phase; the dot product of row segment r for sequence b is the
+// sum of the eight warps' column shares accw[w][r][b], taken in warp order.
+template <int BT>
+__device__ void finish_rows(const FusedParams& p, const Own& o, const float* src, const float* accw,
+                            const float* inv, int tid) {
+  const int B = p.B;
+  auto rowsum = [&](int r, int b) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kFC; ++w) t += accw[(w * kMaxOwnSegs + r) * BT + b];
+    return t;
+  };
+  for (int idx = tid; idx < o.n * B; idx += kFC * 32) {
+    const int r = idx / B, b = idx - r * B, n = o.lo + r;
+    const float acc = rowsum(r, b);
+    if (o.kind == kTower) {
+      p.u[((size_t)o.tower * B + b) * kT + n] = silu(acc * inv[b] + p.w.tower_b[o.tower][n]);
+    } else if (o.kind == kFuse) {
+      const float mean = (src[(0 * BT + b) * kT + n] + src[(1 * BT + b) * kT + n] +
+                          src[(2 * BT + b) * kT + n]) / 3.0f;
+      p.f[(size_t)b * kT + n] = acc + p.w.fuse_b[n] + mean;
+    } else if (o.kind == kUp) {
+      const float ga = acc * inv[b], ua = rowsum(o.n + r, b) * inv[b];
+      p.act[(size_t)b * kF + n] = silu(ga) * ua;
+    } else {
+      p.f[((size_t)(o.blk + 1) * B + b) * kT + n] =
+          __ldcg(p.f + ((size_t)o.blk * B + b) * kT + n) + acc;
+    }
+  }
+}
+
+// Grid-wide barrier for one thread per CTA, after a CTA barrier: a release add on the counter,
+// then acquire loads until `target` CTAs have arrived (bounded).  Returns false when the wait
+// gave up.
+__device__ __forceinline__ bool grid_barrier(int32_t* ctr, int target) {
+  red_release_add_gpu(ctr, 1);
+  if (ld_acquire_gpu(ctr) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (ld_acquire_gpu(ctr) >= target) return true;
+    if (global_timer_ns() - t0 > kGridWaitNs) return false;
+  }
+}
+
+template <int BT>
+__global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedParams p) {
+  extern __shared__ __align__(16) uint8_t fsm[];
+  const int R = p.ring;
+  uint8_t* ring = fsm;
+  float* src = reinterpret_cast<float*>(fsm + (size_t)R * kFStageBytes);
+  float* accw = src + (size_t)max(p.D, 3 * kT) * BT;     // [kFC][kMaxOwnSegs][BT]
+  __shared__ __align__(8) uint64_t full[kMaxRing];
+  __shared__ __align__(8) uint64_t empty[kMaxRing];
+  __shared__ __align__(8) uint64_t src_bar;
+  __shared__ float red[kFC * BT];
+  __shared__ float s_inv[BT];
+  __shared__ int s_last, s_any;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x, G = gridDim.x, B = p.B;
+  if (tid == 0) {
+    for (int i = 0; i < R; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kFC);
+    }
+    mbar_init(&src_bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kFC) {
+    // ---- producer.  First the tower input rows x_i[b] of this CTA's tower (they may come from
+    // the previous kernel), then every weight segment of every phase in the order the consumers
+    // take them; the segments of phase ph+1 are pulled toward L2 when phase ph starts, so HBM
+    // keeps streaming while the grid waits between phases.
+    grid_dependency_wait();
+    const Own o0 = own_rows(0, c, G, p.D);
+    if (lane == 0) mbar_arrive_expect_tx(&src_bar, (uint32_t)(B * p.D * sizeof(float)));
+    __syncwarp();
+    if (lane < B)
+      bulk_load(src + (size_t)lane * p.D, p.x[o0.tower] + (size_t)lane * p.D,
+                (uint32_t)(p.D * sizeof(float)), &src_bar);
+    int k = 0;
+    for (int ph = 0; ph < 6; ++ph) {
+      const Own o = own_rows(ph, c, G, p.D);
+      if (ph + 1 < 6) prefetch_phase(p, own_rows(ph + 1, c, G, p.D), lane);
+      const int ngrp = (o.nseg + kFC - 1) / kFC;
+      for (int ch = 0; ch < o.nchunk; ++ch)
+        for (int g = 0; g < ngrp; ++g, ++k) {
+          const int s = k % R;
+          if (k >= R && !mbar_wait_bounded(&empty[s], (uint32_t)(k / R - 1) & 1u, kFWaitNs) && lane == 0)
+            atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
+          const int n = min(kFC, o.nseg - g * kFC);
+          if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(n * kSegBytes));
+          __syncwarp();
+          if (lane < n)
+            bulk_load(ring + (size_t)s * kFStageBytes + lane * kSegBytes, seg_ptr(p, o, ch, g * kFC + lane),
+                      kSegBytes, &full[s]);
+        }
+    }
+    return;
+  }
+
+  // ---- consumers: warp w owns columns [128w, 128w + 128) of every segment
+  grid_dependency_wait();
+  grid_dependents_launch();
+  float* acc = accw + (size_t)warp * kMaxOwnSegs * BT;
+  const int col4 = 32 * warp + lane;
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  int k = 0;
+  for (int ph = 0; ph < 6; ++ph) {
+    const Own o = own_rows(ph, c, G, p.D);
+    for (int i = lane; i < kMaxOwnSegs * BT; i += 32) acc[i] = 0.f;
+    const bool tower = o.kind == kTower;
+    const float4* gam4 = reinterpret_cast<const float4*>(p.w.tower_norm[o.tower]);
+    float4 gnext = tower ? __ldg(gam4 + col4) : zero;
+    if (tower) {
+      if (!mbar_wait_bounded(&src_bar, 0u, kFWaitNs) && lane == 0) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
+    } else {
+      load_source<BT>(p, o, src, red, s_inv, tid);
+    }
+    __syncwarp();
+    float ssl[BT];
+#pragma unroll
+    for (int bb = 0; bb < BT; ++bb) ssl[bb] = 0.f;
+    const int ngrp = (o.nseg + kFC - 1) / kFC;
+    for (int ch = 0; ch < o.nchunk; ++ch) {
+      const float4 gam = gnext;
+      if (tower && ch + 1 < o.nchunk) gnext = __ldg(gam4 + (ch + 1) * (kSeg / 4) + col4);
+      float4 xs[BT];
+      input_slice<BT>(o, B, p.D, src, ch, col4, gam, ssl, xs);
+      for (int g = 0; g < ngrp; ++g, ++k) {
+        const int s = k % R;
+        if (!mbar_wait_bounded(&full[s], (uint32_t)(k / R) & 1u, kFWaitNs) && lane == 0)
+          atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
+        stage_dot<BT>(ring + (size_t)s * kFStageBytes, min(kFC, o.nseg - g * kFC), col4, xs, acc, g, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+    }
+    if (tower) {
+      // 1 / rms(x_i): the warps' column shares of the sum of squares, summed in warp order
+#pragma unroll
+      for (int bb = 0; bb < BT; ++bb)
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ssl[bb] += __shfl_xor_sync(0xffffffffu, ssl[bb], off);
+      if (lane == 0)
+#pragma unroll
+        for (int bb = 0; bb < BT; ++bb) red[warp * BT + bb] = ssl[bb];
+      consumer_sync();
+      if (tid < BT) {
+        float t = 0.f;
+        for (int w = 0; w < kFC; ++w) t += red[w * BT + tid];
+        s_inv[tid] = rsqrtf(t / p.D + kEps);
+      }
+    }
+    consumer_sync();
+    finish_rows<BT>(p, o, src, accw, s_inv, tid);
+    consumer_sync();
+    if (ph < 5) {
+      if (tid == 0 && !grid_barrier(p.cnt, (ph + 1) * G)) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
+      consumer_sync();
+    }
+  }
+
+  // ---- the last CTA to finish computes q and the gate, then returns the counters to zero
+  if (tid == 0) {
+    s_last = atom_add_acq_rel_gpu(p.cnt + 1, 1) == G - 1;
+    s_any = 0;
+  }
+  consumer_sync();
+  if (!s_last) return;
+  for (int b = warp; b < B; b += kFC)
+    score_and_gate(p.w, p.f + ((size_t)2 * B + b) * kT, b, p.sched, p.theta, p.score, p.flag,
+                   &s_any, lane);
+  consumer_sync();
+  if (tid == 0) {
+    *p.any_flag = s_any;
+    p.cnt[0] = 0;
+    p.cnt[1] = 0;
   }
 }
 
@@ -442,6 +865,39 @@ int head_counter_count(int D) {
   return m + 1;
 }
 
+namespace {
+// device properties and the fused kernels' static shared memory, read by prepare_head_kernel
+int g_fused_static[2] = {-1, -1};   // head_fused_kernel<4>, <8>
+int g_smem_optin = 0;
+int g_coop = 0;
+
+// Fused-head plan: sequence tile, ring depth and dynamic shared memory; bt = 0 where the fused
+// kernel does not apply (batch above 8, D not a multiple of 1024, fewer than 128 SMs, no
+// cooperative launch, or too little shared memory for a ring of two stages), and the six phase
+// kernels run instead.
+struct FusedPlan {
+  int bt, ring;
+  size_t smem;
+};
+
+FusedPlan fused_plan(int B, int D, int n_sms) {
+  FusedPlan pl = {0, 0, 0};
+  if (B < 1 || B > kBTMax || D % kSeg != 0 || n_sms < 128 || !g_coop) return pl;
+  const int bt = B <= 4 ? 4 : 8;
+  const int stat = g_fused_static[bt == 4 ? 0 : 1];
+  if (stat < 0) return pl;
+  const size_t src = (size_t)std::max(D, 3 * kT) * bt * sizeof(float);
+  const size_t res = (size_t)kFC * kMaxOwnSegs * bt * sizeof(float);   // per-warp row sums
+  const long long room = (long long)g_smem_optin - stat - (long long)(src + res);
+  const int ring = (int)std::min<long long>(kMaxRing, room / kFStageBytes);
+  if (ring < 2) return pl;
+  pl.bt = bt;
+  pl.ring = ring;
+  pl.smem = (size_t)ring * kFStageBytes + src + res;
+  return pl;
+}
+}  // namespace
+
 oda_status prepare_head_kernel() {
   // largest input tile: the tower phase with D = 8192 (Kc = 4096)
   oda_status st = check_cuda(cudaFuncSetAttribute(head_phase_kernel<8, 2>,
@@ -449,10 +905,33 @@ oda_status prepare_head_kernel() {
                                                   8 * 4096 * (int)sizeof(float)),
                              "cudaFuncSetAttribute(head)");
   if (st != ODA_OK) return st;
-  return check_cuda(cudaFuncSetAttribute(head_phase_kernel<4, 4>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         4 * 4096 * (int)sizeof(float)),
+  st = check_cuda(cudaFuncSetAttribute(head_phase_kernel<4, 4>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       4 * 4096 * (int)sizeof(float)),
+                  "cudaFuncSetAttribute(head)");
+  if (st != ODA_OK) return st;
+  int dev = 0;
+  st = check_cuda(cudaGetDevice(&dev), "cudaGetDevice");
+  if (st == ODA_OK)
+    st = check_cuda(cudaDeviceGetAttribute(&g_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev),
+                    "cudaDeviceGetAttribute");
+  if (st == ODA_OK)
+    st = check_cuda(cudaDeviceGetAttribute(&g_coop, cudaDevAttrCooperativeLaunch, dev),
+                    "cudaDeviceGetAttribute");
+  if (st != ODA_OK) return st;
+  const void* kernels[2] = {reinterpret_cast<const void*>(head_fused_kernel<4>),
+                            reinterpret_cast<const void*>(head_fused_kernel<8>)};
+  for (int i = 0; i < 2; ++i) {
+    cudaFuncAttributes fa;
+    st = check_cuda(cudaFuncGetAttributes(&fa, kernels[i]), "cudaFuncGetAttributes(head)");
+    if (st != ODA_OK) return st;
+    g_fused_static[i] = (int)fa.sharedSizeBytes;
+    st = check_cuda(cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         g_smem_optin - g_fused_static[i]),
                     "cudaFuncSetAttribute(head)");
+    if (st != ODA_OK) return st;
+  }
+  return ODA_OK;
 }
 
 oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const float* h_prev,
@@ -475,6 +954,49 @@ oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const flo
   for (const void* q : mats)
     if (reinterpret_cast<uintptr_t>(q) & 15)
       return set_error(ODA_ERR_INVALID_ARG, "recall_score: matrices and inputs must be 16-byte aligned");
+  const FusedPlan pl = fused_plan(ctx->cfg.batch, ctx->cfg.head_in_dim, ctx->n_sms);
+  int per_sm = 0;
+  if (pl.bt) {
+    const void* kern = pl.bt == 4 ? reinterpret_cast<const void*>(head_fused_kernel<4>)
+                                  : reinterpret_cast<const void*>(head_fused_kernel<8>);
+    oda_status st = check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFThreads, pl.smem),
+                               "cudaOccupancyMaxActiveBlocksPerMultiprocessor(head)");
+    if (st != ODA_OK) return st;
+  }
+  if (pl.bt && per_sm >= 1) {
+    // one CTA per SM, all resident at once (cooperative launch): the grid barrier needs that
+    FusedParams f;
+    f.w = *w;
+    f.x[0] = h_prev;
+    f.x[1] = emb;
+    f.x[2] = h_loc;
+    f.sched = sched;
+    f.score = score;
+    f.flag = flag;
+    f.any_flag = any_flag;
+    f.u = ctx->head_u;
+    f.f = ctx->head_f;
+    f.act = ctx->head_act;
+    f.cnt = ctx->head_cnt;
+    f.err = ctx->err;
+    f.B = ctx->cfg.batch;
+    f.D = ctx->cfg.head_in_dim;
+    f.ring = pl.ring;
+    f.theta = ctx->cfg.theta;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(ctx->n_sms);
+    lc.blockDim = dim3(kFThreads);
+    lc.dynamicSmemBytes = pl.smem;
+    lc.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    return check_cuda(pl.bt == 4 ? cudaLaunchKernelEx(&lc, head_fused_kernel<4>, f)
+                                 : cudaLaunchKernelEx(&lc, head_fused_kernel<8>, f),
+                      "recall head launch");
+  }
   HeadParams p;
   p.w = *w;
   p.x[0] = h_prev;

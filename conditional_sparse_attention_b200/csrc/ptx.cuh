@@ -1,4 +1,4 @@
-// Thin inline-PTX wrappers for sm_100a: mbarriers, 2-D / 4-D TMA tile loads, ldmatrix, movmatrix,
+// Thin inline-PTX wrappers for sm_100a: mbarriers, 2-D / 4-D TMA tile loads, bulk copies, ldmatrix, movmatrix,
 // bf16 mma.sync, proxy fences and the global timer.  Each wrapper is one instruction.
 #pragma once
 #include <cuda.h>
@@ -94,6 +94,38 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
       ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w),
         "r"(smem_u32(bar))
       : "memory");
+}
+
+// Contiguous bulk copy global -> this CTA's shared memory (both addresses 16-byte aligned, size
+// a multiple of 16), completion counted in bytes on `bar`.  No multicast.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Pulls a contiguous global range (16-byte aligned, size a multiple of 16) toward L2.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+               ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes) : "memory");
+}
+
+// Global counter operations at gpu scope, for the grid-wide barrier: an acquire load, a
+// release add without result, and an acquire-release add that returns the old value.
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(reinterpret_cast<uint64_t>(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_add_gpu(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;"
+               : "=r"(old) : "l"(reinterpret_cast<uint64_t>(p)), "r"(v) : "memory");
+  return old;
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
