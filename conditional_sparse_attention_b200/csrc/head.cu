@@ -609,14 +609,15 @@ __device__ void load_source(const FusedParams& p, const Own& o, float* src, floa
   if (o.kind == kUp) {
     float ss[BT];
     const float4* g4 = reinterpret_cast<const float4*>(p.w.ffn_norm[o.blk]);
+    float4 v[BT];   // kT / 4 == 256 == consumer threads: one float4 of f per sequence each
+#pragma unroll
+    for (int bb = 0; bb < BT; ++bb)
+      v[bb] = bb < B ? __ldcg(reinterpret_cast<const float4*>(p.f + ((size_t)o.blk * B + bb) * kT) + tid) : zero;
+    const float4 g = g4[tid];
 #pragma unroll
     for (int bb = 0; bb < BT; ++bb) {
-      const float4* x4 = reinterpret_cast<const float4*>(p.f + ((size_t)o.blk * B + bb) * kT);
-      const int k4 = tid;   // kT / 4 == 256 == consumer threads
-      const float4 v = bb < B ? __ldcg(x4 + k4) : zero;
-      const float4 g = g4[k4];
-      ss[bb] = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-      s4[bb * (kT / 4) + k4] = make_float4(v.x * g.x, v.y * g.y, v.z * g.z, v.w * g.w);
+      ss[bb] = v[bb].x * v[bb].x + v[bb].y * v[bb].y + v[bb].z * v[bb].z + v[bb].w * v[bb].w;
+      s4[bb * (kT / 4) + tid] = make_float4(v[bb].x * g.x, v[bb].y * g.y, v[bb].z * g.z, v[bb].w * g.w);
     }
 #pragma unroll
     for (int bb = 0; bb < BT; ++bb)
@@ -632,30 +633,55 @@ __device__ void load_source(const FusedParams& p, const Own& o, float* src, floa
       inv[tid] = rsqrtf(t / kT + kEps);
     }
   } else if (o.kind == kFuse) {
+    // every load is issued before the first store
+    float4 v[3][BT];
 #pragma unroll
     for (int i = 0; i < 3; ++i)
 #pragma unroll
-      for (int bb = 0; bb < BT; ++bb) {
-        const float4* u4 = reinterpret_cast<const float4*>(p.u + ((size_t)i * B + bb) * kT);
-        s4[(i * BT + bb) * (kT / 4) + tid] = bb < B ? __ldcg(u4 + tid) : zero;
-      }
+      for (int bb = 0; bb < BT; ++bb)
+        v[i][bb] = bb < B ? __ldcg(reinterpret_cast<const float4*>(p.u + ((size_t)i * B + bb) * kT) + tid)
+                          : zero;
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+#pragma unroll
+      for (int bb = 0; bb < BT; ++bb) s4[(i * BT + bb) * (kT / 4) + tid] = v[i][bb];
   } else {
+    float4 v[BT][2];
 #pragma unroll
-    for (int bb = 0; bb < BT; ++bb) {
-      const float4* a4 = reinterpret_cast<const float4*>(p.act + (size_t)bb * kF);
+    for (int bb = 0; bb < BT; ++bb)
 #pragma unroll
-      for (int k4 = tid; k4 < kF / 4; k4 += kFC * 32)
-        s4[bb * (kF / 4) + k4] = bb < B ? __ldcg(a4 + k4) : zero;
-    }
+      for (int j = 0; j < 2; ++j)
+        v[bb][j] = bb < B ? __ldcg(reinterpret_cast<const float4*>(p.act + (size_t)bb * kF) + tid + j * kFC * 32)
+                          : zero;
+#pragma unroll
+    for (int bb = 0; bb < BT; ++bb)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) s4[bb * (kF / 4) + tid + j * kFC * 32] = v[bb][j];
   }
   consumer_sync();
 }
 
+// The operand of output item idx (row idx / B, sequence idx % B) of the phase that comes from
+// global memory: the tower or fusion bias, or the residual f_j of a down projection (written two
+// phases earlier).  Each thread loads the one for its own item while the phase's stages stream.
+__device__ __forceinline__ float finish_operand(const FusedParams& p, const Own& o, int idx) {
+  const int B = p.B;
+  if (idx >= o.n * B) return 0.f;
+  const int r = idx / B, b = idx - r * B, n = o.lo + r;
+  switch (o.kind) {
+    case kTower: return p.w.tower_b[o.tower][n];
+    case kFuse: return p.w.fuse_b[n];
+    case kUp: return 0.f;
+    default: return __ldcg(p.f + ((size_t)o.blk * B + b) * kT + n);
+  }
+}
+
 // Finishes the CTA's rows of the phase; the dot product of row segment r for sequence b is the
-// sum of the eight warps' column shares accw[w][r][b], taken in warp order.
+// sum of the eight warps' column shares accw[w][r][b], taken in warp order.  `pre` is this
+// thread's finish_operand.
 template <int BT>
 __device__ void finish_rows(const FusedParams& p, const Own& o, const float* src, const float* accw,
-                            const float* inv, int tid) {
+                            const float* inv, float pre, int tid) {
   const int B = p.B;
   auto rowsum = [&](int r, int b) {
     float t = 0.f;
@@ -666,18 +692,18 @@ __device__ void finish_rows(const FusedParams& p, const Own& o, const float* src
   for (int idx = tid; idx < o.n * B; idx += kFC * 32) {
     const int r = idx / B, b = idx - r * B, n = o.lo + r;
     const float acc = rowsum(r, b);
+    const float opnd = idx == tid ? pre : finish_operand(p, o, idx);
     if (o.kind == kTower) {
-      p.u[((size_t)o.tower * B + b) * kT + n] = silu(acc * inv[b] + p.w.tower_b[o.tower][n]);
+      p.u[((size_t)o.tower * B + b) * kT + n] = silu(acc * inv[b] + opnd);
     } else if (o.kind == kFuse) {
       const float mean = (src[(0 * BT + b) * kT + n] + src[(1 * BT + b) * kT + n] +
                           src[(2 * BT + b) * kT + n]) / 3.0f;
-      p.f[(size_t)b * kT + n] = acc + p.w.fuse_b[n] + mean;
+      p.f[(size_t)b * kT + n] = acc + opnd + mean;
     } else if (o.kind == kUp) {
       const float ga = acc * inv[b], ua = rowsum(o.n + r, b) * inv[b];
       p.act[(size_t)b * kF + n] = silu(ga) * ua;
     } else {
-      p.f[((size_t)(o.blk + 1) * B + b) * kT + n] =
-          __ldcg(p.f + ((size_t)o.blk * B + b) * kT + n) + acc;
+      p.f[((size_t)(o.blk + 1) * B + b) * kT + n] = opnd + acc;
     }
   }
 }
@@ -725,8 +751,10 @@ __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedPar
   if (warp == kFC) {
     // ---- producer.  First the tower input rows x_i[b] of this CTA's tower (they may come from
     // the previous kernel), then every weight segment of every phase in the order the consumers
-    // take them; the segments of phase ph+1 are pulled toward L2 when phase ph starts, so HBM
-    // keeps streaming while the grid waits between phases.
+    // take them.  When the producer reaches a phase (its ring is then a few stages ahead of the
+    // consumers, who may still be finishing the previous phase or waiting at the barrier), it
+    // first pulls all of the phase's segments toward L2, so HBM streams at full rate beyond the
+    // ring's depth.
     grid_dependency_wait();
     const Own o0 = own_rows(0, c, G, p.D);
     if (lane == 0) mbar_arrive_expect_tx(&src_bar, (uint32_t)(B * p.D * sizeof(float)));
@@ -737,7 +765,7 @@ __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedPar
     int k = 0;
     for (int ph = 0; ph < 6; ++ph) {
       const Own o = own_rows(ph, c, G, p.D);
-      if (ph + 1 < 6) prefetch_phase(p, own_rows(ph + 1, c, G, p.D), lane);
+      prefetch_phase(p, o, lane);
       const int ngrp = (o.nseg + kFC - 1) / kFC;
       for (int ch = 0; ch < o.nchunk; ++ch)
         for (int g = 0; g < ngrp; ++g, ++k) {
@@ -774,6 +802,7 @@ __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedPar
       load_source<BT>(p, o, src, red, s_inv, tid);
     }
     __syncwarp();
+    const float pre = finish_operand(p, o, tid);
     float ssl[BT];
 #pragma unroll
     for (int bb = 0; bb < BT; ++bb) ssl[bb] = 0.f;
@@ -809,7 +838,7 @@ __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedPar
       }
     }
     consumer_sync();
-    finish_rows<BT>(p, o, src, accw, s_inv, tid);
+    finish_rows<BT>(p, o, src, accw, s_inv, pre, tid);
     consumer_sync();
     if (ph < 5) {
       if (tid == 0 && !grid_barrier(p.cnt, (ph + 1) * G)) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
