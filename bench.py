@@ -306,8 +306,9 @@ def time_head(dec, reps: int = 5) -> float:
 
 
 def run_kernel_only(args, wl, local_rank):
-    """Profiling mode: set up the workload, stage step 0, launch one attention kernel
-    ``--kernel-reps`` times (full: every sequence flagged) and exit."""
+    """Profiling mode: set up the workload, stage step 0, launch one kernel ``--kernel-reps``
+    times (full: the full-set attention with every sequence flagged; local: the local-set
+    attention; head: the recall head on the local hidden state) and exit."""
     import torch
     from conditional_sparse_attention_b200 import oda
     from conditional_sparse_attention_b200.engine import OdaDecoder
@@ -322,9 +323,13 @@ def run_kernel_only(args, wl, local_rank):
             oda.oda_attend_full_if(dec.ctx, dec.layers[a], dec.page_table, dec.pos, ones,
                                    dec.sv["q"][1, a], dec.sv["k"][1, a], dec.sv["v"][1, a],
                                    dec.o[1, a], dec.stream)
-        else:
+        elif args.kernel_only == "local":
             oda.oda_attend_local(dec.ctx, dec.layers[a], dec.page_table, dec.pos, dec.sv["q"][0, a],
                                  dec.sv["k"][0, a], dec.sv["v"][0, a], dec.o[0, a], dec.stream)
+        else:
+            oda.oda_recall_score(dec.ctx, dec.head_w, dec.h_prev, dec.sv["emb"], dec.h[0],
+                                 dec.sv["sched"] if dec.routing_scheduled else None, dec.score,
+                                 dec.flag, dec.any_flag, dec.stream)
     dec.synchronize()
     err = dec.device_error()
     print(json.dumps({"kernel_only": args.kernel_only, "workload": wl.name,
@@ -435,9 +440,7 @@ def run_ours(args, wl, rank, world, local_rank):
     e2e = e2e_detail = None
     if args.e2e:
         host = [b.cpu().pin_memory() for b in store]
-        out_h = torch.empty((wl.B, wl.D), dtype=torch.float32).pin_memory()
-        out_f = torch.empty(wl.B, dtype=torch.int32).pin_memory()
-        out_s = torch.empty(wl.B, dtype=torch.float32).pin_memory()
+        out_r = torch.empty(dec.results.numel(), dtype=torch.float32).pin_memory()
         # the same step inputs (and so the same scheduled flags) as the device-timed loop
         for i in range(2):
             dec.step(host[(W - 1 + i) % n_store])
@@ -451,16 +454,14 @@ def run_ours(args, wl, rank, world, local_rank):
             h0 = time.perf_counter()
             for i in range(n_e2e):
                 dec.step(host[(1 + W + i) % n_store])
-                out_h.copy_(dec.h_prev, non_blocking=True)
-                out_f.copy_(dec.flag, non_blocking=True)
-                out_s.copy_(dec.score, non_blocking=True)
+                dec.read_results(out_r)   # h_prev, score and flags in one device-to-host copy
             host_issue_s = time.perf_counter() - h0
             e1.record(dec.stream)
         torch.cuda.synchronize(dev)
         e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         e2e = {"value": world * n_e2e / (e_ms * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": dec.layout.nbytes,
-               "d2h_bytes_per_step": out_h.numel() * 4 + out_f.numel() * 4 + out_s.numel() * 4}
+               "d2h_bytes_per_step": out_r.numel() * 4}
         # the copies alone, for reading the end-to-end number: uploads back to back on the copy
         # stream, and the read-backs on the step stream
         c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -474,9 +475,7 @@ def run_ours(args, wl, rank, world, local_rank):
         with torch.cuda.stream(dec.stream):
             d0.record(dec.stream)
             for i in range(n_e2e):
-                out_h.copy_(dec.h_prev, non_blocking=True)
-                out_f.copy_(dec.flag, non_blocking=True)
-                out_s.copy_(dec.score, non_blocking=True)
+                dec.read_results(out_r)
             d1.record(dec.stream)
         d1.synchronize()
         e2e_detail = {"upload_us_per_step": c0.elapsed_time(c1) * 1e3 / n_e2e,
@@ -571,8 +570,8 @@ def main():
     ap.add_argument("--eager", action="store_true",
                     help="issue every step's kernels directly instead of replaying a CUDA graph "
                          "(profilers cannot see kernel nodes of graphs with conditional nodes)")
-    ap.add_argument("--kernel-only", choices=["full", "local"], default=None,
-                    help="profiling mode: launch one attention kernel --kernel-reps times and exit")
+    ap.add_argument("--kernel-only", choices=["full", "local", "head"], default=None,
+                    help="profiling mode: launch one kernel (full or local attention, or the recall head) --kernel-reps times and exit")
     ap.add_argument("--kernel-reps", type=int, default=3)
     args = ap.parse_args()
     if args.warmup < 3:

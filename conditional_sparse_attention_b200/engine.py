@@ -118,15 +118,19 @@ class OdaDecoder:
             self.v_pool.append(v)
         self.layers = [oda.kv_layer(self.k_pool[a], self.v_pool[a]) for a in range(L)]
         self.pos = torch.tensor([c + 1 for c in wl.ctx], dtype=torch.int32, device=dev)
-        self.h_prev = torch.from_numpy(inputs.h_prev0(wl)).to(dev)
+        # the step's results (h_{t-1} after the commit, q_t, the routing flags) share one
+        # device block, so they come back to the host in a single copy (read_results)
+        self.results = torch.zeros(B * D + 2 * B, dtype=torch.float32, device=dev)
+        self.h_prev = self.results[:B * D].view(B, D)
+        self.h_prev.copy_(torch.from_numpy(inputs.h_prev0(wl)))
         hp = head_params if head_params is not None else inputs.head_weights(wl, perturb_head)
         self.head_params = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in hp.items()}
         self.head_w = oda.head_weights(self.head_params)
         n_layers = wl.n_layers
         self.o = torch.zeros((2, n_layers, B, D), dtype=torch.float32, device=dev)
         self.h = torch.zeros((2, B, D), dtype=torch.float32, device=dev)
-        self.score = torch.zeros(B, dtype=torch.float32, device=dev)
-        self.flag = torch.zeros(B, dtype=torch.int32, device=dev)
+        self.score = self.results[B * D:B * D + B]
+        self.flag = self.results[B * D + B:].view(torch.int32)
         self.any_flag = torch.zeros(1, dtype=torch.int32, device=dev)
         self.layout = StepLayout(wl)
         # Two staging buffers, used by alternate steps (and one captured graph each): host inputs
@@ -265,6 +269,13 @@ class OdaDecoder:
         if src is not None:
             self.stage(src)
         self.launch()
+
+    def read_results(self, out: torch.Tensor) -> None:
+        """Copies the last step's results (h_prev [B][D], then score [B], then flag [B] as
+        int32 bits) into `out`, a pinned float32 host tensor of B*D + 2B elements, in the step
+        stream's order (asynchronous: synchronize before reading it)."""
+        with torch.cuda.stream(self.stream):
+            out.copy_(self.results, non_blocking=True)
 
     def synchronize(self):
         self.stream.synchronize()

@@ -139,10 +139,18 @@ def test_pinned_host_inputs_equal_device_inputs():
         with torch.cuda.stream(dec.stream):
             for k, t in rec.items():
                 t.copy_(getattr(dec, k), non_blocking=True)
+        # and the single-copy result block: h_prev, then score, then the flags' int32 bits
+        rec["block"] = torch.empty(dec.results.numel(), dtype=torch.float32).pin_memory()
+        dec.read_results(rec["block"])
         outs.append(rec)
     dec.synchronize()
     assert dec.device_error() == 0
+    B, D = wl.B, wl.D
     for s in range(wl.steps):
         for k in ("score", "flag", "h_prev", "pos"):
             assert np.array_equal(outs[s][k].numpy(), ref[s][k]), (s, k)
+        blk = outs[s]["block"].numpy()
+        assert np.array_equal(blk[:B * D].reshape(B, D), ref[s]["h_prev"]), s
+        assert np.array_equal(blk[B * D:B * D + B], ref[s]["score"]), s
+        assert np.array_equal(blk[B * D + B:].view(np.int32), ref[s]["flag"]), s
     dec.close()
