@@ -37,6 +37,7 @@ NCU_FULL_KERNEL_TRAFFIC = {"attention_cu_sha256": "9a82954d8deaa4c9", "bytes": 5
                            "cached_tokens": 4 * 32768}
 UNIT = "steps/s"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e specification; `frac` uses the measured copy peak
 
 
 def traffic_per_token():
@@ -336,6 +337,73 @@ def run_kernel_only(args, wl, local_rank):
                       "launches": args.kernel_reps, "device_error": err}), flush=True)
     dec.close()
 
+SWEEP_CTX = (4096, 16384, 32768, 65536, 131072)
+SWEEP_RHO = (0.0, 0.125, 0.25, 0.5, 1.0)
+
+
+def run_sweep(args, wl0, local_rank):
+    """Recall-rate x context sweep of the decode step on the workload's shapes (batch, heads,
+    layers).  Per context: the whole step (local pass, head, conditional full retry, commit; CUDA
+    graph) at each recall rate, with Bernoulli flags drawn per (sequence, step), and, as the
+    always-full reference, the full-set attention of every sequence and layer (kernels alone: no
+    local pass, no head).  One JSON line per point, then one summary line."""
+    import torch
+    from conditional_sparse_attention_b200.engine import OdaDecoder, fill_step_inputs
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    W, K = args.warmup, args.steps
+    per = W + K
+    points = []
+    for ctx in SWEEP_CTX:
+        wl = wl0.replace(name=f"{wl0.name}_sweep_ctx{ctx}", ctx=(ctx,) * wl0.B, routing="bernoulli",
+                         rates=(0.0,) * wl0.B, steps=per * len(SWEEP_RHO))
+        dec = OdaDecoder(wl, device=dev, capacity_steps=per * len(SWEEP_RHO) + 4)
+        dec.capture()
+        step = 0
+        ones = torch.ones(wl.B, dtype=torch.int32, device=dev)
+        full_ms = None
+        for rho in SWEEP_RHO:
+            wr = wl.replace(rates=(rho,) * wl.B)   # same inputs, the schedule drawn at rate rho
+            bufs = []
+            for i in range(per):
+                buf = torch.zeros(dec.layout.nbytes, dtype=torch.uint8, device=dev)
+                fill_step_inputs(wr, step + i, dec.layout.views(buf))
+                bufs.append(buf)
+            for i in range(W):
+                dec.step(bufs[i])
+            flags = torch.zeros((K, wl.B), dtype=torch.int32, device=dev)
+            dec.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(dec.stream):
+                e0.record(dec.stream)
+                for i in range(K):
+                    dec.step(bufs[W + i])
+                    flags[i].copy_(dec.flag, non_blocking=True)
+                e1.record(dec.stream)
+            e1.synchronize()
+            step += per
+            step_ms = e0.elapsed_time(e1) / K
+            if full_ms is None:
+                full_ms = time_layer_kernels(dec, 1, ones, reps=2) * wl.L
+            pt = {"sweep": True, "ctx": ctx, "rho": rho, "realized_rho": float(flags.float().mean()),
+                  "oda_step_ms": step_ms, "always_full_attention_ms": full_ms,
+                  "oda_over_full": step_ms / full_ms, "steps": K, "warmup": W,
+                  "device_error": dec.device_error()}
+            points.append(pt)
+            print(json.dumps(pt), flush=True)
+        dec.close()
+        del dec, bufs
+        torch.cuda.empty_cache()
+    # per context: the largest swept rate at which the whole ODA step is still faster than the
+    # always-full attention kernels alone
+    cross = {}
+    for ctx in SWEEP_CTX:
+        ok = [p["rho"] for p in points if p["ctx"] == ctx and p["oda_step_ms"] < p["always_full_attention_ms"]]
+        cross[str(ctx)] = max(ok) if ok else None
+    print(json.dumps({"sweep_summary": True, "workload": wl0.name, "B": wl0.B, "layers": wl0.L,
+                      "max_rho_where_oda_is_faster": cross}), flush=True)
+
+
 def run_ours(args, wl, rank, world, local_rank):
     import torch
     from conditional_sparse_attention_b200 import oda
@@ -531,19 +599,22 @@ def run_ours(args, wl, rank, world, local_rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(wl, world, args.eager),
             "roofline": {"bound": "hbm", "achieved": full_gbs, "peak": hbm, "unit": "GB/s",
-                         "frac": full_gbs / hbm, "traffic": full_traffic,
+                         "frac": full_gbs / hbm, "frac_of_nominal": full_gbs / NOMINAL_HBM_GBS,
+                         "traffic": full_traffic,
                          "algorithmic_bytes_per_launch": full_bytes / n_pat_launches,
                          "kernel": "attn_full_kernel (full set, flagged sequences)",
                          "peak_source": peak_src, "launches_timed": n_full,
                          "us_per_launch": full_ms * 1000.0 / sum(pats.values()),
                          "flag_patterns": {"".join(map(str, k)): v for k, v in pats.items()}},
             "step_roofline": {"algorithmic_gb_per_step": total_bytes / K / 1e9,
-                              "achieved_gbs": step_gbs, "frac": step_gbs / hbm},
+                              "achieved_gbs": step_gbs, "frac": step_gbs / hbm,
+                              "frac_of_nominal": step_gbs / NOMINAL_HBM_GBS},
             "local_kernel": {"achieved_gbs": loc_gbs, "frac": loc_gbs / hbm,
                              "us_per_launch": loc_ms * 1000.0},
             # both attention kernels over the timed steps: K local passes and the full-set
             # launches of the realised flag patterns (one per layer of a flagged step)
             "attention_kernels": {"achieved_gbs": att_gbs, "frac": att_gbs / hbm,
+                                  "frac_of_nominal": att_gbs / NOMINAL_HBM_GBS,
                                   "us_per_step": att_us_per_step},
             "recall_head": {"us_per_score": head_ms * 1000.0,
                             "achieved_gbs": head_bytes / (head_ms * 1e-3) / 1e9,
@@ -573,6 +644,8 @@ def main():
     ap.add_argument("--kernel-only", choices=["full", "local", "head"], default=None,
                     help="profiling mode: launch one kernel (full or local attention, or the recall head) --kernel-reps times and exit")
     ap.add_argument("--kernel-reps", type=int, default=3)
+    ap.add_argument("--sweep", action="store_true",
+                    help="recall-rate x context sweep of the step against always-full attention")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -586,6 +659,9 @@ def main():
         return
     if args.kernel_only:
         run_kernel_only(args, wl, local_rank)
+        return
+    if args.sweep:
+        run_sweep(args, wl, local_rank)
         return
     import torch
     if world > 1:

@@ -37,7 +37,11 @@ def _run(B, D, perturb=True, seed=500, sched=None, theta=0.0, bias=0.0, inputs_o
     return P, xs, score.cpu().numpy(), flag.cpu().numpy(), int(anyf.item())
 
 
-@pytest.mark.parametrize("B,D", [(1, 2048), (4, 4096), (8, 2048), (13, 2048), (32, 2048)])
+# fused single-launch head for B <= 8 (ring depth from the shared memory the inputs leave:
+# 5 stages at (1, 2048), 4 at (4, 4096), 3 at (8, 2048) and (2, 8192), 2 at (8, 4096)); the six
+# phase launches for B > 8 and where the inputs do not fit (8, 8192)
+@pytest.mark.parametrize("B,D", [(1, 2048), (4, 4096), (8, 2048), (2, 8192), (8, 4096), (8, 8192),
+                                 (13, 2048), (32, 2048)])
 def test_scores_and_gate_match_oracle(B, D):
     P, xs, score, flag, anyf = _run(B, D, perturb=True, seed=500 + B + D)
     ref = np.array([recall_head(P, xs[0][b], xs[1][b], xs[2][b]) for b in range(B)])
@@ -46,6 +50,31 @@ def test_scores_and_gate_match_oracle(B, D):
         if abs(ref[b]) >= TIE_BAND:
             assert flag[b] == int(route_full(ref[b]))
     assert anyf == int(flag.any())
+
+
+def test_repeated_scores_are_bitwise_stable():
+    """The fused head returns its grid-barrier counters to zero: back-to-back scores on one
+    context (eager, no synchronisation between them) give the same bits."""
+    from conditional_sparse_attention_b200 import oda
+    B, D = 4, 4096
+    Hq = D // 128
+    wl = configs.cfg0().replace(name="t_head_rep", seed=700, B=B, Hq=Hq, Hkv=Hq // 2, ctx=(10,) * B)
+    P = inputs.head_weights(wl, perturb=True)
+    xs = [gen.normal_f32(gen.key(700, 90, i), B * D).reshape(B, D) for i in range(3)]
+    Pd = {k: torch.from_numpy(v).to("cuda") for k, v in P.items()}
+    c = oda.oda_create(oda.make_config(B, wl.Hq, wl.Hkv, 4, D))
+    hx = [torch.from_numpy(np.ascontiguousarray(x)).to("cuda") for x in xs]
+    outs = []
+    for _ in range(5):
+        score = torch.zeros(B, device="cuda")
+        flag = torch.zeros(B, dtype=torch.int32, device="cuda")
+        anyf = torch.zeros(1, dtype=torch.int32, device="cuda")
+        oda.oda_recall_score(c, oda.head_weights(Pd), hx[0], hx[1], hx[2], None, score, flag, anyf)
+        outs.append(score)
+    torch.cuda.synchronize()
+    assert oda.oda_get_error(c) == 0
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
 
 
 def test_unperturbed_init_and_bias_shift():
