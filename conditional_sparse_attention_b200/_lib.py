@@ -42,6 +42,10 @@ class OdaHeadWeights(ctypes.Structure):
                 ("out_norm", c_void_p), ("out_w", c_void_p), ("out_b", c_void_p)]
 
 
+class OdaHeadGrads(ctypes.Structure):
+    _fields_ = OdaHeadWeights._fields_
+
+
 class OdaState(ctypes.Structure):
     _fields_ = [("rec", c_void_p), ("conv", c_void_p), ("n_layers", c_int32), ("heads", c_int32),
                 ("dk", c_int32), ("dv", c_int32), ("conv_taps", c_int32), ("conv_width", c_int32)]
@@ -62,6 +66,10 @@ _SIGS = {
                              c_void_p], c_int32),
     "oda_recall_score": ([c_void_p, _P(OdaHeadWeights), c_void_p, c_void_p, c_void_p, c_void_p,
                           c_void_p, c_void_p, c_void_p, c_void_p], c_int32),
+    "oda_recall_grad_workspace_bytes": ([c_int32, c_int32], ctypes.c_size_t),
+    "oda_recall_grad": ([_P(OdaHeadWeights), _P(OdaHeadGrads), c_int32, c_int32, c_void_p, c_void_p,
+                         c_void_p, c_void_p, c_void_p, c_void_p, ctypes.c_float, c_void_p, c_void_p,
+                         c_void_p, c_void_p, ctypes.c_size_t, c_void_p], c_int32),
     "oda_commit": ([c_void_p, _P(OdaKVLayer), c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
                     c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p], c_int32),
     "oda_snapshot": ([c_void_p, _P(OdaState), _P(OdaState), c_void_p], c_int32),

@@ -220,6 +220,21 @@ oda_status oda_recall_score(oda_ctx* ctx, const oda_head_weights* w, const float
   return oda::launch_recall_head(ctx, w, h_prev, emb, h_loc, sched, score, flag, any_flag, stream);
 }
 
+size_t oda_recall_grad_workspace_bytes(int32_t batch, int32_t head_in_dim) {
+  if (batch < 1 || head_in_dim < 1) return 0;
+  return oda::recall_grad_workspace_bytes(batch, head_in_dim);
+}
+
+oda_status oda_recall_grad(const oda_head_weights* w, const oda_head_grads* grad, int32_t batch,
+                           int32_t head_in_dim, const float* h_prev, const float* emb,
+                           const float* h_loc, const float* p_full, const float* p_local,
+                           const int32_t* valid, float lambda, float* loss, float* q, float* y,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!(lambda >= 0.f)) return set_error(ODA_ERR_INVALID_ARG, "recall_grad: lambda must be >= 0");
+  return oda::launch_recall_grad(w, grad, batch, head_in_dim, h_prev, emb, h_loc, p_full, p_local,
+                                 valid, lambda, loss, q, y, workspace, workspace_bytes, stream);
+}
+
 oda_status oda_commit(oda_ctx* ctx, const oda_kv_layer* layers, int32_t n_layers,
                       const int32_t* page_table, int32_t* pos, const int32_t* flag,
                       const void* k_stage_local, const void* v_stage_local,

@@ -68,6 +68,14 @@ oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const flo
 size_t head_part_floats(int B, int D);
 int head_counter_count(int D);
 
+// head_grad.cu
+size_t recall_grad_workspace_bytes(int B, int D);
+oda_status launch_recall_grad(const oda_head_weights* w, const oda_head_grads* gr, int B, int D,
+                              const float* h_prev, const float* emb, const float* h_loc,
+                              const float* p_full, const float* p_local, const int32_t* valid,
+                              float lam, float* loss, float* q, float* y, void* workspace,
+                              size_t workspace_bytes, cudaStream_t s);
+
 // commit.cu
 oda_status launch_commit(oda_ctx* ctx, const oda_kv_layer* layers, int32_t n_layers,
                          const int32_t* page_table, int32_t* pos, const int32_t* flag,

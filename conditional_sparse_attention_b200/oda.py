@@ -12,7 +12,8 @@ from typing import Optional, Sequence
 import torch
 
 from . import _lib
-from ._lib import OdaConfig, OdaError, OdaHeadWeights, OdaKVLayer, OdaState, check  # noqa: F401
+from ._lib import (OdaConfig, OdaError, OdaHeadGrads, OdaHeadWeights, OdaKVLayer,  # noqa: F401
+                   OdaState, check)
 
 _c = ctypes.c_void_p
 
@@ -66,9 +67,9 @@ def kv_layer(k: torch.Tensor, v: torch.Tensor) -> OdaKVLayer:
     return OdaKVLayer(k.data_ptr(), v.data_ptr(), int(k.shape[0]))
 
 
-def head_weights(P: dict) -> OdaHeadWeights:
+def head_weights(P: dict, cls=OdaHeadWeights):
     """Descriptor from a dict of device fp32 tensors named as in include/oda.h."""
-    w = OdaHeadWeights()
+    w = cls()
     for i in range(3):
         w.tower_norm[i] = P[f"tower_norm{i}"].data_ptr()
         w.tower_w[i] = P[f"tower_w{i}"].data_ptr()
@@ -82,6 +83,11 @@ def head_weights(P: dict) -> OdaHeadWeights:
     w.out_norm, w.out_w, w.out_b = (P["out_norm"].data_ptr(), P["out_w"].data_ptr(),
                                     P["out_b"].data_ptr())
     return w
+
+
+def head_grads(G: dict) -> OdaHeadGrads:
+    """Gradient-buffer descriptor from a dict of device fp32 tensors (names as the weights)."""
+    return head_weights(G, OdaHeadGrads)
 
 
 def state(rec: torch.Tensor, conv: torch.Tensor) -> OdaState:
@@ -131,6 +137,19 @@ def oda_recall_score(ctx, w: OdaHeadWeights, h_prev, emb, h_loc, sched, score, f
                      stream=None):
     check(_lib.load().oda_recall_score(ctx.handle, ctypes.byref(w), _p(h_prev), _p(emb), _p(h_loc),
                                        _p(sched), _p(score), _p(flag), _p(any_flag), _s(stream)))
+
+
+def oda_recall_grad_workspace_bytes(batch: int, head_in_dim: int) -> int:
+    return int(_lib.load().oda_recall_grad_workspace_bytes(batch, head_in_dim))
+
+
+def oda_recall_grad(w: OdaHeadWeights, grad: OdaHeadGrads, batch: int, head_in_dim: int, h_prev,
+                    emb, h_loc, p_full, p_local, valid, lam: float, loss, q, y, workspace,
+                    stream=None):
+    check(_lib.load().oda_recall_grad(ctypes.byref(w), ctypes.byref(grad), batch, head_in_dim,
+                                      _p(h_prev), _p(emb), _p(h_loc), _p(p_full), _p(p_local),
+                                      _p(valid), float(lam), _p(loss), _p(q), _p(y), _p(workspace),
+                                      workspace.numel() * workspace.element_size(), _s(stream)))
 
 
 def oda_commit(ctx, layers: Sequence[OdaKVLayer], page_table, pos, flag, k_stage_local,

@@ -116,6 +116,23 @@ typedef struct {
   const float* out_b;          /* [1]                                                   */
 } oda_head_weights;
 
+/* Gradient buffers of the recall head: the same tensors and shapes as oda_head_weights,
+ * written (overwritten) by oda_recall_grad. */
+typedef struct {
+  float* tower_norm[3];
+  float* tower_w[3];
+  float* tower_b[3];
+  float* fuse_w;
+  float* fuse_b;
+  float* ffn_norm[2];
+  float* ffn_gate[2];
+  float* ffn_up[2];
+  float* ffn_down[2];
+  float* out_norm;
+  float* out_w;
+  float* out_b;
+} oda_head_grads;
+
 /* Recurrent and conv state of the linear-recurrent layers of a hybrid backbone, fp32.
  * rec: [B][n_layers][heads][dv][dk]; conv: [B][n_layers][conv_taps][conv_width]. */
 typedef struct {
@@ -196,6 +213,28 @@ oda_status oda_index_positions(oda_ctx* ctx, int32_t mode, const int32_t* pos, c
 oda_status oda_recall_score(oda_ctx* ctx, const oda_head_weights* w, const float* h_prev,
                             const float* emb, const float* h_loc, const int32_t* sched,
                             float* score, int32_t* flag, int32_t* any_flag, cudaStream_t stream);
+
+/* Training-side arithmetic of the recall head (the head is the only trained part).
+ * [notes §2.1, eq. g_t]: gain g = ln p_full - ln p_local (nats), where p_full and p_local are
+ * the probabilities of the next token under the full and the local pass; [notes §2.2, eqs.
+ * d_t, y_t]: d = g - lambda, label y = sign(d) ln(1 + |d|); [notes §2.2, eq. L(psi)]: loss =
+ * mean over the valid sequences (valid[b] != 0: reference label valid and the two access sets
+ * different) of Huber with threshold 1 of q - y, 0 when none is valid.  Computes, on `stream`:
+ * q [B] (the head's scores, as oda_recall_score computes them up to rounding order), y [B]
+ * (0 where not valid), loss [1], and the gradient of the loss with respect to every head
+ * parameter into `grad` (summed over the batch; every buffer overwritten).  The absolute
+ * differences of the interaction take sign(0) = 0.  h_prev, emb, h_loc: fp32 [B][D] device.
+ * All arithmetic fp32 with fixed reduction orders (deterministic).
+ * Limits: 1 <= batch <= 16; head_in_dim a multiple of 1024 in 1024..8192.  Matrices, their
+ * gradients, the inputs and the workspace must be 16-byte aligned.  `workspace` is device
+ * memory of at least oda_recall_grad_workspace_bytes(batch, head_in_dim) bytes, owned by the
+ * caller, not used across calls.  No context is needed (the call allocates nothing). */
+size_t oda_recall_grad_workspace_bytes(int32_t batch, int32_t head_in_dim);
+oda_status oda_recall_grad(const oda_head_weights* w, const oda_head_grads* grad, int32_t batch,
+                           int32_t head_in_dim, const float* h_prev, const float* emb,
+                           const float* h_loc, const float* p_full, const float* p_local,
+                           const int32_t* valid, float lambda, float* loss, float* q, float* y,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------- commit -------------- */
 
