@@ -29,7 +29,7 @@ constexpr int kGT = 1024;         // tower width
 constexpr int kGF = 2048;         // FFN width
 constexpr int kGZ = 9 * kGT;      // interaction width
 constexpr int kCol = 1024;        // columns per chunk
-constexpr int kRowsFwd = 32;      // rows per CTA in the forward GEMV (8 warps x 4)
+constexpr int kRowsFwd = 16;      // rows per CTA in the forward GEMV (8 warps x 2)
 constexpr int kRowsBwd = 16;      // rows per CTA in the backward pass
 constexpr int kGB = 16;           // largest batch
 constexpr float kGEps = 1e-6f;
@@ -63,7 +63,8 @@ __device__ float block_sum_f(float v, float* red) {
 
 // ------------------------------------------------------------------ forward GEMV
 // part[c][b][n] = sum_{k in chunk c} W[n][k] X[b][k]  for rows n of the CTA's block; X rows
-// are ldx floats apart.  Grid (N / 32, K / 1024), 256 threads: warp w takes rows 4w..4w+3.
+// are ldx floats apart.  Grid (N / 16, K / 1024), 256 threads: warp w takes rows 2w, 2w+1, whose
+// loads are all issued before the first product.
 __global__ void __launch_bounds__(256) gemv_rows_kernel(const float* W, int N, int K, const float* X,
                                                         int ldx, int B, float* part) {
   extern __shared__ float xs[];   // [B][1024]
@@ -75,21 +76,27 @@ __global__ void __launch_bounds__(256) gemv_rows_kernel(const float* W, int N, i
   }
   __syncthreads();
   const float4* x4 = reinterpret_cast<const float4*>(xs);
-  for (int r = 0; r < 4; ++r) {
-    const int n = rb * kRowsFwd + warp * 4 + r;
-    const float4* w4 = reinterpret_cast<const float4*>(W + (size_t)n * K + k0);
-    float4 wv[kCol / 128];
+  const int n0 = rb * kRowsFwd + warp * 2;
+  float4 wv[2][kCol / 128];
 #pragma unroll
-    for (int j = 0; j < kCol / 128; ++j) wv[j] = __ldcs(w4 + lane + 32 * j);
-    for (int b = 0; b < B; ++b) {
-      float acc = 0.f;
+  for (int r = 0; r < 2; ++r) {
+    const float4* w4 = reinterpret_cast<const float4*>(W + (size_t)(n0 + r) * K + k0);
 #pragma unroll
-      for (int j = 0; j < kCol / 128; ++j) {
-        const float4 xv = x4[b * (kCol / 4) + lane + 32 * j];
-        acc += wv[j].x * xv.x + wv[j].y * xv.y + wv[j].z * xv.z + wv[j].w * xv.w;
-      }
-      acc = warp_sum_f(acc);
-      if (lane == 0) part[((size_t)c * B + b) * N + n] = acc;
+    for (int j = 0; j < kCol / 128; ++j) wv[r][j] = __ldcs(w4 + lane + 32 * j);
+  }
+  for (int b = 0; b < B; ++b) {
+    float acc[2] = {0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < kCol / 128; ++j) {
+      const float4 xv = x4[b * (kCol / 4) + lane + 32 * j];
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+        acc[r] += wv[r][j].x * xv.x + wv[r][j].y * xv.y + wv[r][j].z * xv.z + wv[r][j].w * xv.w;
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const float t = warp_sum_f(acc[r]);
+      if (lane == 0) part[((size_t)c * B + b) * N + n0 + r] = t;
     }
   }
 }
@@ -146,7 +153,8 @@ __global__ void fwd_reduce_kernel(const FwdArgs a) {
 // For rows [16 rb, 16 rb + 16) of W [N][K] and columns [1024 c, 1024 c + 1024):
 //   dW[n][k]        = sum_b dY[b][n] X[b][k]          (each (n, k) written by one thread)
 //   part[rb][b][k]  = sum_{n in the block} W[n][k] dY[b][n]
-// 256 threads; thread t owns the four columns 1024 c + 4t .. +3.  Grid (N / 16, K / 1024).
+// 256 threads; thread t owns the four columns 1024 c + 4t .. +3.  Grid (N / 16, K / 1024).  The
+// weight loads of RB rows (16 for batches up to 8, else 8) are issued before their products.
 template <int BM>
 __global__ void __launch_bounds__(256) bwd_rows_kernel(const float* W, int N, int K, const float* dY,
                                                        int ldy, const float* X, int ldx, int B,
@@ -166,26 +174,33 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(const float* W, int N, in
     acc[b] = zero;
   }
   __syncthreads();
-#pragma unroll 4
-  for (int r = 0; r < kRowsBwd; ++r) {
-    const size_t off = (size_t)(n0 + r) * K + col;
-    const float4 w = __ldcs(reinterpret_cast<const float4*>(W + off));
-    float4 g = zero;
+  constexpr int RB = BM <= 8 ? 16 : 8;
+#pragma unroll 1
+  for (int r0 = 0; r0 < kRowsBwd; r0 += RB) {
+    float4 wv[RB];
 #pragma unroll
-    for (int b = 0; b < BM; ++b) {
-      if (b < B) {
-        const float d = dys[r * BM + b];
-        g.x += d * x[b].x;
-        g.y += d * x[b].y;
-        g.z += d * x[b].z;
-        g.w += d * x[b].w;
-        acc[b].x += d * w.x;
-        acc[b].y += d * w.y;
-        acc[b].z += d * w.z;
-        acc[b].w += d * w.w;
+    for (int r = 0; r < RB; ++r)
+      wv[r] = __ldcs(reinterpret_cast<const float4*>(W + (size_t)(n0 + r0 + r) * K + col));
+#pragma unroll
+    for (int r = 0; r < RB; ++r) {
+      const float4 w = wv[r];
+      float4 g = zero;
+#pragma unroll
+      for (int b = 0; b < BM; ++b) {
+        if (b < B) {
+          const float d = dys[(r0 + r) * BM + b];
+          g.x += d * x[b].x;
+          g.y += d * x[b].y;
+          g.z += d * x[b].z;
+          g.w += d * x[b].w;
+          acc[b].x += d * w.x;
+          acc[b].y += d * w.y;
+          acc[b].z += d * w.z;
+          acc[b].w += d * w.w;
+        }
       }
+      __stcs(reinterpret_cast<float4*>(dW + (size_t)(n0 + r0 + r) * K + col), g);
     }
-    __stcs(reinterpret_cast<float4*>(dW + off), g);
   }
 #pragma unroll
   for (int b = 0; b < BM; ++b)
