@@ -318,6 +318,22 @@ def run_kernel_only(args, wl, local_rank):
     dec.stage(dec.make_step_buffer(0))
     dec.synchronize()
     ones = torch.ones(wl.B, dtype=torch.int32, device=dev)
+    if args.kernel_only == "grad":
+        # one training step of the recall head on the step's inputs, with synthetic next-token
+        # probabilities of the two passes (every position valid)
+        grads = {k: torch.empty_like(v) for k, v in dec.head_params.items()}
+        gw = oda.head_grads(grads)
+        p_full = torch.linspace(0.2, 0.8, wl.B, device=dev)
+        p_local = torch.linspace(0.7, 0.1, wl.B, device=dev)
+        loss = torch.zeros(1, device=dev)
+        q = torch.zeros(wl.B, device=dev)
+        y = torch.zeros(wl.B, device=dev)
+        ws = torch.empty(oda.oda_recall_grad_workspace_bytes(wl.B, wl.D), dtype=torch.uint8,
+                         device=dev)
+
+        def grad_step(d):
+            oda.oda_recall_grad(d.head_w, gw, wl.B, wl.D, d.h_prev, d.sv["emb"], d.h[0], p_full,
+                                p_local, ones, 0.01, loss, q, y, ws, d.stream)
     for r in range(args.kernel_reps):
         a = r % wl.L
         if args.kernel_only == "full":
@@ -327,10 +343,12 @@ def run_kernel_only(args, wl, local_rank):
         elif args.kernel_only == "local":
             oda.oda_attend_local(dec.ctx, dec.layers[a], dec.page_table, dec.pos, dec.sv["q"][0, a],
                                  dec.sv["k"][0, a], dec.sv["v"][0, a], dec.o[0, a], dec.stream)
-        else:
+        elif args.kernel_only == "head":
             oda.oda_recall_score(dec.ctx, dec.head_w, dec.h_prev, dec.sv["emb"], dec.h[0],
                                  dec.sv["sched"] if dec.routing_scheduled else None, dec.score,
                                  dec.flag, dec.any_flag, dec.stream)
+        else:
+            grad_step(dec)
     dec.synchronize()
     err = dec.device_error()
     print(json.dumps({"kernel_only": args.kernel_only, "workload": wl.name,
@@ -641,8 +659,9 @@ def main():
     ap.add_argument("--eager", action="store_true",
                     help="issue every step's kernels directly instead of replaying a CUDA graph "
                          "(profilers cannot see kernel nodes of graphs with conditional nodes)")
-    ap.add_argument("--kernel-only", choices=["full", "local", "head"], default=None,
-                    help="profiling mode: launch one kernel (full or local attention, or the recall head) --kernel-reps times and exit")
+    ap.add_argument("--kernel-only", choices=["full", "local", "head", "grad"], default=None,
+                    help="profiling mode: launch one kernel (full or local attention, the recall "
+                         "head) or one recall-head training step --kernel-reps times and exit")
     ap.add_argument("--kernel-reps", type=int, default=3)
     ap.add_argument("--sweep", action="store_true",
                     help="recall-rate x context sweep of the step against always-full attention")

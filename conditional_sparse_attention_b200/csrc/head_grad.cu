@@ -48,7 +48,7 @@ __device__ __forceinline__ float warp_sum_f(float v) {
   return v;
 }
 
-// Block-wide sum (256 threads) in a fixed order; every thread receives the total.
+// Block-wide sum (up to 1024 threads) in a fixed order; every thread receives the total.
 __device__ float block_sum_f(float v, float* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   v = warp_sum_f(v);
@@ -154,9 +154,10 @@ __global__ void fwd_reduce_kernel(const FwdArgs a) {
 //   dW[n][k]        = sum_b dY[b][n] X[b][k]          (each (n, k) written by one thread)
 //   part[rb][b][k]  = sum_{n in the block} W[n][k] dY[b][n]
 // 256 threads; thread t owns the four columns 1024 c + 4t .. +3.  Grid (N / 16, K / 1024).  The
-// weight loads of RB rows (16 for batches up to 8, else 8) are issued before their products.
+// weight loads of 8 rows are issued before their products; with batches up to 8 two CTAs share
+// an SM, so one CTA's loads overlap the other's products and stores.
 template <int BM>
-__global__ void __launch_bounds__(256) bwd_rows_kernel(const float* W, int N, int K, const float* dY,
+__global__ void __launch_bounds__(256, BM <= 8 ? 2 : 1) bwd_rows_kernel(const float* W, int N, int K, const float* dY,
                                                        int ldy, const float* X, int ldx, int B,
                                                        float* dW, float* part) {
   __shared__ float dys[kRowsBwd * BM];   // [row][b]
@@ -174,7 +175,7 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(const float* W, int N, in
     acc[b] = zero;
   }
   __syncthreads();
-  constexpr int RB = BM <= 8 ? 16 : 8;
+  constexpr int RB = 8;
 #pragma unroll 1
   for (int r0 = 0; r0 < kRowsBwd; r0 += RB) {
     float4 wv[RB];
@@ -220,15 +221,25 @@ struct BwdArgs {
   float* out2;           // gate: dv
 };
 
-// Sums the partials in row-block order (then the second set) and applies the epilogue:
-// gate: da -> dg = da v SiLU'(g), dv = da SiLU(g).  One thread per (b, k).
-__global__ void bwd_reduce_kernel(const BwdArgs a) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= a.B * a.K) return;
+// Sums the partials and applies the epilogue (gate: da -> dg = da v SiLU'(g), dv = da
+// SiLU(g)).  A CTA of 256 takes 32 consecutive outputs (b, k); its eight warps each sum every
+// eighth row block (the second set continues the numbering), and warp 0 adds the eight slices
+// in order: a fixed order, with eight times the loads in flight of one thread per output.
+__global__ void __launch_bounds__(256) bwd_reduce_kernel(const BwdArgs a) {
+  __shared__ float sl[8][33];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int i = blockIdx.x * 32 + lane;   // B * K is a multiple of 32
   const int b = i / a.K, k = i - b * a.K;
   float acc = 0.f;
-  for (int r = 0; r < a.nrb; ++r) acc += a.part[((size_t)r * a.B + b) * a.K + k];
-  for (int r = 0; r < a.nrb2; ++r) acc += a.part2[((size_t)r * a.B + b) * a.K + k];
+  for (int r = w; r < a.nrb + a.nrb2; r += 8)
+    acc += r < a.nrb ? a.part[((size_t)r * a.B + b) * a.K + k]
+                     : a.part2[((size_t)(r - a.nrb) * a.B + b) * a.K + k];
+  sl[w][lane] = acc;
+  __syncthreads();
+  if (w != 0) return;
+  acc = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc += sl[j][lane];
   if (a.epi == kBwdStore) {
     a.out[i] = acc;
   } else {
@@ -239,9 +250,9 @@ __global__ void bwd_reduce_kernel(const BwdArgs a) {
 }
 
 // ------------------------------------------------------------------ small kernels
-// Per sequence (one CTA of 256 per b): s[b] = 1 / rms(x_b), y_b = x_b s gamma.
+// Per sequence (one CTA of 1024 per b): s[b] = 1 / rms(x_b), y_b = x_b s gamma.
 __global__ void rms_kernel(const float* x, int K, const float* gamma, float* s, float* y) {
-  __shared__ float red[8];
+  __shared__ float red[32];
   const int b = blockIdx.x;
   const float* xb = x + (size_t)b * K;
   float ss = 0.f;
@@ -270,10 +281,10 @@ __global__ void interaction_kernel(const float* u, int B, float* z) {
   zb[8 * kGT] = fabsf(u1 - u2);
 }
 
-// Per sequence b (one CTA of 256): the score q = w_o . (f2 s gamma_o) + b_o; keeps s_o and n_o.
+// Per sequence b (one CTA of 1024): the score q = w_o . (f2 s gamma_o) + b_o; keeps s_o and n_o.
 __global__ void score_kernel(const float* f2, const float* gamma, const float* w_o, const float* b_o,
                              float* s_o, float* n_o, float* q) {
-  __shared__ float red[8];
+  __shared__ float red[32];
   const int b = blockIdx.x;
   const float* fb = f2 + (size_t)b * kGT;
   float ss = 0.f;
@@ -335,7 +346,7 @@ __global__ void labels_kernel(const float* q, const float* p_full, const float* 
 __global__ void rms_backward_kernel(const float* dy, const float* dq, const float* w_o,
                                     const float* x, const float* s, const float* gamma, int K,
                                     bool accumulate, float* dx_out) {
-  __shared__ float red[8];
+  __shared__ float red[32];
   const int b = blockIdx.x;
   const float sc = s[b];
   const float* xb = x + (size_t)b * K;
@@ -522,14 +533,14 @@ oda_status launch_recall_grad(const oda_head_weights* w, const oda_head_grads* g
   };
   auto red = [&](BwdArgs a) {
     a.B = B;
-    bwd_reduce_kernel<<<(B * a.K + 255) / 256, 256, 0, s>>>(a);
+    bwd_reduce_kernel<<<B * a.K / 32, 256, 0, s>>>(a);
   };
   float* f[3] = {ws.f, ws.f + (size_t)B * kGT, ws.f + 2 * (size_t)B * kGT};
 
   // ---- forward recompute, keeping every activation the backward needs
   for (int i = 0; i < 3; ++i) {
     float* nx = ws.nx + (size_t)i * B * D;
-    rms_kernel<<<B, 256, 0, s>>>(xs[i], D, w->tower_norm[i], ws.sx + i * B, nx);
+    rms_kernel<<<B, 1024, 0, s>>>(xs[i], D, w->tower_norm[i], ws.sx + i * B, nx);
     gemv(w->tower_w[i], kGT, D, nx);
     FwdArgs a = {};
     a.nchunk = D / kCol;
@@ -557,7 +568,7 @@ oda_status launch_recall_grad(const oda_head_weights* w, const oda_head_grads* g
     float* g = ws.g + (size_t)j * B * kGF;
     float* v = ws.v + (size_t)j * B * kGF;
     float* act = ws.a + (size_t)j * B * kGF;
-    rms_kernel<<<B, 256, 0, s>>>(f[j], kGT, w->ffn_norm[j], ws.sf + j * B, m);
+    rms_kernel<<<B, 1024, 0, s>>>(f[j], kGT, w->ffn_norm[j], ws.sf + j * B, m);
     gemv(w->ffn_gate[j], kGF, kGT, m);
     FwdArgs a = {};
     a.nchunk = 1;
@@ -580,14 +591,14 @@ oda_status launch_recall_grad(const oda_head_weights* w, const oda_head_grads* g
     d.out = f[j + 1];
     fwd(d);
   }
-  score_kernel<<<B, 256, 0, s>>>(f[2], w->out_norm, w->out_w, w->out_b, ws.so, ws.no, q);
+  score_kernel<<<B, 1024, 0, s>>>(f[2], w->out_norm, w->out_w, w->out_b, ws.so, ws.no, q);
   labels_kernel<<<1, 32, 0, s>>>(q, p_full, p_local, valid, B, lam, y, ws.dq, loss);
 
   // ---- backward
   out_grad_kernel<<<kGT / 256, 256, 0, s>>>(ws.dq, ws.no, B, gr->out_w, gr->out_b);
   norm_weight_grad_kernel<<<kGT / 256, 256, 0, s>>>(nullptr, ws.dq, w->out_w, f[2], ws.so, B, kGT,
                                                     gr->out_norm);
-  rms_backward_kernel<<<B, 256, 0, s>>>(nullptr, ws.dq, w->out_w, f[2], ws.so, w->out_norm, kGT, false,
+  rms_backward_kernel<<<B, 1024, 0, s>>>(nullptr, ws.dq, w->out_w, f[2], ws.so, w->out_norm, kGT, false,
                                         ws.dF);
   for (int j = 1; j >= 0; --j) {
     const float* m = ws.m + (size_t)j * B * kGT;
@@ -615,7 +626,7 @@ oda_status launch_recall_grad(const oda_head_weights* w, const oda_head_grads* g
     red(b2);
     norm_weight_grad_kernel<<<kGT / 256, 256, 0, s>>>(ws.dM, nullptr, nullptr, f[j], ws.sf + j * B, B, kGT,
                                                       gr->ffn_norm[j]);
-    rms_backward_kernel<<<B, 256, 0, s>>>(ws.dM, nullptr, nullptr, f[j], ws.sf + j * B, w->ffn_norm[j],
+    rms_backward_kernel<<<B, 1024, 0, s>>>(ws.dM, nullptr, nullptr, f[j], ws.sf + j * B, w->ffn_norm[j],
                                           kGT, true, ws.dF);
   }
   batch_sum_kernel<<<kGT / 256, 256, 0, s>>>(ws.dF, B, kGT, gr->fuse_b);
