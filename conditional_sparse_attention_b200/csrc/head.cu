@@ -15,13 +15,13 @@
 // in one cooperative launch of all six phases (head_fused_kernel, further down).  Larger batches
 // run six phase launches, each a split-K GEMV: a CTA streams a 32-row x Kc slab of one weight
 // matrix exactly once with 16-byte non-allocating loads and multiplies it against a
-// shared-memory tile of up to 8 sequences' inputs; lanes reduce with a 31-shuffle butterfly.  The input transform of a phase (RMSNorm
-// scale, the interaction vector, the gated activation) is applied while the tile is built, and
-// the output epilogue (bias, SiLU, residual) runs in the last CTA of each row block, which sums
-// the split-K partials in a fixed order (deterministic results).  The last row block of the
-// final phase also computes q and the gate.  Six launches per score; each may start while the
-// previous one finishes (programmatic dependent launch) and pulls its weight slab toward L2
-// before waiting for the previous phase's outputs.
+// shared-memory tile of up to 8 sequences' inputs; lanes reduce with a 31-shuffle butterfly.
+// The input transform of a phase (RMSNorm scale, the interaction vector, the gated activation)
+// is applied while the tile is built, and the output epilogue (bias, SiLU, residual) runs in the
+// last CTA of each row block, which sums the split-K partials in a fixed order (deterministic
+// results).  The last row block of the final phase also computes q and the gate.  Each phase
+// launch may start while the previous one finishes (programmatic dependent launch) and pulls its
+// weight slab toward L2 before waiting for the previous phase's outputs.
 #include <algorithm>
 #include <cmath>
 
