@@ -82,6 +82,7 @@ _SIGS = {
     "oda_graph_destroy": ([c_void_p], c_int32),
     "oda_get_error": ([c_void_p, _P(c_int32)], c_int32),
     "oda_clear_error": ([c_void_p, c_void_p], c_int32),
+    "oda_probe_wait": ([c_void_p, c_int32, ctypes.c_int64, c_void_p], c_int32),
     "oda_status_string": ([c_int32], ctypes.c_char_p),
     "oda_last_error": ([], ctypes.c_char_p),
     "oda_version": ([], c_int32),

@@ -29,9 +29,45 @@ oda_status check_cuda(cudaError_t e, const char* what) {
   return set_error(ODA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
+oda_status validate_attention_config(const oda_config& c, const char* who) {
+  if (c.batch < 1 || c.batch > ODA_MAX_BATCH)
+    return set_error(ODA_ERR_UNSUPPORTED, "%s: batch must be 1..%d", who, ODA_MAX_BATCH);
+  if (c.n_q_heads < 1 || c.n_kv_heads < 1 || c.n_q_heads % c.n_kv_heads != 0 ||
+      c.n_q_heads / c.n_kv_heads > 8)
+    return set_error(ODA_ERR_UNSUPPORTED, "%s: need Hq %% Hkv == 0 and Hq/Hkv <= 8", who);
+  if (c.head_dim != 128) return set_error(ODA_ERR_UNSUPPORTED, "%s: head_dim must be 128", who);
+  if (c.page_size != 16) return set_error(ODA_ERR_UNSUPPORTED, "%s: page_size must be 16", who);
+  if (c.max_pages < 1 || (int64_t)c.max_pages * 16 > INT32_MAX - 1)
+    return set_error(ODA_ERR_INVALID_ARG, "%s: max_pages out of range", who);
+  if (c.sinks < 0 || c.sinks > 16) return set_error(ODA_ERR_UNSUPPORTED, "%s: sinks must be 0..16", who);
+  if (c.window < 1) return set_error(ODA_ERR_INVALID_ARG, "%s: window must be >= 1", who);
+  if (c.deterministic != 0 && c.deterministic != 1)
+    return set_error(ODA_ERR_INVALID_ARG, "%s: deterministic must be 0 or 1", who);
+  return ODA_OK;
+}
+
 __global__ void set_condition_kernel(cudaGraphConditionalHandle h, const int32_t* any_flag) {
   grid_dependency_wait();   // any_flag comes from the kernel before (programmatic launch)
   cudaGraphSetConditional(h, *any_flag != 0 ? 1u : 0u);
+}
+
+// Diagnostic: one bounded wait that can never complete, through the same helpers the kernels
+// use.  which = 0: an mbarrier that nothing arrives on (the copy-ring waits); which = 1: a
+// grid barrier whose target is one CTA more than the grid (the fused head's phase barrier).
+// The wait gives up after limit_ns and sets ODA_DEVERR_WAIT_TIMEOUT; the counter is handed
+// back to zero before the kernel returns.
+__global__ void wait_probe_kernel(int which, uint64_t limit_ns, int32_t* ctr, int32_t* err) {
+  __shared__ __align__(8) uint64_t bar;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  bool ok;
+  if (which == 0) {
+    ok = mbar_wait_bounded(&bar, 0u, limit_ns);
+  } else {
+    ok = grid_barrier_bounded(ctr, (int)gridDim.x + 1, limit_ns);
+    atomicSub(ctr, 1);
+  }
+  if (!ok) atomicOr(err, ODA_DEVERR_WAIT_TIMEOUT);
 }
 
 oda_status launch_set_condition(cudaGraphConditionalHandle h, const int32_t* any_flag,
@@ -110,21 +146,12 @@ oda_status oda_create(const oda_config* cfg, oda_ctx** out) {
   *out = nullptr;
   if (!cfg) return set_error(ODA_ERR_INVALID_ARG, "create: cfg is NULL");
   const oda_config& c = *cfg;
-  if (c.batch < 1 || c.batch > ODA_MAX_BATCH)
-    return set_error(ODA_ERR_UNSUPPORTED, "create: batch must be 1..%d", ODA_MAX_BATCH);
-  if (c.n_q_heads < 1 || c.n_kv_heads < 1 || c.n_q_heads % c.n_kv_heads != 0 ||
-      c.n_q_heads / c.n_kv_heads > 8)
-    return set_error(ODA_ERR_UNSUPPORTED, "create: need Hq %% Hkv == 0 and Hq/Hkv <= 8");
-  if (c.head_dim != 128) return set_error(ODA_ERR_UNSUPPORTED, "create: head_dim must be 128");
-  if (c.page_size != 16) return set_error(ODA_ERR_UNSUPPORTED, "create: page_size must be 16");
-  if (c.max_pages < 1 || (int64_t)c.max_pages * 16 > INT32_MAX - 1)
-    return set_error(ODA_ERR_INVALID_ARG, "create: max_pages out of range");
-  if (c.sinks < 0 || c.sinks > 16) return set_error(ODA_ERR_UNSUPPORTED, "create: sinks must be 0..16");
-  if (c.window < 1) return set_error(ODA_ERR_INVALID_ARG, "create: window must be >= 1");
+  oda_status vs = oda::validate_attention_config(c, "create");
+  if (vs != ODA_OK) return vs;
   if (c.head_in_dim < 512 || c.head_in_dim > 8192 || c.head_in_dim % 512 != 0)
     return set_error(ODA_ERR_UNSUPPORTED, "create: head_in_dim must be a multiple of 512 in 512..8192");
-  if ((c.overlap_layers != 0 && c.overlap_layers != 1) || (c.deterministic != 0 && c.deterministic != 1))
-    return set_error(ODA_ERR_INVALID_ARG, "create: overlap_layers and deterministic must be 0 or 1");
+  if (c.overlap_layers != 0 && c.overlap_layers != 1)
+    return set_error(ODA_ERR_INVALID_ARG, "create: overlap_layers must be 0 or 1");
 
   oda_ctx* x = new oda_ctx();
   x->cfg = c;
@@ -373,6 +400,16 @@ oda_status oda_graph_destroy(oda_graph* g) {
   if (g->graph) cudaGraphDestroy(g->graph);
   delete g;
   return ODA_OK;
+}
+
+oda_status oda_probe_wait(oda_ctx* ctx, int32_t which, int64_t limit_ns, cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "probe_wait: ctx is NULL");
+  if ((which != 0 && which != 1) || limit_ns < 1000 || limit_ns > 1000000000)
+    return set_error(ODA_ERR_INVALID_ARG, "probe_wait: which must be 0 or 1, limit 1 us .. 1 s");
+  ctx->prev_attention = false;
+  // the fused head's barrier counter: zero between launches, and back to zero after the probe
+  oda::wait_probe_kernel<<<1, 1, 0, stream>>>(which, (uint64_t)limit_ns, ctx->head_cnt, ctx->err);
+  return check_cuda(cudaGetLastError(), "probe_wait launch");
 }
 
 oda_status oda_get_error(oda_ctx* ctx, int32_t* device_error) {

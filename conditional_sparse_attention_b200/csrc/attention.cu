@@ -1263,11 +1263,15 @@ int attention_smem_bytes(int g) {
 // 38 KB at g = 8, within the 192 KB of stages)
 int local_smem_bytes(int) { return 1024 + kStagesBytesL; }
 
-// Sets the shared-memory limits and returns the persistent grid size for group size g.
+// Sets the shared-memory limits and returns the persistent grid size for group size g.  The
+// limit is a per-function setting shared by every context of the process, so it is always set
+// to the largest group's need (g = 8): a context created later with a smaller g must not lower
+// it under a launch of an earlier context.
 oda_status prepare_attention_kernel(int g, int n_sms, int* ctas) {
   const int smem = attention_smem_bytes(g);
   oda_status st = check_cuda(
-      cudaFuncSetAttribute(attn_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+      cudaFuncSetAttribute(attn_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           attention_smem_bytes(8)),
       "cudaFuncSetAttribute(full attention)");
   if (st == ODA_OK)
     st = check_cuda(cudaFuncSetAttribute(attn_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1397,7 +1401,8 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 struct NoAllocDevice {
   unsigned char* scratch = nullptr;   // device address of g_noalloc_scratch on this device
-  int ctas = 0;                       // persistent grid size of the full-set kernel
+  int n_sms = 0;
+  int ctas[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};   // persistent grid size per group size g
   bool ready = false;
 };
 constexpr int kNoAllocMaxDevices = 64;
@@ -1405,8 +1410,10 @@ NoAllocDevice g_noalloc[kNoAllocMaxDevices];
 std::mutex g_noalloc_mu;
 
 // Once per device, with that device current: the array's device address (host code only
-// sees a stand-in symbol) and the grid size.
-oda_status noalloc_setup(int g, NoAllocDevice** out) {
+// sees a stand-in symbol); once per (device, g): the kernel's shared-memory limit and the
+// persistent grid size, from the same occupancy query a context uses, so both entry points
+// launch the same grid and split the work the same way.
+oda_status noalloc_setup(int g, NoAllocDevice** out, int* ctas) {
   int dev = 0;
   oda_status st = check_cuda(cudaGetDevice(&dev), "cudaGetDevice");
   if (st != ODA_OK) return st;
@@ -1419,16 +1426,21 @@ oda_status noalloc_setup(int g, NoAllocDevice** out) {
     void* ptr = nullptr;
     st = check_cuda(cudaGetSymbolAddress(&ptr, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
     if (st != ODA_OK) return st;
-    int n_sms = 0;
-    st = check_cuda(cudaDeviceGetAttribute(&n_sms, cudaDevAttrMultiProcessorCount, dev),
+    st = check_cuda(cudaDeviceGetAttribute(&d.n_sms, cudaDevAttrMultiProcessorCount, dev),
                     "cudaDeviceGetAttribute");
     if (st != ODA_OK) return st;
     d.scratch = static_cast<unsigned char*>(ptr);
-    d.ctas = n_sms;   // one CTA per SM: fits the shared memory of every g
     d.ready = true;
   }
-  (void)g;
+  if (d.ctas[g] == 0) {
+    st = prepare_attention_kernel(g, d.n_sms, &d.ctas[g]);
+    if (st != ODA_OK) {
+      d.ctas[g] = 0;
+      return st;
+    }
+  }
   *out = &d;
+  *ctas = d.ctas[g];
   return ODA_OK;
 }
 
@@ -1443,10 +1455,8 @@ oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* l
                                     cudaStream_t stream) {
   if (!cfg) return set_error(ODA_ERR_INVALID_ARG, "noalloc: cfg is NULL");
   const oda_config& cf = *cfg;
-  if (cf.batch < 1 || cf.batch > ODA_MAX_BATCH || cf.n_q_heads < 1 || cf.n_kv_heads < 1 ||
-      cf.n_q_heads % cf.n_kv_heads != 0 || cf.n_q_heads / cf.n_kv_heads > 8 || cf.head_dim != 128 ||
-      cf.page_size != 16 || cf.max_pages < 1 || (int64_t)cf.max_pages * 16 > INT32_MAX - 1)
-    return set_error(ODA_ERR_UNSUPPORTED, "noalloc: configuration outside what the kernel supports");
+  oda_status st = validate_attention_config(cf, "noalloc");
+  if (st != ODA_OK) return st;
   if (!layer || !layer->k || !layer->v || !page_table || !pos || !flag || !q || !k_new || !v_new ||
       !out)
     return set_error(ODA_ERR_INVALID_ARG, "noalloc: null pointer argument");
@@ -1459,18 +1469,13 @@ oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* l
     return set_error(ODA_ERR_INVALID_ARG, "noalloc: q/k_new/v_new/out must be 4-byte aligned");
   const int g = cf.n_q_heads / cf.n_kv_heads;
   NoAllocDevice* d = nullptr;
-  oda_status st = noalloc_setup(g, &d);
-  if (st != ODA_OK) return st;
-  // the shared-memory limit is a per-function setting that a context created later may have
-  // lowered: raise it to this call's need (host-side, no allocation)
-  st = check_cuda(cudaFuncSetAttribute(attn_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       attention_smem_bytes(8)),
-                  "cudaFuncSetAttribute(full attention)");
+  int ctas = 0;
+  st = noalloc_setup(g, &d, &ctas);
   if (st != ODA_OK) return st;
   // scratch layout: completion counters [B*Hkv] | claim counters [B*Hkv] | error word |
   // partial (m, l) | partial O
   const size_t pairs = (size_t)cf.batch * cf.n_kv_heads;
-  const size_t slots = (size_t)d->ctas + pairs;
+  const size_t slots = (size_t)ctas + pairs;
   const size_t cnt_bytes = ((2 * pairs + 1) * sizeof(int32_t) + 255) / 256 * 256;
   const size_t ml_bytes = (slots * g * 2 * sizeof(float) + 255) / 256 * 256;
   const size_t o_bytes = slots * g * 128 * sizeof(float);
@@ -1519,8 +1524,8 @@ oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* l
   p.mode = 1;
   p.cluster = 1;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(128.0));
-  p.cta_perm = cta_stride(d->ctas);
-  attn_full_kernel<<<d->ctas, kThreads, attention_smem_bytes(g), stream>>>(tmA, tmB, p);
+  p.cta_perm = cta_stride(ctas);
+  attn_full_kernel<<<ctas, kThreads, attention_smem_bytes(g), stream>>>(tmA, tmB, p);
   return check_cuda(cudaGetLastError(), "noalloc full attention launch");
 }
 

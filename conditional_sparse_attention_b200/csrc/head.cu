@@ -708,21 +708,6 @@ __device__ void finish_rows(const FusedParams& p, const Own& o, const float* src
   }
 }
 
-// Grid-wide barrier for one thread per CTA, after a CTA barrier: a release add on the counter,
-// then acquire loads until `target` CTAs have arrived (bounded).  Returns false when the wait
-// gave up.
-__device__ __forceinline__ bool grid_barrier(int32_t* ctr, int target) {
-  red_release_add_gpu(ctr, 1);
-  if (ld_acquire_gpu(ctr) >= target) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (ld_acquire_gpu(ctr) >= target) return true;
-    if (global_timer_ns() - t0 > kGridWaitNs) return false;
-  }
-}
-
 template <int BT>
 __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedParams p) {
   extern __shared__ __align__(16) uint8_t fsm[];
@@ -841,7 +826,7 @@ __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedPar
     finish_rows<BT>(p, o, src, accw, s_inv, pre, tid);
     consumer_sync();
     if (ph < 5) {
-      if (tid == 0 && !grid_barrier(p.cnt, (ph + 1) * G)) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
+      if (tid == 0 && !grid_barrier_bounded(p.cnt, (ph + 1) * G, kGridWaitNs)) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
       consumer_sync();
     }
   }

@@ -44,6 +44,9 @@ namespace oda {
 
 oda_status set_error(oda_status s, const char* fmt, ...);
 oda_status check_cuda(cudaError_t e, const char* what);
+// Shape checks shared by oda_create and the allocation-free attention entry point: every field
+// of oda_config except head_in_dim, theta and overlap_layers.
+oda_status validate_attention_config(const oda_config& c, const char* who);
 
 // attention.cu
 oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32_t* page_table,

@@ -1,8 +1,10 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, 2-D / 4-D TMA tile loads, bulk copies, ldmatrix, movmatrix,
-// bf16 mma.sync, proxy fences and the global timer.  Each wrapper is one instruction.
+// bf16 / f16 mma.sync, e4m3 conversions, proxy fences and the global timer.  Each wrapper is one
+// instruction (plus the register moves its operand widths need).
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace oda {
@@ -128,6 +130,21 @@ __device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
   return old;
 }
 
+// Grid-wide barrier for one thread per CTA, after a CTA barrier: a release add on the counter,
+// then acquire loads until `target` arrivals are counted; gives up after `limit_ns` of wall
+// time and returns false (the caller records a device error).
+__device__ __forceinline__ bool grid_barrier_bounded(int* ctr, int target, uint64_t limit_ns) {
+  red_release_add_gpu(ctr, 1);
+  if (ld_acquire_gpu(ctr) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (ld_acquire_gpu(ctr) >= target) return true;
+    if (global_timer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -159,6 +176,47 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       " {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D += A(16x16, row) * B(16x8, col); f16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9},"
+      " {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two e4m3 codes (bits 0-7 and 8-15 of x) -> f16x2 (the low code in the low half); exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t x) {
+  uint32_t y;
+  asm("{\n .reg .b16 lo;\n cvt.u16.u32 lo, %1;\n cvt.rn.f16x2.e4m3x2 %0, lo;\n}\n"
+      : "=r"(y) : "r"(x));
+  return y;
+}
+
+// Two fp32 values -> e4m3 codes with round-to-nearest-even and saturation to +-448; lo in bits
+// 0-7, hi in bits 8-15.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint32_t y;
+  asm("{\n .reg .b16 r;\n cvt.rn.satfinite.e4m3x2.f32 r, %1, %2;\n cvt.u32.u16 %0, r;\n}\n"
+      : "=r"(y) : "f"(hi), "f"(lo));
+  return y;
+}
+
+// f16x2 from two fp32 values (lo in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t y;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(y) : "f"(hi), "f"(lo));
+  return y;
+}
+
+__device__ __forceinline__ float f16_lo_to_f32(uint32_t x) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(x & 0xFFFFu)));
+}
+__device__ __forceinline__ float f16_hi_to_f32(uint32_t x) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(x >> 16)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 lo, __nv_bfloat16 hi) {

@@ -230,6 +230,10 @@ def oda_clear_error(ctx, stream=None):
     check(_lib.load().oda_clear_error(ctx.handle, _s(stream)))
 
 
+def oda_probe_wait(ctx, which: int, limit_ns: int, stream=None):
+    check(_lib.load().oda_probe_wait(ctx.handle, which, int(limit_ns), _s(stream)))
+
+
 def oda_version() -> int:
     return int(_lib.load().oda_version())
 

@@ -177,14 +177,21 @@ oda_status oda_attend_full_if(oda_ctx* ctx, const oda_kv_layer* layer, const int
  * It is meant for callers that cannot allocate device memory: code running inside a host
  * framework that only lends it buffers, or a latency-critical loop where cudaMalloc's
  * implicit device synchronisation is not acceptable.
- *   - cfg: the shape (same rules as oda_create; overlap_layers and head_in_dim are ignored).
+ *   - cfg: the shape, checked by the same rules as oda_create except that head_in_dim, theta
+ *     and overlap_layers are ignored.
+ *   - It launches the same persistent grid as a context on the same device would (two CTAs
+ *     per SM where the group's shared memory allows it, else one), so with
+ *     cfg->deterministic = 1 its outputs are bit-identical to oda_attend_full_if's; with 0
+ *     both round within the attention tolerance of each other.
  *   - device_error: optional device int32 that receives sticky ODA_DEVERR_* bits (OR-ed in,
  *     never cleared by the call); NULL keeps them in the static scratch, unread.
- *   - Returns ODA_ERR_UNSUPPORTED, launching nothing, when the shape needs more scratch than
- *     the array holds (about (SMs + B*Hkv) * g * 520 bytes plus 4 * B*Hkv).
- *   - The first call on a device looks up the array's device address and sets the kernel's
- *     shared-memory limit (with that device current); make that first call before any stream
- *     capture.  Each call clears the counters it needs with cudaMemsetAsync on `stream`.
+ *   - Scratch needed, in bytes, with P = B*Hkv, S = grid + P (grid as above, 148 or 296 CTAs
+ *     on a B200) and g = Hq/Hkv:  roundup256(8*P + 4) + roundup256(8*g*S) + 512*g*S.  A shape
+ *     needing more than the array holds is refused with ODA_ERR_UNSUPPORTED, launching nothing.
+ *   - The first call on a device (and the first for each group size g) looks up the array's
+ *     device address and sets the kernel's shared-memory limit (with that device current);
+ *     make that first call before any stream capture.  Each call clears the counters it needs
+ *     with cudaMemsetAsync on `stream`.
  *   - All calls share the one array: calls that may overlap on the GPU (other streams, other
  *     host threads) race and must be serialised by the caller. */
 oda_status oda_attend_full_if_noalloc(const oda_config* cfg, const oda_kv_layer* layer,
@@ -288,6 +295,15 @@ oda_status oda_graph_launch(oda_graph* g, cudaStream_t stream);
 oda_status oda_graph_destroy(oda_graph* g);
 
 /* ------------------------------------------------------------- errors -------------- */
+
+/* Diagnostic of the bounded waits (no counterpart in the method notes): runs, on `stream`,
+ * one wait that can never complete, through the same device helpers the kernels use, with a
+ * limit of limit_ns (1 us .. 1 s).  which = 0: an mbarrier wait with no arrival (the page and
+ * weight copy rings); which = 1: the grid-wide phase barrier of the fused recall head, with a
+ * target one CTA above the grid.  The wait gives up after the limit, sets
+ * ODA_DEVERR_WAIT_TIMEOUT in the context's error word and returns; the context stays usable
+ * (clear the word with oda_clear_error).  No fault, trap or endless loop is involved. */
+oda_status oda_probe_wait(oda_ctx* ctx, int32_t which, int64_t limit_ns, cudaStream_t stream);
 
 /* Waits for all work on the device, then reads (and keeps) the sticky device error word into
  * *device_error (host int32).  Returns ODA_ERR_DEVICE if it is non-zero. */

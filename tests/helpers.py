@@ -3,7 +3,8 @@ from __future__ import annotations
 
 import numpy as np
 
-# Tolerances (the attention and score bars of the decode-path target):
+# Tolerances: attention outputs within max-abs 1e-2 and relative L2 2e-3, recall scores within
+# relative 1e-4 (a floor of 1e-3 on |q|), routing compared outside the |q| < 1e-5 tie band:
 ATTN_MAX_ABS = 1e-2     # per (sequence, layer) output
 ATTN_REL_L2 = 2e-3
 SCORE_REL = 1e-4        # |dq| <= 1e-4 * max(|q_ref|, 1e-3)

@@ -215,3 +215,22 @@ def test_full_set_fixed_pattern_is_bitwise_repeatable():
     for b in range(s.wl.B):
         ok, ma, rel = attn_close(outs[0][b], s.oracle(b, 1))
         assert ok, f"b={b} ctx={ctx[b]} max_abs={ma:.3g} rel_l2={rel:.3g}"
+
+
+def test_context_with_smaller_group_keeps_earlier_context_working():
+    """The full-set kernel's shared-memory limit is one setting per process: creating a context
+    with g = 1 after one with g = 8 must not break the g = 8 context's launches."""
+    from conditional_sparse_attention_b200 import oda
+    ctx = [3000, 131]
+    s8 = Setup(_wl(ctx, 64, 8, seed=85))           # g = 8: the largest shared-memory need
+    c1 = oda.oda_create(oda.make_config(2, 4, 4, s8.max_pages, 512))   # g = 1, created later
+    flag = torch.ones(2, dtype=torch.int32, device="cuda")
+    out = torch.full((2, 64, 128), 7.0, device="cuda")
+    s8.oda.oda_attend_full_if(s8.ctx, s8.layer, s8.pt, s8.pos, flag, s8.q, s8.kn, s8.vn, out)
+    torch.cuda.synchronize()
+    assert s8.oda.oda_get_error(s8.ctx) == 0
+    got = out.cpu().numpy()
+    for b in range(2):
+        ok, ma, rel = attn_close(got[b], s8.oracle(b, 1))
+        assert ok, (b, ma, rel)
+    c1.close()

@@ -71,6 +71,39 @@ def test_noalloc_matches_context_entry_point_twice():
                 assert np.all(out[b] == 5.0), f"unflagged row {b} was written"
 
 
+def test_noalloc_bit_identical_in_deterministic_mode():
+    """With deterministic = 1 both entry points launch the same grid with the same page
+    pattern, so their outputs agree bit for bit (on two calls in a row)."""
+    from conditional_sparse_attention_b200 import oda
+    ctx_lens = [60000, 900, 2053, 4097, 33]
+    wl, cfg, layer, pt, pos, q, kn, vn, _keep = _setup(ctx_lens, seed=101)
+    cfg.deterministic = 1
+    flag = torch.ones(wl.B, dtype=torch.int32, device="cuda")
+    ref = torch.zeros((wl.B, wl.Hq, 128), device="cuda")
+    c = oda.oda_create(cfg)
+    oda.oda_attend_full_if(c, layer, pt, pos, flag, q, kn, vn, ref)
+    torch.cuda.synchronize()
+    assert oda.oda_get_error(c) == 0
+    for _ in range(2):
+        out = torch.zeros_like(ref)
+        oda.oda_attend_full_if_noalloc(cfg, layer, pt, pos, flag, q, kn, vn, out)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+    c.close()
+
+
+def test_noalloc_refuses_invalid_config_fields():
+    from conditional_sparse_attention_b200 import _lib, oda
+    wl, cfg, layer, pt, pos, q, kn, vn, _keep = _setup([100, 200])
+    out = torch.zeros((2, 32, 128), device="cuda")
+    flag = torch.ones(2, dtype=torch.int32, device="cuda")
+    for field, val in (("deterministic", 2), ("sinks", -1), ("window", 0)):
+        bad = oda.make_config(2, 32, 8, cfg.max_pages, 4096)
+        setattr(bad, field, val)
+        with pytest.raises(_lib.OdaError):
+            oda.oda_attend_full_if_noalloc(bad, layer, pt, pos, flag, q, kn, vn, out)
+
+
 def test_noalloc_refuses_shapes_beyond_its_scratch():
     from conditional_sparse_attention_b200 import _lib, oda
     wl, cfg, layer, pt, pos, q, kn, vn, _keep = _setup([100, 200])
