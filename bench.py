@@ -29,10 +29,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "ODA decode-attn steps/s + % of HBM peak, 128K ctx, 12.5% recall, 1 B200"
 
-# DRAM bytes (read + write) of one full-set attention launch from the ncu capture summarised in
-# profiles/attn_full_kernel_cfg2_ctx32k_l2.md (4 flagged sequences x 32768 cached tokens); the
-# bench scales it to its own launches by cached tokens processed.  Valid only for the kernel
-# source it was taken from (first 16 hex digits of the file's SHA-256).
+# DRAM bytes (read + write) of one full-set attention launch from an ncu capture of the
+# 32K-context, 2-layer profiling workload (4 flagged sequences x 32768 cached tokens); the bench
+# scales it to its own launches by cached tokens processed.  Valid only for the kernel source it
+# was taken from (first 16 hex digits of the file's SHA-256).
 NCU_FULL_KERNEL_TRAFFIC = {"attention_cu_sha256": "9a82954d8deaa4c9", "bytes": 541364992,
                            "cached_tokens": 4 * 32768}
 UNIT = "steps/s"
@@ -165,58 +165,83 @@ def max_over_ranks(ms: float, world: int, device=None) -> float:
 
 
 # --------------------------------------------------------------------- oracle sample
-class OracleSample:
-    """A bounded sample of one step of the workload for the CPU oracle: sequence 0 of layer 0,
-    the first ``kv_heads`` KV heads (with their query-head groups), local and full attention,
-    plus one recall-head score.  Inputs are generated once, outside the timed region."""
+def timed_steps(W: int, K: int) -> list:
+    """Step indices whose inputs the K timed steps of the GPU arm use (after the first step and
+    W warm-up steps, cycling through W + K stored step inputs)."""
+    n_store = W + K
+    return [(1 + W + i) % n_store for i in range(K)]
 
-    def __init__(self, wl, kv_heads: int = 1):
+
+class OracleStepSample:
+    """The CPU oracle's cost of one decode step of the workload, composed from timed parts.
+
+    Each part is one call of the oracle exactly as its decode step (oracle.step.run_pass)
+    makes it, on sequence 0 / attention layer 0 of the workload's step-0 inputs:
+      * local attention of one (sequence, layer) over S^L, all KV heads;
+      * full attention of one (sequence, layer) over S^F, all KV heads;
+      * one recall-head score (the oracle scores sequence by sequence).
+    A step costs L*B local calls, one full call per flagged (sequence, layer) and B head
+    scores; the flags are the workload's seeded schedule for the GPU arm's timed steps (the
+    head's own gate where the workload routes on the head, counted at the workload's expected
+    rate).  Full calls are scaled from sequence 0's context to each flagged sequence's by the
+    cached tokens, the only size that changes their work; so are the local calls, because the
+    oracle's decode step hands every call the whole cache of its sequence.  Inputs are generated
+    once, outside the timed region."""
+
+    def __init__(self, wl, W: int, K: int):
         import numpy as np
         from workload import inputs
         self.wl = wl
-        self.kv_heads = kv_heads
-        g = wl.Hq // wl.Hkv
         self.t = wl.ctx[0] + 1
-        q, kn, vn = inputs.step_qkv(wl, 0, 0, 0)
-        self.q = np.ascontiguousarray(q[0, :kv_heads * g])
-        self.kn = np.ascontiguousarray(kn[0, :kv_heads])
-        self.vn = np.ascontiguousarray(vn[0, :kv_heads])
-        self.kc = np.ascontiguousarray(inputs.cache_tokens(wl, "k", 0, 0, self.t - 1)[:, :kv_heads])
-        self.vc = np.ascontiguousarray(inputs.cache_tokens(wl, "v", 0, 0, self.t - 1)[:, :kv_heads])
+        q, kn, vn = inputs.step_qkv(wl, 0, wl.attn_layers[0], 0)
+        self.q, self.kn, self.vn = q[0], kn[0], vn[0]
+        self.kc = inputs.cache_tokens(wl, "k", 0, 0, self.t - 1)
+        self.vc = inputs.cache_tokens(wl, "v", 0, 0, self.t - 1)
         self.P = inputs.head_weights(wl)
         self.e = inputs.emb(wl, 0).astype(np.float64)[0]
         self.hp = inputs.h_prev0(wl).astype(np.float64)[0]
-        per_tok = wl.Hkv * 128 * 2 * 2
-        self.head_bytes = inputs.head_param_count(wl.D) * 4
-        rates = list(wl.rates) if wl.rates else [0.4] * wl.B
-        self.exp_step_bytes = sum(min(self.t, wl.sinks + wl.window) * per_tok * wl.L +
-                                  r * self.t * per_tok * wl.L for r in rates) + self.head_bytes
+        # flagged (sequence, step) pairs of the timed steps -> full calls per step, in units of
+        # sequence 0's context
+        if wl.routing == "bernoulli":
+            steps = timed_steps(W, K)
+            fl = np.array([inputs.schedule(wl, s) for s in steps])
+        else:
+            fl = np.full((1, wl.B), 0.4)
+        rel = np.array([(c + 1) / self.t for c in wl.ctx])
+        self.full_units = float((fl * rel[None, :]).sum(axis=1).mean())
+        self.local_units = float(rel.sum())
+        self.flagged_per_step = float(fl.sum(axis=1).mean())
 
-    def run(self):
-        """Returns (algorithmic bytes processed, seconds)."""
+    def run(self) -> dict:
+        """Seconds of each part (one timed call each)."""
         import numpy as np
         from oracle.attention import attend_bits
         from oracle.head import recall_head
         from oracle.sets import full_set, local_set
         wl, t = self.wl, self.t
-        per_head_tok = 128 * 2 * 2
         t0 = time.perf_counter()
         o_l = attend_bits(self.q, self.kc, self.vc, self.kn, self.vn, local_set(t, wl.sinks, wl.window))
+        t1 = time.perf_counter()
         o_f = attend_bits(self.q, self.kc, self.vc, self.kn, self.vn, full_set(t))
+        t2 = time.perf_counter()
         sc = recall_head(self.P, self.hp, self.e, self.e)
-        dt = time.perf_counter() - t0
+        t3 = time.perf_counter()
         assert np.isfinite(o_l).all() and np.isfinite(o_f).all() and np.isfinite(sc)
-        nbytes = (min(t, wl.sinks + wl.window) + t) * per_head_tok * self.kv_heads + self.head_bytes
-        return nbytes, dt
+        return {"local_s": t1 - t0, "full_s": t2 - t1, "head_s": t3 - t2}
 
-    def describe(self, nbytes, dt):
-        return (f"fp64 oracle on sequence 0, layer 0, {self.kv_heads} of {self.wl.Hkv} KV heads: "
-                f"local attention (|S^L|={min(self.t, 2052)}) + full attention (t={self.t}) + one "
-                f"recall-head score = {nbytes / 1e6:.0f} MB of algorithmic bytes in {dt:.2f} s; "
-                f"steps/s = bytes/s / {self.exp_step_bytes / 1e9:.2f} GB (expected bytes per step)")
+    def step_seconds(self, part: dict) -> float:
+        wl = self.wl
+        return (wl.L * self.local_units * part["local_s"] + wl.L * self.full_units * part["full_s"] +
+                wl.B * part["head_s"])
 
-    def steps_per_s(self, nbytes, dt):
-        return (nbytes / dt) / self.exp_step_bytes
+    def describe(self, part: dict) -> str:
+        wl = self.wl
+        return (f"fp64 oracle, one call of each part as its decode step makes it (sequence 0, "
+                f"attention layer 0, all {wl.Hkv} KV heads, t={self.t}): local attention "
+                f"{part['local_s']:.3f} s, full attention {part['full_s']:.3f} s, recall-head score "
+                f"{part['head_s']:.3f} s; step = {wl.L}x{wl.B} local + {wl.L}x"
+                f"{self.flagged_per_step:.3f} full (the schedule's flagged sequences per timed "
+                f"step) + {wl.B} head scores = {self.step_seconds(part):.1f} s")
 
 
 def cpu_cores() -> int:
@@ -235,21 +260,22 @@ def workload_config(wl, world: int, eager: bool) -> dict:
 def run_reference(args, wl, rank, world):
     if rank != 0:
         return
-    smp = OracleSample(wl, kv_heads=1)
-    vals, desc = [], ""
+    smp = OracleStepSample(wl, args.warmup, args.steps)
+    vals, parts = [], []
     for i in range(args.warmup + args.steps):
-        nb, dt = smp.run()
+        part = smp.run()
         if i >= args.warmup:
-            vals.append(smp.steps_per_s(nb, dt))
-            desc = smp.describe(nb, dt)
+            parts.append(part)
+            vals.append(1.0 / smp.step_seconds(part))
     value = statistics.median(vals)
+    mid = parts[vals.index(sorted(vals)[len(vals) // 2])]
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000.0 / value, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(wl, world, args.eager),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-                             "sample": desc},
+                             "sample": smp.describe(mid) + f"; median of {args.steps} samples"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -597,16 +623,40 @@ def run_ours(args, wl, rank, world, local_rank):
         step_detail = {"unflagged_step_us": quiet_us, "local_pass_us": loc_ms * 1e3 * wl.L,
                        "head_us": head_ms * 1e3, "staging_copy_us": stage_us,
                        "glue_us": quiet_us - loc_ms * 1e3 * wl.L - head_ms * 1e3 - stage_us}
+        # a step with exactly one flagged sequence: its extra time over the unflagged step is the
+        # retry of one sequence (every layer's full-set attention, the retry's hidden-state
+        # glue and the conditional's launch)
+        one = dec.make_step_buffer(0)
+        ov = dec.layout.views(one)["sched"]
+        ov.zero_()
+        ov[0] = 1
+        dec.step(one)
+        dec.synchronize()
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        r0.record(dec.stream)
+        for _ in range(2):
+            dec.step(one)
+        r1.record(dec.stream)
+        r1.synchronize()
+        one_us = r0.elapsed_time(r1) * 1e3 / 2
+        rho = statistics.mean(wl.rates) if wl.rates else 0.0
+        retry_us = one_us - quiet_us
+        norm_us = quiet_us + rho * wl.B * retry_us
+        rate_normalized = {"value": 1e6 / norm_us, "unit": UNIT, "rho": rho,
+                           "unflagged_step_us": quiet_us, "one_flag_step_us": one_us,
+                           "retry_us_per_sequence": retry_us,
+                           "formula": "1 / (unflagged step + rho * B * (one-flag step - unflagged step))"}
     else:
         step_detail = None
+        rate_normalized = None
     err = dec.device_error()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        smp = OracleSample(wl, kv_heads=wl.Hkv)
-        nb, dt = smp.run()
-        cpu = {"value": smp.steps_per_s(nb, dt), "unit": UNIT, "cores": cpu_cores(),
-               "kind": "oracle", "sample": smp.describe(nb, dt)}
+        smp = OracleStepSample(wl, W, K)
+        part = smp.run()
+        cpu = {"value": 1.0 / smp.step_seconds(part), "unit": UNIT, "cores": cpu_cores(),
+               "kind": "oracle", "sample": smp.describe(part)}
 
     if rank == 0:
         value = world * K / (elapsed_ms * 1e-3)
@@ -641,6 +691,7 @@ def run_ours(args, wl, rank, world, local_rank):
             "first_step_ms_incl_capture": first_ms, "setup_s": setup_s,
             "gpu_launches": launches, "device_error": err,
             "clocks": clocks, "e2e": e2e, "e2e_detail": e2e_detail, "step_detail": step_detail,
+            "rate_normalized": rate_normalized,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
