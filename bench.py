@@ -118,10 +118,14 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------ accounting
-def step_bytes(wl, pos_list, flags):
+KV_BYTES_PER_TOKEN_HEAD = {"bf16": 128 * 2 * 2,       # K and V rows, bf16
+                           "fp8": 128 * 2 + 2 * 4}     # K and V e4m3 codes + two fp32 scales
+
+
+def step_bytes(wl, pos_list, flags, kv="bf16"):
     """Algorithmic bytes of one step: local KV + flagged full KV + head weights."""
     from workload import inputs
-    per_tok = wl.Hkv * 128 * 2 * 2
+    per_tok = wl.Hkv * KV_BYTES_PER_TOKEN_HEAD[kv]
     b = 0
     for bi, t in enumerate(pos_list):
         b += min(t, wl.sinks + wl.window) * per_tok * wl.L
@@ -248,12 +252,17 @@ def cpu_cores() -> int:
     return len(os.sched_getaffinity(0))
 
 
-def workload_config(wl, world: int, eager: bool) -> dict:
+def workload_config(wl, world: int, eager: bool, kv: str = "bf16") -> dict:
     """The `config` object of both arms' JSON lines (the workload and how the GPU arm runs it)."""
+    n_pages = sum((c + 1 + 15) // 16 for c in wl.ctx)
+    cache_gb = n_pages * 16 * wl.Hkv * KV_BYTES_PER_TOKEN_HEAD[kv] * wl.L / 1e9
     return {"workload": wl.name, "B": wl.B, "layers": wl.L, "Hq": wl.Hq, "Hkv": wl.Hkv,
-            "head_dim": 128, "ctx": wl.ctx[0], "recall_rate": wl.rates[0] if wl.rates else None,
-            "page_tokens": 16, "parallelism": f"replicas{world}",
-            "l2": "inputs larger than L2 (77 GB resident KV cache), no flush",
+            "head_dim": 128, "ctx": wl.ctx[0] if len(set(wl.ctx)) == 1 else
+            f"{min(wl.ctx)}..{max(wl.ctx)}",
+            "recall_rate": (wl.rates[0] if len(set(wl.rates)) == 1 else
+                            f"{min(wl.rates):.3f}..{max(wl.rates):.3f}") if wl.rates else None,
+            "page_tokens": 16, "kv_cache": kv, "parallelism": f"replicas{world}",
+            "l2": f"inputs larger than L2 ({cache_gb:.0f} GB resident KV cache), no flush",
             "launch": "eager" if eager else "cuda-graph with conditional IF node"}
 
 
@@ -273,7 +282,7 @@ def run_reference(args, wl, rank, world):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000.0 / value, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(wl, world, args.eager),
+            "config": workload_config(wl, world, args.eager, args.kv),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
                              "sample": smp.describe(mid) + f"; median of {args.steps} samples"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -292,12 +301,12 @@ def time_layer_kernels(dec, mode: int, flag, reps: int = 3) -> float:
     oda.oda_graph_begin(s)
     for a in range(wl.L):
         if mode == 0:
-            oda.oda_attend_local(dec.ctx, dec.layers[a], dec.page_table, dec.pos, dec.sv["q"][0, a],
-                                 dec.sv["k"][0, a], dec.sv["v"][0, a], dec.o[0, a], s)
+            dec._attend_local(dec.ctx, dec.layers[a], dec.page_table, dec.pos, dec.sv["q"][0, a],
+                              dec.sv["k"][0, a], dec.sv["v"][0, a], dec.o[0, a], s)
         else:
-            oda.oda_attend_full_if(dec.ctx, dec.layers[a], dec.page_table, dec.pos, flag,
-                                   dec.sv["q"][1, a], dec.sv["k"][1, a], dec.sv["v"][1, a],
-                                   dec.o[1, a], s)
+            dec._attend_full(dec.ctx, dec.layers[a], dec.page_table, dec.pos, flag,
+                             dec.sv["q"][1, a], dec.sv["k"][1, a], dec.sv["v"][1, a],
+                             dec.o[1, a], s)
     g = oda.oda_graph_end(s)
     g.launch(s)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -340,7 +349,7 @@ def run_kernel_only(args, wl, local_rank):
     from conditional_sparse_attention_b200 import oda
     from conditional_sparse_attention_b200.engine import OdaDecoder
     dev = torch.device("cuda", local_rank)
-    dec = OdaDecoder(wl, device=dev, capacity_steps=4)
+    dec = OdaDecoder(wl, device=dev, capacity_steps=4, kv_format=args.kv)
     dec.stage(dec.make_step_buffer(0))
     dec.synchronize()
     ones = torch.ones(wl.B, dtype=torch.int32, device=dev)
@@ -363,12 +372,12 @@ def run_kernel_only(args, wl, local_rank):
     for r in range(args.kernel_reps):
         a = r % wl.L
         if args.kernel_only == "full":
-            oda.oda_attend_full_if(dec.ctx, dec.layers[a], dec.page_table, dec.pos, ones,
-                                   dec.sv["q"][1, a], dec.sv["k"][1, a], dec.sv["v"][1, a],
-                                   dec.o[1, a], dec.stream)
+            dec._attend_full(dec.ctx, dec.layers[a], dec.page_table, dec.pos, ones,
+                             dec.sv["q"][1, a], dec.sv["k"][1, a], dec.sv["v"][1, a],
+                             dec.o[1, a], dec.stream)
         elif args.kernel_only == "local":
-            oda.oda_attend_local(dec.ctx, dec.layers[a], dec.page_table, dec.pos, dec.sv["q"][0, a],
-                                 dec.sv["k"][0, a], dec.sv["v"][0, a], dec.o[0, a], dec.stream)
+            dec._attend_local(dec.ctx, dec.layers[a], dec.page_table, dec.pos, dec.sv["q"][0, a],
+                              dec.sv["k"][0, a], dec.sv["v"][0, a], dec.o[0, a], dec.stream)
         elif args.kernel_only == "head":
             oda.oda_recall_score(dec.ctx, dec.head_w, dec.h_prev, dec.sv["emb"], dec.h[0],
                                  dec.sv["sched"] if dec.routing_scheduled else None, dec.score,
@@ -377,7 +386,7 @@ def run_kernel_only(args, wl, local_rank):
             grad_step(dec)
     dec.synchronize()
     err = dec.device_error()
-    print(json.dumps({"kernel_only": args.kernel_only, "workload": wl.name,
+    print(json.dumps({"kernel_only": args.kernel_only, "workload": wl.name, "kv": args.kv,
                       "launches": args.kernel_reps, "device_error": err}), flush=True)
     dec.close()
 
@@ -461,7 +470,7 @@ def run_ours(args, wl, rank, world, local_rank):
     n_e2e = K if args.e2e else 0
     cap = W + K + W + n_e2e + 4
     t_setup = time.perf_counter()
-    dec = OdaDecoder(wl, device=dev, capacity_steps=cap)
+    dec = OdaDecoder(wl, device=dev, capacity_steps=cap, kv_format=args.kv)
     n_store = min(cap, W + K)
     store = [dec.make_step_buffer(s) for s in range(n_store)]
     torch.cuda.synchronize(dev)
@@ -509,14 +518,14 @@ def run_ours(args, wl, rank, world, local_rank):
     elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     flags = flag_hist.cpu().numpy()
     poss = pos_hist.cpu().numpy()
-    total_bytes = sum(step_bytes(wl, poss[i].tolist(), flags[i].tolist()) for i in range(K))
+    total_bytes = sum(step_bytes(wl, poss[i].tolist(), flags[i].tolist(), args.kv) for i in range(K))
     realized_rate = float(flags.mean())
     launches = sum(kernel_launches(wl, bool(flags[i].any())) for i in range(K))
 
     # ---------------- per-kernel timing: each attention kernel replayed as a graph of one launch
     # per layer (no host gaps), CUDA events on the launching stream
     hbm, peak_src = peaks()
-    per_tok = wl.Hkv * 128 * 2 * 2
+    per_tok = wl.Hkv * KV_BYTES_PER_TOKEN_HEAD[args.kv]
     pos_now = dec.pos.cpu().numpy()
     pats = {}
     for f in flags:
@@ -534,7 +543,7 @@ def run_ours(args, wl, rank, world, local_rank):
         full_bytes += count * sum(int(pos_now[b]) * per_tok for b in range(wl.B) if pat[b])
         n_full += 2 * wl.L
     full_gbs = full_bytes / (full_ms * 1e-3) / 1e9
-    tpt = traffic_per_token()
+    tpt = traffic_per_token() if args.kv == "bf16" else None
     n_pat_launches = sum(pats.values())
     full_traffic = (tpt * (full_bytes / per_tok) / n_pat_launches) if tpt else None
     loc_ms = time_layer_kernels(dec, 0, None, reps=3)
@@ -664,13 +673,14 @@ def run_ours(args, wl, rank, world, local_rank):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(wl, world, args.eager),
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if args.kv == "bf16" else "fp8",
+            "data": "synthetic",
+            "config": workload_config(wl, world, args.eager, args.kv),
             "roofline": {"bound": "hbm", "achieved": full_gbs, "peak": hbm, "unit": "GB/s",
                          "frac": full_gbs / hbm, "frac_of_nominal": full_gbs / NOMINAL_HBM_GBS,
                          "traffic": full_traffic,
                          "algorithmic_bytes_per_launch": full_bytes / n_pat_launches,
-                         "kernel": "attn_full_kernel (full set, flagged sequences)",
+                         "kernel": f"attn_full_kernel<{args.kv} pages> (full set, flagged sequences)",
                          "peak_source": peak_src, "launches_timed": n_full,
                          "us_per_launch": full_ms * 1000.0 / sum(pats.values()),
                          "flag_patterns": {"".join(map(str, k)): v for k, v in pats.items()}},
@@ -705,6 +715,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="cfg2")
+    ap.add_argument("--kv", choices=["bf16", "fp8"], default="bf16",
+                    help="KV cache page format (fp8: e4m3 codes with per-row fp32 scales)")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true",

@@ -35,6 +35,10 @@ class OdaKVLayer(ctypes.Structure):
     _fields_ = [("k", c_void_p), ("v", c_void_p), ("n_pages", c_int64)]
 
 
+class OdaKV8Layer(ctypes.Structure):
+    _fields_ = [("kv", c_void_p), ("n_pages", c_int64)]
+
+
 class OdaHeadWeights(ctypes.Structure):
     _fields_ = [("tower_norm", c_void_p * 3), ("tower_w", c_void_p * 3), ("tower_b", c_void_p * 3),
                 ("fuse_w", c_void_p), ("fuse_b", c_void_p), ("ffn_norm", c_void_p * 2),
@@ -62,6 +66,14 @@ _SIGS = {
     "oda_attend_full_if_noalloc": ([_P(OdaConfig), _P(OdaKVLayer), c_void_p, c_void_p, c_void_p,
                                     c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p],
                                    c_int32),
+    "oda_attend_local_fp8": ([c_void_p, _P(OdaKV8Layer), c_void_p, c_void_p, c_void_p, c_void_p,
+                              c_void_p, c_void_p, c_void_p], c_int32),
+    "oda_attend_full_if_fp8": ([c_void_p, _P(OdaKV8Layer), c_void_p, c_void_p, c_void_p, c_void_p,
+                                c_void_p, c_void_p, c_void_p, c_void_p], c_int32),
+    "oda_kv8_pack": ([_P(OdaKVLayer), _P(OdaKV8Layer), c_int32, c_void_p], c_int32),
+    "oda_commit_fp8": ([c_void_p, _P(OdaKV8Layer), c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
+                        c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p],
+                       c_int32),
     "oda_index_positions": ([c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_int32, c_void_p,
                              c_void_p], c_int32),
     "oda_recall_score": ([c_void_p, _P(OdaHeadWeights), c_void_p, c_void_p, c_void_p, c_void_p,

@@ -1,6 +1,7 @@
 // C ABI entry points: argument validation, context scratch, conditional capture, graphs,
 // error reporting.  Every compute step is one of the kernels in attention.cu, head.cu,
 // commit.cu and glue.cu.
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -160,14 +161,14 @@ oda_status oda_create(const oda_config* cfg, oda_ctx** out) {
   if (st == ODA_OK)
     st = check_cuda(cudaDeviceGetAttribute(&x->n_sms, cudaDevAttrMultiProcessorCount, x->device),
                     "cudaDeviceGetAttribute");
-  if (st == ODA_OK) st = oda::prepare_attention_kernel(x->g, x->n_sms, &x->attn_ctas);
+  if (st == ODA_OK) st = oda::prepare_attention_kernel(x->g, x->n_sms, x->attn_ctas);
   if (st == ODA_OK) st = oda::prepare_head_kernel();
   if (st != ODA_OK) {
     free_ctx(x);
     return st;
   }
   const int64_t B = c.batch, Hkv = c.n_kv_heads, D = c.head_in_dim;
-  x->n_slots = (int)(x->attn_ctas + B * Hkv);
+  x->n_slots = (int)(std::max(x->attn_ctas[0], x->attn_ctas[1]) + B * Hkv);
   const int64_t ms = x->n_slots;
   const int gch = oda::glue_chunks(c.head_in_dim);
   st = dev_alloc(&x->part_o, (size_t)ms * x->g * 128, "cudaMalloc(partials)");
@@ -211,16 +212,40 @@ oda_status oda_destroy(oda_ctx* ctx) {
 oda_status oda_attend_local(oda_ctx* ctx, const oda_kv_layer* layer, const int32_t* page_table,
                             const int32_t* pos, const void* q, const void* k_new,
                             const void* v_new, float* out, cudaStream_t stream) {
-  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "attend_local: ctx is NULL");
-  return oda::launch_attention(ctx, layer, page_table, pos, nullptr, q, k_new, v_new, out, 0, stream);
+  if (!ctx || !layer) return set_error(ODA_ERR_INVALID_ARG, "attend_local: ctx or layer is NULL");
+  const oda::KvPool pool{0, layer->k, layer->v, layer->n_pages};
+  return oda::launch_attention(ctx, pool, page_table, pos, nullptr, q, k_new, v_new, out, 0, stream);
 }
 
 oda_status oda_attend_full_if(oda_ctx* ctx, const oda_kv_layer* layer, const int32_t* page_table,
                               const int32_t* pos, const int32_t* flag, const void* q,
                               const void* k_new, const void* v_new, float* out,
                               cudaStream_t stream) {
-  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "attend_full_if: ctx is NULL");
-  return oda::launch_attention(ctx, layer, page_table, pos, flag, q, k_new, v_new, out, 1, stream);
+  if (!ctx || !layer) return set_error(ODA_ERR_INVALID_ARG, "attend_full_if: ctx or layer is NULL");
+  const oda::KvPool pool{0, layer->k, layer->v, layer->n_pages};
+  return oda::launch_attention(ctx, pool, page_table, pos, flag, q, k_new, v_new, out, 1, stream);
+}
+
+oda_status oda_attend_local_fp8(oda_ctx* ctx, const oda_kv8_layer* layer, const int32_t* page_table,
+                                const int32_t* pos, const void* q, const void* k_new,
+                                const void* v_new, float* out, cudaStream_t stream) {
+  if (!ctx || !layer) return set_error(ODA_ERR_INVALID_ARG, "attend_local_fp8: ctx or layer is NULL");
+  const oda::KvPool pool{1, layer->kv, nullptr, layer->n_pages};
+  return oda::launch_attention(ctx, pool, page_table, pos, nullptr, q, k_new, v_new, out, 0, stream);
+}
+
+oda_status oda_attend_full_if_fp8(oda_ctx* ctx, const oda_kv8_layer* layer, const int32_t* page_table,
+                                  const int32_t* pos, const int32_t* flag, const void* q,
+                                  const void* k_new, const void* v_new, float* out,
+                                  cudaStream_t stream) {
+  if (!ctx || !layer) return set_error(ODA_ERR_INVALID_ARG, "attend_full_if_fp8: ctx or layer is NULL");
+  const oda::KvPool pool{1, layer->kv, nullptr, layer->n_pages};
+  return oda::launch_attention(ctx, pool, page_table, pos, flag, q, k_new, v_new, out, 1, stream);
+}
+
+oda_status oda_kv8_pack(const oda_kv_layer* src, const oda_kv8_layer* dst, int32_t n_kv_heads,
+                        cudaStream_t stream) {
+  return oda::launch_kv8_pack(src, dst, n_kv_heads, stream);
 }
 
 oda_status oda_attend_full_if_noalloc(const oda_config* cfg, const oda_kv_layer* layer,
@@ -269,8 +294,29 @@ oda_status oda_commit(oda_ctx* ctx, const oda_kv_layer* layers, int32_t n_layers
                       const float* h_local, const float* h_full, float* h_prev,
                       cudaStream_t stream) {
   if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "commit: ctx is NULL");
+  if (!layers || n_layers < 1 || n_layers > ODA_MAX_LAYERS)
+    return set_error(ODA_ERR_INVALID_ARG, "commit: n_layers must be 1..%d", ODA_MAX_LAYERS);
   ctx->prev_attention = false;
-  return oda::launch_commit(ctx, layers, n_layers, page_table, pos, flag, k_stage_local,
+  oda::KvPool pools[ODA_MAX_LAYERS];
+  for (int l = 0; l < n_layers; ++l) pools[l] = {0, layers[l].k, layers[l].v, layers[l].n_pages};
+  return oda::launch_commit(ctx, pools, n_layers, page_table, pos, flag, k_stage_local,
+                            v_stage_local, k_stage_full, v_stage_full, h_local, h_full, h_prev,
+                            stream);
+}
+
+oda_status oda_commit_fp8(oda_ctx* ctx, const oda_kv8_layer* layers, int32_t n_layers,
+                          const int32_t* page_table, int32_t* pos, const int32_t* flag,
+                          const void* k_stage_local, const void* v_stage_local,
+                          const void* k_stage_full, const void* v_stage_full,
+                          const float* h_local, const float* h_full, float* h_prev,
+                          cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "commit_fp8: ctx is NULL");
+  if (!layers || n_layers < 1 || n_layers > ODA_MAX_LAYERS)
+    return set_error(ODA_ERR_INVALID_ARG, "commit_fp8: n_layers must be 1..%d", ODA_MAX_LAYERS);
+  ctx->prev_attention = false;
+  oda::KvPool pools[ODA_MAX_LAYERS];
+  for (int l = 0; l < n_layers; ++l) pools[l] = {1, layers[l].kv, nullptr, layers[l].n_pages};
+  return oda::launch_commit(ctx, pools, n_layers, page_table, pos, flag, k_stage_local,
                             v_stage_local, k_stage_full, v_stage_full, h_local, h_full, h_prev,
                             stream);
 }

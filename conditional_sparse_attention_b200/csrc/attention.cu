@@ -26,6 +26,7 @@
 // a launch prefetches its first pages before waiting for the previous one.
 #include <cmath>
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 
 #include <cooperative_groups.h>
@@ -48,19 +49,17 @@ constexpr int kRL = 3;                // local set: pages in flight per warp
 constexpr int kThreadsL = kWL * 32;
 constexpr int kPageTok = 16;
 constexpr int kStageBytes = 8192;     // K (4 KiB) + V (4 KiB) of one (page, KV head)
-constexpr int kStagesBytes = kW * kR * kStageBytes;
-constexpr int kStagesBytesL = kWL * kRL * kStageBytes;
 constexpr int kMergeStride = 132;     // floats per (warp, head) row of the merge area
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kMaxCluster = 8;
 constexpr int kChunk = 4;             // full set: pages per claimed chunk
-constexpr int kQueueLow = kR + kChunk;   // full set: queue length that triggers the next claim
 constexpr int kMergeRows = 20;        // full set: partial rows folded per round of the merge
 
 struct AttnParams {
   const int32_t* page_table;
   const int32_t* pos;
   const int32_t* flag;
+  const uint8_t* kv8;     // fp8 pages: blocks [n_pages][Hkv][kF8Block] (unused for bf16 pages)
   const uint32_t* q;      // bf16 pairs [B][Hq][64]
   const uint32_t* k_new;  // bf16 pairs [B][Hkv][64]
   const uint32_t* v_new;
@@ -420,6 +419,227 @@ __device__ __forceinline__ void page_compute2(WarpAcc& A, const uint32_t (&qf)[8
   }
 }
 
+// ------------------------------------------------------------------ fp8 (e4m3) pages
+// One (page, KV head) block of an fp8 pool is kF8Block contiguous bytes, brought in by one bulk
+// copy:
+//   [0, 2048)     K codes, token-major: token j's 128 codes at 128*j, its 16-dim chunk k stored
+//                 at chunk position k ^ (j & 7) (so ldmatrix rows of 8 tokens hit 8 bank groups);
+//   [2048, 4096)  V codes transposed: dim d's 16 codes at 2048 + 16*d, slot s holding token
+//                 tau(s) = 2*(s/4) + (s&1) + 8*((s>>1)&1), i.e. slots 4c..4c+3 hold tokens
+//                 2c, 2c+1, 2c+8, 2c+9 (the token order of a P^T fragment);
+//   [4096, 4160)  K scales, fp32 [16], token order;  [4160, 4224)  V scales, fp32 [16].
+// Cached value = scale * e4m3 value of its code.  The codes convert exactly to f16 for the
+// tensor-core products; the K scale multiplies each token's score after the QK^T product; the
+// V scale multiplies each token's probability before the PV product (normalised per page by a
+// power of two that is multiplied back into the accumulator, so f16 keeps its range).
+constexpr int kF8Block = 4224;
+constexpr int kF8V = 2048;
+constexpr int kF8SK = 4096;
+constexpr int kF8SV = 4160;
+
+// q of one KV head's group as f16 B fragments in the fp8 dimension order, scaled per head by a
+// power of two 2^e_n (max |q_n| * 2^e_n in [2^14, 2^15)); fs0 / fs1 undo it (times log2(e)/sqrt(d))
+// for the heads 2c, 2c + 1 of this lane's score columns.
+struct QF8 {
+  uint32_t qf[8][2];
+  float fs0, fs1;
+};
+
+__device__ __forceinline__ void load_q8(QF8& Q, const AttnParams& p, int b, int h, int lane) {
+  const int n = lane >> 2, c = lane & 3;
+  float v[8][4];
+  float mx = 0.f;
+  if (n < p.g) {
+    const uint32_t* qrow = p.q + ((size_t)b * p.Hq + h * p.g + n) * 64;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint32_t w0 = qrow[8 * kk + 2 * c], w1 = qrow[8 * kk + 2 * c + 1];
+      v[kk][0] = bf16_lo_to_f32(w0);
+      v[kk][1] = bf16_hi_to_f32(w0);
+      v[kk][2] = bf16_lo_to_f32(w1);
+      v[kk][3] = bf16_hi_to_f32(w1);
+      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v[kk][0]), fabsf(v[kk][1])), fmaxf(fabsf(v[kk][2]), fabsf(v[kk][3]))));
+    }
+  } else {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) v[kk][0] = v[kk][1] = v[kk][2] = v[kk][3] = 0.f;
+  }
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  int e = 0;
+  if (mx > 0.f && mx <= 3.0e38f) {
+    const int ex = (int)((__float_as_uint(mx) >> 23) & 0xFF) - 127;   // floor(log2(mx)), normal mx
+    e = min(60, max(-60, 14 - ex));
+  }
+  const float up = __uint_as_float((uint32_t)(127 + e) << 23);
+  const float down = (n < p.g) ? p.scale_log2 * __uint_as_float((uint32_t)(127 - e) << 23) : 0.f;
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    Q.qf[kk][0] = pack_f16x2(v[kk][0] * up, v[kk][1] * up);
+    Q.qf[kk][1] = pack_f16x2(v[kk][2] * up, v[kk][3] * up);
+  }
+  Q.fs0 = __shfl_sync(0xffffffffu, down, 8 * c);
+  Q.fs1 = __shfl_sync(0xffffffffu, down, 8 * c + 4);
+}
+
+// Raw scores K q^T of one fp8 page (tokens as M in natural order, heads as N), before scales.
+__device__ __forceinline__ void page_scores8(float (&sacc)[4], const QF8& Q, uint32_t sb, int lane) {
+  const int mi = lane >> 3, rr = lane & 7;
+  const int tok = ((mi & 1) << 3) + rr;
+  float sa[4] = {0.f, 0.f, 0.f, 0.f}, sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int kk = 0; kk < 8; kk += 2) {
+    uint32_t r[4];
+    const int ch = kk + (mi >> 1);
+    ldsm_x4(r, sb + tok * 128 + ((ch ^ rr) << 4));
+    const uint32_t a0[4] = {e4m3x2_to_f16x2(r[0]), e4m3x2_to_f16x2(r[1]),
+                            e4m3x2_to_f16x2(r[0] >> 16), e4m3x2_to_f16x2(r[1] >> 16)};
+    const uint32_t a1[4] = {e4m3x2_to_f16x2(r[2]), e4m3x2_to_f16x2(r[3]),
+                            e4m3x2_to_f16x2(r[2] >> 16), e4m3x2_to_f16x2(r[3] >> 16)};
+    mma_f16_16816(sa, a0, Q.qf[kk][0], Q.qf[kk][1]);
+    mma_f16_16816(sc, a1, Q.qf[kk + 1][0], Q.qf[kk + 1][1]);
+  }
+  sacc[0] = sa[0] + sc[0];
+  sacc[1] = sa[1] + sc[1];
+  sacc[2] = sa[2] + sc[2];
+  sacc[3] = sa[3] + sc[3];
+}
+
+// Keep-masks of this lane's V^T fragment halves for a page whose token set is given by the
+// lanes' (in0, in1): the low word of a fragment holds tokens 2c, 2c+1, the high word 2c+8, 2c+9.
+__device__ __forceinline__ void v8_masks(bool in0, bool in1, int lane, uint32_t& mlo, uint32_t& mhi) {
+  auto squeeze = [](uint32_t x) {   // bits 0, 4, ..., 28 -> bits 0..7
+    x &= 0x11111111u;
+    x = (x | (x >> 3)) & 0x03030303u;
+    x = (x | (x >> 6)) & 0x000F000Fu;
+    return (x | (x >> 12)) & 0xFFu;
+  };
+  const uint32_t t_lo = squeeze(__ballot_sync(0xffffffffu, in0));   // tokens 0..7
+  const uint32_t t_hi = squeeze(__ballot_sync(0xffffffffu, in1));   // tokens 8..15
+  const int c = lane & 3;
+  const uint32_t a = (t_lo >> (2 * c)) & 3u, bb = (t_hi >> (2 * c)) & 3u;
+  mlo = ((a & 1u) ? 0x0000FFFFu : 0u) | ((a & 2u) ? 0xFFFF0000u : 0u);
+  mhi = ((bb & 1u) ? 0x0000FFFFu : 0u) | ((bb & 2u) ? 0xFFFF0000u : 0u);
+}
+
+// PV of one fp8 page into (hi, lo) accumulators: P'' fragments (hi / lo f16) times V^T codes.
+__device__ __forceinline__ void page_pv8(float (&th)[8][4], float (&tl)[8][4], uint32_t vb,
+                                         uint32_t bh0, uint32_t bh1, uint32_t bl0, uint32_t bl1,
+                                         bool masked, uint32_t mlo, uint32_t mhi, int lane) {
+  const int mi = lane >> 3, rr = lane & 7;
+  const int row = ((mi & 1) << 3) + rr;   // dim within the 16-dim tile
+#pragma unroll
+  for (int mt = 0; mt < 8; mt += 2) {
+    uint32_t r[4];
+    ldsm_x4(r, vb + (16 * (mt + (mi >> 1)) + row) * 16);
+    uint32_t a0[4] = {e4m3x2_to_f16x2(r[0]), e4m3x2_to_f16x2(r[1]),
+                      e4m3x2_to_f16x2(r[0] >> 16), e4m3x2_to_f16x2(r[1] >> 16)};
+    uint32_t a1[4] = {e4m3x2_to_f16x2(r[2]), e4m3x2_to_f16x2(r[3]),
+                      e4m3x2_to_f16x2(r[2] >> 16), e4m3x2_to_f16x2(r[3] >> 16)};
+    if (masked) {   // tokens outside the set: their codes may be stale (even NaN); P'' is 0 there
+      a0[0] &= mlo; a0[1] &= mlo; a0[2] &= mhi; a0[3] &= mhi;
+      a1[0] &= mlo; a1[1] &= mlo; a1[2] &= mhi; a1[3] &= mhi;
+    }
+    mma_f16_16816(th[mt], a0, bh0, bh1);
+    mma_f16_16816(tl[mt], a0, bl0, bl1);
+    mma_f16_16816(th[mt + 1], a1, bh0, bh1);
+    mma_f16_16816(tl[mt + 1], a1, bl0, bl1);
+  }
+}
+
+// NP (1 or 2) fp8 pages in one online-softmax step (one maximum and rescale for 16 * NP tokens).
+// in[i][0] / in[i][1]: whether this lane's token rows r and r + 8 of page i belong to the set.
+template <int NP>
+__device__ __forceinline__ void page_step8(WarpAcc& A, const QF8& Q, uint8_t* const (&st)[2],
+                                           const bool (&in)[2][2], int lane) {
+  const int r = lane >> 2;
+  float x[2][4], svv[2][2];
+  bool any_masked = false;
+  float svmax = 0.f;
+#pragma unroll
+  for (int i = 0; i < NP; ++i) {
+    const uint32_t sb = smem_u32(st[i]);
+    float sacc[4];
+    page_scores8(sacc, Q, sb, lane);
+    const float* sk = reinterpret_cast<const float*>(st[i] + kF8SK);
+    const float* sv = reinterpret_cast<const float*>(st[i] + kF8SV);
+    const float k0 = sk[r], k1 = sk[r + 8];
+    x[i][0] = in[i][0] ? sacc[0] * k0 * Q.fs0 : -INFINITY;
+    x[i][1] = in[i][0] ? sacc[1] * k0 * Q.fs1 : -INFINITY;
+    x[i][2] = in[i][1] ? sacc[2] * k1 * Q.fs0 : -INFINITY;
+    x[i][3] = in[i][1] ? sacc[3] * k1 * Q.fs1 : -INFINITY;
+    svv[i][0] = in[i][0] ? sv[r] : 0.f;
+    svv[i][1] = in[i][1] ? sv[r + 8] : 0.f;
+    svmax = fmaxf(svmax, fmaxf(svv[i][0], svv[i][1]));
+    any_masked |= !(in[i][0] && in[i][1]);
+  }
+  float mx0 = fmaxf(x[0][0], x[0][2]), mx1 = fmaxf(x[0][1], x[0][3]);
+  if (NP == 2) {
+    mx0 = fmaxf(mx0, fmaxf(x[1][0], x[1][2]));
+    mx1 = fmaxf(mx1, fmaxf(x[1][1], x[1][3]));
+  }
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    svmax = fmaxf(svmax, __shfl_xor_sync(0xffffffffu, svmax, off));
+  }
+  // the pages' V-scale binade: P'' = p * sv * 2^-E stays below 2 in f16
+  const int E = (svmax > 0.f && svmax <= 3.0e38f) ? (int)((__float_as_uint(svmax) >> 23) & 0xFF) - 127 : 0;
+  const int Ec = min(126, max(-126, E));
+  const float down = __uint_as_float((uint32_t)(127 - Ec) << 23);
+  const float upE = __uint_as_float((uint32_t)(127 + Ec) << 23);
+  const float mn0 = fmaxf(A.m0, mx0), mn1 = fmaxf(A.m1, mx1);
+  if (mn0 > A.m0 || mn1 > A.m1) {
+    const float al0 = exp2f(A.m0 - mn0), al1 = exp2f(A.m1 - mn1);
+    A.l0 *= al0;
+    A.l1 *= al1;
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      A.o[mt][0] *= al0;
+      A.o[mt][1] *= al1;
+      A.o[mt][2] *= al0;
+      A.o[mt][3] *= al1;
+    }
+    A.m0 = mn0;
+    A.m1 = mn1;
+  }
+  const bool masked = __any_sync(0xffffffffu, any_masked);
+  float th[8][4], tl[8][4];
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt)
+    th[mt][0] = th[mt][1] = th[mt][2] = th[mt][3] = tl[mt][0] = tl[mt][1] = tl[mt][2] = tl[mt][3] = 0.f;
+#pragma unroll
+  for (int i = 0; i < NP; ++i) {
+    const float p0 = exp2f(x[i][0] - A.m0), p1 = exp2f(x[i][1] - A.m1);
+    const float p2 = exp2f(x[i][2] - A.m0), p3 = exp2f(x[i][3] - A.m1);
+    A.l0 += p0 + p2;
+    A.l1 += p1 + p3;
+    const float s0 = svv[i][0] * down, s1 = svv[i][1] * down;
+    const float q0 = p0 * s0, q1 = p1 * s0, q2 = p2 * s1, q3 = p3 * s1;
+    const uint32_t h01 = pack_f16x2(q0, q1), h23 = pack_f16x2(q2, q3);
+    const uint32_t l01 = pack_f16x2(q0 - f16_lo_to_f32(h01), q1 - f16_hi_to_f32(h01));
+    const uint32_t l23 = pack_f16x2(q2 - f16_lo_to_f32(h23), q3 - f16_hi_to_f32(h23));
+    const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
+    const uint32_t bl0 = movmatrix_trans(l01), bl1 = movmatrix_trans(l23);
+    uint32_t mlo = 0xFFFFFFFFu, mhi = 0xFFFFFFFFu;
+    if (masked) v8_masks(in[i][0], in[i][1], lane, mlo, mhi);
+    page_pv8(th, tl, smem_u32(st[i] + kF8V), bh0, bh1, bl0, bl1, masked, mlo, mhi, lane);
+  }
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) A.o[mt][j] = fmaf(th[mt][j] + tl[mt][j], upE, A.o[mt][j]);
+}
+
+// Issues the bulk copy of one fp8 (page, KV head) block into a stage.
+__device__ __forceinline__ void issue_page8(uint8_t* dst, uint64_t* bar, const uint8_t* kv8,
+                                            int phys, int Hkv, int h) {
+  fence_proxy_async_smem();
+  mbar_arrive_expect_tx(bar, kF8Block);
+  bulk_load(dst, kv8 + ((size_t)phys * Hkv + h) * kF8Block, kF8Block, bar);
+}
+
 // Reduces l over the token rows and writes the warp's state to its merge slot:
 // mo [g][kMergeStride] (O^T columns), ml [8][2] (m, l).
 __device__ __forceinline__ void warp_flush(WarpAcc& A, float* mo, float* ml, int g, int lane) {
@@ -523,17 +743,76 @@ __device__ __forceinline__ int cta_of(long long u, long long U, long long G) {
   return (int)(((u + 1) * G - 1) / U);
 }
 
+// Page formats: F = 0 bf16 pools (one 4-D / two 3-D TMA tile copies of 8 KiB per page),
+// F = 1 fp8 blocks (one bulk copy of kF8Block bytes).  The fp8 stages are about half the size,
+// so the rings hold twice as many pages and the bytes in flight stay the same.
+template <int F> struct Fmt;
+template <> struct Fmt<0> {
+  static constexpr int kStage = kStageBytes, kR = 3, kRL = 3, kAlign = 1024;
+};
+template <> struct Fmt<1> {
+  static constexpr int kStage = kF8Block, kR = 6, kRL = 6, kAlign = 128;
+};
+constexpr int kMaxR = 6;
+constexpr int kMaxRL = 6;
+
+// Query fragments of either format.
+template <int F> struct QFrag;
+template <> struct QFrag<0> { uint32_t qf[8][2]; };
+template <> struct QFrag<1> { QF8 q; };
+
+template <int F>
+__device__ __forceinline__ void load_q(QFrag<F>& Q, const AttnParams& p, int b, int h, int lane) {
+  if constexpr (F == 0) load_qf(Q.qf, p, b, h, lane);
+  else load_q8(Q.q, p, b, h, lane);
+}
+
+template <int F>
+__device__ __forceinline__ void issue_any(uint8_t* dst, uint64_t* bar, const CUtensorMap* tmA,
+                                          const CUtensorMap* tmB, const AttnParams& p, int phys, int h) {
+  if constexpr (F == 0) issue_page(dst, bar, tmA, tmB, p.kv_single, phys, p.Hkv, h);
+  else issue_page8(dst, bar, p.kv8, phys, p.Hkv, h);
+}
+
+// One page (a1 = a0 = false for b: single) or two pages in one online-softmax step.
+template <int F>
+__device__ __forceinline__ void pages_compute(WarpAcc& A, const QFrag<F>& Q, uint8_t* stA, bool a0,
+                                              bool a1, uint8_t* stB, bool b0, bool b1, bool pair,
+                                              float scale_log2, int lane) {
+  if constexpr (F == 0) {
+    if (pair) page_compute2(A, Q.qf, stA, a0, a1, stB, b0, b1, scale_log2, lane);
+    else page_compute(A, Q.qf, stA, a0, a1, scale_log2, lane);
+  } else {
+    uint8_t* const st[2] = {stA, stB};
+    const bool in[2][2] = {{a0, a1}, {b0, b1}};
+    const bool anyA = __any_sync(0xffffffffu, a0 || a1);
+    const bool anyB = pair && __any_sync(0xffffffffu, b0 || b1);
+    if (anyA && anyB) {
+      page_step8<2>(A, Q.q, st, in, lane);
+    } else if (anyA) {
+      page_step8<1>(A, Q.q, st, in, lane);
+    } else if (anyB) {
+      uint8_t* const stb[2] = {stB, stB};
+      const bool inb[2][2] = {{b0, b1}, {b0, b1}};
+      page_step8<1>(A, Q.q, stb, inb, lane);
+    }
+  }
+}
+
 // ---------------------------------------------------------------- local set: clusters
 // Cluster of p.cluster CTAs per (b, h); CTA `rank` takes the contiguous share
 // [rank*nv/C, (rank+1)*nv/C) of the visited pages; warps take every kWL-th page of it.  After a
 // cluster barrier each rank finishes its share of the g*128 outputs from all ranks' partials
 // (read through distributed shared memory).
+template <int F>
 __global__ void __launch_bounds__(kThreadsL, 1)
 attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const AttnParams p) {
+  constexpr int kRL = Fmt<F>::kRL;
+  constexpr int kStg = Fmt<F>::kStage;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+      (reinterpret_cast<uintptr_t>(smem_raw) + (Fmt<F>::kAlign - 1)) & ~uintptr_t(Fmt<F>::kAlign - 1));
   const int g = p.g;
   // the merge areas reuse the stages: they are written only after every copy has landed
   float* merge_o = reinterpret_cast<float*>(stages);                   // [W][g][132]
@@ -552,8 +831,10 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 #pragma unroll
     for (int i = 0; i < kWL * kRL; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
-    prefetch_tensormap(&tmA);
-    if (!p.kv_single) prefetch_tensormap(&tmB);
+    if (F == 0) {
+      prefetch_tensormap(&tmA);
+      if (!p.kv_single) prefetch_tensormap(&tmB);
+    }
   }
   const int t = __ldcg(p.pos + b);
   const Geom ge = make_geom(t, 0, p.sinks, p.window, p.max_pages, true);
@@ -562,7 +843,7 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   const int v_lo = (int)((long long)rank * nv / C), v_hi = (int)((long long)(rank + 1) * nv / C);
   const int cw = (v_hi - v_lo - warp > 0) ? (v_hi - v_lo - warp + kWL - 1) / kWL : 0;
   const int* ptab = p.page_table + (size_t)b * p.max_pages;
-  uint8_t* my_stages = stages + warp * kRL * kStageBytes;
+  uint8_t* my_stages = stages + warp * kRL * kStg;
   uint64_t* my_bars = bars + warp * kRL;
   __syncthreads();
 
@@ -585,7 +866,7 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     const int phys = __shfl_sync(0xffffffffu, pt_phys, k - pt_base);
     if (lane == k - pt_base) {
       if (phys >= 0)
-        issue_page(my_stages + st * kStageBytes, my_bars + st, &tmA, &tmB, p.kv_single, phys, p.Hkv, h);
+        issue_any<F>(my_stages + st * kStg, my_bars + st, &tmA, &tmB, p, phys, h);
       else
         mbar_arrive(my_bars + st);
     }
@@ -596,8 +877,8 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   grid_dependency_wait();
   grid_dependents_launch();
 
-  uint32_t qf[8][2];
-  load_qf(qf, p, b, h, lane);
+  QFrag<F> qf;
+  load_q<F>(qf, p, b, h, lane);
   // staged current token: its q . k words (heads warp, warp + kWL) and the value this thread
   // combines first are loaded now and used after the page loop, off the critical path
   __shared__ float s_snew[8];
@@ -639,16 +920,18 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       const int lp1 = geom_page(ge, v_lo + warp + (k + 1) * kWL);
       const bool ok1 = (vbits >> st1) & 1u;
       const int j1 = lp1 * kPageTok + r;
-      page_compute2(A, qf, my_stages + st * kStageBytes, ok && geom_has(ge, j0),
-                    ok && geom_has(ge, j0 + 8), my_stages + st1 * kStageBytes,
-                    ok1 && geom_has(ge, j1), ok1 && geom_has(ge, j1 + 8), p.scale_log2, lane);
+      pages_compute<F>(A, qf, my_stages + st * kStg, ok && geom_has(ge, j0),
+                       ok && geom_has(ge, j0 + 8), my_stages + st1 * kStg,
+                       ok1 && geom_has(ge, j1), ok1 && geom_has(ge, j1 + 8), true, p.scale_log2,
+                       lane);
       __syncwarp();
       if (k + kRL < cw) issue(k + kRL);
       if (k + 1 + kRL < cw) issue(k + 1 + kRL);
       k += 2;
     } else {
-      page_compute(A, qf, my_stages + st * kStageBytes, ok && geom_has(ge, j0),
-                   ok && geom_has(ge, j0 + 8), p.scale_log2, lane);
+      pages_compute<F>(A, qf, my_stages + st * kStg, ok && geom_has(ge, j0),
+                       ok && geom_has(ge, j0 + 8), nullptr, false, false, false, p.scale_log2,
+                       lane);
       __syncwarp();
       if (k + kRL < cw) issue(k + kRL);
       k += 1;
@@ -726,14 +1009,18 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 }
 
 // ------------------------------------------------------------ full set: persistent grid
+template <int F>
 __global__ void __launch_bounds__(kThreads, 2)
 attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const AttnParams p) {
+  constexpr int kR = Fmt<F>::kR;
+  constexpr int kStg = Fmt<F>::kStage;
+  constexpr int kQueueLow = kR + kChunk;   // queue length that triggers the next claim
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+      (reinterpret_cast<uintptr_t>(smem_raw) + (Fmt<F>::kAlign - 1)) & ~uintptr_t(Fmt<F>::kAlign - 1));
   const int g = p.g;
-  float* merge_o = reinterpret_cast<float*>(stages + kStagesBytes);   // [W][g][132]
+  float* merge_o = reinterpret_cast<float*>(stages + kW * kR * kStg);   // [W][g][132]
   float* merge_ml = merge_o + kW * g * kMergeStride;                  // [W][8][2]
   float* cpart_o = merge_ml + kW * 16;                                // combine scratch
   __shared__ __align__(8) uint64_t bars[kW * kR];
@@ -749,8 +1036,10 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 #pragma unroll
     for (int i = 0; i < kW * kR; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
-    prefetch_tensormap(&tmA);
-    if (!p.kv_single) prefetch_tensormap(&tmB);
+    if (F == 0) {
+      prefetch_tensormap(&tmA);
+      if (!p.kv_single) prefetch_tensormap(&tmB);
+    }
   }
   // ---- per-sequence geometry and unit prefix sums (identical in every CTA)
   for (int b = tid; b < B; b += kThreads) {
@@ -792,7 +1081,7 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     u0 = (int)(vc * U / G);
     u1 = (int)((vc + 1) * U / G);
   }
-  uint8_t* my_stages = stages + warp * kR * kStageBytes;
+  uint8_t* my_stages = stages + warp * kR * kStg;
   uint64_t* my_bars = bars + warp * kR;
 
   // ---- this warp's copy stream.  The pages of a (b, h) are split into chunks of kChunk
@@ -913,7 +1202,7 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const uint32_t st = issued % kR;
     if (lane == src) {
       if (phys >= 0)
-        issue_page(my_stages + st * kStageBytes, my_bars + st, &tmA, &tmB, p.kv_single, phys, Hkv, hh);
+        issue_any<F>(my_stages + st * kStg, my_bars + st, &tmA, &tmB, p, phys, hh);
       else
         mbar_arrive(my_bars + st);
     }
@@ -957,8 +1246,8 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const Seg cs = decode_seg(seg_u, u1, s_us, s_nv, B, Hkv);
     const int b = cs.b, h = cs.h;
     const int n_cache = s_t[b] - 1;
-    uint32_t qf[8][2];
-    load_qf(qf, p, b, h, lane);
+    QFrag<F> qf;
+    load_q<F>(qf, p, b, h, lane);
     WarpAcc A;
     acc_init(A);
     const int r = lane >> 2;
@@ -977,8 +1266,8 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const bool ok = (vbits >> st) & 1u;
       const int lp = __shfl_sync(0xffffffffu, st_lp, (int)st);
       const int j0 = lp * kPageTok + r;
-      page_compute(A, qf, my_stages + st * kStageBytes, ok && j0 < n_cache, ok && j0 + 8 < n_cache,
-                   p.scale_log2, lane);
+      pages_compute<F>(A, qf, my_stages + st * kStg, ok && j0 < n_cache, ok && j0 + 8 < n_cache,
+                       nullptr, false, false, false, p.scale_log2, lane);
       ++consumed;
       __syncwarp();
       top_up();
@@ -1255,61 +1544,84 @@ int cta_stride(int grid) {
 }
 
 // stages | merge_o [W][g][132] | merge_ml [W][16] | CTA partial / combine scratch
-int attention_smem_bytes(int g) {
+template <int F>
+int full_smem_bytes(int g) {
   const int tail = g * 130 > kW * 132 ? g * 130 : kW * 132;
-  return 1024 + kStagesBytes + (kW * g * kMergeStride + kW * 16 + tail) * (int)sizeof(float);
+  return Fmt<F>::kAlign + kW * Fmt<F>::kR * Fmt<F>::kStage +
+         (kW * g * kMergeStride + kW * 16 + tail) * (int)sizeof(float);
 }
+int attention_smem_bytes(int g) { return full_smem_bytes<0>(g); }
 // local set: the merge areas live in the stages (kWL * g * 132 + kWL * 16 + g * 130 floats,
-// 38 KB at g = 8, within the 192 KB of stages)
-int local_smem_bytes(int) { return 1024 + kStagesBytesL; }
+// 38 KB at g = 8, within the ~200 KB of stages)
+template <int F>
+int local_smem_bytes() { return Fmt<F>::kAlign + kWL * Fmt<F>::kRL * Fmt<F>::kStage; }
 
-// Sets the shared-memory limits and returns the persistent grid size for group size g.  The
+// Sets the shared-memory limits of both kernels in both page formats and returns the
+// persistent full-set grid size for group size g per format (ctas[0] bf16, ctas[1] fp8).  The
 // limit is a per-function setting shared by every context of the process, so it is always set
 // to the largest group's need (g = 8): a context created later with a smaller g must not lower
 // it under a launch of an earlier context.
 oda_status prepare_attention_kernel(int g, int n_sms, int* ctas) {
-  const int smem = attention_smem_bytes(g);
   oda_status st = check_cuda(
-      cudaFuncSetAttribute(attn_full_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           attention_smem_bytes(8)),
+      cudaFuncSetAttribute(attn_full_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           full_smem_bytes<0>(8)),
       "cudaFuncSetAttribute(full attention)");
   if (st == ODA_OK)
-    st = check_cuda(cudaFuncSetAttribute(attn_local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         local_smem_bytes(g)),
+    st = check_cuda(cudaFuncSetAttribute(attn_full_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         full_smem_bytes<1>(8)),
+                    "cudaFuncSetAttribute(full attention, fp8)");
+  if (st == ODA_OK)
+    st = check_cuda(cudaFuncSetAttribute(attn_local_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         local_smem_bytes<0>()),
                     "cudaFuncSetAttribute(local attention)");
+  if (st == ODA_OK)
+    st = check_cuda(cudaFuncSetAttribute(attn_local_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         local_smem_bytes<1>()),
+                    "cudaFuncSetAttribute(local attention, fp8)");
   if (st != ODA_OK) return st;
-  int occ = 0;
-  st = check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, attn_full_kernel, kThreads, smem),
-                  "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
-  if (st != ODA_OK) return st;
-  occ = std::max(1, std::min(occ, 2));
-  *ctas = n_sms * occ;
-  // the combine keeps one weight per partial and head in the merge area
-  if (*ctas > kW * kMergeStride) return set_error(ODA_ERR_UNSUPPORTED, "too many CTAs for the merge area");
+  for (int f = 0; f < 2; ++f) {
+    int occ = 0;
+    st = f == 0 ? check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, attn_full_kernel<0>,
+                                                                          kThreads, full_smem_bytes<0>(g)),
+                             "cudaOccupancyMaxActiveBlocksPerMultiprocessor")
+                : check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, attn_full_kernel<1>,
+                                                                          kThreads, full_smem_bytes<1>(g)),
+                             "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (st != ODA_OK) return st;
+    occ = std::max(1, std::min(occ, 2));
+    ctas[f] = n_sms * occ;
+    // the combine keeps one weight per partial and head in the merge area
+    if (ctas[f] > kW * kMergeStride) return set_error(ODA_ERR_UNSUPPORTED, "too many CTAs for the merge area");
+  }
   return ODA_OK;
 }
 
-oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32_t* page_table,
+oda_status launch_attention(oda_ctx* ctx, const KvPool& pool, const int32_t* page_table,
                             const int32_t* pos, const int32_t* flag, const void* q,
                             const void* k_new, const void* v_new, float* out, int mode,
                             cudaStream_t stream) {
   const oda_config& cf = ctx->cfg;
-  if (!layer || !layer->k || !layer->v || !page_table || !pos || !q || !k_new || !v_new || !out ||
+  const int F = pool.fmt;
+  if (!pool.k || (F == 0 && !pool.v) || !page_table || !pos || !q || !k_new || !v_new || !out ||
       (mode == 1 && !flag))
     return set_error(ODA_ERR_INVALID_ARG, "attention: null pointer argument");
-  if (layer->n_pages <= 0 || layer->n_pages * (int64_t)cf.n_kv_heads * kPageTok > INT32_MAX)
+  if (pool.n_pages <= 0 || pool.n_pages * (int64_t)cf.n_kv_heads * kPageTok > INT32_MAX)
     return set_error(ODA_ERR_INVALID_ARG, "attention: n_pages out of range (%lld)",
-                     (long long)layer->n_pages);
-  if ((reinterpret_cast<uintptr_t>(layer->k) | reinterpret_cast<uintptr_t>(layer->v)) & 15)
+                     (long long)pool.n_pages);
+  if ((reinterpret_cast<uintptr_t>(pool.k) | reinterpret_cast<uintptr_t>(pool.v)) & 15)
     return set_error(ODA_ERR_INVALID_ARG, "attention: K/V pools must be 16-byte aligned");
   if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k_new) |
        reinterpret_cast<uintptr_t>(v_new) | reinterpret_cast<uintptr_t>(out)) & 3)
     return set_error(ODA_ERR_INVALID_ARG, "attention: q/k_new/v_new/out must be 4-byte aligned");
   CUtensorMap tmA, tmB;
+  memset(&tmA, 0, sizeof tmA);
+  memset(&tmB, 0, sizeof tmB);
   int kv_single = 0;
-  oda_status st = encode_kv(&tmA, &tmB, &kv_single, layer->k, layer->v, layer->n_pages,
-                            cf.n_kv_heads);
-  if (st != ODA_OK) return st;
+  oda_status st = ODA_OK;
+  if (F == 0) {
+    st = encode_kv(&tmA, &tmB, &kv_single, pool.k, pool.v, pool.n_pages, cf.n_kv_heads);
+    if (st != ODA_OK) return st;
+  }
   AttnParams p;
   p.kv_single = kv_single;
   p.cta_perm = 1;
@@ -1317,6 +1629,7 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
   p.page_table = page_table;
   p.pos = pos;
   p.flag = flag;
+  p.kv8 = F == 1 ? static_cast<const uint8_t*>(pool.k) : nullptr;
   p.q = static_cast<const uint32_t*>(q);
   p.k_new = static_cast<const uint32_t*>(k_new);
   p.v_new = static_cast<const uint32_t*>(v_new);
@@ -1326,7 +1639,7 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
   p.counters = ctx->attn_cnt;
   p.claims = ctx->attn_cnt + (size_t)cf.batch * cf.n_kv_heads;
   p.err = ctx->err;
-  p.n_pool_pages = layer->n_pages;
+  p.n_pool_pages = pool.n_pages;
   p.B = cf.batch;
   p.Hq = cf.n_q_heads;
   p.Hkv = cf.n_kv_heads;
@@ -1346,7 +1659,8 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
   // before reading q or writing.
   cudaLaunchConfig_t lc = {};
   lc.blockDim = dim3(mode == 0 ? kThreadsL : kThreads);
-  lc.dynamicSmemBytes = mode == 0 ? local_smem_bytes(ctx->g) : attention_smem_bytes(ctx->g);
+  lc.dynamicSmemBytes = mode == 0 ? (F == 0 ? local_smem_bytes<0>() : local_smem_bytes<1>())
+                                  : (F == 0 ? full_smem_bytes<0>(ctx->g) : full_smem_bytes<1>(ctx->g));
   lc.stream = stream;
   cudaLaunchAttribute attr[2];
   int na = 0;
@@ -1363,14 +1677,17 @@ oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32
     ++na;
     lc.gridDim = dim3(pairs * p.cluster);
   } else {
-    lc.gridDim = dim3(ctx->attn_ctas);
-    p.cta_perm = cta_stride(ctx->attn_ctas);
+    lc.gridDim = dim3(ctx->attn_ctas[F]);
+    p.cta_perm = cta_stride(ctx->attn_ctas[F]);
   }
   lc.attrs = attr;
   lc.numAttrs = na;
-  st = (mode == 0)
-           ? check_cuda(cudaLaunchKernelEx(&lc, attn_local_kernel, tmA, tmB, p), "local attention launch")
-           : check_cuda(cudaLaunchKernelEx(&lc, attn_full_kernel, tmA, tmB, p), "full attention launch");
+  if (mode == 0)
+    st = F == 0 ? check_cuda(cudaLaunchKernelEx(&lc, attn_local_kernel<0>, tmA, tmB, p), "local attention launch")
+                : check_cuda(cudaLaunchKernelEx(&lc, attn_local_kernel<1>, tmA, tmB, p), "local attention launch");
+  else
+    st = F == 0 ? check_cuda(cudaLaunchKernelEx(&lc, attn_full_kernel<0>, tmA, tmB, p), "full attention launch")
+                : check_cuda(cudaLaunchKernelEx(&lc, attn_full_kernel<1>, tmA, tmB, p), "full attention launch");
   ctx->prev_attention = (st == ODA_OK);
   return st;
 }
@@ -1402,7 +1719,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 struct NoAllocDevice {
   unsigned char* scratch = nullptr;   // device address of g_noalloc_scratch on this device
   int n_sms = 0;
-  int ctas[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};   // persistent grid size per group size g
+  int ctas[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};   // persistent bf16 grid size per group size g
   bool ready = false;
 };
 constexpr int kNoAllocMaxDevices = 64;
@@ -1433,11 +1750,10 @@ oda_status noalloc_setup(int g, NoAllocDevice** out, int* ctas) {
     d.ready = true;
   }
   if (d.ctas[g] == 0) {
-    st = prepare_attention_kernel(g, d.n_sms, &d.ctas[g]);
-    if (st != ODA_OK) {
-      d.ctas[g] = 0;
-      return st;
-    }
+    int both[2] = {0, 0};
+    st = prepare_attention_kernel(g, d.n_sms, both);
+    if (st != ODA_OK) return st;
+    d.ctas[g] = both[0];
   }
   *out = &d;
   *ctas = d.ctas[g];
@@ -1524,8 +1840,9 @@ oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* l
   p.mode = 1;
   p.cluster = 1;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt(128.0));
+  p.kv8 = nullptr;
   p.cta_perm = cta_stride(ctas);
-  attn_full_kernel<<<ctas, kThreads, attention_smem_bytes(g), stream>>>(tmA, tmB, p);
+  attn_full_kernel<0><<<ctas, kThreads, attention_smem_bytes(g), stream>>>(tmA, tmB, p);
   return check_cuda(cudaGetLastError(), "noalloc full attention launch");
 }
 

@@ -13,8 +13,8 @@ struct oda_ctx {
   int n_sms = 0;
   int g = 1;
   // split-KV attention scratch
-  int attn_ctas = 0;          // persistent grid size of the attention kernel
-  int n_slots = 0;            // partial slots: attn_ctas + B*Hkv
+  int attn_ctas[2] = {0, 0};  // persistent grid size of the full-set kernel: bf16, fp8 pages
+  int n_slots = 0;            // partial slots: max(attn_ctas) + B*Hkv
   float* part_o = nullptr;    // [n_slots][g][128]
   float* part_ml = nullptr;   // [n_slots][g][2]
   int32_t* attn_cnt = nullptr;  // [2][B*Hkv] completion and chunk-claim counters (self-resetting)
@@ -48,8 +48,17 @@ oda_status check_cuda(cudaError_t e, const char* what);
 // of oda_config except head_in_dim, theta and overlap_layers.
 oda_status validate_attention_config(const oda_config& c, const char* who);
 
+// Where one layer's cached pages live: fmt 0 = bf16 K and V pools (k, v), fmt 1 = fp8 page
+// blocks (k; v unused).
+struct KvPool {
+  int fmt;
+  const void* k;
+  const void* v;
+  int64_t n_pages;
+};
+
 // attention.cu
-oda_status launch_attention(oda_ctx* ctx, const oda_kv_layer* layer, const int32_t* page_table,
+oda_status launch_attention(oda_ctx* ctx, const KvPool& pool, const int32_t* page_table,
                             const int32_t* pos, const int32_t* flag, const void* q,
                             const void* k_new, const void* v_new, float* out, int mode,
                             cudaStream_t stream);
@@ -57,7 +66,7 @@ oda_status launch_index_positions(oda_ctx* ctx, int mode, const int32_t* pos, co
                                   int32_t* positions, int32_t cap, int32_t* counts,
                                   cudaStream_t stream);
 int attention_smem_bytes(int g);
-oda_status prepare_attention_kernel(int g, int n_sms, int* ctas);
+oda_status prepare_attention_kernel(int g, int n_sms, int* ctas /* [2] */);
 oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* layer,
                                     const int32_t* page_table, const int32_t* pos,
                                     const int32_t* flag, const void* q, const void* k_new,
@@ -80,7 +89,9 @@ oda_status launch_recall_grad(const oda_head_weights* w, const oda_head_grads* g
                               size_t workspace_bytes, cudaStream_t s);
 
 // commit.cu
-oda_status launch_commit(oda_ctx* ctx, const oda_kv_layer* layers, int32_t n_layers,
+oda_status launch_kv8_pack(const oda_kv_layer* src, const oda_kv8_layer* dst, int32_t n_kv_heads,
+                           cudaStream_t stream);
+oda_status launch_commit(oda_ctx* ctx, const KvPool* layers, int32_t n_layers,
                          const int32_t* page_table, int32_t* pos, const int32_t* flag,
                          const void* ksl, const void* vsl, const void* ksf, const void* vsf,
                          const float* h_local, const float* h_full, float* h_prev,

@@ -86,7 +86,7 @@ class OdaDecoder:
 
     def __init__(self, wl: Workload, device="cuda", capacity_steps: int = 0,
                  perturb_head: bool = False, head_params: dict = None, fill_cache: bool = True,
-                 overlap_layers: bool = True, deterministic: bool = False):
+                 overlap_layers: bool = True, deterministic: bool = False, kv_format: str = "bf16"):
         if not torch.cuda.is_available():
             raise RuntimeError("OdaDecoder needs a CUDA device (the CUDA path has no fallback)")
         self.wl = wl
@@ -105,7 +105,10 @@ class OdaDecoder:
         dev = self.device
         self.stream = torch.cuda.Stream(dev)
         self.page_table = torch.from_numpy(inputs.page_table(wl, self.max_pages)).to(dev)
-        self.k_pool, self.v_pool = [], []
+        if kv_format not in ("bf16", "fp8"):
+            raise ValueError("kv_format must be 'bf16' or 'fp8'")
+        self.kv_format = kv_format
+        self.k_pool, self.v_pool, self.kv8_pool = [], [], []
         for a in range(L):
             k = torch.empty((self.n_pool, Hkv, configs.PAGE, 128), dtype=torch.bfloat16, device=dev)
             v = torch.empty_like(k)
@@ -114,9 +117,24 @@ class OdaDecoder:
                              [inputs.cache_key(wl, "k", a, b) for b in range(B)], Hkv)
                 wdev.fill_kv(v, self.page_table, wl.ctx,
                              [inputs.cache_key(wl, "v", a, b) for b in range(B)], Hkv)
-            self.k_pool.append(k)
-            self.v_pool.append(v)
-        self.layers = [oda.kv_layer(self.k_pool[a], self.v_pool[a]) for a in range(L)]
+            if kv_format == "bf16":
+                self.k_pool.append(k)
+                self.v_pool.append(v)
+            else:
+                # the seeded bf16 cache of this layer, packed into fp8 page blocks by the library
+                kv8 = torch.empty((self.n_pool, Hkv, oda.KV8_BLOCK_BYTES), dtype=torch.uint8, device=dev)
+                oda.oda_kv8_pack(oda.kv_layer(k, v), oda.kv8_layer(kv8), Hkv)
+                torch.cuda.synchronize(dev)
+                self.kv8_pool.append(kv8)
+                del k, v
+        if kv_format == "bf16":
+            self.layers = [oda.kv_layer(self.k_pool[a], self.v_pool[a]) for a in range(L)]
+        else:
+            self.layers = [oda.kv8_layer(self.kv8_pool[a]) for a in range(L)]
+        fp8 = kv_format == "fp8"
+        self._attend_local = oda.oda_attend_local_fp8 if fp8 else oda.oda_attend_local
+        self._attend_full = oda.oda_attend_full_if_fp8 if fp8 else oda.oda_attend_full_if
+        self._commit = oda.oda_commit_fp8 if fp8 else oda.oda_commit
         self.pos = torch.tensor([c + 1 for c in wl.ctx], dtype=torch.int32, device=dev)
         # the step's results (h_{t-1} after the commit, q_t, the routing flags) share one
         # device block, so they come back to the host in a single copy (read_results)
@@ -201,8 +219,8 @@ class OdaDecoder:
         a = j = 0
         for layer in range(n_layers):
             if layer in wl.attn_layers:
-                oda.oda_attend_local(ctx, self.layers[a], self.page_table, self.pos, sv["q"][LOCAL, a],
-                                     sv["k"][LOCAL, a], sv["v"][LOCAL, a], self.o[LOCAL, layer], s)
+                self._attend_local(ctx, self.layers[a], self.page_table, self.pos, sv["q"][LOCAL, a],
+                                   sv["k"][LOCAL, a], sv["v"][LOCAL, a], self.o[LOCAL, layer], s)
                 a += 1
             else:
                 oda.oda_glue_gdn(ctx, self.live, j, sv["gc"][LOCAL, j], sv["gv"][LOCAL, j],
@@ -219,9 +237,9 @@ class OdaDecoder:
         a = j = 0
         for layer in range(n_layers):
             if layer in wl.attn_layers:
-                oda.oda_attend_full_if(ctx, self.layers[a], self.page_table, self.pos, self.flag,
-                                       sv["q"][FULL, a], sv["k"][FULL, a], sv["v"][FULL, a],
-                                       self.o[FULL, layer], body)
+                self._attend_full(ctx, self.layers[a], self.page_table, self.pos, self.flag,
+                                  sv["q"][FULL, a], sv["k"][FULL, a], sv["v"][FULL, a],
+                                  self.o[FULL, layer], body)
                 a += 1
             else:
                 oda.oda_glue_gdn(ctx, self.live, j, sv["gc"][FULL, j], sv["gv"][FULL, j],
@@ -230,9 +248,9 @@ class OdaDecoder:
                 j += 1
         oda.oda_glue_hidden(ctx, sv["emb"], self.o[FULL], n_layers, self.flag, self.h[FULL], body)
         oda.oda_cond_end(ctx, s)
-        oda.oda_commit(ctx, self.layers, self.page_table, self.pos, self.flag, sv["k"][LOCAL],
-                       sv["v"][LOCAL], sv["k"][FULL], sv["v"][FULL], self.h[LOCAL], self.h[FULL],
-                       self.h_prev, s)
+        self._commit(ctx, self.layers, self.page_table, self.pos, self.flag, sv["k"][LOCAL],
+                     sv["v"][LOCAL], sv["k"][FULL], sv["v"][FULL], self.h[LOCAL], self.h[FULL],
+                     self.h_prev, s)
 
     def capture(self) -> None:
         """Records one step (with the retry under a conditional node) as a CUDA graph, once per
@@ -285,6 +303,8 @@ class OdaDecoder:
         return oda.oda_get_error(self.ctx)
 
     def attention_layers_bytes(self) -> int:
+        if self.kv_format == "fp8":
+            return sum(p.numel() for p in self.kv8_pool)
         return sum(k.numel() * 2 * 2 for k in self.k_pool)
 
     def close(self):

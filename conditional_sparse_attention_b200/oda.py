@@ -12,8 +12,8 @@ from typing import Optional, Sequence
 import torch
 
 from . import _lib
-from ._lib import (OdaConfig, OdaError, OdaHeadGrads, OdaHeadWeights, OdaKVLayer,  # noqa: F401
-                   OdaState, check)
+from ._lib import (OdaConfig, OdaError, OdaHeadGrads, OdaHeadWeights, OdaKV8Layer,  # noqa: F401
+                   OdaKVLayer, OdaState, check)
 
 _c = ctypes.c_void_p
 
@@ -65,6 +65,14 @@ def make_config(batch, n_q_heads, n_kv_heads, max_pages, head_in_dim, sinks=4, w
 def kv_layer(k: torch.Tensor, v: torch.Tensor) -> OdaKVLayer:
     """Pool descriptor: k, v bf16 [n_pages, Hkv, 16, 128]."""
     return OdaKVLayer(k.data_ptr(), v.data_ptr(), int(k.shape[0]))
+
+
+KV8_BLOCK_BYTES = 4224
+
+
+def kv8_layer(kv: torch.Tensor) -> OdaKV8Layer:
+    """fp8 pool descriptor: kv uint8 [n_pages, Hkv, 4224] (page blocks, see include/oda.h)."""
+    return OdaKV8Layer(kv.data_ptr(), int(kv.shape[0]))
 
 
 def head_weights(P: dict, cls=OdaHeadWeights):
@@ -126,6 +134,34 @@ def oda_attend_full_if_noalloc(cfg: OdaConfig, layer: OdaKVLayer, page_table, po
                                                  _p(page_table), _p(pos), _p(flag), _p(q),
                                                  _p(k_new), _p(v_new), _p(out), _p(device_error),
                                                  _s(stream)))
+
+
+def oda_attend_local_fp8(ctx, layer: OdaKV8Layer, page_table, pos, q, k_new, v_new, out,
+                         stream=None):
+    check(_lib.load().oda_attend_local_fp8(ctx.handle, ctypes.byref(layer), _p(page_table),
+                                           _p(pos), _p(q), _p(k_new), _p(v_new), _p(out),
+                                           _s(stream)))
+
+
+def oda_attend_full_if_fp8(ctx, layer: OdaKV8Layer, page_table, pos, flag, q, k_new, v_new, out,
+                           stream=None):
+    check(_lib.load().oda_attend_full_if_fp8(ctx.handle, ctypes.byref(layer), _p(page_table),
+                                             _p(pos), _p(flag), _p(q), _p(k_new), _p(v_new),
+                                             _p(out), _s(stream)))
+
+
+def oda_kv8_pack(src: OdaKVLayer, dst: OdaKV8Layer, n_kv_heads: int, stream=None):
+    check(_lib.load().oda_kv8_pack(ctypes.byref(src), ctypes.byref(dst), n_kv_heads, _s(stream)))
+
+
+def oda_commit_fp8(ctx, layers: Sequence[OdaKV8Layer], page_table, pos, flag, k_stage_local,
+                   v_stage_local, k_stage_full, v_stage_full, h_local, h_full, h_prev,
+                   stream=None):
+    arr = (OdaKV8Layer * len(layers))(*layers)
+    check(_lib.load().oda_commit_fp8(ctx.handle, arr, len(layers), _p(page_table), _p(pos),
+                                     _p(flag), _p(k_stage_local), _p(v_stage_local),
+                                     _p(k_stage_full), _p(v_stage_full), _p(h_local), _p(h_full),
+                                     _p(h_prev), _s(stream)))
 
 
 def oda_index_positions(ctx, mode: int, pos, flag, positions, cap: int, counts, stream=None):

@@ -99,6 +99,29 @@ typedef struct {
   int64_t n_pages;      /* pages in this layer's pool (bounds every page-table entry)   */
 } oda_kv_layer;
 
+/* fp8 (OCP E4M3FN) KV pages.  The method notes suggest (summary and limits, section 4; the
+ * review page's section 六 likewise) combining the access policy with a quantised KV cache
+ * without fixing a format; this library's format keeps one fp32 scale per (token, KV head) row
+ * of 128 values: s = max|x| / 448 (1 for an all-zero row; NaN values ignored), code =
+ * round-to-nearest-even(x / s) saturating at +-448, both divisions in fp32 with IEEE rounding;
+ * cached value = s * e4m3(code).  One layer's pool is an array of page blocks
+ * [n_pages][Hkv][ODA_KV8_BLOCK_BYTES bytes]; the block of one (page, KV head) is
+ *   bytes [0, 2048)     K codes: token j (0..15) of the page at 128*j; the 16-value chunk k
+ *                       (0..7) of the token's 128 values is stored at chunk position k ^ (j & 7)
+ *                       within its row (an XOR swizzle for conflict-free shared-memory reads);
+ *   bytes [2048, 4096)  V codes transposed: dimension d (0..127) at 2048 + 16*d, 16 slots per
+ *                       dimension, slot s holding token 2*(s/4) + (s%2) + 8*((s/2)%2)
+ *                       (slots 4c..4c+3 hold tokens 2c, 2c+1, 2c+8, 2c+9);
+ *   bytes [4096, 4160)  K scales, fp32 [16], token order;
+ *   bytes [4160, 4224)  V scales, fp32 [16], token order.
+ * A block holds 16 tokens in 4224 bytes: 264 bytes per token and KV head, 51.6% of bf16's 512. */
+#define ODA_KV8_BLOCK_BYTES 4224
+
+typedef struct {
+  void* kv;             /* page blocks [n_pages][Hkv][4224 bytes], 16-byte aligned          */
+  int64_t n_pages;      /* pages in this layer's pool (bounds every page-table entry)       */
+} oda_kv8_layer;
+
 /* Recall-head parameters, fp32, row-major [out][in] matrices.  Towers i = 0,1,2 read
  * h_{t-1}, E(x_t), h^L_t.  D = head_in_dim, T = 1024 (tower width), F = 2048 (FFN width). */
 typedef struct {
@@ -200,6 +223,26 @@ oda_status oda_attend_full_if_noalloc(const oda_config* cfg, const oda_kv_layer*
                                       const void* v_new, float* out, int32_t* device_error,
                                       cudaStream_t stream);
 
+/* The same two attention calls over an fp8 pool (format above): identical arguments and
+ * semantics, with `layer` an fp8 pool.  The current token (position t) still comes from the
+ * bf16 staging, exactly as computed by the branch (it is quantised only when committed).
+ * Scores and outputs use the decoded cache values s * e4m3(code); arithmetic: codes and q
+ * (scaled per head by a power of two) as f16 tensor-core operands with fp32 accumulation. */
+oda_status oda_attend_local_fp8(oda_ctx* ctx, const oda_kv8_layer* layer,
+                                const int32_t* page_table, const int32_t* pos, const void* q,
+                                const void* k_new, const void* v_new, float* out,
+                                cudaStream_t stream);
+oda_status oda_attend_full_if_fp8(oda_ctx* ctx, const oda_kv8_layer* layer,
+                                  const int32_t* page_table, const int32_t* pos,
+                                  const int32_t* flag, const void* q, const void* k_new,
+                                  const void* v_new, float* out, cudaStream_t stream);
+
+/* Packs a bf16 cache layer (pools [n_pages][Hkv][16][128], as oda_kv_layer) into fp8 page
+ * blocks, every slot of every page (slots not yet written are packed too; they are never
+ * read).  src and dst must have the same n_pages.  Asynchronous on `stream`; no context. */
+oda_status oda_kv8_pack(const oda_kv_layer* src, const oda_kv8_layer* dst, int32_t n_kv_heads,
+                        cudaStream_t stream);
+
 /* The index sets as the attention kernels visit them (same work decomposition): for each
  * sequence b (mode 0: all, S^L; mode 1: flag[b] != 0, S^F), positions[b*cap + i] receives the
  * 1-based cache positions read, in page order, followed by t (the staged token);
@@ -258,6 +301,17 @@ oda_status oda_commit(oda_ctx* ctx, const oda_kv_layer* layers, int32_t n_layers
                       const void* k_stage_full, const void* v_stage_full,
                       const float* h_local, const float* h_full, float* h_prev,
                       cudaStream_t stream);
+
+/* oda_commit for an fp8 cache: the chosen branch's staged K,V (bf16) of every layer are
+ * quantised (the format above: one scale per (token, KV head) row) into the page slot of
+ * position t; h_prev and pos as oda_commit.  The codes and scales written are a deterministic
+ * function of the staged bf16 values. */
+oda_status oda_commit_fp8(oda_ctx* ctx, const oda_kv8_layer* layers, int32_t n_layers,
+                          const int32_t* page_table, int32_t* pos, const int32_t* flag,
+                          const void* k_stage_local, const void* v_stage_local,
+                          const void* k_stage_full, const void* v_stage_full,
+                          const float* h_local, const float* h_full, float* h_prev,
+                          cudaStream_t stream);
 
 /* ----------------------------------------------------- snapshot / restore ---------- */
 

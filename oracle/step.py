@@ -28,7 +28,8 @@ import numpy as np
 from workload import inputs as wi
 from workload.configs import Workload
 
-from .attention import attend_bits
+from . import kv_fp8
+from .attention import append_current, attend, attend_bits, bf16_to_f64
 from .delta import gdn_layer
 from .gate import route_full
 from .head import recall_head, rmsnorm
@@ -45,6 +46,8 @@ class OracleState:
     v_cache: list
     gdn_S: np.ndarray = None       # [B, n_gdn, 16, 128, 128] fp64
     gdn_conv: np.ndarray = None    # [B, n_gdn, 4, 2048] fp64
+    kv: str = "bf16"               # "bf16": caches hold bf16 bits; "fp8": caches hold the
+                                   # decoded values (fp64) of rows stored as e4m3 + scale
 
 
 @dataclass
@@ -57,14 +60,24 @@ class StepRecord:
     staged_v: dict = field(default_factory=dict)
 
 
-def initial_state(wl: Workload) -> OracleState:
-    """Prefilled caches (ctx_b tokens each), h_{t-1} and recurrent state from the generator."""
+def _stored(bits: np.ndarray, kv: str) -> np.ndarray:
+    """A cache row block as the cache holds it: bf16 bits, or (fp8) the decoded values of its
+    quantised rows (oracle.kv_fp8's format)."""
+    if kv == "bf16":
+        return bits
+    codes, scales = kv_fp8.quantize_rows(bf16_to_f64(bits))
+    return kv_fp8.dequantize_rows(codes, scales)
+
+
+def initial_state(wl: Workload, kv: str = "bf16") -> OracleState:
+    """Prefilled caches (ctx_b tokens each), h_{t-1} and recurrent state from the generator.
+    kv = "fp8": the prefilled rows are stored quantised (the cache holds their decoded values)."""
     kc, vc = [], []
     for a in range(wl.L):
-        kc.append([wi.cache_tokens(wl, "k", a, b, wl.ctx[b]) for b in range(wl.B)])
-        vc.append([wi.cache_tokens(wl, "v", a, b, wl.ctx[b]) for b in range(wl.B)])
+        kc.append([_stored(wi.cache_tokens(wl, "k", a, b, wl.ctx[b]), kv) for b in range(wl.B)])
+        vc.append([_stored(wi.cache_tokens(wl, "v", a, b, wl.ctx[b]), kv) for b in range(wl.B)])
     st = OracleState(pos=[c + 1 for c in wl.ctx], h_prev=wi.h_prev0(wl).astype(np.float64),
-                     k_cache=kc, v_cache=vc)
+                     k_cache=kc, v_cache=vc, kv=kv)
     if wl.hybrid:
         S, C = wi.gdn_state0(wl)
         st.gdn_S = S.astype(np.float64)
@@ -110,7 +123,12 @@ def run_pass(wl: Workload, state: OracleState, step: int, branch: int, active, r
             for b in active:
                 t = state.pos[b]
                 S = local_set(t, wl.sinks, wl.window) if branch == LOCAL else full_set(t)
-                o[b] = attend_bits(q[b], state.k_cache[a][b], state.v_cache[a][b], k[b], v[b], S)
+                if state.kv == "bf16":
+                    o[b] = attend_bits(q[b], state.k_cache[a][b], state.v_cache[a][b], k[b], v[b], S)
+                else:   # stored rows decoded; the current token exactly as this branch computed it
+                    o[b] = attend(bf16_to_f64(q[b]),
+                                  append_current(state.k_cache[a][b], bf16_to_f64(k[b])),
+                                  append_current(state.v_cache[a][b], bf16_to_f64(v[b])), S)
                 x[b] += o[b].reshape(D)
             rec.o[(branch, a)] = o
             a += 1
@@ -159,9 +177,9 @@ def commit(wl: Workload, state: OracleState, rec: StepRecord) -> None:
         br = FULL if rec.flags[b] else LOCAL
         for a in range(wl.L):
             state.k_cache[a][b] = np.concatenate(
-                [state.k_cache[a][b], rec.staged_k[(br, a)][b][None]], axis=0)
+                [state.k_cache[a][b], _stored(rec.staged_k[(br, a)][b], state.kv)[None]], axis=0)
             state.v_cache[a][b] = np.concatenate(
-                [state.v_cache[a][b], rec.staged_v[(br, a)][b][None]], axis=0)
+                [state.v_cache[a][b], _stored(rec.staged_v[(br, a)][b], state.kv)[None]], axis=0)
         state.h_prev[b] = rec.h[br][b]
         state.pos[b] += 1
 

@@ -38,3 +38,41 @@ def logical_cache(pool_u16: np.ndarray, page_table: np.ndarray, b: int, n_tokens
     pages = page_table[b, :(n_tokens + 15) // 16]
     toks = pool_u16[pages].transpose(0, 2, 1, 3).reshape(-1, pool_u16.shape[1], 128)
     return toks[:n_tokens]
+
+
+def v8_slot_token(s: int) -> int:
+    """Token held by slot s of a V row of an fp8 page block (layout stated in include/oda.h)."""
+    return 2 * (s // 4) + (s % 2) + 8 * ((s // 2) % 2)
+
+
+def decode_kv8_block(blk: np.ndarray):
+    """(K codes [16,128], V codes [16,128], K scales [16], V scales [16]) of one fp8 page block,
+    read by the layout stated in include/oda.h."""
+    blk = np.ascontiguousarray(blk, dtype=np.uint8)
+    K = np.empty((16, 128), np.uint8)
+    for j in range(16):
+        row = blk[128 * j:128 * (j + 1)].reshape(8, 16)
+        K[j] = row[[k ^ (j & 7) for k in range(8)]].reshape(128)
+    Vt = blk[2048:4096].reshape(128, 16)
+    V = np.empty((16, 128), np.uint8)
+    for s in range(16):
+        V[v8_slot_token(s)] = Vt[:, s]
+    sk = blk[4096:4160].view(np.float32).astype(np.float64)
+    sv = blk[4160:4224].view(np.float32).astype(np.float64)
+    return K, V, sk, sv
+
+
+def logical_cache8(pool: np.ndarray, page_table: np.ndarray, b: int, n_tokens: int, table):
+    """Decoded values (fp64 [n, Hkv, 128]) of tokens 0..n-1 of sequence b from an fp8 pool
+    [n_pages, Hkv, 4224]; `table` maps codes to values."""
+    Hkv = pool.shape[1]
+    K = np.empty((n_tokens, Hkv, 128))
+    V = np.empty((n_tokens, Hkv, 128))
+    for tok in range(n_tokens):
+        phys = page_table[b, tok // 16]
+        for h in range(Hkv):
+            kc, vc, sk, sv = decode_kv8_block(pool[phys, h])
+            j = tok % 16
+            K[tok, h] = table[kc[j]] * sk[j]
+            V[tok, h] = table[vc[j]] * sv[j]
+    return K, V

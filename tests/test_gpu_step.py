@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import TIE_BAND, attn_close, build_all, logical_cache, score_close
+from helpers import TIE_BAND, attn_close, build_all, logical_cache, logical_cache8, score_close
 from oracle import step as OS
 from workload import configs, inputs
 
@@ -46,9 +46,9 @@ def _gpu_record(dec):
                 h_prev=dec.h_prev.cpu().numpy().copy(), pos=dec.pos.cpu().numpy().copy())
 
 
-def _run_gpu(wl, graph: bool, perturb=True, deterministic=False):
+def _run_gpu(wl, graph: bool, perturb=True, deterministic=False, kv_format="bf16"):
     from conditional_sparse_attention_b200.engine import OdaDecoder
-    dec = OdaDecoder(wl, perturb_head=perturb, deterministic=deterministic)
+    dec = OdaDecoder(wl, perturb_head=perturb, deterministic=deterministic, kv_format=kv_format)
     if graph:
         dec.capture()
     recs = []
@@ -59,6 +59,12 @@ def _run_gpu(wl, graph: bool, perturb=True, deterministic=False):
     caches = []
     pt = dec.page_table.cpu().numpy()
     for a in range(wl.L):
+        if kv_format == "fp8":
+            from oracle.kv_fp8 import E4M3_TABLE
+            pool = dec.kv8_pool[a].cpu().numpy()
+            caches.append([logical_cache8(pool, pt, b, wl.ctx[b] + wl.steps, E4M3_TABLE)
+                           for b in range(wl.B)])
+            continue
         kp = dec.k_pool[a].cpu().view(torch.int16).numpy().view(np.uint16)
         vp = dec.v_pool[a].cpu().view(torch.int16).numpy().view(np.uint16)
         caches.append([(logical_cache(kp, pt, b, wl.ctx[b] + wl.steps),
@@ -68,11 +74,13 @@ def _run_gpu(wl, graph: bool, perturb=True, deterministic=False):
     return recs, caches, head
 
 
-@pytest.mark.parametrize("name", ["cfg0", "cfg1_small", "cfg2_small", "cfg3_small", "cfg4_small"])
-def test_trajectory_matches_oracle(name):
+@pytest.mark.parametrize("name,kv", [("cfg0", "bf16"), ("cfg1_small", "bf16"), ("cfg2_small", "bf16"),
+                                     ("cfg3_small", "bf16"), ("cfg4_small", "bf16"),
+                                     ("cfg0", "fp8"), ("cfg2_small", "fp8"), ("cfg4_small", "fp8")])
+def test_trajectory_matches_oracle(name, kv):
     wl = _small(name)
-    recs, caches, P = _run_gpu(wl, graph=True)
-    st = OS.initial_state(wl)
+    recs, caches, P = _run_gpu(wl, graph=True, kv_format=kv)
+    st = OS.initial_state(wl, kv=kv)
     for s in range(wl.steps):
         sched = inputs.schedule(wl, s)
         st, rec = OS.decode_step(wl, st, s, P, sched=sched)

@@ -68,7 +68,40 @@ def test_row_scales_and_error_bound():
     # the row maximum maps to 448 exactly; every element is within half a step of its binade
     assert np.allclose(np.max(np.abs(xd[[0, 1]]), axis=1), np.max(np.abs(x[[0, 1]]), axis=1))
     rel = np.abs(xd - x) / np.maximum(np.abs(x), s[:, None] * 2.0 ** -6)
-    assert np.max(rel) <= 2.0 ** -4 + 1e-12
+    assert np.max(rel) <= 2.0 ** -4 + 1e-6      # + the fp32 rounding of x and of x / s
+
+
+def test_scale_and_scaled_values_are_fp32():
+    """The decisions are taken in fp32: the scale is an fp32 number, and a value whose fp64
+    quotient x / s lies just past a rounding midpoint but whose fp32 quotient lands on it rounds
+    as the fp32 quotient says."""
+    rng = np.random.default_rng(3)
+    x = rng.normal(0, 1, (16, 128)).astype(np.float32)
+    _, s = kv_fp8.quantize_rows(x)
+    assert np.array_equal(s, s.astype(np.float32).astype(np.float64))
+    # a row with max 448 (s = 1): x / s = x exactly, so the codes are the plain encoding
+    row = np.zeros(128, np.float32)
+    row[0], row[1], row[2] = 448.0, 1.0625, 1.1875
+    c, s1 = kv_fp8.quantize_rows(row)
+    assert s1 == 1.0 and c[1] == 0x38 and c[2] == 0x3A and c[0] == 0x7E
+    # fp32 division: 1 / fl32(1/3) rounded in fp32 is exactly 3 (the fp64 quotient is not)
+    amax = np.float32(448.0) * np.float32(3.0)
+    r2 = np.zeros(128, np.float32)
+    r2[0] = amax
+    r2[1] = np.float32(1.0)
+    c2, s2 = kv_fp8.quantize_rows(r2)
+    assert s2 == np.float32(amax / np.float32(448.0))
+    assert kv_fp8.e4m3_decode(c2[1]) == kv_fp8.e4m3_decode(kv_fp8.e4m3_encode(
+        float(np.float32(1.0) / np.float32(s2))))
+
+
+def test_nan_entries_do_not_set_the_scale():
+    x = np.ones((1, 128))
+    x[0, 5] = np.nan
+    x[0, 7] = 2.0
+    c, s = kv_fp8.quantize_rows(x)
+    assert s[0] == np.float32(2.0 / 448.0)
+    assert c[0, 5] == 0x7F and kv_fp8.e4m3_decode(c[0, 7]) * s[0] == pytest.approx(2.0)
 
 
 def test_attention_over_a_quantised_cache_is_the_plain_definition():
@@ -90,3 +123,32 @@ def test_attention_over_a_quantised_cache_is_the_plain_definition():
     # and it stays close to attention over the unquantised cache (e4m3 keeps 3 mantissa bits)
     o_ref = attend(q[None, :], K[:, None, :], V[:, None, :], S)[0]
     assert np.linalg.norm(o - o_ref) / np.linalg.norm(o_ref) < 0.08
+
+
+def test_attend_quantized_is_attention_over_the_decoded_cache_plus_the_exact_current_token():
+    from oracle.attention import append_current, bf16_to_f64
+    from oracle.sets import full_set, local_set
+    from workload import gen
+    t = 70
+    bits = lambda tag, n: gen.normal_bf16(gen.key(5, tag), n)  # noqa: E731
+    q = bits(1, 4 * 128).reshape(4, 128)
+    kc = bits(2, (t - 1) * 2 * 128).reshape(t - 1, 2, 128)
+    vc = bits(3, (t - 1) * 2 * 128).reshape(t - 1, 2, 128)
+    kn, vn = bits(4, 256).reshape(2, 128), bits(5, 256).reshape(2, 128)
+    for S in (full_set(t), local_set(t, 4, 32)):
+        got = kv_fp8.attend_quantized(q, kc, vc, kn, vn, S)
+        Kc, Ks = kv_fp8.quantize_rows(bf16_to_f64(kc))
+        Vc, Vs = kv_fp8.quantize_rows(bf16_to_f64(vc))
+        K = append_current(kv_fp8.dequantize_rows(Kc, Ks), bf16_to_f64(kn))
+        V = append_current(kv_fp8.dequantize_rows(Vc, Vs), bf16_to_f64(vn))
+        # written out directly: per head, scores over the set's rows, softmax, weighted values
+        rows = np.array(sorted(S)) - 1
+        for h in range(4):
+            kh = h // 2
+            sc = K[rows, kh] @ bf16_to_f64(q[h]) / math.sqrt(128)
+            w = np.exp(sc - sc.max())
+            w /= w.sum()
+            assert np.allclose(got[h], w @ V[rows, kh], rtol=1e-12, atol=1e-12)
+        # the current token is not quantised: changing its value moves the output exactly as
+        # the exact value says (position t always belongs to both sets)
+        assert t in S

@@ -146,3 +146,35 @@ def test_multi_step_trajectory_counts():
     assert st.pos == [c + 1 + wl.steps for c in wl.ctx]
     assert [st.k_cache[0][b].shape[0] for b in range(2)] == [c + wl.steps for c in wl.ctx]
     assert n_routed == wl.steps
+
+
+def test_fp8_cache_commits_the_decoded_quantised_row_and_tracks_bf16():
+    """fp8 mode: the commit appends the chosen row as stored (quantised, decoded), the cache's
+    older rows are untouched, and every attention output stays within the format's error of the
+    bf16-cache step (same inputs, same routing)."""
+    from oracle import kv_fp8
+    from oracle.attention import bf16_to_f64
+    wl = _small_attn(ctx=(40, 2100), L=2, rates=(1.0, 1.0))
+    P = _small_head(wl)
+    s8 = S.initial_state(wl, kv="fp8")
+    s16 = S.initial_state(wl)
+    # prefilled rows: every stored row is within e4m3's half step (2^-4 relative) of bf16's
+    for a in range(wl.L):
+        for b in range(wl.B):
+            x = bf16_to_f64(s16.k_cache[a][b])
+            d = np.abs(s8.k_cache[a][b] - x)
+            assert np.all(d <= 2.0 ** -4 * np.maximum(np.abs(x), np.max(np.abs(x), axis=-1, keepdims=True) / 448 * 2.0 ** -6) + 1e-12)
+    n8, rec8 = S.decode_step(wl, s8, 0, P, sched=_force(wl, [1, 0]))
+    n16, rec16 = S.decode_step(wl, s16, 0, P, sched=_force(wl, [1, 0]))
+    for b, br in ((0, S.FULL), (1, S.LOCAL)):
+        for a in range(wl.L):
+            row = rec8.staged_k[(br, a)][b]
+            c, sc = kv_fp8.quantize_rows(bf16_to_f64(row))
+            assert np.array_equal(n8.k_cache[a][b][-1], kv_fp8.dequantize_rows(c, sc))
+            assert np.array_equal(n8.k_cache[a][b][:-1], s8.k_cache[a][b])
+    for key, o in rec8.o.items():
+        for b in range(wl.B):
+            if key[0] == S.FULL and b == 1:
+                continue
+            r = np.linalg.norm(o[b] - rec16.o[key][b]) / np.linalg.norm(rec16.o[key][b])
+            assert r < 0.08, (key, b, r)
