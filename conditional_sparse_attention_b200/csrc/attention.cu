@@ -145,9 +145,11 @@ __device__ __forceinline__ float warp_sum(float v) {
 struct WarpAcc {
   float m0, m1, l0, l1;
   float o[8][4];
+  int e;   // fp8 pages: o is held in units of 2^e (the V-scale binade of the last page step)
 };
 
 __device__ __forceinline__ void acc_init(WarpAcc& A) {
+  A.e = 0;
   A.m0 = A.m1 = -INFINITY;
   A.l0 = A.l1 = 0.f;
 #pragma unroll
@@ -482,22 +484,44 @@ __device__ __forceinline__ void load_q8(QF8& Q, const AttnParams& p, int b, int 
   Q.fs1 = __shfl_sync(0xffffffffu, down, 8 * c + 4);
 }
 
-// Raw scores K q^T of one fp8 page (tokens as M in natural order, heads as N), before scales.
-__device__ __forceinline__ void page_scores8(float (&sacc)[4], const QF8& Q, uint32_t sb, int lane) {
+// K fragments of one fp8 page (tokens as M in natural order, dims in the q fragment order) and
+// V^T fragments (dims as M, tokens in the P^T fragment order), converted to f16.
+struct Page8 {
+  uint32_t k[8][4];   // A fragments of the 8 k-steps of K q^T
+  uint32_t v[8][4];   // A fragments of the 8 dim tiles of V^T P^T
+};
+
+__device__ __forceinline__ void load_page8(Page8& P, uint32_t sb, int lane) {
   const int mi = lane >> 3, rr = lane & 7;
-  const int tok = ((mi & 1) << 3) + rr;
-  float sa[4] = {0.f, 0.f, 0.f, 0.f}, sc[4] = {0.f, 0.f, 0.f, 0.f};
+  const int tok = ((mi & 1) << 3) + rr;          // K: token row this lane addresses
+  const int drow = ((mi & 1) << 3) + rr;         // V^T: dim row within a 16-dim tile
 #pragma unroll
   for (int kk = 0; kk < 8; kk += 2) {
     uint32_t r[4];
-    const int ch = kk + (mi >> 1);
-    ldsm_x4(r, sb + tok * 128 + ((ch ^ rr) << 4));
-    const uint32_t a0[4] = {e4m3x2_to_f16x2(r[0]), e4m3x2_to_f16x2(r[1]),
-                            e4m3x2_to_f16x2(r[0] >> 16), e4m3x2_to_f16x2(r[1] >> 16)};
-    const uint32_t a1[4] = {e4m3x2_to_f16x2(r[2]), e4m3x2_to_f16x2(r[3]),
-                            e4m3x2_to_f16x2(r[2] >> 16), e4m3x2_to_f16x2(r[3] >> 16)};
-    mma_f16_16816(sa, a0, Q.qf[kk][0], Q.qf[kk][1]);
-    mma_f16_16816(sc, a1, Q.qf[kk + 1][0], Q.qf[kk + 1][1]);
+    ldsm_x4(r, sb + tok * 128 + (((kk + (mi >> 1)) ^ rr) << 4));
+    e4m3x4_to_f16x2x2(r[0], P.k[kk][0], P.k[kk][2]);
+    e4m3x4_to_f16x2x2(r[1], P.k[kk][1], P.k[kk][3]);
+    e4m3x4_to_f16x2x2(r[2], P.k[kk + 1][0], P.k[kk + 1][2]);
+    e4m3x4_to_f16x2x2(r[3], P.k[kk + 1][1], P.k[kk + 1][3]);
+  }
+#pragma unroll
+  for (int mt = 0; mt < 8; mt += 2) {
+    uint32_t r[4];
+    ldsm_x4(r, sb + kF8V + (16 * (mt + (mi >> 1)) + drow) * 16);
+    e4m3x4_to_f16x2x2(r[0], P.v[mt][0], P.v[mt][2]);
+    e4m3x4_to_f16x2x2(r[1], P.v[mt][1], P.v[mt][3]);
+    e4m3x4_to_f16x2x2(r[2], P.v[mt + 1][0], P.v[mt + 1][2]);
+    e4m3x4_to_f16x2x2(r[3], P.v[mt + 1][1], P.v[mt + 1][3]);
+  }
+}
+
+// Raw scores K q^T of one converted page, before scales.
+__device__ __forceinline__ void page_scores8(float (&sacc)[4], const QF8& Q, const Page8& P) {
+  float sa[4] = {0.f, 0.f, 0.f, 0.f}, sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int kk = 0; kk < 8; kk += 2) {
+    mma_f16_16816(sa, P.k[kk], Q.qf[kk][0], Q.qf[kk][1]);
+    mma_f16_16816(sc, P.k[kk + 1], Q.qf[kk + 1][0], Q.qf[kk + 1][1]);
   }
   sacc[0] = sa[0] + sc[0];
   sacc[1] = sa[1] + sc[1];
@@ -522,45 +546,26 @@ __device__ __forceinline__ void v8_masks(bool in0, bool in1, int lane, uint32_t&
   mhi = ((bb & 1u) ? 0x0000FFFFu : 0u) | ((bb & 2u) ? 0xFFFF0000u : 0u);
 }
 
-// PV of one fp8 page into (hi, lo) accumulators: P'' fragments (hi / lo f16) times V^T codes.
-__device__ __forceinline__ void page_pv8(float (&th)[8][4], float (&tl)[8][4], uint32_t vb,
-                                         uint32_t bh0, uint32_t bh1, uint32_t bl0, uint32_t bl1,
-                                         bool masked, uint32_t mlo, uint32_t mhi, int lane) {
-  const int mi = lane >> 3, rr = lane & 7;
-  const int row = ((mi & 1) << 3) + rr;   // dim within the 16-dim tile
-#pragma unroll
-  for (int mt = 0; mt < 8; mt += 2) {
-    uint32_t r[4];
-    ldsm_x4(r, vb + (16 * (mt + (mi >> 1)) + row) * 16);
-    uint32_t a0[4] = {e4m3x2_to_f16x2(r[0]), e4m3x2_to_f16x2(r[1]),
-                      e4m3x2_to_f16x2(r[0] >> 16), e4m3x2_to_f16x2(r[1] >> 16)};
-    uint32_t a1[4] = {e4m3x2_to_f16x2(r[2]), e4m3x2_to_f16x2(r[3]),
-                      e4m3x2_to_f16x2(r[2] >> 16), e4m3x2_to_f16x2(r[3] >> 16)};
-    if (masked) {   // tokens outside the set: their codes may be stale (even NaN); P'' is 0 there
-      a0[0] &= mlo; a0[1] &= mlo; a0[2] &= mhi; a0[3] &= mhi;
-      a1[0] &= mlo; a1[1] &= mlo; a1[2] &= mhi; a1[3] &= mhi;
-    }
-    mma_f16_16816(th[mt], a0, bh0, bh1);
-    mma_f16_16816(tl[mt], a0, bl0, bl1);
-    mma_f16_16816(th[mt + 1], a1, bh0, bh1);
-    mma_f16_16816(tl[mt + 1], a1, bl0, bl1);
-  }
-}
-
 // NP (1 or 2) fp8 pages in one online-softmax step (one maximum and rescale for 16 * NP tokens).
 // in[i][0] / in[i][1]: whether this lane's token rows r and r + 8 of page i belong to the set.
+// The accumulator is kept in units of 2^A.e, the binade of the largest V scale of the step's
+// tokens, so P'' = p * sv * 2^-e stays below 2 and f16 keeps its precision; when the binade
+// changes the accumulator is rescaled by the (exact) power of two, together with the softmax's
+// own rescale.
 template <int NP>
 __device__ __forceinline__ void page_step8(WarpAcc& A, const QF8& Q, uint8_t* const (&st)[2],
                                            const bool (&in)[2][2], int lane) {
   const int r = lane >> 2;
+  Page8 P[NP];
+#pragma unroll
+  for (int i = 0; i < NP; ++i) load_page8(P[i], smem_u32(st[i]), lane);
   float x[2][4], svv[2][2];
   bool any_masked = false;
   float svmax = 0.f;
 #pragma unroll
   for (int i = 0; i < NP; ++i) {
-    const uint32_t sb = smem_u32(st[i]);
     float sacc[4];
-    page_scores8(sacc, Q, sb, lane);
+    page_scores8(sacc, Q, P[i]);
     const float* sk = reinterpret_cast<const float*>(st[i] + kF8SK);
     const float* sv = reinterpret_cast<const float*>(st[i] + kF8SV);
     const float k0 = sk[r], k1 = sk[r + 8];
@@ -584,31 +589,29 @@ __device__ __forceinline__ void page_step8(WarpAcc& A, const QF8& Q, uint8_t* co
     mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
     svmax = fmaxf(svmax, __shfl_xor_sync(0xffffffffu, svmax, off));
   }
-  // the pages' V-scale binade: P'' = p * sv * 2^-E stays below 2 in f16
-  const int E = (svmax > 0.f && svmax <= 3.0e38f) ? (int)((__float_as_uint(svmax) >> 23) & 0xFF) - 127 : 0;
-  const int Ec = min(126, max(-126, E));
-  const float down = __uint_as_float((uint32_t)(127 - Ec) << 23);
-  const float upE = __uint_as_float((uint32_t)(127 + Ec) << 23);
+  const int E = (svmax > 0.f && svmax <= 3.0e38f)
+                    ? min(126, max(-126, (int)((__float_as_uint(svmax) >> 23) & 0xFF) - 127))
+                    : A.e;
+  const float down = __uint_as_float((uint32_t)(127 - E) << 23);
   const float mn0 = fmaxf(A.m0, mx0), mn1 = fmaxf(A.m1, mx1);
-  if (mn0 > A.m0 || mn1 > A.m1) {
+  if (mn0 > A.m0 || mn1 > A.m1 || E != A.e) {
+    // o in units of 2^A.e -> units of 2^E, with the softmax rescale; -inf maxima give 0
     const float al0 = exp2f(A.m0 - mn0), al1 = exp2f(A.m1 - mn1);
     A.l0 *= al0;
     A.l1 *= al1;
+    const float f0 = ldexpf(al0, A.e - E), f1 = ldexpf(al1, A.e - E);
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
-      A.o[mt][0] *= al0;
-      A.o[mt][1] *= al1;
-      A.o[mt][2] *= al0;
-      A.o[mt][3] *= al1;
+      A.o[mt][0] *= f0;
+      A.o[mt][1] *= f1;
+      A.o[mt][2] *= f0;
+      A.o[mt][3] *= f1;
     }
     A.m0 = mn0;
     A.m1 = mn1;
+    A.e = E;
   }
   const bool masked = __any_sync(0xffffffffu, any_masked);
-  float th[8][4], tl[8][4];
-#pragma unroll
-  for (int mt = 0; mt < 8; ++mt)
-    th[mt][0] = th[mt][1] = th[mt][2] = th[mt][3] = tl[mt][0] = tl[mt][1] = tl[mt][2] = tl[mt][3] = 0.f;
 #pragma unroll
   for (int i = 0; i < NP; ++i) {
     const float p0 = exp2f(x[i][0] - A.m0), p1 = exp2f(x[i][1] - A.m1);
@@ -622,14 +625,23 @@ __device__ __forceinline__ void page_step8(WarpAcc& A, const QF8& Q, uint8_t* co
     const uint32_t l23 = pack_f16x2(q2 - f16_lo_to_f32(h23), q3 - f16_hi_to_f32(h23));
     const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
     const uint32_t bl0 = movmatrix_trans(l01), bl1 = movmatrix_trans(l23);
-    uint32_t mlo = 0xFFFFFFFFu, mhi = 0xFFFFFFFFu;
-    if (masked) v8_masks(in[i][0], in[i][1], lane, mlo, mhi);
-    page_pv8(th, tl, smem_u32(st[i] + kF8V), bh0, bh1, bl0, bl1, masked, mlo, mhi, lane);
+    if (masked) {   // tokens outside the set: their codes may be stale (even NaN); P'' is 0 there
+      uint32_t mlo, mhi;
+      v8_masks(in[i][0], in[i][1], lane, mlo, mhi);
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        P[i].v[mt][0] &= mlo;
+        P[i].v[mt][1] &= mlo;
+        P[i].v[mt][2] &= mhi;
+        P[i].v[mt][3] &= mhi;
+      }
+    }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      mma_f16_16816(A.o[mt], P[i].v[mt], bh0, bh1);
+      mma_f16_16816(A.o[mt], P[i].v[mt], bl0, bl1);
+    }
   }
-#pragma unroll
-  for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) A.o[mt][j] = fmaf(th[mt][j] + tl[mt][j], upE, A.o[mt][j]);
 }
 
 // Issues the bulk copy of one fp8 (page, KV head) block into a stage.
@@ -647,6 +659,17 @@ __device__ __forceinline__ void warp_flush(WarpAcc& A, float* mo, float* ml, int
   for (int off = 4; off < 32; off <<= 1) {
     A.l0 += __shfl_xor_sync(0xffffffffu, A.l0, off);
     A.l1 += __shfl_xor_sync(0xffffffffu, A.l1, off);
+  }
+  if (A.e != 0) {   // warp-uniform
+    const float u = __uint_as_float((uint32_t)(127 + A.e) << 23);
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      A.o[mt][0] *= u;
+      A.o[mt][1] *= u;
+      A.o[mt][2] *= u;
+      A.o[mt][3] *= u;
+    }
+    A.e = 0;
   }
   const int r = lane >> 2, c = lane & 3;
   const int n0 = 2 * c, n1 = 2 * c + 1;
@@ -1266,9 +1289,31 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const bool ok = (vbits >> st) & 1u;
       const int lp = __shfl_sync(0xffffffffu, st_lp, (int)st);
       const int j0 = lp * kPageTok + r;
-      pages_compute<F>(A, qf, my_stages + st * kStg, ok && j0 < n_cache, ok && j0 + 8 < n_cache,
-                       nullptr, false, false, false, p.scale_log2, lane);
-      ++consumed;
+      // An even page and the next page of its chunk go through one softmax step.  Chunks are
+      // queued whole and copies run kR >= 2 ahead, so the partner is always issued by now: the
+      // pairing depends only on page numbers, never on copy timing.
+      bool pair = false;
+      const uint32_t st1 = (consumed + 1) % kR;
+      if ((lp & 1) == 0 && consumed + 1 < issued)
+        pair = __shfl_sync(0xffffffffu, st_seg, (int)st1) == cseg &&
+               __shfl_sync(0xffffffffu, st_lp, (int)st1) == lp + 1;
+      if (pair) {
+        if (!mbar_wait_bounded(my_bars + st1, ((consumed + 1) / kR) & 1u, kWaitNs)) {
+          if (lane == 0) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
+          dead = true;
+          break;
+        }
+        const bool ok1 = (vbits >> st1) & 1u;
+        const int j1 = j0 + kPageTok;
+        pages_compute<F>(A, qf, my_stages + st * kStg, ok && j0 < n_cache, ok && j0 + 8 < n_cache,
+                         my_stages + st1 * kStg, ok1 && j1 < n_cache, ok1 && j1 + 8 < n_cache, true,
+                         p.scale_log2, lane);
+        consumed += 2;
+      } else {
+        pages_compute<F>(A, qf, my_stages + st * kStg, ok && j0 < n_cache, ok && j0 + 8 < n_cache,
+                         nullptr, false, false, false, p.scale_log2, lane);
+        ++consumed;
+      }
       __syncwarp();
       top_up();
       pump();

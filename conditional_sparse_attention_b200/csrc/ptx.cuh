@@ -188,12 +188,12 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Two e4m3 codes (bits 0-7 and 8-15 of x) -> f16x2 (the low code in the low half); exact.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t x) {
-  uint32_t y;
-  asm("{\n .reg .b16 lo;\n cvt.u16.u32 lo, %1;\n cvt.rn.f16x2.e4m3x2 %0, lo;\n}\n"
-      : "=r"(y) : "r"(x));
-  return y;
+// Four e4m3 codes (byte i of x) -> two f16x2: lo = (code 0, code 1), hi = (code 2, code 3), each
+// first code in the low half; exact.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n cvt.rn.f16x2.e4m3x2 %0, l;\n"
+      " cvt.rn.f16x2.e4m3x2 %1, h;\n}\n"
+      : "=r"(lo), "=r"(hi) : "r"(x));
 }
 
 // Two fp32 values -> e4m3 codes with round-to-nearest-even and saturation to +-448; lo in bits
