@@ -457,6 +457,109 @@ def run_sweep(args, wl0, local_rank):
                       "max_rho_where_oda_is_faster": cross}), flush=True)
 
 
+BB_CTX = (4096, 16384, 32768, 65536, 131072)
+BB_RHO = (0.0, 0.125, 0.5, 1.0)
+
+
+def run_backbone(args, local_rank):
+    """Whole-model decode steps of the synthetic Qwen3-1.7B-shaped model (batch 1): every layer's
+    projections and attention, the recall head, the conditional full pass, the commit and the LM
+    head - the scope of the method notes' throughput measurement (§3.3) - at each context and
+    recall rate, beside the always-full model (full attention everywhere, no head).  Per point:
+    the first step including graph capture and the warm median; one JSON line per point, then a
+    summary with the speed-up over always-full at each context."""
+    import torch
+    from conditional_sparse_attention_b200 import oda
+    from conditional_sparse_attention_b200.engine import OdaDecoder, fill_step_inputs
+    from workload import configs
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    W, K = args.warmup, args.steps
+    hbm, peak_src = peaks()
+    ctxs = BB_CTX if args.backbone_ctx is None else tuple(int(c) for c in args.backbone_ctx.split(","))
+    out = []
+    for ctx in ctxs:
+        wl0 = configs.bb_qwen3_1p7b(ctx=ctx)
+        per = W + K
+        total = per * (len(BB_RHO) + 2) + 8
+        wl = wl0.replace(steps=total)
+        dec = OdaDecoder(wl, device=dev, capacity_steps=total)
+        weight_bytes = dec.backbone_bytes()
+        lm_bytes = wl.vocab * wl.D * 2
+        head_bytes = __import__("workload.inputs", fromlist=["x"]).head_param_count(wl.D) * 4
+        per_tok = wl.Hkv * KV_BYTES_PER_TOKEN_HEAD["bf16"]
+        t0 = time.perf_counter()
+        dec.capture()
+        dec.step(dec.make_step_buffer(0))
+        dec.synchronize()
+        first_ms = (time.perf_counter() - t0) * 1e3
+        step = 1
+        res = {"ctx": ctx, "first_step_ms_incl_capture": first_ms}
+        for rho in BB_RHO:
+            wr = wl.replace(rates=(rho,) * wl.B)
+            bufs = []
+            for i in range(per):
+                buf = torch.zeros(dec.layout.nbytes, dtype=torch.uint8, device=dev)
+                fill_step_inputs(wr, step + i, dec.layout.views(buf))
+                bufs.append(buf)
+            for i in range(W):
+                dec.step(bufs[i])
+            flags = torch.zeros((K, wl.B), dtype=torch.int32, device=dev)
+            dec.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(dec.stream):
+                e0.record(dec.stream)
+                for i in range(K):
+                    dec.step(bufs[W + i])
+                    flags[i].copy_(dec.flag, non_blocking=True)
+                e1.record(dec.stream)
+            e1.synchronize()
+            step += per
+            ms = e0.elapsed_time(e1) / K
+            f = flags.float().mean().item()
+            t = ctx + step
+            bytes_step = (weight_bytes * (1 + f) + lm_bytes + head_bytes +
+                          wl.L * min(t, wl.sinks + wl.window) * per_tok + f * wl.L * t * per_tok)
+            res[f"rho_{rho}"] = {"ms_per_step": ms, "tokens_per_s": wl.B * 1e3 / ms,
+                                 "realized_rho": f, "gb_per_step": bytes_step / 1e9,
+                                 "achieved_gbs": bytes_step / (ms * 1e-3) / 1e9}
+        # always-full model: its own graph
+        s_ = dec.stream
+        torch.cuda.synchronize(dev)
+        oda.oda_graph_begin(s_)
+        dec.issue_always_full()
+        g = oda.oda_graph_end(s_)
+        for _ in range(W):
+            g.launch(s_)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s_)
+        for _ in range(K):
+            g.launch(s_)
+        e1.record(s_)
+        e1.synchronize()
+        g.close()
+        ms_full = e0.elapsed_time(e1) / K
+        t = ctx + step + W + K
+        full_bytes = weight_bytes + lm_bytes + wl.L * t * per_tok
+        res["always_full"] = {"ms_per_step": ms_full, "tokens_per_s": wl.B * 1e3 / ms_full,
+                              "gb_per_step": full_bytes / 1e9,
+                              "achieved_gbs": full_bytes / (ms_full * 1e-3) / 1e9}
+        res["speedup_at_rho_0.125"] = ms_full / res["rho_0.125"]["ms_per_step"]
+        res["device_error"] = dec.device_error()
+        res["backbone_weight_gb"] = weight_bytes / 1e9
+        print(json.dumps({"backbone_sweep": True, "workload": wl0.name, **res}), flush=True)
+        out.append(res)
+        dec.close()
+        del dec
+        torch.cuda.empty_cache()
+    print(json.dumps({"backbone_summary": True, "model": "synthetic Qwen3-1.7B-shaped, batch 1",
+                      "peak_gbs": hbm, "peak_source": peak_src,
+                      "speedup_over_always_full_at_rho_0.125": {str(r["ctx"]): r["speedup_at_rho_0.125"] for r in out},
+                      "tokens_per_s_at_rho_0.125": {str(r["ctx"]): r["rho_0.125"]["tokens_per_s"] for r in out},
+                      "always_full_tokens_per_s": {str(r["ctx"]): r["always_full"]["tokens_per_s"] for r in out}}),
+          flush=True)
+
+
 def run_ours(args, wl, rank, world, local_rank):
     import torch
     from conditional_sparse_attention_b200 import oda
@@ -728,6 +831,11 @@ def main():
     ap.add_argument("--kernel-reps", type=int, default=3)
     ap.add_argument("--sweep", action="store_true",
                     help="recall-rate x context sweep of the step against always-full attention")
+    ap.add_argument("--backbone", action="store_true",
+                    help="whole-model steps of the synthetic Qwen3-1.7B-shaped model (projections, "
+                         "attention, head, retry, commit, LM head) at 4K..128K against always-full")
+    ap.add_argument("--backbone-ctx", default=None,
+                    help="comma-separated contexts for --backbone (default 4K,16K,32K,64K,128K)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -744,6 +852,9 @@ def main():
         return
     if args.sweep:
         run_sweep(args, wl, local_rank)
+        return
+    if args.backbone:
+        run_backbone(args, local_rank)
         return
     import torch
     if world > 1:

@@ -39,6 +39,12 @@ class OdaKV8Layer(ctypes.Structure):
     _fields_ = [("kv", c_void_p), ("n_pages", c_int64)]
 
 
+class OdaBBLayer(ctypes.Structure):
+    _fields_ = [("attn_norm", c_void_p), ("w_qkv", c_void_p), ("w_o", c_void_p),
+                ("mlp_norm", c_void_p), ("w_gate", c_void_p), ("w_up", c_void_p),
+                ("w_down", c_void_p), ("ffn", c_int32)]
+
+
 class OdaHeadWeights(ctypes.Structure):
     _fields_ = [("tower_norm", c_void_p * 3), ("tower_w", c_void_p * 3), ("tower_b", c_void_p * 3),
                 ("fuse_w", c_void_p), ("fuse_b", c_void_p), ("ffn_norm", c_void_p * 2),
@@ -74,6 +80,15 @@ _SIGS = {
     "oda_commit_fp8": ([c_void_p, _P(OdaKV8Layer), c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
                         c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p],
                        c_int32),
+    "oda_bb_begin": ([c_void_p, c_void_p, c_void_p, c_void_p], c_int32),
+    "oda_bb_qkv": ([c_void_p, _P(OdaBBLayer), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p],
+                   c_int32),
+    "oda_bb_attn_out": ([c_void_p, _P(OdaBBLayer), c_void_p, c_void_p, c_void_p], c_int32),
+    "oda_bb_mlp": ([c_void_p, _P(OdaBBLayer), c_void_p, c_void_p, c_void_p], c_int32),
+    "oda_bb_final_norm": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p], c_int32),
+    "oda_bb_lm_head": ([c_void_p, c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
+                        c_void_p], c_int32),
+    "oda_bb_embed": ([c_void_p, c_void_p, c_int32, c_void_p, c_void_p, c_void_p], c_int32),
     "oda_index_positions": ([c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_int32, c_void_p,
                              c_void_p], c_int32),
     "oda_recall_score": ([c_void_p, _P(OdaHeadWeights), c_void_p, c_void_p, c_void_p, c_void_p,

@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "lib", "liboda.so")
-SOURCES = ["api.cu", "attention.cu", "head.cu", "head_grad.cu", "commit.cu", "glue.cu"]
+SOURCES = ["api.cu", "attention.cu", "head.cu", "head_grad.cu", "commit.cu", "glue.cu", "backbone.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-DNDEBUG",
          "-I" + INCLUDE, "-I" + CSRC]

@@ -176,7 +176,7 @@ oda_status oda_create(const oda_config* cfg, oda_ctx** out) {
   if (st == ODA_OK) st = dev_alloc(&x->attn_cnt, (size_t)2 * B * Hkv, "cudaMalloc(counters)");
   if (st == ODA_OK) st = dev_alloc(&x->err, 1, "cudaMalloc(error word)");
   if (st == ODA_OK) st = dev_alloc(&x->head_part, oda::head_part_floats((int)B, (int)D), "cudaMalloc(head)");
-  if (st == ODA_OK) st = dev_alloc(&x->head_ss, (size_t)96 * (D / 512) * B, "cudaMalloc(head)");
+  if (st == ODA_OK) st = dev_alloc(&x->head_ss, oda::head_ss_floats((int)B, (int)D), "cudaMalloc(head)");
   if (st == ODA_OK) st = dev_alloc(&x->head_cnt, (size_t)oda::head_counter_count((int)D), "cudaMalloc(head)");
   if (st == ODA_OK) st = dev_alloc(&x->head_u, (size_t)3 * B * 1024, "cudaMalloc(head)");
   if (st == ODA_OK) st = dev_alloc(&x->head_f, (size_t)3 * B * 1024, "cudaMalloc(head)");
@@ -349,6 +349,47 @@ oda_status oda_glue_gdn(oda_ctx* ctx, const oda_state* st, int32_t layer, const 
   if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "glue_gdn: ctx is NULL");
   ctx->prev_attention = false;
   return oda::launch_glue_gdn(ctx, st, layer, c, v, alpha, beta, taps, flag, o, stream);
+}
+
+oda_status oda_bb_begin(oda_ctx* ctx, const float* emb, float* x, cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "bb_begin: ctx is NULL");
+  return oda::launch_bb_begin(ctx, emb, x, stream);
+}
+
+oda_status oda_bb_qkv(oda_ctx* ctx, const oda_bb_layer* layer, const float* x, void* q,
+                      void* k_new, void* v_new, cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "bb_qkv: ctx is NULL");
+  return oda::launch_bb_qkv(ctx, layer, x, q, k_new, v_new, stream);
+}
+
+oda_status oda_bb_attn_out(oda_ctx* ctx, const oda_bb_layer* layer, const float* o, float* x,
+                           cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "bb_attn_out: ctx is NULL");
+  return oda::launch_bb_attn_out(ctx, layer, o, x, stream);
+}
+
+oda_status oda_bb_mlp(oda_ctx* ctx, const oda_bb_layer* layer, float* x, void* act,
+                      cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "bb_mlp: ctx is NULL");
+  return oda::launch_bb_mlp(ctx, layer, x, act, stream);
+}
+
+oda_status oda_bb_final_norm(oda_ctx* ctx, const float* gamma, const float* x, float* h,
+                             cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "bb_final_norm: ctx is NULL");
+  return oda::launch_bb_final_norm(ctx, gamma, x, h, stream);
+}
+
+oda_status oda_bb_lm_head(oda_ctx* ctx, const void* embed, int32_t vocab, const float* h,
+                          float* logits, int32_t* token, float* next_emb, cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "bb_lm_head: ctx is NULL");
+  return oda::launch_bb_lm_head(ctx, embed, vocab, h, logits, token, next_emb, stream);
+}
+
+oda_status oda_bb_embed(oda_ctx* ctx, const void* embed, int32_t vocab, int32_t* token,
+                        float* emb, cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "bb_embed: ctx is NULL");
+  return oda::launch_bb_embed(ctx, embed, vocab, token, emb, stream);
 }
 
 oda_status oda_cond_begin(oda_ctx* ctx, cudaStream_t stream, const int32_t* any_flag,

@@ -42,10 +42,8 @@ namespace {
 // full set: 4 warps per CTA, two CTAs per SM; local set: 8 warps, one CTA per SM (its
 // launch is latency-bound, so more warps in flight beat the room for a second CTA)
 constexpr int kW = 4;                 // full set: warps per CTA (each streams its own pages)
-constexpr int kR = 3;                 // pages in flight per warp
 constexpr int kThreads = kW * 32;
 constexpr int kWL = 8;                // local set: warps per CTA
-constexpr int kRL = 3;                // local set: pages in flight per warp
 constexpr int kThreadsL = kWL * 32;
 constexpr int kPageTok = 16;
 constexpr int kStageBytes = 8192;     // K (4 KiB) + V (4 KiB) of one (page, KV head)
@@ -714,19 +712,6 @@ __device__ __forceinline__ void cta_merge(const float* merge_o, const float* mer
   }
 }
 
-// q . k_new of head n of the group, in the exp2 domain (whole warp; result in every lane).
-__device__ __forceinline__ float staged_score(const AttnParams& p, int b, int h, int n, int lane) {
-  const uint32_t* qrow = p.q + ((size_t)b * p.Hq + h * p.g + n) * 64;
-  const uint32_t* krow = p.k_new + ((size_t)b * p.Hkv + h) * 64;
-  const uint32_t qa0 = qrow[lane], qa1 = qrow[lane + 32];
-  const uint32_t ka0 = krow[lane], ka1 = krow[lane + 32];
-  const float acc = bf16_lo_to_f32(qa0) * bf16_lo_to_f32(ka0) +
-                    bf16_hi_to_f32(qa0) * bf16_hi_to_f32(ka0) +
-                    bf16_lo_to_f32(qa1) * bf16_lo_to_f32(ka1) +
-                    bf16_hi_to_f32(qa1) * bf16_hi_to_f32(ka1);
-  return warp_sum(acc) * p.scale_log2;
-}
-
 __device__ __forceinline__ float staged_value(const AttnParams& p, int b, int h, int d) {
   const uint32_t vv = p.v_new[((size_t)b * p.Hkv + h) * 64 + (d >> 1)];
   return (d & 1) ? bf16_hi_to_f32(vv) : bf16_lo_to_f32(vv);
@@ -776,8 +761,6 @@ template <> struct Fmt<0> {
 template <> struct Fmt<1> {
   static constexpr int kStage = kF8Block, kR = 6, kRL = 6, kAlign = 128;
 };
-constexpr int kMaxR = 6;
-constexpr int kMaxRL = 6;
 
 // Query fragments of either format.
 template <int F> struct QFrag;

@@ -873,6 +873,12 @@ size_t head_part_floats(int B, int D) {
   return m;
 }
 
+// Per-chunk sums of squares of the tower inputs: (row block, chunk, sequence) of the tower phase.
+size_t head_ss_floats(int B, int D) {
+  const PhaseShape s = phase_shape(kTower, D);
+  return (size_t)s.row_blocks * s.nchunks * B;
+}
+
 int head_counter_count(int D) {
   int m = 0;
   for (int ph = 0; ph < 4; ++ph) m = std::max(m, phase_shape(ph, D).row_blocks);

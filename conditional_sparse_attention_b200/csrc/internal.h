@@ -6,6 +6,7 @@
 
 #include "oda.h"
 #include "oda_glue.h"
+#include "oda_backbone.h"
 
 struct oda_ctx {
   oda_config cfg;
@@ -78,6 +79,7 @@ oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const flo
                               const float* emb, const float* h_loc, const int32_t* sched,
                               float* score, int32_t* flag, int32_t* any_flag, cudaStream_t s);
 size_t head_part_floats(int B, int D);
+size_t head_ss_floats(int B, int D);
 int head_counter_count(int D);
 
 // head_grad.cu
@@ -106,6 +108,18 @@ oda_status launch_glue_gdn(oda_ctx* ctx, const oda_state* st, int layer, const f
                            const float* v, const float* alpha, const float* beta,
                            const float* taps, const int32_t* flag, float* o, cudaStream_t s);
 int glue_chunks(int D);
+
+// backbone.cu
+oda_status launch_bb_qkv(oda_ctx* ctx, const oda_bb_layer* w, const float* x, void* q, void* k_new,
+                         void* v_new, cudaStream_t s);
+oda_status launch_bb_attn_out(oda_ctx* ctx, const oda_bb_layer* w, const float* o, float* x, cudaStream_t s);
+oda_status launch_bb_mlp(oda_ctx* ctx, const oda_bb_layer* w, float* x, void* act, cudaStream_t s);
+oda_status launch_bb_begin(oda_ctx* ctx, const float* emb, float* x, cudaStream_t s);
+oda_status launch_bb_final_norm(oda_ctx* ctx, const float* gamma, const float* x, float* h, cudaStream_t s);
+oda_status launch_bb_lm_head(oda_ctx* ctx, const void* embed, int32_t vocab, const float* h,
+                             float* logits, int32_t* token, float* next_emb, cudaStream_t s);
+oda_status launch_bb_embed(oda_ctx* ctx, const void* embed, int32_t vocab, const int32_t* token,
+                           float* emb, cudaStream_t s);
 
 // cond.cu
 oda_status launch_set_condition(cudaGraphConditionalHandle h, const int32_t* any_flag,

@@ -36,9 +36,14 @@ class StepLayout:
     def __init__(self, wl: Workload):
         B, L, Hq, Hkv, D = wl.B, wl.L, wl.Hq, wl.Hkv, wl.D
         G = len(wl.gdn_layers)
-        ent = [("q", (2, L, B, Hq, 128), torch.bfloat16), ("k", (2, L, B, Hkv, 128), torch.bfloat16),
-               ("v", (2, L, B, Hkv, 128), torch.bfloat16), ("emb", (B, D), torch.float32),
-               ("sched", (B,), torch.int32)]
+        if wl.backbone:
+            # q/k/v come from the backbone's projections and E(x_t) from the previous step's LM
+            # head: a step's only host input is the schedule
+            ent = [("sched", (B,), torch.int32)]
+        else:
+            ent = [("q", (2, L, B, Hq, 128), torch.bfloat16), ("k", (2, L, B, Hkv, 128), torch.bfloat16),
+                   ("v", (2, L, B, Hkv, 128), torch.bfloat16), ("emb", (B, D), torch.float32),
+                   ("sched", (B,), torch.int32)]
         if G:
             ent += [("gc", (2, G, B, configs.CONV_WIDTH), torch.float32),
                     ("gv", (2, G, B, configs.GDN_HEADS, configs.GDN_DIM), torch.float32),
@@ -62,6 +67,10 @@ class StepLayout:
 def fill_step_inputs(wl: Workload, step: int, views: dict) -> None:
     """Writes step ``step``'s seeded inputs into device views (bit-identical to the host
     generator: q/k/v by the device generator, fp32 inputs generated on the host)."""
+    sched = inputs.schedule(wl, step)
+    views["sched"].copy_(torch.from_numpy(sched if sched is not None else np.zeros(wl.B, np.int32)))
+    if wl.backbone:
+        return
     for br in (LOCAL, FULL):
         for a, layer in enumerate(wl.attn_layers):
             kq, kk, kv = inputs.qkv_keys(wl, step, layer, br)
@@ -69,8 +78,6 @@ def fill_step_inputs(wl: Workload, step: int, views: dict) -> None:
             wdev.fill_normal_bf16(views["k"][br, a], kk)
             wdev.fill_normal_bf16(views["v"][br, a], kv)
     views["emb"].copy_(torch.from_numpy(inputs.emb(wl, step)))
-    sched = inputs.schedule(wl, step)
-    views["sched"].copy_(torch.from_numpy(sched if sched is not None else np.zeros(wl.B, np.int32)))
     for br in (LOCAL, FULL):
         for j, layer in enumerate(wl.gdn_layers):
             c, v, a, b = inputs.gdn_step_inputs(wl, step, layer, br)
@@ -173,8 +180,49 @@ class OdaDecoder:
             self.snap = oda.state(self.rec_snap, self.conv_snap)
             self.taps = torch.from_numpy(
                 np.stack([inputs.gdn_taps(wl, layer) for layer in wl.gdn_layers])).to(dev)
+        if wl.backbone:
+            self._init_backbone()
         self.graph = None
         torch.cuda.synchronize(dev)
+
+    def _init_backbone(self) -> None:
+        """Seeded random weights of the synthetic backbone (bf16 projections filled on the device,
+        bit-identical to workload.inputs), its buffers, and E(x_1) of the first tokens."""
+        wl, dev = self.wl, self.device
+        B, D, F, V, L = wl.B, wl.D, wl.ffn, wl.vocab, wl.L
+        shapes = inputs.bb_shapes(wl)
+        self.bb_w, self.bb_layers = [], []
+        for a, layer in enumerate(wl.attn_layers):
+            ws = {}
+            for name in inputs.BB_TENSORS:
+                R, C = shapes[name]
+                t = torch.empty((R, C), dtype=torch.bfloat16, device=dev)
+                wdev.fill_normal_bf16(t, inputs.bb_weight_key(wl, layer, name), 0, inputs.bb_log2_scale(C))
+                ws[name] = t
+            ga, gm = inputs.bb_norms(wl, layer)
+            ws["attn_norm"] = torch.from_numpy(ga).to(dev)
+            ws["mlp_norm"] = torch.from_numpy(gm).to(dev)
+            self.bb_w.append(ws)
+            self.bb_layers.append(oda.bb_layer(ws["attn_norm"], ws["w_qkv"], ws["w_o"], ws["mlp_norm"],
+                                               ws["w_gate"], ws["w_up"], ws["w_down"]))
+        self.bb_final_norm = torch.from_numpy(inputs.bb_norms(wl, -1)[0]).to(dev)
+        self.bb_embed = torch.empty((V, D), dtype=torch.bfloat16, device=dev)
+        wdev.fill_normal_bf16(self.bb_embed, inputs.bb_embed_key(wl), 0, inputs.BB_EMBED_LOG2_SCALE)
+        self.bb_x = torch.zeros((2, B, D), dtype=torch.float32, device=dev)
+        self.bb_act = torch.zeros((B, F), dtype=torch.bfloat16, device=dev)
+        self.bb_logits = torch.zeros((B, V), dtype=torch.float32, device=dev)
+        self.bb_q = torch.zeros((2, L, B, wl.Hq, 128), dtype=torch.bfloat16, device=dev)
+        self.bb_k = torch.zeros((2, L, B, wl.Hkv, 128), dtype=torch.bfloat16, device=dev)
+        self.bb_v = torch.zeros_like(self.bb_k)
+        self.token = torch.from_numpy(inputs.bb_token0(wl)).to(dev)
+        self.emb = torch.zeros((B, D), dtype=torch.float32, device=dev)
+        oda.oda_bb_embed(self.ctx, self.bb_embed, V, self.token, self.emb, self.stream)
+        self.stream.synchronize()
+
+    def backbone_bytes(self) -> int:
+        """Weight bytes one backbone pass streams (projections of every layer)."""
+        return sum(t.numel() * t.element_size() for ws in self.bb_w
+                   for n, t in ws.items() if n.startswith("w_"))
 
     # ---------------------------------------------------------------- inputs
     def make_step_buffer(self, step: int) -> torch.Tensor:
@@ -209,8 +257,63 @@ class OdaDecoder:
         self.stream.wait_event(self.staged[i])
 
     # ------------------------------------------------------------------ step
+    def _bb_pass(self, br: int, stream, flag=None) -> None:
+        """One backbone pass of branch br: the residual starts from E(x_t); every layer projects
+        q/k/v from it, attends (S^L or, for flagged sequences, S^F), adds o_proj and the MLP;
+        then the final norm gives h^br."""
+        wl, ctx = self.wl, self.ctx
+        x = self.bb_x[br]
+        oda.oda_bb_begin(ctx, self.emb, x, stream)
+        for a, layer in enumerate(wl.attn_layers):
+            q, k, v = self.bb_q[br, a], self.bb_k[br, a], self.bb_v[br, a]
+            oda.oda_bb_qkv(ctx, self.bb_layers[a], x, q, k, v, stream)
+            if br == LOCAL:
+                self._attend_local(ctx, self.layers[a], self.page_table, self.pos, q, k, v,
+                                   self.o[br, layer], stream)
+            else:
+                self._attend_full(ctx, self.layers[a], self.page_table, self.pos, flag, q, k, v,
+                                  self.o[br, layer], stream)
+            oda.oda_bb_attn_out(ctx, self.bb_layers[a], self.o[br, layer], x, stream)
+            oda.oda_bb_mlp(ctx, self.bb_layers[a], x, self.bb_act, stream)
+        oda.oda_bb_final_norm(ctx, self.bb_final_norm, x, self.h[br], stream)
+
+    def _issue_backbone(self) -> None:
+        """One decode step of the whole synthetic model: local pass, recall head, conditional full
+        pass, commit, then the LM head on the committed hidden state (its greedy token's embedding
+        is E(x_{t+1}) of the next step)."""
+        wl, s, sv, ctx = self.wl, self.stream, self.sv, self.ctx
+        self._bb_pass(LOCAL, s)
+        oda.oda_recall_score(ctx, self.head_w, self.h_prev, self.emb, self.h[LOCAL],
+                             sv["sched"] if self.routing_scheduled else None, self.score,
+                             self.flag, self.any_flag, s)
+        body = oda.oda_cond_begin(ctx, s, self.any_flag)
+        self._bb_pass(FULL, body, self.flag)
+        oda.oda_cond_end(ctx, s)
+        self._commit(ctx, self.layers, self.page_table, self.pos, self.flag, self.bb_k[LOCAL],
+                     self.bb_v[LOCAL], self.bb_k[FULL], self.bb_v[FULL], self.h[LOCAL], self.h[FULL],
+                     self.h_prev, s)
+        oda.oda_bb_lm_head(ctx, self.bb_embed, wl.vocab, self.h_prev, self.bb_logits, self.token,
+                           self.emb, s)
+
+    def issue_always_full(self) -> None:
+        """The reference decoder the method is measured against: every step one backbone pass with
+        full attention in every layer for every sequence, no local pass and no recall head, then
+        the commit of that pass and the LM head (synthetic-backbone workloads only)."""
+        wl, s, ctx = self.wl, self.stream, self.ctx
+        if not hasattr(self, "ones"):
+            self.ones = torch.ones(wl.B, dtype=torch.int32, device=self.device)
+        self._bb_pass(FULL, s, self.ones)
+        self._commit(ctx, self.layers, self.page_table, self.pos, self.ones, self.bb_k[FULL],
+                     self.bb_v[FULL], self.bb_k[FULL], self.bb_v[FULL], self.h[FULL], self.h[FULL],
+                     self.h_prev, s)
+        oda.oda_bb_lm_head(ctx, self.bb_embed, wl.vocab, self.h_prev, self.bb_logits, self.token,
+                           self.emb, s)
+
     def issue(self) -> None:
         """Enqueues one decode step on self.stream (eagerly or into a capture)."""
+        if self.wl.backbone:
+            self._issue_backbone()
+            return
         wl, s, sv = self.wl, self.stream, self.sv
         ctx = self.ctx
         n_layers = wl.n_layers

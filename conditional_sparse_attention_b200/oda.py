@@ -12,8 +12,8 @@ from typing import Optional, Sequence
 import torch
 
 from . import _lib
-from ._lib import (OdaConfig, OdaError, OdaHeadGrads, OdaHeadWeights, OdaKV8Layer,  # noqa: F401
-                   OdaKVLayer, OdaState, check)
+from ._lib import (OdaBBLayer, OdaConfig, OdaError, OdaHeadGrads, OdaHeadWeights,  # noqa: F401
+                   OdaKV8Layer, OdaKVLayer, OdaState, check)
 
 _c = ctypes.c_void_p
 
@@ -282,3 +282,41 @@ def oda_glue_hidden(ctx, emb, terms, n_terms: int, flag, h, stream=None):
 def oda_glue_gdn(ctx, st: OdaState, layer: int, c, v, alpha, beta, taps, flag, o, stream=None):
     check(_lib.load().oda_glue_gdn(ctx.handle, ctypes.byref(st), layer, _p(c), _p(v), _p(alpha),
                                    _p(beta), _p(taps), _p(flag), _p(o), _s(stream)))
+
+
+# ------------------------------------------------------------------ synthetic backbone
+def bb_layer(attn_norm, w_qkv, w_o, mlp_norm, w_gate, w_up, w_down) -> OdaBBLayer:
+    """Layer descriptor from device tensors (norm weights fp32 [D]; projections bf16 or int16
+    [out, in]); F is taken from w_gate."""
+    return OdaBBLayer(attn_norm.data_ptr(), w_qkv.data_ptr(), w_o.data_ptr(), mlp_norm.data_ptr(),
+                      w_gate.data_ptr(), w_up.data_ptr(), w_down.data_ptr(), int(w_gate.shape[0]))
+
+
+def oda_bb_begin(ctx, emb, x, stream=None):
+    check(_lib.load().oda_bb_begin(ctx.handle, _p(emb), _p(x), _s(stream)))
+
+
+def oda_bb_qkv(ctx, layer: OdaBBLayer, x, q, k_new, v_new, stream=None):
+    check(_lib.load().oda_bb_qkv(ctx.handle, ctypes.byref(layer), _p(x), _p(q), _p(k_new), _p(v_new),
+                                 _s(stream)))
+
+
+def oda_bb_attn_out(ctx, layer: OdaBBLayer, o, x, stream=None):
+    check(_lib.load().oda_bb_attn_out(ctx.handle, ctypes.byref(layer), _p(o), _p(x), _s(stream)))
+
+
+def oda_bb_mlp(ctx, layer: OdaBBLayer, x, act, stream=None):
+    check(_lib.load().oda_bb_mlp(ctx.handle, ctypes.byref(layer), _p(x), _p(act), _s(stream)))
+
+
+def oda_bb_final_norm(ctx, gamma, x, h, stream=None):
+    check(_lib.load().oda_bb_final_norm(ctx.handle, _p(gamma), _p(x), _p(h), _s(stream)))
+
+
+def oda_bb_lm_head(ctx, embed, vocab: int, h, logits, token, next_emb, stream=None):
+    check(_lib.load().oda_bb_lm_head(ctx.handle, _p(embed), vocab, _p(h), _p(logits), _p(token),
+                                     _p(next_emb), _s(stream)))
+
+
+def oda_bb_embed(ctx, embed, vocab: int, token, emb, stream=None):
+    check(_lib.load().oda_bb_embed(ctx.handle, _p(embed), vocab, _p(token), _p(emb), _s(stream)))

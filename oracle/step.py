@@ -28,6 +28,9 @@ import numpy as np
 from workload import inputs as wi
 from workload.configs import Workload
 
+import functools
+
+from . import backbone as BB
 from . import kv_fp8
 from .attention import append_current, attend, attend_bits, bf16_to_f64
 from .delta import gdn_layer
@@ -48,6 +51,8 @@ class OracleState:
     gdn_conv: np.ndarray = None    # [B, n_gdn, 4, 2048] fp64
     kv: str = "bf16"               # "bf16": caches hold bf16 bits; "fp8": caches hold the
                                    # decoded values (fp64) of rows stored as e4m3 + scale
+    tokens: np.ndarray = None      # synthetic backbone: the current token x_t of each sequence
+    emb: np.ndarray = None         # synthetic backbone: E(x_t) [B, D] fp64
 
 
 @dataclass
@@ -58,6 +63,9 @@ class StepRecord:
     h: dict = field(default_factory=dict)      # branch -> [B, D]
     staged_k: dict = field(default_factory=dict)   # (branch, ordinal) -> uint16 [B, Hkv, 128]
     staged_v: dict = field(default_factory=dict)
+    staged_q: dict = field(default_factory=dict)   # synthetic backbone: (branch, ordinal) -> q bits
+    logits: np.ndarray = None      # synthetic backbone: LM head on the committed hidden
+    tokens: np.ndarray = None      # synthetic backbone: x_{t+1} (greedy)
 
 
 def _stored(bits: np.ndarray, kv: str) -> np.ndarray:
@@ -78,6 +86,9 @@ def initial_state(wl: Workload, kv: str = "bf16") -> OracleState:
         vc.append([_stored(wi.cache_tokens(wl, "v", a, b, wl.ctx[b]), kv) for b in range(wl.B)])
     st = OracleState(pos=[c + 1 for c in wl.ctx], h_prev=wi.h_prev0(wl).astype(np.float64),
                      k_cache=kc, v_cache=vc, kv=kv)
+    if wl.backbone:
+        st.tokens = wi.bb_token0(wl)
+        st.emb = bf16_to_f64(wi.bb_embed_rows(wl, st.tokens))
     if wl.hybrid:
         S, C = wi.gdn_state0(wl)
         st.gdn_S = S.astype(np.float64)
@@ -102,6 +113,50 @@ def restore(snap, state: OracleState, flags) -> None:
             state.gdn_conv[b] = snap[1][b]
 
 
+@functools.lru_cache(maxsize=2)
+def backbone_weights(wl: Workload):
+    """The synthetic backbone's weights (bf16 bits / fp32 norms) per attention layer, the final
+    norm weight and the embedding table, from the seeded generators."""
+    layers = []
+    for layer in wl.attn_layers:
+        w = {name: wi.bb_weight(wl, layer, name) for name in wi.BB_TENSORS}
+        w["attn_norm"], w["mlp_norm"] = wi.bb_norms(wl, layer)
+        layers.append(w)
+    return layers, wi.bb_norms(wl, -1)[0], wi.bb_embed(wl)
+
+
+def run_backbone_pass(wl: Workload, state: OracleState, branch: int, active, rec: StepRecord):
+    """One pass of the synthetic backbone (oracle.backbone) from the pre-step residual E(x_t):
+    per layer q/k/v from the residual, attention over S^L or S^F for the sequences in
+    ``active``, o_proj and the MLP; returns h = the final norm of the residual."""
+    layers, g_final, _ = backbone_weights(wl)
+    B, D = wl.B, wl.D
+    x = state.emb.copy()
+    for a, layer in enumerate(wl.attn_layers):
+        w = layers[a]
+        q, k, v = BB.attn_in(x, w["attn_norm"], w["w_qkv"], wl.Hq, wl.Hkv)
+        rec.staged_q[(branch, a)] = q
+        rec.staged_k[(branch, a)] = k
+        rec.staged_v[(branch, a)] = v
+        o = np.full((B, wl.Hq, wl.d), np.nan)
+        for b in active:
+            t = state.pos[b]
+            S = local_set(t, wl.sinks, wl.window) if branch == LOCAL else full_set(t)
+            if state.kv == "bf16":
+                o[b] = attend_bits(q[b], state.k_cache[a][b], state.v_cache[a][b], k[b], v[b], S)
+            else:
+                o[b] = attend(bf16_to_f64(q[b]), append_current(state.k_cache[a][b], bf16_to_f64(k[b])),
+                              append_current(state.v_cache[a][b], bf16_to_f64(v[b])), S)
+        rec.o[(branch, a)] = o
+        x = BB.attn_out(x, o.reshape(B, D), w["w_o"])
+        x = BB.mlp(x, w["mlp_norm"], w["w_gate"], w["w_up"], w["w_down"])
+    h = np.full((B, D), np.nan)
+    for b in active:
+        h[b] = BB.rmsnorm(x[b], g_final)
+    rec.h[branch] = h
+    return h
+
+
 def run_pass(wl: Workload, state: OracleState, step: int, branch: int, active, rec: StepRecord):
     """One forward pass of the synthetic backbone for the sequences in ``active``.
 
@@ -109,6 +164,8 @@ def run_pass(wl: Workload, state: OracleState, step: int, branch: int, active, r
     S^L (local) or S^F (full); recurrent layers advance ``state``'s gdn arrays in place.
     Returns h [B, D] (rows of inactive sequences are NaN).
     """
+    if wl.backbone:
+        return run_backbone_pass(wl, state, branch, active, rec)
     B, D = wl.B, wl.D
     e = wi.emb(wl, step).astype(np.float64)
     x = e.copy()
@@ -159,7 +216,7 @@ def decode_step(wl: Workload, state: OracleState, step: int, head_params: dict,
     snap = snapshot(live)
     rec = StepRecord(scores=np.zeros(B), flags=np.zeros(B, dtype=np.int32))
     h_loc = run_pass(wl, live, step, LOCAL, range(B), rec)
-    e = wi.emb(wl, step).astype(np.float64)
+    e = live.emb if wl.backbone else wi.emb(wl, step).astype(np.float64)
     for b in range(B):
         rec.scores[b] = recall_head(head_params, live.h_prev[b], e[b], h_loc[b])
         full = route_full(rec.scores[b], wl.theta) if sched is None else bool(sched[b])
@@ -168,6 +225,12 @@ def decode_step(wl: Workload, state: OracleState, step: int, head_params: dict,
     restore(snap, live, rec.flags)
     run_pass(wl, live, step, FULL, flagged, rec)
     commit(wl, live, rec)
+    if wl.backbone:
+        # [notes §2.3, eq. p_t]: the output distribution once, from the committed hidden h_t
+        _, _, E = backbone_weights(wl)
+        rec.logits, rec.tokens = BB.lm_head(live.h_prev, E)
+        live.tokens = rec.tokens
+        live.emb = bf16_to_f64(E[rec.tokens])
     return live, rec
 
 

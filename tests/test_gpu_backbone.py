@@ -1,0 +1,225 @@
+"""GPU parity of the synthetic-backbone calls (include/oda_backbone.h) and of whole decode
+steps of the synthetic model against the oracle (oracle.backbone, oracle.step).
+
+The stand-in's definition rounds projection inputs, q/k/v and the MLP activation to bf16; the GPU
+takes those roundings from fp32 values and the oracle from fp64 ones, so a value within an fp32
+rounding error of a bf16 midpoint can land one bf16 step apart.  bf16 outputs are therefore
+compared as: equal except for at most 0.5% of the elements, and those within one bf16 step; fp32
+outputs within relative L2 1e-4 (projections) or the attention tolerance (attention outputs).
+Greedy tokens are compared where the oracle's two largest logits differ by more than 1e-3.
+Along a trajectory the two residual streams (fp32 here, fp64 in the oracle) drift apart by the
+roundings of every layer.  So the kernels are checked teacher-forced - every attention output
+against the oracle on the GPU's own q/k/v and committed cache, the recall score on the GPU's own
+inputs - and the independent oracle trajectory within a drift bound; the cache must hold exactly
+the GPU's own committed rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+from helpers import TIE_BAND, attn_close, build_all, logical_cache, score_close
+from oracle import backbone as BB
+from oracle import step as OS
+from oracle.attention import bf16_to_f64
+from oracle.head import recall_head
+from workload import configs, device as wdev, gen, inputs
+
+pytestmark = pytest.mark.gpu
+TOKEN_TIE = 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _build():
+    build_all()
+
+
+def _bits_t(a):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+
+def bf16_close(got_bits, ref_bits, frac=5e-3):
+    g, r = bf16_to_f64(got_bits), bf16_to_f64(ref_bits)
+    diff = g != r
+    step = np.abs(r) * 2.0 ** -7 + 1e-30
+    return diff.mean() <= frac and np.all(np.abs(g - r)[diff] <= step[diff] * 1.01)
+
+
+def rel_l2(a, b):
+    return float(np.linalg.norm(np.asarray(a) - np.asarray(b)) / max(np.linalg.norm(b), 1e-30))
+
+
+def _wl(B=3, Hq=4, Hkv=2, F=1024, V=2000, seed=300):
+    return configs.bb_qwen3_1p7b().replace(name=f"t_bb_{B}_{Hq}_{F}", seed=seed, B=B, n_layers=1,
+                                           attn_layers=(0,), Hq=Hq, Hkv=Hkv, ctx=(10,) * B,
+                                           ffn=F, vocab=V, rates=(0.5,) * B)
+
+
+class Layer:
+    def __init__(self, wl):
+        from conditional_sparse_attention_b200 import oda
+        self.oda = oda
+        self.wl = wl
+        self.w = {n: inputs.bb_weight(wl, 0, n) for n in inputs.BB_TENSORS}
+        self.ga, self.gm = inputs.bb_norms(wl, 0)
+        d = {n: _bits_t(v) for n, v in self.w.items()}
+        self.d = d
+        self.tga, self.tgm = torch.from_numpy(self.ga).cuda(), torch.from_numpy(self.gm).cuda()
+        self.layer = oda.bb_layer(self.tga, d["w_qkv"], d["w_o"], self.tgm, d["w_gate"], d["w_up"],
+                                  d["w_down"])
+        self.ctx = oda.oda_create(oda.make_config(wl.B, wl.Hq, wl.Hkv, 8, max(512, wl.D)))
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,F", [(1, 4, 2, 1024), (3, 4, 2, 1536), (8, 8, 2, 512),
+                                        (1, 16, 8, 6144)])
+def test_projections_match_oracle(B, Hq, Hkv, F):
+    wl = _wl(B, Hq, Hkv, F)
+    L = Layer(wl)
+    oda, D = L.oda, wl.D
+    rng = np.random.default_rng(B + F)
+    x = rng.normal(0, 2, (B, D)).astype(np.float32)
+    o = rng.normal(0, 1, (B, D)).astype(np.float32)
+    tx = torch.from_numpy(x).cuda()
+    q = torch.zeros((B, Hq, 128), dtype=torch.int16, device="cuda")
+    k = torch.zeros((B, Hkv, 128), dtype=torch.int16, device="cuda")
+    v = torch.zeros_like(k)
+    oda.oda_bb_qkv(L.ctx, L.layer, tx, q, k, v)
+    x1 = tx.clone()
+    oda.oda_bb_attn_out(L.ctx, L.layer, torch.from_numpy(o).cuda(), x1)
+    x2 = tx.clone()
+    act = torch.zeros((B, F), dtype=torch.bfloat16, device="cuda")
+    oda.oda_bb_mlp(L.ctx, L.layer, x2, act)
+    h = torch.zeros_like(tx)
+    oda.oda_bb_final_norm(L.ctx, L.tgm, tx, h)
+    torch.cuda.synchronize()
+    assert oda.oda_get_error(L.ctx) == 0
+    rq, rk, rv = BB.attn_in(x.astype(np.float64), L.ga, L.w["w_qkv"], Hq, Hkv)
+    u16 = lambda t: t.cpu().numpy().view(np.uint16)  # noqa: E731
+    assert bf16_close(u16(q), rq) and bf16_close(u16(k), rk) and bf16_close(u16(v), rv)
+    assert rel_l2(x1.cpu().numpy(), BB.attn_out(x, o, L.w["w_o"])) < 1e-5
+    ref2 = BB.mlp(x.astype(np.float64), L.gm, L.w["w_gate"], L.w["w_up"], L.w["w_down"])
+    assert rel_l2(x2.cpu().numpy() - x, ref2 - x) < 1e-3
+    assert rel_l2(h.cpu().numpy(), BB.rmsnorm(x.astype(np.float64), L.gm)) < 1e-6
+    L.ctx.close()
+
+
+@pytest.mark.parametrize("B,V", [(1, 2000), (5, 4096), (8, 151936)])
+def test_lm_head_matches_oracle(B, V):
+    wl = _wl(B, 16, 8, 512, V, seed=301)
+    from conditional_sparse_attention_b200 import oda
+    D = wl.D
+    ctx = oda.oda_create(oda.make_config(B, wl.Hq, wl.Hkv, 8, D))
+    E = inputs.bb_embed(wl)
+    tE = torch.empty((V, D), dtype=torch.int16, device="cuda")
+    wdev.fill_normal_bf16(tE, inputs.bb_embed_key(wl), 0, inputs.BB_EMBED_LOG2_SCALE)
+    assert np.array_equal(tE.cpu().numpy().view(np.uint16), E)
+    rng = np.random.default_rng(V)
+    h = rng.normal(0, 1, (B, D)).astype(np.float32)
+    logits = torch.zeros((B, V), device="cuda")
+    tok = torch.zeros(B, dtype=torch.int32, device="cuda")
+    emb = torch.zeros((B, D), device="cuda")
+    oda.oda_bb_lm_head(ctx, tE, V, torch.from_numpy(h).cuda(), logits, tok, emb)
+    torch.cuda.synchronize()
+    ref, rtok = BB.lm_head(h.astype(np.float64), E)
+    assert rel_l2(logits.cpu().numpy(), ref) < 1e-5
+    top2 = np.sort(ref, axis=1)[:, -2:]
+    for b in range(B):
+        if top2[b, 1] - top2[b, 0] > TOKEN_TIE:
+            assert tok[b].item() == rtok[b]
+        assert np.array_equal(emb[b].cpu().numpy(), bf16_to_f64(E[tok[b].item()]).astype(np.float32))
+    # embedding lookup alone, with an out-of-range token taken as 0
+    t2 = torch.tensor([3, V + 7, 0, 1, 2, 3, 4, 5][:B], dtype=torch.int32, device="cuda")
+    oda.oda_bb_embed(ctx, tE, V, t2, emb)
+    torch.cuda.synchronize()
+    want = [3, 0, 0, 1, 2, 3, 4, 5][:B]
+    assert t2.cpu().tolist() == want
+    assert np.array_equal(emb.cpu().numpy(), bf16_to_f64(E[want]).astype(np.float32))
+    ctx.close()
+
+
+def _small_model(kv="bf16", seed=2005):
+    return configs.bb_qwen3_1p7b().replace(name=f"t_bb_traj_{kv}", seed=seed, B=2, n_layers=2,
+                                           attn_layers=(0, 1), Hq=4, Hkv=2, ctx=(100, 3000),
+                                           steps=4, rates=(0.5, 0.5), ffn=1024, vocab=2000)
+
+
+# Drift bound of the independent trajectory: every layer re-rounds four bf16 vectors from an fp32
+# stream (the oracle from fp64), each rounding moving ~2^-9 of an element when it flips; over the
+# two layers and four steps here the outputs stay within 1e-2 relative L2.
+DRIFT = 1e-2
+
+
+@pytest.mark.parametrize("kv,graph", [("bf16", True), ("bf16", False), ("fp8", True)])
+def test_backbone_trajectory_matches_oracle(kv, graph):
+    from conditional_sparse_attention_b200.engine import OdaDecoder
+    from oracle.attention import attend_bits
+    from oracle.kv_fp8 import attend_quantized
+    from oracle.sets import full_set, local_set
+    wl = _small_model(kv)
+    dec = OdaDecoder(wl, perturb_head=True, kv_format=kv)
+    P = {k: v.cpu().numpy() for k, v in dec.head_params.items()}
+    if graph:
+        dec.capture()
+    st = OS.initial_state(wl, kv=kv)
+    assert dec.token.cpu().tolist() == st.tokens.tolist()
+    # the GPU's own committed rows per (layer, sequence): the cache the kernels read
+    own_k = [[inputs.cache_tokens(wl, "k", a, b, wl.ctx[b]) for b in range(wl.B)] for a in range(wl.L)]
+    own_v = [[inputs.cache_tokens(wl, "v", a, b, wl.ctx[b]) for b in range(wl.B)] for a in range(wl.L)]
+    u16 = lambda t: t.cpu().view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    for s in range(wl.steps):
+        sched = inputs.schedule(wl, s)
+        # the head is teacher-forced: scored by the oracle on the GPU's own inputs
+        hp = dec.h_prev.cpu().numpy().astype(np.float64)
+        em = dec.emb.cpu().numpy().astype(np.float64)
+        pos = dec.pos.cpu().numpy().copy()
+        dec.step(dec.make_step_buffer(s))
+        dec.synchronize()
+        st, rec = OS.decode_step(wl, st, s, P, sched=sched)
+        flags = dec.flag.cpu().numpy()
+        assert flags.tolist() == rec.flags.tolist(), s
+        sc = dec.score.cpu().numpy()
+        hl = dec.h[0].cpu().numpy().astype(np.float64)
+        for b in range(wl.B):
+            ref = recall_head(P, hp[b], em[b], hl[b])
+            assert score_close(sc[b], ref), (s, b, sc[b], ref)
+        o = dec.o.cpu().numpy()
+        q_all, k_all, v_all = u16(dec.bb_q), u16(dec.bb_k), u16(dec.bb_v)
+        for a in range(wl.L):
+            for br in (0, 1):
+                rows = [b for b in range(wl.B) if br == 0 or flags[b]]
+                for b in rows:
+                    t = int(pos[b])
+                    S = local_set(t, wl.sinks, wl.window) if br == 0 else full_set(t)
+                    # kernel parity: the oracle attends with the GPU's own q/k/v and cache
+                    args = (q_all[br, a, b], own_k[a][b], own_v[a][b], k_all[br, a, b], v_all[br, a, b], S)
+                    ref = attend_bits(*args) if kv == "bf16" else attend_quantized(*args)
+                    ok, ma, rel = attn_close(o[br, a, b], ref.reshape(-1))
+                    assert ok, ("teacher-forced", s, a, br, b, ma, rel)
+                    # drift of the independent trajectory
+                    r = rel_l2(o[br, a, b], rec.o[(br, a)][b].reshape(-1))
+                    assert r < DRIFT, ("drift", s, a, br, b, r)
+                if a == 0 and rows:   # from the exact embedding: equal up to rounding edges
+                    assert bf16_close(k_all[br, a][rows], rec.staged_k[(br, a)][rows]), (s, br, "k")
+        for b in range(wl.B):
+            br = 1 if flags[b] else 0
+            for a in range(wl.L):
+                own_k[a][b] = np.concatenate([own_k[a][b], k_all[br, a, b][None]])
+                own_v[a][b] = np.concatenate([own_v[a][b], v_all[br, a, b][None]])
+            assert rel_l2(hl[b], rec.h[0][b]) < DRIFT, (s, b)
+        top2 = np.sort(rec.logits, axis=1)[:, -2:]
+        tok = dec.token.cpu().numpy()
+        if np.any(top2[:, 1] - top2[:, 0] <= TOKEN_TIE):
+            pytest.skip(f"near-tie of the greedy token at step {s}; trajectories may part")
+        assert tok.tolist() == rec.tokens.tolist(), (s, tok, rec.tokens)
+        assert dec.pos.cpu().tolist() == st.pos
+    assert dec.device_error() == 0
+    # the commit wrote the GPU's own chosen-branch rows into the cache, bit for bit (bf16)
+    if kv == "bf16":
+        pt = dec.page_table.cpu().numpy()
+        for a in range(wl.L):
+            kp = dec.k_pool[a].cpu().view(torch.int16).numpy().view(np.uint16)
+            vp = dec.v_pool[a].cpu().view(torch.int16).numpy().view(np.uint16)
+            for b in range(wl.B):
+                n = wl.ctx[b] + wl.steps
+                assert np.array_equal(logical_cache(kp, pt, b, n), own_k[a][b])
+                assert np.array_equal(logical_cache(vp, pt, b, n), own_v[a][b])
+    dec.close()

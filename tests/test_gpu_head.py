@@ -39,9 +39,10 @@ def _run(B, D, perturb=True, seed=500, sched=None, theta=0.0, bias=0.0, inputs_o
 
 # fused single-launch head for B <= 8 (ring depth from the shared memory the inputs leave:
 # 5 stages at (1, 2048), 4 at (4, 4096), 3 at (8, 2048) and (2, 8192), 2 at (8, 4096)); the six
-# phase launches for B > 8 and where the inputs do not fit (8, 8192)
+# phase launches for B > 8, where the inputs do not fit (8, 8192) and where D is not a multiple of
+# 1024 (512, 1536: the tower phase's per-chunk sums of squares fill their whole scratch at D = 512)
 @pytest.mark.parametrize("B,D", [(1, 2048), (4, 4096), (8, 2048), (2, 8192), (8, 4096), (8, 8192),
-                                 (13, 2048), (32, 2048)])
+                                 (13, 2048), (32, 2048), (2, 512), (8, 512), (3, 1536)])
 def test_scores_and_gate_match_oracle(B, D):
     P, xs, score, flag, anyf = _run(B, D, perturb=True, seed=500 + B + D)
     ref = np.array([recall_head(P, xs[0][b], xs[1][b], xs[2][b]) for b in range(B)])

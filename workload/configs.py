@@ -48,7 +48,15 @@ class Workload:
     sinks: int = SINKS
     window: int = WINDOW
     d: int = HEAD_DIM
+    ffn: int = 0                  # synthetic backbone: gated-MLP width (0: no backbone weights)
+    vocab: int = 0                # synthetic backbone: vocabulary (tied embedding / LM head)
     note: str = ""
+
+    @property
+    def backbone(self) -> bool:
+        """True when every layer runs random-weight projections around attention (QKV from the
+        residual, o_proj, gated MLP) and each step ends with the LM head."""
+        return self.ffn > 0
 
     @property
     def D(self) -> int:
@@ -140,6 +148,17 @@ def cfg4() -> Workload:
                     note="hybrid: 6 attention + 18 gated-delta layers, snapshot/restore, recall 0.4")
 
 
+def bb_qwen3_1p7b(ctx: int = 131072, B: int = 1) -> Workload:
+    """Whole decode step of a Qwen3-1.7B-shaped model with a synthetic frozen backbone: 28
+    layers, hidden 2048 (16 query / 8 KV heads of 128), gated MLP 6144, vocabulary 151936 with
+    tied embeddings, random bf16 weights; batch 1 and about 1/8 scheduled full calls as in the
+    method notes' throughput setup, the head still run."""
+    return Workload(f"bb_qwen3_1p7b_ctx{ctx // 1024}k_b{B}_r0.125", 1005, B=B, n_layers=28,
+                    attn_layers=tuple(range(28)), Hq=16, Hkv=8, ctx=(ctx,) * B, steps=32,
+                    routing="bernoulli", rates=(0.125,) * B, ffn=6144, vocab=151936,
+                    note="synthetic Qwen3-1.7B-shaped backbone, LM head, Bernoulli(0.125) recall")
+
+
 def cfg2_ctx32k_l2() -> Workload:
     """Profiling case of the 128K workload's kernels: same heads and batch, 2 layers, context
     32768 (1 GiB of cache: larger than L2, small enough for a many-pass profiler capture)."""
@@ -148,7 +167,7 @@ def cfg2_ctx32k_l2() -> Workload:
 
 
 ALL = {"cfg0": cfg0, "cfg1": cfg1, "cfg2": cfg2, "cfg3": cfg3, "cfg4": cfg4,
-       "cfg2_ctx32k_l2": cfg2_ctx32k_l2}
+       "cfg2_ctx32k_l2": cfg2_ctx32k_l2, "bb": bb_qwen3_1p7b}
 
 
 def get(name: str) -> Workload:

@@ -52,24 +52,25 @@ def lib():
     return _lib
 
 
-def table(device) -> torch.Tensor:
+def table(device, log2_scale: int = 0) -> torch.Tensor:
     device = torch.device(device)
-    if device not in _tables:
-        t = torch.from_numpy(gen.normal_bf16_table().astype(np.int16)).to(device)
-        _tables[device] = t
-    return _tables[device]
+    if (device, log2_scale) not in _tables:
+        t = torch.from_numpy(gen.normal_bf16_table(log2_scale).view(np.int16)).to(device)
+        _tables[(device, log2_scale)] = t
+    return _tables[(device, log2_scale)]
 
 
 def _stream(device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
-def fill_normal_bf16(out: torch.Tensor, key: int, start: int = 0) -> torch.Tensor:
-    """Fill a contiguous 2-byte tensor (bf16 or int16) with draws start.. of stream ``key``."""
+def fill_normal_bf16(out: torch.Tensor, key: int, start: int = 0, log2_scale: int = 0) -> torch.Tensor:
+    """Fill a contiguous 2-byte tensor (bf16 or int16) with draws start.. of stream ``key``
+    (N(0,1) times 2^log2_scale, as gen.normal_bf16)."""
     assert out.is_cuda and out.is_contiguous() and out.element_size() == 2
     rc = lib().odagen_fill_normal_bf16(ctypes.c_void_p(out.data_ptr()), out.numel(),
                                        ctypes.c_uint64(key & (2**64 - 1)), ctypes.c_uint64(start),
-                                       ctypes.c_void_p(table(out.device).data_ptr()),
+                                       ctypes.c_void_p(table(out.device, log2_scale).data_ptr()),
                                        _stream(out.device))
     if rc != 0:
         raise RuntimeError(f"odagen_fill_normal_bf16 failed: cudaError {rc}")

@@ -51,6 +51,10 @@ class Tag(IntEnum):
     GDN_TAPS = 17
     GDN_STATE0 = 18
     GDN_CONV0 = 19
+    BB_W = 20        # synthetic backbone weights, ids (layer, tensor)
+    BB_NORM = 21     # synthetic backbone norm weights, ids (layer, tensor)
+    BB_EMBED = 22    # token embedding table (tied output projection)
+    TOKEN0 = 23      # first token of each sequence
 
 
 def mix64(z: np.ndarray) -> np.ndarray:
@@ -100,18 +104,20 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
-@functools.lru_cache(maxsize=1)
-def normal_bf16_table() -> np.ndarray:
-    """65536 bf16 bit patterns: N(0,1) quantiles at the midpoints (j + 0.5) / 65536."""
+@functools.lru_cache(maxsize=8)
+def normal_bf16_table(log2_scale: int = 0) -> np.ndarray:
+    """65536 bf16 bit patterns: N(0,1) quantiles at the midpoints (j + 0.5) / 65536, times
+    2^log2_scale (an exact power of two, so the scaled table is the unscaled one with its
+    exponents shifted)."""
     p = (np.arange(65536, dtype=np.float64) + 0.5) / 65536.0
-    t = f32_to_bf16_bits(ndtri(p).astype(np.float32))
+    t = f32_to_bf16_bits((ndtri(p) * 2.0 ** log2_scale).astype(np.float32))
     t.setflags(write=False)
     return t
 
 
-def normal_bf16(k: int, n: int, start: int = 0) -> np.ndarray:
-    """n bf16 N(0,1) draws (uint16 bit patterns) from stream ``k``."""
-    table = normal_bf16_table()
+def normal_bf16(k: int, n: int, start: int = 0, log2_scale: int = 0) -> np.ndarray:
+    """n bf16 N(0, 4^log2_scale) draws (uint16 bit patterns) from stream ``k``."""
+    table = normal_bf16_table(log2_scale)
     out = np.empty(n, dtype=np.uint16)
     for c0 in range(0, n, _CHUNK):
         c1 = min(n, c0 + _CHUNK)

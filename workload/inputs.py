@@ -163,3 +163,70 @@ def gdn_state0(wl: Workload):
 
 def n_pages_for(tokens: int) -> int:
     return (tokens + PAGE - 1) // PAGE
+
+
+# ------------------------------------------------------------ synthetic backbone weights
+BB_TENSORS = ("w_qkv", "w_o", "w_gate", "w_up", "w_down")
+
+
+def bb_shapes(wl: Workload) -> dict:
+    """[rows, cols] of each bf16 projection of one layer (row-major [out][in])."""
+    D, F = wl.D, wl.ffn
+    return {"w_qkv": ((wl.Hq + 2 * wl.Hkv) * wl.d, D), "w_o": (D, wl.Hq * wl.d),
+            "w_gate": (F, D), "w_up": (F, D), "w_down": (D, F)}
+
+
+def bb_log2_scale(fan_in: int) -> int:
+    """Weights are N(0,1) times 2^-floor(log2(fan_in) / 2), about 1/sqrt(fan_in) as an exact
+    power of two, so the device fill and this generator agree bit for bit."""
+    return -(int(np.log2(fan_in)) // 2)
+
+
+def bb_weight_key(wl: Workload, layer: int, name: str) -> int:
+    return gen.key(wl.seed, Tag.BB_W, layer, BB_TENSORS.index(name))
+
+
+def bb_weight(wl: Workload, layer: int, name: str, rows=None) -> np.ndarray:
+    """One projection (bf16 bits [rows, cols]), or rows r0..r1-1 of it if rows = (r0, r1)."""
+    R, C = bb_shapes(wl)[name]
+    r0, r1 = rows if rows is not None else (0, R)
+    v = gen.normal_bf16(bb_weight_key(wl, layer, name), (r1 - r0) * C, r0 * C, bb_log2_scale(C))
+    return v.reshape(r1 - r0, C)
+
+
+def bb_norms(wl: Workload, layer: int) -> tuple:
+    """(attention-input norm weight, MLP-input norm weight), fp32 [D] ~ U(0.5, 1.5); layer -1
+    gives the final norm's weight in both slots."""
+    a = gen.uniform_f32(gen.key(wl.seed, Tag.BB_NORM, layer, 0), wl.D, 0.5, 1.5)
+    m = gen.uniform_f32(gen.key(wl.seed, Tag.BB_NORM, layer, 1), wl.D, 0.5, 1.5)
+    return a, m
+
+
+# The embedding table is N(0,1) * 2^-3: with tied N(0,1) rows the token's own row dominates the
+# residual stream and greedy decoding of random weights repeats one token; at 1/8 the layers'
+# contributions decide the next token.
+BB_EMBED_LOG2_SCALE = -3
+
+
+def bb_embed_key(wl: Workload) -> int:
+    return gen.key(wl.seed, Tag.BB_EMBED)
+
+
+def bb_embed_rows(wl: Workload, tokens) -> np.ndarray:
+    """Rows of the embedding table (bf16 bits [len(tokens), D])."""
+    out = np.empty((len(tokens), wl.D), np.uint16)
+    for i, t in enumerate(tokens):
+        out[i] = gen.normal_bf16(bb_embed_key(wl), wl.D, int(t) * wl.D, BB_EMBED_LOG2_SCALE)
+    return out
+
+
+def bb_embed(wl: Workload) -> np.ndarray:
+    """The whole embedding table, bf16 bits [vocab, D] (small vocabularies only)."""
+    return gen.normal_bf16(bb_embed_key(wl), wl.vocab * wl.D, 0,
+                           BB_EMBED_LOG2_SCALE).reshape(wl.vocab, wl.D)
+
+
+def bb_token0(wl: Workload) -> np.ndarray:
+    """First token of each sequence, int32 [B] uniform over the vocabulary."""
+    u = gen.uniform_f64(gen.key(wl.seed, Tag.TOKEN0), wl.B)
+    return np.minimum((u * wl.vocab).astype(np.int64), wl.vocab - 1).astype(np.int32)
