@@ -349,6 +349,19 @@ def run_kernel_only(args, wl, local_rank):
     from conditional_sparse_attention_b200 import oda
     from conditional_sparse_attention_b200.engine import OdaDecoder
     dev = torch.device("cuda", local_rank)
+    if args.kernel_only == "bbstep":
+        # whole-model steps of the synthetic backbone, issued kernel by kernel (a profiler lists
+        # every launch; graphs with conditional nodes hide theirs)
+        from workload import configs
+        wl = configs.bb_qwen3_1p7b(ctx=4096)
+        dec = OdaDecoder(wl, device=dev, capacity_steps=args.kernel_reps + 2)
+        for r in range(args.kernel_reps):
+            dec.step(dec.make_step_buffer(r))
+        dec.synchronize()
+        print(json.dumps({"kernel_only": "bbstep", "workload": wl.name, "steps": args.kernel_reps,
+                          "device_error": dec.device_error()}), flush=True)
+        dec.close()
+        return
     dec = OdaDecoder(wl, device=dev, capacity_steps=4, kv_format=args.kv)
     dec.stage(dec.make_step_buffer(0))
     dec.synchronize()
@@ -825,7 +838,7 @@ def main():
     ap.add_argument("--eager", action="store_true",
                     help="issue every step's kernels directly instead of replaying a CUDA graph "
                          "(profilers cannot see kernel nodes of graphs with conditional nodes)")
-    ap.add_argument("--kernel-only", choices=["full", "local", "head", "grad"], default=None,
+    ap.add_argument("--kernel-only", choices=["full", "local", "head", "grad", "bbstep"], default=None,
                     help="profiling mode: launch one kernel (full or local attention, the recall "
                          "head) or one recall-head training step --kernel-reps times and exit")
     ap.add_argument("--kernel-reps", type=int, default=3)

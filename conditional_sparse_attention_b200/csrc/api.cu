@@ -109,7 +109,7 @@ void free_ctx(oda_ctx* c) {
   if (!c) return;
   void* ptrs[] = {c->part_o, c->part_ml, c->attn_cnt, c->err, c->head_part, c->head_ss,
                   c->head_cnt, c->head_u, c->head_f, c->head_act, c->glue_x, c->glue_ss,
-                  c->glue_cnt};
+                  c->glue_cnt, c->bb_part, c->bb_cnt};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   if (c->body_stream) cudaStreamDestroy(c->body_stream);
@@ -184,6 +184,12 @@ oda_status oda_create(const oda_config* cfg, oda_ctx** out) {
   if (st == ODA_OK) st = dev_alloc(&x->glue_x, (size_t)B * D, "cudaMalloc(glue)");
   if (st == ODA_OK) st = dev_alloc(&x->glue_ss, (size_t)B * gch, "cudaMalloc(glue)");
   if (st == ODA_OK) st = dev_alloc(&x->glue_cnt, (size_t)2 * B, "cudaMalloc(glue)");
+  // backbone projections: split-K partials (up to 1M floats) and per-tile counters
+  x->bb_part_floats = (size_t)1 << 20;
+  x->bb_cnt_n = 4096;
+  if (st == ODA_OK) st = dev_alloc(&x->bb_part, x->bb_part_floats, "cudaMalloc(backbone)");
+  if (st == ODA_OK) st = dev_alloc(&x->bb_cnt, (size_t)x->bb_cnt_n, "cudaMalloc(backbone)");
+  if (st == ODA_OK) st = check_cuda(cudaMemset(x->bb_cnt, 0, x->bb_cnt_n * sizeof(int32_t)), "cudaMemset");
   if (st == ODA_OK) st = check_cuda(cudaMemset(x->attn_cnt, 0, 2 * B * Hkv * sizeof(int32_t)), "cudaMemset");
   if (st == ODA_OK) st = check_cuda(cudaMemset(x->err, 0, sizeof(int32_t)), "cudaMemset");
   if (st == ODA_OK)

@@ -32,10 +32,8 @@ namespace oda {
 namespace {
 
 constexpr int kBW = 8;                 // warps per CTA (they split K)
-constexpr int kBThreads = kBW * 32;
 constexpr int kTile = 16;              // output rows per tile
 constexpr int kMaxB = 8;               // sequences: the MMA's N
-constexpr int kPad = 32;               // bf16 padding of an input row in shared memory
 constexpr float kEps = 1e-6f;
 
 enum Epi { kEpiQKV = 0, kEpiResid = 1, kEpiGateUp = 2, kEpiLogits = 3 };
@@ -53,142 +51,157 @@ struct GemvParams {
   float* resid;           // kEpiResid: [B][N], += W a
   uint16_t* act;          // kEpiGateUp: [B][N] bf16
   float* logits;          // kEpiLogits: [B][N]
+  int32_t* err;
   int B, N, K, Hq, Hkv, n_tiles;
+  int kst;                // K values per stage (a K chunk of one tile)
+  int ring;               // stages in the ring
 };
 
-__device__ __forceinline__ uint4 ldg_stream(const uint16_t* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(reinterpret_cast<uint64_t>(p)));
-  return v;
-}
+constexpr int kXPad = 8;            // bf16 padding of an input row (rows 4 banks apart)
+constexpr int kRowPad = 8;          // bf16 padding of a staged weight row
+constexpr int kGThreads = (kBW + 1) * 32;   // 8 consumer warps + 1 producer warp
+constexpr int kMaxRing = 6;
+constexpr uint64_t kGWaitNs = 2000000000ull;
 
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
-// Weight chunk of 32 K values for one tile: rows g and g + 8 of this lane, 8 values each.
-struct WChunk {
-  uint4 lo, hi;
-};
-
-// Two MMA k-steps over one 32-value chunk: physical K offsets 8c .. 8c+7 of the lane hold the
-// logical k-step 0 values {2c, 2c+1 | 2c+8, 2c+9} at 8c+0..3 and k-step 1 at 8c+4..7.
-__device__ __forceinline__ void chunk_mma(float (&acc)[4], const WChunk& w, const uint4& xs) {
-  const uint32_t a0[4] = {w.lo.x, w.hi.x, w.lo.y, w.hi.y};
-  const uint32_t a1[4] = {w.lo.z, w.hi.z, w.lo.w, w.hi.w};
-  mma_bf16_16816(acc, a0, xs.x, xs.y);
-  mma_bf16_16816(acc, a1, xs.z, xs.w);
+__device__ __forceinline__ void consumers_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kBW * 32) : "memory");
 }
 
+// Persistent projection: one CTA per SM takes tiles t = blockIdx.x, + gridDim.x, ...  A producer
+// warp streams each tile's rows, K chunk by K chunk, through a ring of shared-memory stages with
+// one bulk copy per row segment (completion counted on the stage's mbarrier); it only reads
+// weights, so it fills the ring before the previous kernel has finished.  The 8 consumer warps
+// each take 1/8 of every chunk's columns: A fragments of the 16 rows by ldmatrix, B fragments of
+// the bf16 inputs (in shared memory) by ldmatrix, mma.sync bf16 -> fp32.  At the end of a tile
+// the warps' partial sums are added in warp order and the epilogue writes the outputs.
 template <int EPI, int IN>
-__global__ void __launch_bounds__(kBThreads, 2) bb_gemv_kernel(const GemvParams p) {
-  extern __shared__ __align__(16) uint8_t bsm[];
-  const int K = p.K, ldx = K + kPad;
-  uint16_t* xs = reinterpret_cast<uint16_t*>(bsm);                        // [kMaxB][K + kPad]
-  float* red = reinterpret_cast<float*>(bsm + (size_t)kMaxB * ldx * 2);  // [kBW][2][16][8]
+__global__ void __launch_bounds__(kGThreads, 1) bb_gemv_kernel(const GemvParams p) {
+  extern __shared__ __align__(128) uint8_t bsm[];
+  constexpr int kRows = EPI == kEpiGateUp ? 2 * kTile : kTile;
+  const int K = p.K, kst = p.kst, R = p.ring, nck = K / kst;
+  const int ldx = K + kXPad, ldw = kst + kRowPad;
+  const size_t stage_bytes = (size_t)kRows * ldw * 2;
+  uint8_t* stages = bsm;
+  uint16_t* xs = reinterpret_cast<uint16_t*>(bsm + R * stage_bytes);              // [8][K + pad]
+  float* red = reinterpret_cast<float*>(bsm + R * stage_bytes + (size_t)kMaxB * ldx * 2);
+  __shared__ __align__(8) uint64_t full[kMaxRing];
+  __shared__ __align__(8) uint64_t empty[kMaxRing];
   __shared__ float s_inv[kMaxB];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, c = lane & 3;
-  const size_t tile_bytes = (size_t)kTile * K * 2;
-
-  // weights never depend on the previous kernel: pull this CTA's tiles toward L2 first
-  // (the first two tiles only: a large projection, such as the LM head, would not fit in L2)
   if (tid == 0) {
-    for (int t = blockIdx.x, i = 0; t < p.n_tiles && i < 2; t += gridDim.x, ++i) {
-      prefetch_l2_bulk(p.W + (size_t)t * kTile * K, (uint32_t)tile_bytes);
-      if (EPI == kEpiGateUp) prefetch_l2_bulk(p.W2 + (size_t)t * kTile * K, (uint32_t)tile_bytes);
+    for (int i = 0; i < R; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kBW);
     }
+    fence_mbar_init();
   }
+  __syncthreads();
+
+  if (warp == kBW) {
+    // ---- producer: every (tile, chunk) of this CTA in order
+    int k = 0;
+    for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x) {
+      for (int ch = 0; ch < nck; ++ch, ++k) {
+        const int s = k % R;
+        if (k >= R && !mbar_wait_bounded(&empty[s], (uint32_t)(k / R - 1) & 1u, kGWaitNs)) {
+          if (lane == 0) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
+          return;
+        }
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(kRows * kst * 2));
+        __syncwarp();
+        if (lane < kRows) {
+          const uint16_t* src = (EPI == kEpiGateUp && lane >= kTile)
+                                    ? p.W2 + (size_t)(t * kTile + lane - kTile) * K + ch * kst
+                                    : p.W + (size_t)(t * kTile + lane) * K + ch * kst;
+          fence_proxy_async_smem();
+          bulk_load(stages + s * stage_bytes + (size_t)lane * ldw * 2, src, (uint32_t)(kst * 2), &full[s]);
+        }
+      }
+    }
+    return;
+  }
+
+  // ---- consumers
   grid_dependency_wait();
   grid_dependents_launch();
-
-  // ---- the bf16 input vectors of the batch, in shared memory (rows >= B are zero)
   if (IN == kInNorm) {
     if (warp < kMaxB) {
       float ss = 0.f;
       if (warp < p.B)
-        for (int k = lane; k < K; k += 32) {
-          const float v = p.x[(size_t)warp * K + k];
-          ss = fmaf(v, v, ss);
+        for (int kk = 4 * lane; kk < K; kk += 128) {
+          const float4 v = *reinterpret_cast<const float4*>(p.x + (size_t)warp * K + kk);
+          ss = fmaf(v.x, v.x, ss);
+          ss = fmaf(v.y, v.y, ss);
+          ss = fmaf(v.z, v.z, ss);
+          ss = fmaf(v.w, v.w, ss);
         }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       if (lane == 0) s_inv[warp] = rsqrtf(ss / (float)K + kEps);
     }
-    __syncthreads();
+    consumers_sync();
   }
-  for (int i = tid; i < kMaxB * (K / 2); i += kBThreads) {
-    const int b = i / (K / 2), k = 2 * (i - b * (K / 2));
+  for (int i = tid; i < kMaxB * (K / 2); i += kBW * 32) {
+    const int b = i / (K / 2), kk = 2 * (i - b * (K / 2));
     uint32_t w = 0u;
     if (b < p.B) {
       if (IN == kInBf16) {
-        w = *reinterpret_cast<const uint32_t*>(p.xb + (size_t)b * K + k);
+        w = *reinterpret_cast<const uint32_t*>(p.xb + (size_t)b * K + kk);
       } else {
-        const float2 v = *reinterpret_cast<const float2*>(p.x + (size_t)b * K + k);
+        const float2 v = *reinterpret_cast<const float2*>(p.x + (size_t)b * K + kk);
         float v0 = v.x, v1 = v.y;
         if (IN == kInNorm) {
-          v0 = v0 * s_inv[b] * p.gamma[k];
-          v1 = v1 * s_inv[b] * p.gamma[k + 1];
+          v0 = v0 * s_inv[b] * p.gamma[kk];
+          v1 = v1 * s_inv[b] * p.gamma[kk + 1];
         }
         w = (uint32_t)f32_to_bf16_bits(v0) | ((uint32_t)f32_to_bf16_bits(v1) << 16);
       }
     }
-    *reinterpret_cast<uint32_t*>(xs + (size_t)b * ldx + k) = w;
+    *reinterpret_cast<uint32_t*>(xs + (size_t)b * ldx + kk) = w;
   }
-  __syncthreads();
+  consumers_sync();
 
-  const int kw = K / kBW;                  // K values per warp
-  const int nch = kw / 32;                 // chunks per warp (a multiple of 2)
-  const uint16_t* xrow = xs + (size_t)g * ldx + warp * kw + 8 * c;
+  const int g = lane >> 2, c = lane & 3;
+  const int mi = lane >> 3, rr = lane & 7;
+  const int kw = kst / kBW;                      // columns of a chunk per warp (multiple of 16)
+  const uint32_t xs_base = smem_u32(xs);
+  // ldmatrix rows: A from the staged weight rows, B from the input rows (batch g)
+  const int arow = ((mi & 1) << 3) + rr, acol = (mi >> 1) << 3;
+  const int brow = rr, bcol = mi << 3;
+  int k = 0;
   for (int t = blockIdx.x; t < p.n_tiles; t += gridDim.x) {
-    const int r0 = t * kTile;
-    const uint16_t* wr0 = p.W + (size_t)(r0 + g) * K + warp * kw + 8 * c;
-    const uint16_t* wr8 = wr0 + (size_t)8 * K;
-    const uint16_t* ur0 = EPI == kEpiGateUp ? p.W2 + (size_t)(r0 + g) * K + warp * kw + 8 * c : nullptr;
-    const uint16_t* ur8 = EPI == kEpiGateUp ? ur0 + (size_t)8 * K : nullptr;
     float acc[4] = {0.f, 0.f, 0.f, 0.f}, accu[4] = {0.f, 0.f, 0.f, 0.f};
-    // two chunks in registers while the next two load
-    WChunk w[2], u[2];
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      w[j].lo = ldg_stream(wr0 + 32 * j);
-      w[j].hi = ldg_stream(wr8 + 32 * j);
-      if (EPI == kEpiGateUp) {
-        u[j].lo = ldg_stream(ur0 + 32 * j);
-        u[j].hi = ldg_stream(ur8 + 32 * j);
+    for (int ch = 0; ch < nck; ++ch, ++k) {
+      const int s = k % R;
+      if (!mbar_wait_bounded(&full[s], (uint32_t)(k / R) & 1u, kGWaitNs)) {
+        if (lane == 0) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
       }
-    }
-    for (int ch = 0; ch < nch; ch += 2) {
-      WChunk wn[2], un[2];
-      const bool more = ch + 2 < nch;
-      if (more) {
+      const uint32_t sb = smem_u32(stages + s * stage_bytes);
+      const int c0 = warp * kw;                  // first column of this warp in the chunk
+#pragma unroll 4
+      for (int kk = 0; kk < kw; kk += 32) {
+        uint32_t xb4[4];
+        ldsm_x4(xb4, xs_base + ((brow * ldx) + ch * kst + c0 + kk + bcol) * 2);
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          wn[j].lo = ldg_stream(wr0 + 32 * (ch + 2 + j));
-          wn[j].hi = ldg_stream(wr8 + 32 * (ch + 2 + j));
+        for (int h = 0; h < 2; ++h) {
+          uint32_t a[4];
+          ldsm_x4(a, sb + ((arow * ldw) + c0 + kk + 16 * h + acol) * 2);
+          mma_bf16_16816(acc, a, xb4[2 * h], xb4[2 * h + 1]);
           if (EPI == kEpiGateUp) {
-            un[j].lo = ldg_stream(ur0 + 32 * (ch + 2 + j));
-            un[j].hi = ldg_stream(ur8 + 32 * (ch + 2 + j));
+            uint32_t au[4];
+            ldsm_x4(au, sb + (((arow + kTile) * ldw) + c0 + kk + 16 * h + acol) * 2);
+            mma_bf16_16816(accu, au, xb4[2 * h], xb4[2 * h + 1]);
           }
         }
       }
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const uint4 xv = *reinterpret_cast<const uint4*>(xrow + 32 * (ch + j));
-        chunk_mma(acc, w[j], xv);
-        if (EPI == kEpiGateUp) chunk_mma(accu, u[j], xv);
-      }
-      if (more) {
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          w[j] = wn[j];
-          if (EPI == kEpiGateUp) u[j] = un[j];
-        }
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
     }
-    // ---- reduce the warps' K slices in warp order; lane (g, c) holds rows g, g + 8 and
+    // ---- the warps' column shares, added in warp order; lane (g, c) holds rows g, g + 8 and
     // sequences 2c, 2c + 1
     float* rw = red + (size_t)warp * 2 * kTile * kMaxB;
     rw[g * kMaxB + 2 * c] = acc[0];
@@ -201,7 +214,7 @@ __global__ void __launch_bounds__(kBThreads, 2) bb_gemv_kernel(const GemvParams 
       rw[kTile * kMaxB + (g + 8) * kMaxB + 2 * c] = accu[2];
       rw[kTile * kMaxB + (g + 8) * kMaxB + 2 * c + 1] = accu[3];
     }
-    __syncthreads();
+    consumers_sync();
     if (tid < kTile * kMaxB) {
       const int row = tid / kMaxB, b = tid - row * kMaxB;
       float y = 0.f, yu = 0.f;
@@ -210,7 +223,7 @@ __global__ void __launch_bounds__(kBThreads, 2) bb_gemv_kernel(const GemvParams 
         y += red[(size_t)ww * 2 * kTile * kMaxB + tid];
         if (EPI == kEpiGateUp) yu += red[(size_t)ww * 2 * kTile * kMaxB + kTile * kMaxB + tid];
       }
-      const int n = r0 + row;
+      const int n = t * kTile + row;
       if (b < p.B) {
         if (EPI == kEpiQKV) {
           const int nq = p.Hq * 128, nk = p.Hkv * 128;
@@ -228,7 +241,7 @@ __global__ void __launch_bounds__(kBThreads, 2) bb_gemv_kernel(const GemvParams 
         }
       }
     }
-    __syncthreads();
+    consumers_sync();
   }
 }
 
@@ -265,27 +278,33 @@ __global__ void __launch_bounds__(1024) bb_norm_kernel(const float* x, const flo
   for (int k = threadIdx.x; k < D; k += blockDim.x) h[(size_t)b * D + k] = x[(size_t)b * D + k] * inv * gamma[k];
 }
 
-// token[b] = the smallest index of the largest logit; emb[b] = fp32(E[token[b]]).  One CTA per
-// sequence.  If token_in is given, the argmax is skipped and its tokens are embedded.
-__global__ void __launch_bounds__(1024) bb_argmax_embed_kernel(const float* logits, int V,
-                                                               const int32_t* token_in,
-                                                               int32_t* token, const uint16_t* E,
-                                                               float* emb, int D) {
+// token[b] = the smallest index of the largest logit; emb[b] = fp32(E[token[b]]).  Grid (slices,
+// B): each CTA finds the first maximum of its slice of the logits; the CTA completing sequence b
+// (a completion counter, no waiting) takes the first maximum over the slices in slice order and
+// writes the token and its embedding row.  With token_in (one slice), the given tokens are
+// embedded instead (a token outside [0, V) is taken as 0).
+__global__ void __launch_bounds__(256) bb_argmax_embed_kernel(const float* logits, int V,
+                                                              const int32_t* token_in,
+                                                              int32_t* token, const uint16_t* E,
+                                                              float* emb, int D, float* part_v,
+                                                              int32_t* part_i, int32_t* cnt) {
   grid_dependency_wait();
   grid_dependents_launch();
-  const int b = blockIdx.x;
-  __shared__ float sv[32];
-  __shared__ int si[32];
-  __shared__ int s_tok;
+  const int sl = blockIdx.x, nsl = gridDim.x, b = blockIdx.y;
+  __shared__ float sv[8];
+  __shared__ int si[8];
+  __shared__ int s_tok, s_last;
+  auto better = [](float v, int i, float bv, int bi) { return v > bv || (v == bv && i < bi); };
   if (token_in) {
     if (threadIdx.x == 0) {
       const int t = token_in[b];
       s_tok = (t >= 0 && t < V) ? t : 0;
     }
   } else {
+    const int lo = (int)((long long)sl * V / nsl), hi = (int)((long long)(sl + 1) * V / nsl);
     float best = -INFINITY;
     int bi = 0x7fffffff;
-    for (int i = threadIdx.x; i < V; i += blockDim.x) {
+    for (int i = lo + threadIdx.x; i < hi; i += blockDim.x) {
       const float v = logits[(size_t)b * V + i];
       if (v > best) {   // i increases per thread: the first maximum is kept
         best = v;
@@ -296,7 +315,7 @@ __global__ void __launch_bounds__(1024) bb_argmax_embed_kernel(const float* logi
     for (int o = 16; o > 0; o >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, best, o);
       const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > best || (ov == best && oi < bi)) {
+      if (better(ov, oi, best, bi)) {
         best = ov;
         bi = oi;
       }
@@ -306,48 +325,68 @@ __global__ void __launch_bounds__(1024) bb_argmax_embed_kernel(const float* logi
       si[threadIdx.x >> 5] = bi;
     }
     __syncthreads();
-    if (threadIdx.x < 32) {
-      const int nw = blockDim.x >> 5;
-      best = threadIdx.x < nw ? sv[threadIdx.x] : -INFINITY;
-      bi = threadIdx.x < nw ? si[threadIdx.x] : 0x7fffffff;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > best || (ov == best && oi < bi)) {
-          best = ov;
-          bi = oi;
+    if (threadIdx.x == 0) {
+      for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
+        if (better(sv[w], si[w], best, bi)) {
+          best = sv[w];
+          bi = si[w];
         }
+      if (nsl > 1) {
+        part_v[(size_t)b * nsl + sl] = best;
+        part_i[(size_t)b * nsl + sl] = bi;
+        __threadfence();
+        s_last = atomicAdd(&cnt[b], 1) == nsl - 1;
+        if (s_last) {
+          __threadfence();
+          best = -INFINITY;
+          bi = 0x7fffffff;
+          for (int j = 0; j < nsl; ++j) {
+            const float v = __ldcg(part_v + (size_t)b * nsl + j);
+            const int i = __ldcg(part_i + (size_t)b * nsl + j);
+            if (better(v, i, best, bi)) {
+              best = v;
+              bi = i;
+            }
+          }
+          cnt[b] = 0;
+        }
+      } else {
+        s_last = 1;
       }
-      if (threadIdx.x == 0) s_tok = (bi >= 0 && bi < V) ? bi : 0;
+      s_tok = (bi >= 0 && bi < V) ? bi : 0;
     }
+    __syncthreads();
+    if (!s_last) return;
   }
   __syncthreads();
   const int t = s_tok;
   if (threadIdx.x == 0) token[b] = t;
-  for (int k = threadIdx.x; k < D; k += blockDim.x)
-    emb[(size_t)b * D + k] = __uint_as_float((uint32_t)E[(size_t)t * D + k] << 16);
+  for (int kk = threadIdx.x; kk < D; kk += blockDim.x)
+    emb[(size_t)b * D + kk] = __uint_as_float((uint32_t)E[(size_t)t * D + kk] << 16);
 }
 
 int g_bb_smem_optin = 0;
 
 template <int EPI, int IN>
-oda_status launch_gemv(oda_ctx* ctx, const GemvParams& p, cudaStream_t s) {
-  const size_t smem = (size_t)kMaxB * (p.K + kPad) * 2 + (size_t)kBW * 2 * kTile * kMaxB * 4;
-  if ((int)smem > g_bb_smem_optin)
+oda_status launch_gemv(oda_ctx* ctx, GemvParams p, cudaStream_t s) {
+  constexpr int rows = EPI == kEpiGateUp ? 2 * kTile : kTile;
+  p.err = ctx->err;
+  // a stage of about 32 KiB: 1024 columns of 16 rows, or 512 of the gate and up rows together
+  p.kst = (EPI != kEpiGateUp && p.K % 1024 == 0) ? 1024 : 512;
+  const size_t stage = (size_t)rows * (p.kst + kRowPad) * 2;
+  const size_t fixed = (size_t)kMaxB * (p.K + kXPad) * 2 + (size_t)kBW * 2 * kTile * kMaxB * 4;
+  const long long room = (long long)g_bb_smem_optin - 1024 - (long long)fixed;
+  p.ring = (int)std::min<long long>(kMaxRing, room / (long long)stage);
+  if (p.ring < 2)
     return set_error(ODA_ERR_UNSUPPORTED, "backbone: input width %d needs more shared memory", p.K);
+  const size_t smem = p.ring * stage + fixed;
   oda_status st = check_cuda(cudaFuncSetAttribute(bb_gemv_kernel<EPI, IN>,
                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
                              "cudaFuncSetAttribute(backbone)");
   if (st != ODA_OK) return st;
-  int occ = 0;
-  st = check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, bb_gemv_kernel<EPI, IN>, kBThreads, smem),
-                  "cudaOccupancyMaxActiveBlocksPerMultiprocessor(backbone)");
-  if (st != ODA_OK) return st;
-  const int grid = std::max(1, std::min(p.n_tiles, ctx->n_sms * std::max(1, occ)));
   cudaLaunchConfig_t lc = {};
-  lc.gridDim = dim3(grid);
-  lc.blockDim = dim3(kBThreads);
+  lc.gridDim = dim3(std::min(p.n_tiles, ctx->n_sms));
+  lc.blockDim = dim3(kGThreads);
   lc.dynamicSmemBytes = smem;
   lc.stream = s;
   cudaLaunchAttribute attr[1];
@@ -511,9 +550,12 @@ oda_status launch_bb_lm_head(oda_ctx* ctx, const void* embed, int32_t vocab, con
   p.n_tiles = vocab / kTile;
   st = launch_gemv<kEpiLogits, kInF32>(ctx, p, s);
   if (st != ODA_OK) return st;
-  return launch_small(ctx, bb_argmax_embed_kernel, dim3(cf.batch), dim3(1024), s, "bb_argmax launch",
+  const int nsl = std::max(1, std::min(64, vocab / 2048));
+  float* part_v = ctx->bb_part;
+  int32_t* part_i = reinterpret_cast<int32_t*>(ctx->bb_part + (size_t)cf.batch * nsl);
+  return launch_small(ctx, bb_argmax_embed_kernel, dim3(nsl, cf.batch), dim3(256), s, "bb_argmax launch",
                       (const float*)logits, (int)vocab, (const int32_t*)nullptr, token,
-                      static_cast<const uint16_t*>(embed), next_emb, D);
+                      static_cast<const uint16_t*>(embed), next_emb, D, part_v, part_i, ctx->bb_cnt);
 }
 
 oda_status launch_bb_embed(oda_ctx* ctx, const void* embed, int32_t vocab, const int32_t* token,
@@ -521,9 +563,10 @@ oda_status launch_bb_embed(oda_ctx* ctx, const void* embed, int32_t vocab, const
   const int D = ctx->cfg.n_q_heads * 128;
   if (!embed || !token || !emb || vocab < 1) return set_error(ODA_ERR_INVALID_ARG, "bb_embed: bad argument");
   // the token buffer is read, and rewritten with the (range-checked) token it used
-  return launch_small(ctx, bb_argmax_embed_kernel, dim3(ctx->cfg.batch), dim3(1024), s, "bb_embed launch",
+  return launch_small(ctx, bb_argmax_embed_kernel, dim3(1, ctx->cfg.batch), dim3(256), s, "bb_embed launch",
                       (const float*)nullptr, (int)vocab, token, const_cast<int32_t*>(token),
-                      static_cast<const uint16_t*>(embed), emb, D);
+                      static_cast<const uint16_t*>(embed), emb, D, ctx->bb_part,
+                      reinterpret_cast<int32_t*>(ctx->bb_part), ctx->bb_cnt);
 }
 
 }  // namespace oda

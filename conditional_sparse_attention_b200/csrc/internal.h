@@ -27,6 +27,11 @@ struct oda_ctx {
   float* head_u = nullptr;      // [3][B][1024]
   float* head_f = nullptr;      // [3][B][1024]: fusion output and the two block outputs
   float* head_act = nullptr;    // [B][2048]
+  // synthetic-backbone scratch: split-K partial sums and per-tile completion counters
+  float* bb_part = nullptr;
+  size_t bb_part_floats = 0;
+  int32_t* bb_cnt = nullptr;
+  int bb_cnt_n = 0;
   // glue scratch
   float* glue_x = nullptr;      // [B][D]
   float* glue_ss = nullptr;     // [B][chunks]
