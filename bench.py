@@ -122,15 +122,26 @@ KV_BYTES_PER_TOKEN_HEAD = {"bf16": 128 * 2 * 2,       # K and V rows, bf16
                            "fp8": 128 * 2 + 2 * 4}     # K and V e4m3 codes + two fp32 scales
 
 
+def hybrid_state_bytes(wl) -> int:
+    """Recurrent + conv state of one sequence over all linear-recurrent layers (fp32)."""
+    from workload import configs
+    n = len(wl.gdn_layers)
+    return n * (configs.GDN_HEADS * configs.GDN_DIM * configs.GDN_DIM +
+                configs.CONV_TAPS * configs.CONV_WIDTH) * 4
+
+
 def step_bytes(wl, pos_list, flags, kv="bf16"):
-    """Algorithmic bytes of one step: local KV + flagged full KV + head weights."""
+    """Algorithmic bytes of one step: local KV + flagged full KV + head weights; hybrid stacks add
+    the recurrent state each pass reads and writes (the local pass for every sequence, the retry
+    for flagged ones; with ping-pong state buffers nothing is snapshotted or restored)."""
     from workload import inputs
     per_tok = wl.Hkv * KV_BYTES_PER_TOKEN_HEAD[kv]
+    st = hybrid_state_bytes(wl) if wl.hybrid else 0
     b = 0
     for bi, t in enumerate(pos_list):
-        b += min(t, wl.sinks + wl.window) * per_tok * wl.L
+        b += min(t, wl.sinks + wl.window) * per_tok * wl.L + 2 * st
         if flags[bi]:
-            b += t * per_tok * wl.L
+            b += t * per_tok * wl.L + 2 * st
     return b + inputs.head_param_count(wl.D) * 4
 
 
@@ -141,12 +152,10 @@ def head_launches(wl) -> int:
 
 
 def kernel_launches(wl, any_flag: bool) -> int:
-    # local layers, glue, head, set-cond, commit
+    # local layers, glue, head, set-cond, commit (hybrid stacks: no snapshot or restore copies)
     n = wl.L + (wl.n_layers - wl.L) + 1 + head_launches(wl) + 1 + 1
-    if wl.hybrid:
-        n += 2
     if any_flag:
-        n += wl.n_layers + 1 + (2 if wl.hybrid else 0)
+        n += wl.n_layers + 1
     return n
 
 

@@ -117,6 +117,8 @@ _SIGS = {
                         c_int32),
     "oda_glue_gdn": ([c_void_p, _P(OdaState), c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
                       c_void_p, c_void_p, c_void_p, c_void_p], c_int32),
+    "oda_glue_gdn_step": ([c_void_p, _P(OdaState), _P(OdaState), c_int32, c_void_p, c_void_p,
+                           c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p], c_int32),
 }
 
 _lib = None

@@ -354,7 +354,16 @@ oda_status oda_glue_gdn(oda_ctx* ctx, const oda_state* st, int32_t layer, const 
                         const float* taps, const int32_t* flag, float* o, cudaStream_t stream) {
   if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "glue_gdn: ctx is NULL");
   ctx->prev_attention = false;
-  return oda::launch_glue_gdn(ctx, st, layer, c, v, alpha, beta, taps, flag, o, stream);
+  return oda::launch_glue_gdn(ctx, st, st, layer, c, v, alpha, beta, taps, flag, o, stream);
+}
+
+oda_status oda_glue_gdn_step(oda_ctx* ctx, const oda_state* src, const oda_state* dst,
+                             int32_t layer, const float* c, const float* v, const float* alpha,
+                             const float* beta, const float* taps, const int32_t* flag, float* o,
+                             cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "glue_gdn_step: ctx is NULL");
+  ctx->prev_attention = false;
+  return oda::launch_glue_gdn(ctx, src, dst, layer, c, v, alpha, beta, taps, flag, o, stream);
 }
 
 oda_status oda_bb_begin(oda_ctx* ctx, const float* emb, float* x, cudaStream_t stream) {

@@ -85,22 +85,25 @@ hidden_kernel(const float* emb, const float* terms, int n_terms, const int32_t* 
   if (threadIdx.x == 0) cnt[b] = 0;
 }
 
-// One (sequence, head) per CTA of 256 threads: thread t owns half of row t/2 of S_h.
+// One (sequence, head) per CTA of 256 threads: thread t owns half of row t/2 of S_h.  The layer's
+// state is read from (rec_in, conv_in) and the advanced state written to (rec_out, conv_out);
+// the two may be the same buffers (in place) or different ones (the pre-step state stays).
 __global__ void __launch_bounds__(256)
-gdn_kernel(float* rec, float* conv, int n_layers, int layer, const float* c, const float* v,
-           const float* alpha, const float* beta, const float* taps, const int32_t* flag,
-           float* o) {
+gdn_kernel(const float* rec_in, const float* conv_in, float* rec, float* conv, int n_layers,
+           int layer, const float* c, const float* v, const float* alpha, const float* beta,
+           const float* taps, const int32_t* flag, float* o) {
   constexpr int H = 16, DK = 128, W = 2048, TAPS = 4;
   const int h = blockIdx.x, b = blockIdx.y;
   if (flag && flag[b] == 0) return;
   __shared__ float k_s[DK];
   __shared__ float red[8];
   const int tid = threadIdx.x;
+  const float* ci = conv_in + ((size_t)b * n_layers + layer) * TAPS * W;
   float* cv = conv + ((size_t)b * n_layers + layer) * TAPS * W;
   float u = 0.f;
   if (tid < DK) {
     const int e = h * DK + tid;
-    const float c0 = cv[1 * W + e], c1 = cv[2 * W + e], c2 = cv[3 * W + e];
+    const float c0 = ci[1 * W + e], c1 = ci[2 * W + e], c2 = ci[3 * W + e];
     const float c3 = c[(size_t)b * W + e];
     cv[0 * W + e] = c0;
     cv[1 * W + e] = c1;
@@ -111,13 +114,14 @@ gdn_kernel(float* rec, float* conv, int n_layers, int layer, const float* c, con
   const float nrm2 = block_sum256(u * u, red);
   if (tid < DK) k_s[tid] = u / sqrtf(nrm2);
   __syncthreads();
+  const float* Si = rec_in + (((size_t)b * n_layers + layer) * H + h) * DK * DK;
   float* S = rec + (((size_t)b * n_layers + layer) * H + h) * DK * DK;
   const int i = tid >> 1, j0 = (tid & 1) * 64;
   float4 row[16];
   float sk = 0.f;
 #pragma unroll
   for (int q = 0; q < 16; ++q) {
-    row[q] = reinterpret_cast<const float4*>(S + (size_t)i * DK + j0)[q];
+    row[q] = reinterpret_cast<const float4*>(Si + (size_t)i * DK + j0)[q];
     const int j = j0 + 4 * q;
     sk += row[q].x * k_s[j] + row[q].y * k_s[j + 1] + row[q].z * k_s[j + 2] + row[q].w * k_s[j + 3];
   }
@@ -165,20 +169,25 @@ oda_status launch_glue_hidden(oda_ctx* ctx, const float* emb, const float* terms
                     "glue_hidden launch");
 }
 
-oda_status launch_glue_gdn(oda_ctx* ctx, const oda_state* st, int layer, const float* c,
-                           const float* v, const float* alpha, const float* beta,
+oda_status launch_glue_gdn(oda_ctx* ctx, const oda_state* src, const oda_state* st, int layer,
+                           const float* c, const float* v, const float* alpha, const float* beta,
                            const float* taps, const int32_t* flag, float* o, cudaStream_t s) {
-  if (!st || !st->rec || !st->conv || !c || !v || !alpha || !beta || !taps || !o)
+  if (!src || !st || !st->rec || !st->conv || !src->rec || !src->conv || !c || !v || !alpha ||
+      !beta || !taps || !o)
     return set_error(ODA_ERR_INVALID_ARG, "glue_gdn: null pointer argument");
   if (st->heads != 16 || st->dk != 128 || st->dv != 128 || st->conv_taps != 4 ||
       st->conv_width != 2048)
     return set_error(ODA_ERR_UNSUPPORTED, "glue_gdn: needs 16 heads of 128x128 and a 4x2048 conv");
+  if (src->n_layers != st->n_layers || src->heads != st->heads || src->dk != st->dk ||
+      src->dv != st->dv || src->conv_taps != st->conv_taps || src->conv_width != st->conv_width)
+    return set_error(ODA_ERR_INVALID_ARG, "glue_gdn: source and destination shapes differ");
   if (layer < 0 || layer >= st->n_layers)
     return set_error(ODA_ERR_INVALID_ARG, "glue_gdn: layer %d out of range", layer);
-  if (reinterpret_cast<uintptr_t>(st->rec) & 15)
+  if ((reinterpret_cast<uintptr_t>(st->rec) | reinterpret_cast<uintptr_t>(src->rec)) & 15)
     return set_error(ODA_ERR_INVALID_ARG, "glue_gdn: state must be 16-byte aligned");
-  gdn_kernel<<<dim3(16, ctx->cfg.batch), 256, 0, s>>>(st->rec, st->conv, st->n_layers, layer, c, v,
-                                                       alpha, beta, taps, flag, o);
+  gdn_kernel<<<dim3(16, ctx->cfg.batch), 256, 0, s>>>(src->rec, src->conv, st->rec, st->conv,
+                                                       st->n_layers, layer, c, v, alpha, beta, taps,
+                                                       flag, o);
   return check_cuda(cudaGetLastError(), "glue_gdn launch");
 }
 

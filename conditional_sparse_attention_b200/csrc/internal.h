@@ -109,8 +109,8 @@ oda_status launch_state_copy(const oda_state* src, const oda_state* dst, int B,
 // glue.cu
 oda_status launch_glue_hidden(oda_ctx* ctx, const float* emb, const float* terms, int n_terms,
                               const int32_t* flag, float* h, cudaStream_t stream);
-oda_status launch_glue_gdn(oda_ctx* ctx, const oda_state* st, int layer, const float* c,
-                           const float* v, const float* alpha, const float* beta,
+oda_status launch_glue_gdn(oda_ctx* ctx, const oda_state* src, const oda_state* st, int layer,
+                           const float* c, const float* v, const float* alpha, const float* beta,
                            const float* taps, const int32_t* flag, float* o, cudaStream_t s);
 int glue_chunks(int D);
 

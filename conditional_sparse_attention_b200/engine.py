@@ -3,12 +3,12 @@
 One step, in the order of the method notes ("On-Demand Attention：让语言模型按需读取完整历史")
 §2.3, issued on one stream with no host synchronisation:
 
-  [hybrid] oda_snapshot(live -> snap)
   local pass : per layer oda_attend_local (S^L) or the recurrent stand-in; oda_glue_hidden -> h^L
+               [hybrid: the recurrent layers read state buffer i and write buffer 1 - i]
   oda_recall_score(h_{t-1}, E(x_t), h^L) -> score, flag, any_flag
   oda_cond_begin(any_flag)          # a CUDA-graph IF node when captured
-     [hybrid] oda_restore(flag, snap -> live)
      full pass: per layer oda_attend_full_if (S^F, flagged sequences only); glue -> h^F
+               [hybrid: the recurrent layers read the untouched pre-step buffer i again]
   oda_cond_end
   oda_commit(flag): chosen branch's staged K,V -> cache slot of position t, h_{t-1} <- h^b, t += 1
 
@@ -170,14 +170,15 @@ class OdaDecoder:
         self.staged = [torch.cuda.Event() for _ in range(2)]
         self.released = [torch.cuda.Event() for _ in range(2)]
         self.routing_scheduled = wl.routing == "bernoulli"
+        self._n_launched = 0
         if wl.hybrid:
+            # two state buffers used alternately (ping-pong): a step reads the pre-step recurrent
+            # and conv state from one and writes the advanced state to the other, so the full
+            # retry reads the untouched pre-step state directly - no snapshot or restore copies
             S0, C0 = inputs.gdn_state0(wl)
-            self.rec = torch.from_numpy(S0).to(dev)
-            self.conv = torch.from_numpy(C0).to(dev)
-            self.rec_snap = torch.empty_like(self.rec)
-            self.conv_snap = torch.empty_like(self.conv)
-            self.live = oda.state(self.rec, self.conv)
-            self.snap = oda.state(self.rec_snap, self.conv_snap)
+            self.rec_buf = [torch.from_numpy(S0).to(dev), torch.empty(S0.shape, dtype=torch.float32, device=dev)]
+            self.conv_buf = [torch.from_numpy(C0).to(dev), torch.empty(C0.shape, dtype=torch.float32, device=dev)]
+            self.states = [oda.state(self.rec_buf[i], self.conv_buf[i]) for i in range(2)]
             self.taps = torch.from_numpy(
                 np.stack([inputs.gdn_taps(wl, layer) for layer in wl.gdn_layers])).to(dev)
         if wl.backbone:
@@ -317,8 +318,8 @@ class OdaDecoder:
         wl, s, sv = self.wl, self.stream, self.sv
         ctx = self.ctx
         n_layers = wl.n_layers
-        if wl.hybrid:
-            oda.oda_snapshot(ctx, self.live, self.snap, s)
+        if wl.hybrid:   # the step with staging slot i reads state i and writes state 1 - i
+            cur, nxt = self.states[self.slot], self.states[1 - self.slot]
         a = j = 0
         for layer in range(n_layers):
             if layer in wl.attn_layers:
@@ -326,17 +327,15 @@ class OdaDecoder:
                                    sv["k"][LOCAL, a], sv["v"][LOCAL, a], self.o[LOCAL, layer], s)
                 a += 1
             else:
-                oda.oda_glue_gdn(ctx, self.live, j, sv["gc"][LOCAL, j], sv["gv"][LOCAL, j],
-                                 sv["ga"][LOCAL, j], sv["gb"][LOCAL, j], self.taps[j], None,
-                                 self.o[LOCAL, layer], s)
+                oda.oda_glue_gdn_step(ctx, cur, nxt, j, sv["gc"][LOCAL, j], sv["gv"][LOCAL, j],
+                                      sv["ga"][LOCAL, j], sv["gb"][LOCAL, j], self.taps[j], None,
+                                      self.o[LOCAL, layer], s)
                 j += 1
         oda.oda_glue_hidden(ctx, sv["emb"], self.o[LOCAL], n_layers, None, self.h[LOCAL], s)
         oda.oda_recall_score(ctx, self.head_w, self.h_prev, sv["emb"], self.h[LOCAL],
                              sv["sched"] if self.routing_scheduled else None, self.score,
                              self.flag, self.any_flag, s)
         body = oda.oda_cond_begin(ctx, s, self.any_flag)
-        if wl.hybrid:
-            oda.oda_restore(ctx, self.flag, self.snap, self.live, body)
         a = j = 0
         for layer in range(n_layers):
             if layer in wl.attn_layers:
@@ -345,9 +344,10 @@ class OdaDecoder:
                                   self.o[FULL, layer], body)
                 a += 1
             else:
-                oda.oda_glue_gdn(ctx, self.live, j, sv["gc"][FULL, j], sv["gv"][FULL, j],
-                                 sv["ga"][FULL, j], sv["gb"][FULL, j], self.taps[j], self.flag,
-                                 self.o[FULL, layer], body)
+                # flagged sequences: from the pre-step state, over the local pass's result
+                oda.oda_glue_gdn_step(ctx, cur, nxt, j, sv["gc"][FULL, j], sv["gv"][FULL, j],
+                                      sv["ga"][FULL, j], sv["gb"][FULL, j], self.taps[j], self.flag,
+                                      self.o[FULL, layer], body)
                 j += 1
         oda.oda_glue_hidden(ctx, sv["emb"], self.o[FULL], n_layers, self.flag, self.h[FULL], body)
         oda.oda_cond_end(ctx, s)
@@ -378,8 +378,17 @@ class OdaDecoder:
         self.slot = slot
         self.graph = graphs
 
+    def live_state(self):
+        """(recurrent, conv) buffers holding the state after the last launched step (hybrid)."""
+        i = self._n_launched % 2
+        return self.rec_buf[i], self.conv_buf[i]
+
     def launch(self) -> None:
         """Runs one step on the most recently staged inputs."""
+        if self.wl.hybrid and self.slot != self._n_launched % 2:
+            raise RuntimeError("hybrid steps alternate their state buffers with the staging "
+                               "buffers: stage new inputs before every step")
+        self._n_launched += 1
         if self.graph is not None:
             self.graph[self.slot].launch(self.stream)
         else:

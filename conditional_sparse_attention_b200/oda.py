@@ -279,6 +279,13 @@ def oda_glue_hidden(ctx, emb, terms, n_terms: int, flag, h, stream=None):
                                       _s(stream)))
 
 
+def oda_glue_gdn_step(ctx, src: OdaState, dst: OdaState, layer: int, c, v, alpha, beta, taps, flag,
+                      o, stream=None):
+    check(_lib.load().oda_glue_gdn_step(ctx.handle, ctypes.byref(src), ctypes.byref(dst), layer,
+                                        _p(c), _p(v), _p(alpha), _p(beta), _p(taps), _p(flag), _p(o),
+                                        _s(stream)))
+
+
 def oda_glue_gdn(ctx, st: OdaState, layer: int, c, v, alpha, beta, taps, flag, o, stream=None):
     check(_lib.load().oda_glue_gdn(ctx.handle, ctypes.byref(st), layer, _p(c), _p(v), _p(alpha),
                                    _p(beta), _p(taps), _p(flag), _p(o), _s(stream)))

@@ -37,6 +37,17 @@ oda_status oda_glue_gdn(oda_ctx* ctx, const oda_state* st, int32_t layer, const 
                         const float* v, const float* alpha, const float* beta,
                         const float* taps, const int32_t* flag, float* o, cudaStream_t stream);
 
+/* The same layer update reading the layer's state from src and writing the advanced state to
+ * dst (same shapes; src == dst is oda_glue_gdn).  With two state buffers used alternately, the
+ * pre-step state of a hybrid backbone stays intact in one of them while the local pass writes
+ * the other: the full retry reads it directly, so neither a snapshot copy nor a restore copy is
+ * needed ([notes §2.3, third paragraph]: the retry must start from the pre-step state and no
+ * state may advance twice). */
+oda_status oda_glue_gdn_step(oda_ctx* ctx, const oda_state* src, const oda_state* dst,
+                             int32_t layer, const float* c, const float* v, const float* alpha,
+                             const float* beta, const float* taps, const int32_t* flag, float* o,
+                             cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

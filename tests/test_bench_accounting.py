@@ -35,3 +35,21 @@ def test_launch_counts():
     assert bench.kernel_launches(wl, False) == 36 + 1 + 1 + 1 + 1
     # plus 36 full-set launches and the retry's hidden-state glue when the IF node fires
     assert bench.kernel_launches(wl, True) == 40 + 36 + 1
+
+
+def test_step_bytes_of_the_hybrid_stack_count_the_state_each_pass_moves():
+    wl = configs.cfg4()
+    per_seq = 18 * (16 * 128 * 128 + 4 * 2048) * 4            # 18 recurrent layers, fp32
+    assert bench.hybrid_state_bytes(wl) == per_seq
+    t = 65537
+    kv = wl.Hkv * 128 * 2 * 2
+    local = 8 * 2052 * kv * 6 + 8 * 2 * per_seq               # every sequence: read + write
+    full = 2 * (t * kv * 6 + 2 * per_seq)                     # two flagged sequences
+    head = inputs.head_param_count(wl.D) * 4
+    flags = [1, 0, 0, 1, 0, 0, 0, 0]
+    assert bench.step_bytes(wl, [t] * 8, flags) == local + full + head
+    # fp8 pages: 264 bytes per token and KV head
+    assert bench.step_bytes(configs.cfg2(), [100] * 4, [0] * 4, "fp8") == (
+        4 * 100 * 8 * 264 * 36 + inputs.head_param_count(4096) * 4)
+    # a hybrid step launches no snapshot or restore kernels
+    assert bench.kernel_launches(wl, True) == bench.kernel_launches(wl, False) + 24 + 1
