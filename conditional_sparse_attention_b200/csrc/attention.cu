@@ -484,47 +484,53 @@ __device__ __forceinline__ void load_q8(QF8& Q, const AttnParams& p, int b, int 
 
 // K fragments of one fp8 page (tokens as M in natural order, dims in the q fragment order) and
 // V^T fragments (dims as M, tokens in the P^T fragment order), converted to f16.
-struct Page8 {
-  uint32_t k[8][4];   // A fragments of the 8 k-steps of K q^T
-  uint32_t v[8][4];   // A fragments of the 8 dim tiles of V^T P^T
-};
-
-__device__ __forceinline__ void load_page8(Page8& P, uint32_t sb, int lane) {
+// Raw scores K q^T of one fp8 page (tokens as M in natural order, dims in the q fragment
+// order), before scales: K fragments by ldmatrix, converted to f16 from the register halves.
+__device__ __forceinline__ void page_scores8(float (&sacc)[4], const QF8& Q, uint32_t sb, int lane) {
   const int mi = lane >> 3, rr = lane & 7;
-  const int tok = ((mi & 1) << 3) + rr;          // K: token row this lane addresses
-  const int drow = ((mi & 1) << 3) + rr;         // V^T: dim row within a 16-dim tile
-#pragma unroll
-  for (int kk = 0; kk < 8; kk += 2) {
-    uint32_t r[4];
-    ldsm_x4(r, sb + tok * 128 + (((kk + (mi >> 1)) ^ rr) << 4));
-    e4m3x4_to_f16x2x2(r[0], P.k[kk][0], P.k[kk][2]);
-    e4m3x4_to_f16x2x2(r[1], P.k[kk][1], P.k[kk][3]);
-    e4m3x4_to_f16x2x2(r[2], P.k[kk + 1][0], P.k[kk + 1][2]);
-    e4m3x4_to_f16x2x2(r[3], P.k[kk + 1][1], P.k[kk + 1][3]);
-  }
-#pragma unroll
-  for (int mt = 0; mt < 8; mt += 2) {
-    uint32_t r[4];
-    ldsm_x4(r, sb + kF8V + (16 * (mt + (mi >> 1)) + drow) * 16);
-    e4m3x4_to_f16x2x2(r[0], P.v[mt][0], P.v[mt][2]);
-    e4m3x4_to_f16x2x2(r[1], P.v[mt][1], P.v[mt][3]);
-    e4m3x4_to_f16x2x2(r[2], P.v[mt + 1][0], P.v[mt + 1][2]);
-    e4m3x4_to_f16x2x2(r[3], P.v[mt + 1][1], P.v[mt + 1][3]);
-  }
-}
-
-// Raw scores K q^T of one converted page, before scales.
-__device__ __forceinline__ void page_scores8(float (&sacc)[4], const QF8& Q, const Page8& P) {
+  const int tok = ((mi & 1) << 3) + rr;          // token row this lane addresses
   float sa[4] = {0.f, 0.f, 0.f, 0.f}, sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int kk = 0; kk < 8; kk += 2) {
-    mma_f16_16816(sa, P.k[kk], Q.qf[kk][0], Q.qf[kk][1]);
-    mma_f16_16816(sc, P.k[kk + 1], Q.qf[kk + 1][0], Q.qf[kk + 1][1]);
+    uint32_t r[4], a0[4], a1[4];
+    ldsm_x4(r, sb + tok * 128 + (((kk + (mi >> 1)) ^ rr) << 4));
+    e4m3x4_to_f16x2x2(r[0], a0[0], a0[2]);
+    e4m3x4_to_f16x2x2(r[1], a0[1], a0[3]);
+    e4m3x4_to_f16x2x2(r[2], a1[0], a1[2]);
+    e4m3x4_to_f16x2x2(r[3], a1[1], a1[3]);
+    mma_f16_16816(sa, a0, Q.qf[kk][0], Q.qf[kk][1]);
+    mma_f16_16816(sc, a1, Q.qf[kk + 1][0], Q.qf[kk + 1][1]);
   }
   sacc[0] = sa[0] + sc[0];
   sacc[1] = sa[1] + sc[1];
   sacc[2] = sa[2] + sc[2];
   sacc[3] = sa[3] + sc[3];
+}
+
+// PV of one fp8 page into the accumulator: V^T fragments (dims as M, tokens in the P^T fragment
+// order) by ldmatrix, converted to f16, masked where tokens are outside the set.
+__device__ __forceinline__ void page_pv8(float (&o)[8][4], uint32_t vb, uint32_t bh0, uint32_t bh1,
+                                         uint32_t bl0, uint32_t bl1, bool masked, uint32_t mlo,
+                                         uint32_t mhi, int lane) {
+  const int mi = lane >> 3, rr = lane & 7;
+  const int drow = ((mi & 1) << 3) + rr;         // dim row within a 16-dim tile
+#pragma unroll
+  for (int mt = 0; mt < 8; mt += 2) {
+    uint32_t r[4], a0[4], a1[4];
+    ldsm_x4(r, vb + (16 * (mt + (mi >> 1)) + drow) * 16);
+    e4m3x4_to_f16x2x2(r[0], a0[0], a0[2]);
+    e4m3x4_to_f16x2x2(r[1], a0[1], a0[3]);
+    e4m3x4_to_f16x2x2(r[2], a1[0], a1[2]);
+    e4m3x4_to_f16x2x2(r[3], a1[1], a1[3]);
+    if (masked) {   // tokens outside the set: their codes may be stale (even NaN); P'' is 0 there
+      a0[0] &= mlo; a0[1] &= mlo; a0[2] &= mhi; a0[3] &= mhi;
+      a1[0] &= mlo; a1[1] &= mlo; a1[2] &= mhi; a1[3] &= mhi;
+    }
+    mma_f16_16816(o[mt], a0, bh0, bh1);
+    mma_f16_16816(o[mt], a0, bl0, bl1);
+    mma_f16_16816(o[mt + 1], a1, bh0, bh1);
+    mma_f16_16816(o[mt + 1], a1, bl0, bl1);
+  }
 }
 
 // Keep-masks of this lane's V^T fragment halves for a page whose token set is given by the
@@ -554,16 +560,13 @@ template <int NP>
 __device__ __forceinline__ void page_step8(WarpAcc& A, const QF8& Q, uint8_t* const (&st)[2],
                                            const bool (&in)[2][2], int lane) {
   const int r = lane >> 2;
-  Page8 P[NP];
-#pragma unroll
-  for (int i = 0; i < NP; ++i) load_page8(P[i], smem_u32(st[i]), lane);
   float x[2][4], svv[2][2];
   bool any_masked = false;
   float svmax = 0.f;
 #pragma unroll
   for (int i = 0; i < NP; ++i) {
     float sacc[4];
-    page_scores8(sacc, Q, P[i]);
+    page_scores8(sacc, Q, smem_u32(st[i]), lane);
     const float* sk = reinterpret_cast<const float*>(st[i] + kF8SK);
     const float* sv = reinterpret_cast<const float*>(st[i] + kF8SV);
     const float k0 = sk[r], k1 = sk[r + 8];
@@ -623,22 +626,9 @@ __device__ __forceinline__ void page_step8(WarpAcc& A, const QF8& Q, uint8_t* co
     const uint32_t l23 = pack_f16x2(q2 - f16_lo_to_f32(h23), q3 - f16_hi_to_f32(h23));
     const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
     const uint32_t bl0 = movmatrix_trans(l01), bl1 = movmatrix_trans(l23);
-    if (masked) {   // tokens outside the set: their codes may be stale (even NaN); P'' is 0 there
-      uint32_t mlo, mhi;
-      v8_masks(in[i][0], in[i][1], lane, mlo, mhi);
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        P[i].v[mt][0] &= mlo;
-        P[i].v[mt][1] &= mlo;
-        P[i].v[mt][2] &= mhi;
-        P[i].v[mt][3] &= mhi;
-      }
-    }
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      mma_f16_16816(A.o[mt], P[i].v[mt], bh0, bh1);
-      mma_f16_16816(A.o[mt], P[i].v[mt], bl0, bl1);
-    }
+    uint32_t mlo = 0xFFFFFFFFu, mhi = 0xFFFFFFFFu;
+    if (masked) v8_masks(in[i][0], in[i][1], lane, mlo, mhi);
+    page_pv8(A.o, smem_u32(st[i] + kF8V), bh0, bh1, bl0, bl1, masked, mlo, mhi, lane);
   }
 }
 
@@ -756,10 +746,10 @@ __device__ __forceinline__ int cta_of(long long u, long long U, long long G) {
 // so the rings hold twice as many pages and the bytes in flight stay the same.
 template <int F> struct Fmt;
 template <> struct Fmt<0> {
-  static constexpr int kStage = kStageBytes, kR = 3, kRL = 3, kAlign = 1024;
+  static constexpr int kStage = kStageBytes, kR = 3, kRL = 3, kAlign = 1024, kMinCtas = 2;
 };
 template <> struct Fmt<1> {
-  static constexpr int kStage = kF8Block, kR = 6, kRL = 6, kAlign = 128;
+  static constexpr int kStage = kF8Block, kR = 3, kRL = 6, kAlign = 128, kMinCtas = 3;
 };
 
 // Query fragments of either format.
@@ -1016,7 +1006,7 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 
 // ------------------------------------------------------------ full set: persistent grid
 template <int F>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, Fmt<F>::kMinCtas)
 attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const AttnParams p) {
   constexpr int kR = Fmt<F>::kR;
@@ -1616,7 +1606,7 @@ oda_status prepare_attention_kernel(int g, int n_sms, int* ctas) {
                                                                           kThreads, full_smem_bytes<1>(g)),
                              "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
     if (st != ODA_OK) return st;
-    occ = std::max(1, std::min(occ, 2));
+    occ = std::max(1, std::min(occ, f == 0 ? Fmt<0>::kMinCtas : Fmt<1>::kMinCtas));
     ctas[f] = n_sms * occ;
     // the combine keeps one weight per partial and head in the merge area
     if (ctas[f] > kW * kMergeStride) return set_error(ODA_ERR_UNSUPPORTED, "too many CTAs for the merge area");
