@@ -505,7 +505,7 @@ def run_backbone(args, local_rank):
         per = W + K
         total = per * (len(BB_RHO) + 2) + 8
         wl = wl0.replace(steps=total)
-        dec = OdaDecoder(wl, device=dev, capacity_steps=total)
+        dec = OdaDecoder(wl, device=dev, capacity_steps=total, bb_fused=not args.bb_separate)
         weight_bytes = dec.backbone_bytes()
         lm_bytes = wl.vocab * wl.D * 2
         head_bytes = __import__("workload.inputs", fromlist=["x"]).head_param_count(wl.D) * 4
@@ -856,6 +856,8 @@ def main():
     ap.add_argument("--backbone", action="store_true",
                     help="whole-model steps of the synthetic Qwen3-1.7B-shaped model (projections, "
                          "attention, head, retry, commit, LM head) at 4K..128K against always-full")
+    ap.add_argument("--bb-separate", action="store_true",
+                    help="--backbone: separate o_proj / MLP / QKV launches instead of the fused one")
     ap.add_argument("--backbone-ctx", default=None,
                     help="comma-separated contexts for --backbone (default 4K,16K,32K,64K,128K)")
     args = ap.parse_args()

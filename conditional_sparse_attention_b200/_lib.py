@@ -85,6 +85,9 @@ _SIGS = {
                    c_int32),
     "oda_bb_attn_out": ([c_void_p, _P(OdaBBLayer), c_void_p, c_void_p, c_void_p], c_int32),
     "oda_bb_mlp": ([c_void_p, _P(OdaBBLayer), c_void_p, c_void_p, c_void_p], c_int32),
+    "oda_bb_pack_weight": ([c_void_p, c_void_p, c_int32, c_int32, c_void_p, c_void_p], c_int32),
+    "oda_bb_post_attention": ([c_void_p, _P(OdaBBLayer), _P(OdaBBLayer), c_void_p, c_void_p, c_void_p,
+                               c_void_p, c_void_p, c_void_p, c_void_p], c_int32),
     "oda_bb_final_norm": ([c_void_p, c_void_p, c_void_p, c_void_p, c_void_p], c_int32),
     "oda_bb_lm_head": ([c_void_p, c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_void_p,
                         c_void_p], c_int32),

@@ -389,6 +389,19 @@ oda_status oda_bb_mlp(oda_ctx* ctx, const oda_bb_layer* layer, float* x, void* a
   return oda::launch_bb_mlp(ctx, layer, x, act, stream);
 }
 
+oda_status oda_bb_post_attention(oda_ctx* ctx, const oda_bb_layer* layer, const oda_bb_layer* next,
+                                 const float* o, float* x, void* act, void* q, void* k_new,
+                                 void* v_new, cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "bb_post_attention: ctx is NULL");
+  return oda::launch_bb_post(ctx, layer, next, o, x, act, q, k_new, v_new, stream);
+}
+
+oda_status oda_bb_pack_weight(oda_ctx* ctx, const void* src, int32_t rows, int32_t cols, void* dst,
+                              cudaStream_t stream) {
+  if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "bb_pack_weight: ctx is NULL");
+  return oda::launch_bb_pack_weight(ctx, src, rows, cols, dst, stream);
+}
+
 oda_status oda_bb_final_norm(oda_ctx* ctx, const float* gamma, const float* x, float* h,
                              cudaStream_t stream) {
   if (!ctx) return set_error(ODA_ERR_INVALID_ARG, "bb_final_norm: ctx is NULL");

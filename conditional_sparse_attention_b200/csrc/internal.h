@@ -120,6 +120,11 @@ oda_status launch_bb_qkv(oda_ctx* ctx, const oda_bb_layer* w, const float* x, vo
 oda_status launch_bb_attn_out(oda_ctx* ctx, const oda_bb_layer* w, const float* o, float* x, cudaStream_t s);
 oda_status launch_bb_mlp(oda_ctx* ctx, const oda_bb_layer* w, float* x, void* act, cudaStream_t s);
 oda_status launch_bb_begin(oda_ctx* ctx, const float* emb, float* x, cudaStream_t s);
+oda_status launch_bb_pack_weight(oda_ctx* ctx, const void* src, int32_t rows, int32_t cols, void* dst,
+                                 cudaStream_t s);
+oda_status launch_bb_post(oda_ctx* ctx, const oda_bb_layer* w, const oda_bb_layer* next,
+                          const float* o, float* x, void* act, void* q, void* k_new, void* v_new,
+                          cudaStream_t s);
 oda_status launch_bb_final_norm(oda_ctx* ctx, const float* gamma, const float* x, float* h, cudaStream_t s);
 oda_status launch_bb_lm_head(oda_ctx* ctx, const void* embed, int32_t vocab, const float* h,
                              float* logits, int32_t* token, float* next_emb, cudaStream_t s);

@@ -93,10 +93,12 @@ class OdaDecoder:
 
     def __init__(self, wl: Workload, device="cuda", capacity_steps: int = 0,
                  perturb_head: bool = False, head_params: dict = None, fill_cache: bool = True,
-                 overlap_layers: bool = True, deterministic: bool = False, kv_format: str = "bf16"):
+                 overlap_layers: bool = True, deterministic: bool = False, kv_format: str = "bf16",
+                 bb_fused: bool = True):
         if not torch.cuda.is_available():
             raise RuntimeError("OdaDecoder needs a CUDA device (the CUDA path has no fallback)")
         self.wl = wl
+        self.bb_fused = bb_fused
         dev = torch.device(device)
         if dev.index is None:
             dev = torch.device("cuda", torch.cuda.current_device())
@@ -192,14 +194,22 @@ class OdaDecoder:
         wl, dev = self.wl, self.device
         B, D, F, V, L = wl.B, wl.D, wl.ffn, wl.vocab, wl.L
         shapes = inputs.bb_shapes(wl)
+        fill_stream = torch.cuda.current_stream(dev)   # the device fills run on torch's stream
+
+        def packed(R, C, key, log2_scale):
+            """A seeded N(0,1) * 2^log2_scale matrix, generated row-major, stored packed."""
+            tmp = torch.empty((R, C), dtype=torch.bfloat16, device=dev)
+            wdev.fill_normal_bf16(tmp, key, 0, log2_scale)
+            out = torch.empty_like(tmp)
+            oda.oda_bb_pack_weight(self.ctx, tmp, out, fill_stream)
+            return out
+
         self.bb_w, self.bb_layers = [], []
         for a, layer in enumerate(wl.attn_layers):
             ws = {}
             for name in inputs.BB_TENSORS:
                 R, C = shapes[name]
-                t = torch.empty((R, C), dtype=torch.bfloat16, device=dev)
-                wdev.fill_normal_bf16(t, inputs.bb_weight_key(wl, layer, name), 0, inputs.bb_log2_scale(C))
-                ws[name] = t
+                ws[name] = packed(R, C, inputs.bb_weight_key(wl, layer, name), inputs.bb_log2_scale(C))
             ga, gm = inputs.bb_norms(wl, layer)
             ws["attn_norm"] = torch.from_numpy(ga).to(dev)
             ws["mlp_norm"] = torch.from_numpy(gm).to(dev)
@@ -207,8 +217,8 @@ class OdaDecoder:
             self.bb_layers.append(oda.bb_layer(ws["attn_norm"], ws["w_qkv"], ws["w_o"], ws["mlp_norm"],
                                                ws["w_gate"], ws["w_up"], ws["w_down"]))
         self.bb_final_norm = torch.from_numpy(inputs.bb_norms(wl, -1)[0]).to(dev)
-        self.bb_embed = torch.empty((V, D), dtype=torch.bfloat16, device=dev)
-        wdev.fill_normal_bf16(self.bb_embed, inputs.bb_embed_key(wl), 0, inputs.BB_EMBED_LOG2_SCALE)
+        self.bb_embed = packed(V, D, inputs.bb_embed_key(wl), inputs.BB_EMBED_LOG2_SCALE)
+        fill_stream.synchronize()
         self.bb_x = torch.zeros((2, B, D), dtype=torch.float32, device=dev)
         self.bb_act = torch.zeros((B, F), dtype=torch.bfloat16, device=dev)
         self.bb_logits = torch.zeros((B, V), dtype=torch.float32, device=dev)
@@ -264,18 +274,30 @@ class OdaDecoder:
         then the final norm gives h^br."""
         wl, ctx = self.wl, self.ctx
         x = self.bb_x[br]
+        n_attn = len(wl.attn_layers)
         oda.oda_bb_begin(ctx, self.emb, x, stream)
+        oda.oda_bb_qkv(ctx, self.bb_layers[0], x, self.bb_q[br, 0], self.bb_k[br, 0], self.bb_v[br, 0],
+                       stream)
         for a, layer in enumerate(wl.attn_layers):
             q, k, v = self.bb_q[br, a], self.bb_k[br, a], self.bb_v[br, a]
-            oda.oda_bb_qkv(ctx, self.bb_layers[a], x, q, k, v, stream)
             if br == LOCAL:
                 self._attend_local(ctx, self.layers[a], self.page_table, self.pos, q, k, v,
                                    self.o[br, layer], stream)
             else:
                 self._attend_full(ctx, self.layers[a], self.page_table, self.pos, flag, q, k, v,
                                   self.o[br, layer], stream)
-            oda.oda_bb_attn_out(ctx, self.bb_layers[a], self.o[br, layer], x, stream)
-            oda.oda_bb_mlp(ctx, self.bb_layers[a], x, self.bb_act, stream)
+            last = a + 1 == n_attn
+            if self.bb_fused:   # o_proj, the MLP and the next layer's QKV in one launch
+                nq = (None, None, None) if last else (self.bb_q[br, a + 1], self.bb_k[br, a + 1],
+                                                      self.bb_v[br, a + 1])
+                oda.oda_bb_post_attention(ctx, self.bb_layers[a], None if last else self.bb_layers[a + 1],
+                                          self.o[br, layer], x, self.bb_act, *nq, stream=stream)
+            else:
+                oda.oda_bb_attn_out(ctx, self.bb_layers[a], self.o[br, layer], x, stream)
+                oda.oda_bb_mlp(ctx, self.bb_layers[a], x, self.bb_act, stream)
+                if not last:
+                    oda.oda_bb_qkv(ctx, self.bb_layers[a + 1], x, self.bb_q[br, a + 1],
+                                   self.bb_k[br, a + 1], self.bb_v[br, a + 1], stream)
         oda.oda_bb_final_norm(ctx, self.bb_final_norm, x, self.h[br], stream)
 
     def _issue_backbone(self) -> None:

@@ -312,8 +312,25 @@ def oda_bb_attn_out(ctx, layer: OdaBBLayer, o, x, stream=None):
     check(_lib.load().oda_bb_attn_out(ctx.handle, ctypes.byref(layer), _p(o), _p(x), _s(stream)))
 
 
+def oda_bb_pack_weight(ctx, src, dst, stream=None):
+    """dst = src ([rows][cols] bf16, row-major) in the projections' packed layout."""
+    rows, cols = src.shape
+    if tuple(dst.shape) != (rows, cols) or src.element_size() != 2 or dst.element_size() != 2:
+        raise ValueError("bb_pack_weight: src and dst must be bf16 matrices of one shape")
+    check(_lib.load().oda_bb_pack_weight(ctx.handle, _p(src), rows, cols, _p(dst), _s(stream)))
+
+
 def oda_bb_mlp(ctx, layer: OdaBBLayer, x, act, stream=None):
     check(_lib.load().oda_bb_mlp(ctx.handle, ctypes.byref(layer), _p(x), _p(act), _s(stream)))
+
+
+def oda_bb_post_attention(ctx, layer: OdaBBLayer, next_layer, o, x, act, q=None, k_new=None, v_new=None,
+                          stream=None):
+    """attn_out(layer) + mlp(layer) + qkv(next_layer) as one cooperative launch; next_layer None
+    stops after the MLP."""
+    nxt = ctypes.byref(next_layer) if next_layer is not None else None
+    check(_lib.load().oda_bb_post_attention(ctx.handle, ctypes.byref(layer), nxt, _p(o), _p(x), _p(act),
+                                            _p(q), _p(k_new), _p(v_new), _s(stream)))
 
 
 def oda_bb_final_norm(ctx, gamma, x, h, stream=None):

@@ -37,6 +37,23 @@ def _bits_t(a):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
 
 
+def packed_index(rows, cols):
+    """Element offset of W[n][k] in the packed layout, as include/oda_backbone.h defines it."""
+    n = np.arange(rows)[:, None]
+    k = np.arange(cols)[None, :]
+    return (((n // 16) * (cols // 512) + k // 512) * 8192 + (n % 16) * 512
+            + (((k % 512) // 8) ^ (n % 8)) * 8 + k % 8)
+
+
+def _packed_t(ctx, a):
+    """Row-major bf16 bits (numpy) -> a packed device matrix (via oda_bb_pack_weight)."""
+    from conditional_sparse_attention_b200 import oda
+    src = _bits_t(a)
+    dst = torch.empty_like(src)
+    oda.oda_bb_pack_weight(ctx, src, dst)
+    return dst
+
+
 def bf16_close(got_bits, ref_bits, frac=5e-3):
     g, r = bf16_to_f64(got_bits), bf16_to_f64(ref_bits)
     diff = g != r
@@ -61,12 +78,12 @@ class Layer:
         self.wl = wl
         self.w = {n: inputs.bb_weight(wl, 0, n) for n in inputs.BB_TENSORS}
         self.ga, self.gm = inputs.bb_norms(wl, 0)
-        d = {n: _bits_t(v) for n, v in self.w.items()}
+        self.ctx = oda.oda_create(oda.make_config(wl.B, wl.Hq, wl.Hkv, 8, max(512, wl.D)))
+        d = {n: _packed_t(self.ctx, v) for n, v in self.w.items()}
         self.d = d
         self.tga, self.tgm = torch.from_numpy(self.ga).cuda(), torch.from_numpy(self.gm).cuda()
         self.layer = oda.bb_layer(self.tga, d["w_qkv"], d["w_o"], self.tgm, d["w_gate"], d["w_up"],
                                   d["w_down"])
-        self.ctx = oda.oda_create(oda.make_config(wl.B, wl.Hq, wl.Hkv, 8, max(512, wl.D)))
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,F", [(1, 4, 2, 1024), (3, 4, 2, 1536), (8, 8, 2, 512),
@@ -109,9 +126,12 @@ def test_lm_head_matches_oracle(B, V):
     D = wl.D
     ctx = oda.oda_create(oda.make_config(B, wl.Hq, wl.Hkv, 8, D))
     E = inputs.bb_embed(wl)
-    tE = torch.empty((V, D), dtype=torch.int16, device="cuda")
-    wdev.fill_normal_bf16(tE, inputs.bb_embed_key(wl), 0, inputs.BB_EMBED_LOG2_SCALE)
-    assert np.array_equal(tE.cpu().numpy().view(np.uint16), E)
+    rowmajor = torch.empty((V, D), dtype=torch.int16, device="cuda")
+    wdev.fill_normal_bf16(rowmajor, inputs.bb_embed_key(wl), 0, inputs.BB_EMBED_LOG2_SCALE)
+    assert np.array_equal(rowmajor.cpu().numpy().view(np.uint16), E)
+    tE = torch.empty_like(rowmajor)
+    oda.oda_bb_pack_weight(ctx, rowmajor, tE)
+    del rowmajor
     rng = np.random.default_rng(V)
     h = rng.normal(0, 1, (B, D)).astype(np.float32)
     logits = torch.zeros((B, V), device="cuda")
@@ -223,3 +243,107 @@ def test_backbone_trajectory_matches_oracle(kv, graph):
                 assert np.array_equal(logical_cache(kp, pt, b, n), own_k[a][b])
                 assert np.array_equal(logical_cache(vp, pt, b, n), own_v[a][b])
     dec.close()
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,F,with_next", [(1, 4, 2, 1024, True), (3, 4, 2, 1536, True),
+                                                  (8, 8, 2, 512, False), (4, 16, 8, 6144, True),
+                                                  (8, 16, 8, 6144, False)])
+def test_post_attention_equals_separate_calls(B, Hq, Hkv, F, with_next):
+    """oda_bb_post_attention does the arithmetic of oda_bb_attn_out, oda_bb_mlp and oda_bb_qkv (of
+    the next layer) in the same order, so its outputs equal theirs bit for bit; the separate calls
+    are the ones checked against the oracle above."""
+    from conditional_sparse_attention_b200 import oda
+    wl = _wl(B, Hq, Hkv, F).replace(n_layers=2, attn_layers=(0, 1))
+    D = wl.D
+    ctx = oda.oda_create(oda.make_config(B, Hq, Hkv, 8, D))
+    layers, keep = [], []
+    for a in range(2):
+        w = {}
+        for n, (R, C) in inputs.bb_shapes(wl).items():
+            rowmajor = torch.empty((R, C), dtype=torch.bfloat16, device="cuda")
+            wdev.fill_normal_bf16(rowmajor, inputs.bb_weight_key(wl, a, n), 0, inputs.bb_log2_scale(C))
+            w[n] = torch.empty_like(rowmajor)
+            oda.oda_bb_pack_weight(ctx, rowmajor, w[n])
+        ga, gm = (torch.from_numpy(g).cuda() for g in inputs.bb_norms(wl, a))
+        keep += [w, ga, gm]
+        layers.append(oda.bb_layer(ga, w["w_qkv"], w["w_o"], gm, w["w_gate"], w["w_up"], w["w_down"]))
+    rng = np.random.default_rng(F + B)
+    x0 = torch.from_numpy(rng.normal(0, 2, (B, D)).astype(np.float32)).cuda()
+    o = torch.from_numpy(rng.normal(0, 1, (B, D)).astype(np.float32)).cuda()
+
+    def outputs():
+        return (torch.zeros((B, Hq, 128), dtype=torch.int16, device="cuda"),
+                torch.zeros((B, Hkv, 128), dtype=torch.int16, device="cuda"),
+                torch.zeros((B, Hkv, 128), dtype=torch.int16, device="cuda"),
+                torch.zeros((B, F), dtype=torch.bfloat16, device="cuda"))
+
+    x1 = x0.clone()
+    q1, k1, v1, act1 = outputs()
+    oda.oda_bb_attn_out(ctx, layers[0], o, x1)
+    oda.oda_bb_mlp(ctx, layers[0], x1, act1)
+    if with_next:
+        oda.oda_bb_qkv(ctx, layers[1], x1, q1, k1, v1)
+    for rep in range(3):   # repeated launches: the barrier counters return to zero
+        x2 = x0.clone()
+        q2, k2, v2, act2 = outputs()
+        if with_next:
+            oda.oda_bb_post_attention(ctx, layers[0], layers[1], o, x2, act2, q2, k2, v2)
+        else:
+            oda.oda_bb_post_attention(ctx, layers[0], None, o, x2, act2)
+        torch.cuda.synchronize()
+        assert oda.oda_get_error(ctx) == 0
+        assert torch.equal(x1, x2), rep
+        assert torch.equal(act1, act2), rep
+        assert torch.equal(q1, q2) and torch.equal(k1, k2) and torch.equal(v1, v2), rep
+    with pytest.raises(oda.OdaError):   # the next layer's outputs are required
+        oda.oda_bb_post_attention(ctx, layers[0], layers[1], o, x2, act2)
+    ctx.close()
+
+
+@pytest.mark.parametrize("graph", [True, False])
+def test_backbone_fused_step_equals_separate_launches(graph):
+    """A whole-model trajectory with the fused post-attention launch equals the one with the
+    separate projection launches, bit for bit (same kernels' arithmetic, fewer launches)."""
+    from conditional_sparse_attention_b200.engine import OdaDecoder
+    wl = _small_model("bf16", seed=2011).replace(n_layers=3, attn_layers=(0, 1, 2))
+    runs = []
+    for fused in (True, False):
+        dec = OdaDecoder(wl, perturb_head=True, bb_fused=fused)
+        if graph:
+            dec.capture()
+        out = []
+        for s in range(wl.steps):
+            dec.step(dec.make_step_buffer(s))
+            dec.synchronize()
+            out.append((dec.token.cpu().clone(), dec.h_prev.cpu().clone(), dec.o.cpu().clone(),
+                        dec.flag.cpu().clone()))
+        assert dec.device_error() == 0
+        runs.append(out)
+        dec.close()
+    for s, (a, b) in enumerate(zip(*runs)):
+        for ta, tb in zip(a, b):
+            assert torch.equal(ta, tb), s
+
+
+@pytest.mark.parametrize("rows,cols", [(16, 512), (48, 1536), (4096, 2048), (2048, 6144)])
+def test_pack_weight_layout(rows, cols):
+    """oda_bb_pack_weight moves every element to the offset the header's formula gives, bit for
+    bit; bad shapes, aliasing and misalignment are rejected."""
+    from conditional_sparse_attention_b200 import oda
+    ctx = oda.oda_create(oda.make_config(1, 4, 2, 8, 512))
+    rng = np.random.default_rng(rows + cols)
+    a = rng.integers(0, 2**16, (rows, cols), dtype=np.uint16)
+    got = _packed_t(ctx, a).cpu().numpy().view(np.uint16).reshape(-1)
+    want = np.empty(rows * cols, dtype=np.uint16)
+    want[packed_index(rows, cols).reshape(-1)] = a.reshape(-1)
+    assert np.array_equal(got, want)
+    t = torch.zeros((32, 1024), dtype=torch.bfloat16, device="cuda")
+    for src, dst in [(t[:24], torch.zeros((24, 1024), dtype=torch.bfloat16, device="cuda")),
+                     (t[:, :768], torch.zeros((32, 768), dtype=torch.bfloat16, device="cuda")),
+                     (t, t)]:
+        with pytest.raises(oda.OdaError):
+            oda.oda_bb_pack_weight(ctx, src.contiguous() if src is not t else src, dst)
+    flat = torch.zeros(32 * 1024 + 8, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(oda.OdaError):   # 2 bytes off 16-byte alignment
+        oda.oda_bb_pack_weight(ctx, flat[1:1 + 32 * 1024].view(32, 1024), torch.zeros_like(t))
+    ctx.close()
