@@ -797,9 +797,11 @@ __device__ __forceinline__ void pages_compute(WarpAcc& A, const QFrag<F>& Q, uin
 
 // ---------------------------------------------------------------- local set: clusters
 // Cluster of p.cluster CTAs per (b, h); CTA `rank` takes the contiguous share
-// [rank*nv/C, (rank+1)*nv/C) of the visited pages; warps take every kWL-th page of it.  After a
-// cluster barrier each rank finishes its share of the g*128 outputs from all ranks' partials
-// (read through distributed shared memory).
+// [rank*nv/C, (rank+1)*nv/C) of the visited pages; warps take every kWL-th page of it.  Each
+// rank merges its warps' partials and writes the result straight into rank 0's inbox (distributed
+// shared memory), then arrives on rank 0's inbox barrier and exits; rank 0 waits for the C - 1
+// arrivals and finishes all g*128 outputs with the staged token.  Nothing but rank 0 waits on
+// another CTA after the pages, and no CTA reads another's shared memory.
 template <int F>
 __global__ void __launch_bounds__(kThreadsL, 1)
 attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -813,9 +815,12 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   // the merge areas reuse the stages: they are written only after every copy has landed
   float* merge_o = reinterpret_cast<float*>(stages);                   // [W][g][132]
   float* merge_ml = merge_o + kWL * g * kMergeStride;                  // [W][8][2]
-  float* cpart_o = merge_ml + kWL * 16;                                // [g][128] CTA partial
-  float* cpart_ml = cpart_o + g * 128;                                // [g][2]
+  // rank 0's inbox (its own region, past the stages: other ranks write it while rank 0 may
+  // still stream pages): the ranks' CTA partials o [C][g][128], then (m, l) [C][g][2]
+  float* inbox_o = reinterpret_cast<float*>(stages + kWL * kRL * kStg);
+  float* inbox_ml = inbox_o + (size_t)p.cluster * g * 128;
   __shared__ __align__(8) uint64_t bars[kWL * kRL];
+  __shared__ __align__(8) uint64_t inbox_bar;
 
   cg::cluster_group cluster = cg::this_cluster();
   const int C = p.cluster;
@@ -826,6 +831,7 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   if (tid == 0) {
 #pragma unroll
     for (int i = 0; i < kWL * kRL; ++i) mbar_init(&bars[i], 1);
+    mbar_init(&inbox_bar, C > 1 ? C - 1 : 1);
     fence_mbar_init();
     if (F == 0) {
       prefetch_tensormap(&tmA);
@@ -842,6 +848,9 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   uint8_t* my_stages = stages + warp * kRL * kStg;
   uint64_t* my_bars = bars + warp * kRL;
   __syncthreads();
+  // rank 0's inbox barrier is initialised before any rank arrives on it: every thread arrives
+  // here and waits (long after) before the merge
+  cluster_arrive();
 
   // lane k holds the physical page of this warp's (pt_base + k)-th page
   int pt_phys = -1, pt_base = -64;
@@ -890,8 +899,11 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       sq[i][1] = qrow[lane + 32];
     }
   }
-  const int o_lo0 = (int)((long long)rank * (g * 128) / C);
-  const float v_first = staged_value(p, b, h, (o_lo0 + tid) & 127);
+  // rank 0 finishes outputs tid, tid + 256, ... (at most 4 for g <= 8): their staged values now
+  float v_staged[(8 * 128) / kThreadsL];
+#pragma unroll
+  for (int i = 0; i < (8 * 128) / kThreadsL; ++i)
+    v_staged[i] = (rank == 0 && tid + i * kThreadsL < g * 128) ? staged_value(p, b, h, (tid + i * kThreadsL) & 127) : 0.f;
   WarpAcc A;
   acc_init(A);
   const int r = lane >> 2;
@@ -954,23 +966,44 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   __syncthreads();
   warp_flush(A, merge_o + warp * g * kMergeStride, merge_ml + warp * 16, g, lane);
   __syncthreads();
+  cluster_wait();
+  // this CTA's merged partial, into slot `rank` of rank 0's inbox (plain stores through the
+  // cluster window for rank != 0)
+  float* dst_o = rank == 0 ? inbox_o : cluster.map_shared_rank(inbox_o, 0);
+  float* dst_ml = rank == 0 ? inbox_ml : cluster.map_shared_rank(inbox_ml, 0);
   for (int idx = tid; idx < g * 128; idx += kThreadsL) {
     const int n = idx >> 7, d = idx & 127;
     float M, L, O;
     cta_merge<kWL>(merge_o, merge_ml, g, n, d, M, L, O);
-    cpart_o[n * 128 + d] = O;
+    dst_o[((size_t)rank * g + n) * 128 + d] = O;
     if (d == 0) {
-      cpart_ml[n * 2] = M;
-      cpart_ml[n * 2 + 1] = L;
+      dst_ml[((size_t)rank * g + n) * 2] = M;
+      dst_ml[((size_t)rank * g + n) * 2 + 1] = L;
     }
   }
-  cluster.sync();
+  __syncthreads();
+  if (rank != 0) {
+    // the barrier above orders every thread's inbox writes before this release
+    if (tid == 0) mbar_arrive_remote(mapa_shared(smem_u32(&inbox_bar), 0));
+    return;
+  }
+  if (C > 1) {
+    // bounded: every other rank arrives after its own bounded page waits
+    bool ok = mbar_try_wait_cluster(&inbox_bar, 0u);
+    if (!ok) {
+      const uint64_t t0 = global_timer_ns();
+      while (!(ok = mbar_try_wait_cluster(&inbox_bar, 0u)))
+        if (global_timer_ns() - t0 > 5 * kWaitNs) break;
+      if (!ok && tid == 0) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
+    }
+  }
   if (ge.active) {
-    // merge the cluster's partials through distributed shared memory plus the staged token;
-    // the g*128 outputs are shared out among the ranks, one output per thread
+    // the cluster's partials plus the staged token, in rank order: g*128 outputs
     const int n_out = g * 128;
-    const int o_lo = (int)((long long)rank * n_out / C), o_hi = (int)((long long)(rank + 1) * n_out / C);
-    for (int idx = o_lo + tid; idx < o_hi; idx += kThreadsL) {
+#pragma unroll
+    for (int i = 0; i < (8 * 128) / kThreadsL; ++i) {
+      const int idx = tid + i * kThreadsL;
+      if (idx >= n_out) break;
       const int n = idx >> 7, d = idx & 127;
       const float snew = s_snew[n];
       float Mr[kMaxCluster], Lr[kMaxCluster], Or[kMaxCluster];
@@ -978,16 +1011,14 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 #pragma unroll
       for (int q = 0; q < kMaxCluster; ++q) {
         if (q < C) {
-          const float* rml = cluster.map_shared_rank(cpart_ml, q);
-          const float* ro = cluster.map_shared_rank(cpart_o, q);
-          Mr[q] = rml[n * 2];
-          Lr[q] = rml[n * 2 + 1];
-          Or[q] = ro[n * 128 + d];
+          Mr[q] = inbox_ml[((size_t)q * g + n) * 2];
+          Lr[q] = inbox_ml[((size_t)q * g + n) * 2 + 1];
+          Or[q] = inbox_o[((size_t)q * g + n) * 128 + d];
           M = fmaxf(M, Mr[q]);
         }
       }
       const float wn = exp2f(snew - M);
-      const float vd = (idx == o_lo + tid) ? v_first : staged_value(p, b, h, d);
+      const float vd = v_staged[i];
       float L = wn, O = wn * vd;
 #pragma unroll
       for (int q = 0; q < kMaxCluster; ++q) {
@@ -1000,8 +1031,6 @@ attn_local_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       p.out[((size_t)b * p.Hq + h * g + n) * 128 + d] = O / L;
     }
   }
-  // keep every CTA's shared memory alive until the other ranks have read it
-  cluster.sync();
 }
 
 // ------------------------------------------------------------ full set: persistent grid
@@ -1572,7 +1601,13 @@ int attention_smem_bytes(int g) { return full_smem_bytes<0>(g); }
 // local set: the merge areas live in the stages (kWL * g * 132 + kWL * 16 + g * 130 floats,
 // 38 KB at g = 8, within the ~200 KB of stages)
 template <int F>
-int local_smem_bytes() { return Fmt<F>::kAlign + kWL * Fmt<F>::kRL * Fmt<F>::kStage; }
+int local_smem_bytes(int C, int g) {
+  return Fmt<F>::kAlign + kWL * Fmt<F>::kRL * Fmt<F>::kStage + C * g * 130 * (int)sizeof(float);
+}
+
+// Dynamic shared memory the local kernels may use (the device's opt-in limit less their static
+// shared memory), set by prepare_attention_kernel; it bounds the cluster size through the inbox.
+int g_local_dyn_max[2] = {0, 0};
 
 // Sets the shared-memory limits of both kernels in both page formats and returns the
 // persistent full-set grid size for group size g per format (ctas[0] bf16, ctas[1] fp8).  The
@@ -1588,14 +1623,24 @@ oda_status prepare_attention_kernel(int g, int n_sms, int* ctas) {
     st = check_cuda(cudaFuncSetAttribute(attn_full_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          full_smem_bytes<1>(8)),
                     "cudaFuncSetAttribute(full attention, fp8)");
+  int dev = 0, optin = 0;
+  if (st == ODA_OK) st = check_cuda(cudaGetDevice(&dev), "cudaGetDevice");
   if (st == ODA_OK)
-    st = check_cuda(cudaFuncSetAttribute(attn_local_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         local_smem_bytes<0>()),
+    st = check_cuda(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev),
+                    "cudaDeviceGetAttribute");
+  const void* local_k[2] = {reinterpret_cast<const void*>(attn_local_kernel<0>),
+                            reinterpret_cast<const void*>(attn_local_kernel<1>)};
+  for (int f = 0; f < 2 && st == ODA_OK; ++f) {
+    cudaFuncAttributes fa;
+    st = check_cuda(cudaFuncGetAttributes(&fa, local_k[f]), "cudaFuncGetAttributes(local attention)");
+    if (st != ODA_OK) break;
+    g_local_dyn_max[f] = optin - (int)fa.sharedSizeBytes;
+    const int base = f == 0 ? local_smem_bytes<0>(1, 1) : local_smem_bytes<1>(1, 1);
+    if (g_local_dyn_max[f] < base) return set_error(ODA_ERR_UNSUPPORTED, "local attention: shared memory too small");
+    st = check_cuda(cudaFuncSetAttribute(local_k[f], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         g_local_dyn_max[f]),
                     "cudaFuncSetAttribute(local attention)");
-  if (st == ODA_OK)
-    st = check_cuda(cudaFuncSetAttribute(attn_local_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         local_smem_bytes<1>()),
-                    "cudaFuncSetAttribute(local attention, fp8)");
+  }
   if (st != ODA_OK) return st;
   for (int f = 0; f < 2; ++f) {
     int occ = 0;
@@ -1671,13 +1716,18 @@ oda_status launch_attention(oda_ctx* ctx, const KvPool& pool, const int32_t* pag
   // an SM's shared memory), at most 8 per (b, h)
   const int pairs = cf.batch * cf.n_kv_heads;
   p.cluster = std::max(1, std::min(kMaxCluster, ctx->n_sms / pairs));
+  // rank 0's inbox holds every rank's partial: a smaller cluster where it would not fit
+  while (p.cluster > 1 && (F == 0 ? local_smem_bytes<0>(p.cluster, ctx->g) : local_smem_bytes<1>(p.cluster, ctx->g)) >
+                              g_local_dyn_max[F])
+    --p.cluster;
 
   // Consecutive attention launches of one context overlap when the context allows it: the
   // later one may start (and prefetch its pages) while the earlier one finishes; it waits
   // before reading q or writing.
   cudaLaunchConfig_t lc = {};
   lc.blockDim = dim3(mode == 0 ? kThreadsL : kThreads);
-  lc.dynamicSmemBytes = mode == 0 ? (F == 0 ? local_smem_bytes<0>() : local_smem_bytes<1>())
+  lc.dynamicSmemBytes = mode == 0 ? (F == 0 ? local_smem_bytes<0>(p.cluster, ctx->g)
+                                              : local_smem_bytes<1>(p.cluster, ctx->g))
                                   : (F == 0 ? full_smem_bytes<0>(ctx->g) : full_smem_bytes<1>(ctx->g));
   lc.stream = stream;
   cudaLaunchAttribute attr[2];
