@@ -33,7 +33,7 @@ METRIC = "ODA decode-attn steps/s + % of HBM peak, 128K ctx, 12.5% recall, 1 B20
 # 32K-context, 2-layer profiling workload (4 flagged sequences x 32768 cached tokens); the bench
 # scales it to its own launches by cached tokens processed.  Valid only for the kernel source it
 # was taken from (first 16 hex digits of the file's SHA-256).
-NCU_FULL_KERNEL_TRAFFIC = {"attention_cu_sha256": "9a82954d8deaa4c9", "bytes": 541364992,
+NCU_FULL_KERNEL_TRAFFIC = {"attention_cu_sha256": "0529ba2eae03a27d", "bytes": 540988416,
                            "cached_tokens": 4 * 32768}
 UNIT = "steps/s"
 FALLBACK_HBM_GBS = 6650.0
@@ -362,7 +362,8 @@ def run_kernel_only(args, wl, local_rank):
         # whole-model steps of the synthetic backbone, issued kernel by kernel (a profiler lists
         # every launch; graphs with conditional nodes hide theirs)
         from workload import configs
-        wl = configs.bb_qwen3_1p7b(ctx=4096)
+        if not wl.backbone:   # default: the whole 28-layer model at 4K context
+            wl = configs.bb_qwen3_1p7b(ctx=4096)
         dec = OdaDecoder(wl, device=dev, capacity_steps=args.kernel_reps + 2)
         for r in range(args.kernel_reps):
             dec.step(dec.make_step_buffer(r))

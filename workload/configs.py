@@ -166,8 +166,14 @@ def cfg2_ctx32k_l2() -> Workload:
                           ctx=(32768,) * 4, steps=8)
 
 
+def bb_qwen3_1p7b_l2() -> Workload:
+    """Profiling case of the synthetic-backbone step: the same layer shapes, 2 layers, 4K
+    context (under 1 GB on the device, so a many-pass profiler capture stays small)."""
+    return bb_qwen3_1p7b(ctx=4096).replace(name="bb_qwen3_1p7b_ctx4k_l2", n_layers=2, attn_layers=(0, 1))
+
+
 ALL = {"cfg0": cfg0, "cfg1": cfg1, "cfg2": cfg2, "cfg3": cfg3, "cfg4": cfg4,
-       "cfg2_ctx32k_l2": cfg2_ctx32k_l2, "bb": bb_qwen3_1p7b}
+       "cfg2_ctx32k_l2": cfg2_ctx32k_l2, "bb": bb_qwen3_1p7b, "bb_l2": bb_qwen3_1p7b_l2}
 
 
 def get(name: str) -> Workload:
