@@ -78,6 +78,22 @@ def test_local_matches_oracle(Hq, Hkv):
         assert ok, f"b={b} ctx={s.wl.ctx[b]} max_abs={ma:.3g} rel_l2={rel:.3g}"
 
 
+@pytest.mark.parametrize("ctx,Hq,Hkv", [([40000], 16, 8), ([65536], 32, 8), ([5000, 70000], 8, 4),
+                                        ([3000], 8, 1), ([2052, 17], 16, 4)])
+def test_local_small_batches_large_clusters(ctx, Hq, Hkv):
+    """Few (sequence, KV head) pairs give the largest clusters (8 CTAs, each rank's partial pushed
+    into rank 0's inbox); the cluster size is cut where the inbox would not fit (g = 8)."""
+    s = Setup(_wl(ctx, Hq, Hkv, seed=80))
+    out = torch.full((s.wl.B, Hq, 128), 7.0, device="cuda")
+    s.oda.oda_attend_local(s.ctx, s.layer, s.pt, s.pos, s.q, s.kn, s.vn, out)
+    torch.cuda.synchronize()
+    assert s.oda.oda_get_error(s.ctx) == 0
+    got = out.cpu().numpy()
+    for b in range(s.wl.B):
+        ok, ma, rel = attn_close(got[b], s.oracle(b, 0))
+        assert ok, f"b={b} ctx={ctx[b]} max_abs={ma:.3g} rel_l2={rel:.3g}"
+
+
 @pytest.mark.parametrize("Hq,Hkv", [(16, 8), (32, 8), (8, 1), (4, 4), (24, 8)])
 def test_full_if_matches_oracle_and_skips_unflagged(Hq, Hkv):
     ctx = [0, 17, 2052, 2053, 2064, 4096, 5000, 9000, 16, 3333]
