@@ -667,7 +667,7 @@ oda_status launch_proj(oda_ctx* ctx, const Phase* ph, int n, cudaStream_t s) {
   lc.blockDim = dim3(kGThreads);
   lc.dynamicSmemBytes = smem;
   lc.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   if (n == 1) {
     lc.gridDim = dim3(std::min(n_tiles, ctx->n_sms));
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -689,6 +689,15 @@ oda_status launch_proj(oda_ctx* ctx, const Phase* ph, int n, cudaStream_t s) {
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
     lc.numAttrs = 1;
+    if (cf.overlap_layers) {
+      // the producers stream weights (which no earlier kernel writes) while the previous
+      // kernel finishes; the consumers wait for it before reading any input.  CTAs that find
+      // no free SM yet are placed as the previous kernel's CTAs leave (they wait on nothing of
+      // this launch), so all of them become resident before any grid barrier can complete.
+      attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[1].val.programmaticStreamSerializationAllowed = 1;
+      lc.numAttrs = 2;
+    }
   }
   lc.attrs = attr;
   oda_status st = check_cuda(cudaLaunchKernelEx(&lc, bb_proj_kernel, p), "backbone projection launch");
