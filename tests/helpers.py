@@ -76,3 +76,13 @@ def logical_cache8(pool: np.ndarray, page_table: np.ndarray, b: int, n_tokens: i
             K[tok, h] = table[kc[j]] * sk[j]
             V[tok, h] = table[vc[j]] * sv[j]
     return K, V
+
+
+def packed_index(rows, cols):
+    """Element offset of W[n][k] in the projections' packed layout, written out from the formula
+    in include/oda_backbone.h (16 x 512 blocks, tile-major; 16-byte chunk j of row r at slot
+    j ^ (r mod 8))."""
+    n = np.arange(rows)[:, None]
+    k = np.arange(cols)[None, :]
+    return (((n // 16) * (cols // 512) + k // 512) * 8192 + (n % 16) * 512
+            + (((k % 512) // 8) ^ (n % 8)) * 8 + k % 8)

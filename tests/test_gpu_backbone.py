@@ -17,7 +17,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import TIE_BAND, attn_close, build_all, logical_cache, score_close
+from helpers import TIE_BAND, attn_close, build_all, logical_cache, packed_index, score_close
 from oracle import backbone as BB
 from oracle import step as OS
 from oracle.attention import bf16_to_f64
@@ -35,14 +35,6 @@ def _build():
 
 def _bits_t(a):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
-
-
-def packed_index(rows, cols):
-    """Element offset of W[n][k] in the packed layout, as include/oda_backbone.h defines it."""
-    n = np.arange(rows)[:, None]
-    k = np.arange(cols)[None, :]
-    return (((n // 16) * (cols // 512) + k // 512) * 8192 + (n % 16) * 512
-            + (((k % 512) // 8) ^ (n % 8)) * 8 + k % 8)
 
 
 def _packed_t(ctx, a):
