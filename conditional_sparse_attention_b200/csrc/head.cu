@@ -521,14 +521,6 @@ __device__ __forceinline__ float butterfly32(float (&v)[32], int lane) {
   return v[0];
 }
 
-// Pulls every weight segment of the CTA's part of a phase toward L2 (lanes share the work).
-__device__ __forceinline__ void prefetch_phase(const FusedParams& p, const Own& o, int lane) {
-  const int total = o.nchunk * o.nseg;
-  for (int i = lane; i < total; i += 32) {
-    const int ch = i / o.nseg, r = i - ch * o.nseg;
-    prefetch_l2_bulk(seg_ptr(p, o, ch, r), kSegBytes);
-  }
-}
 
 // This warp's 128-column slice of K-chunk ch of the phase input, lane l holding columns
 // 4*col4 .. 4*col4+3 of the chunk, for the BT sequences of the tile (zeros beyond B).  Tower:
@@ -736,10 +728,10 @@ __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedPar
   if (warp == kFC) {
     // ---- producer.  First the tower input rows x_i[b] of this CTA's tower (they may come from
     // the previous kernel), then every weight segment of every phase in the order the consumers
-    // take them.  When the producer reaches a phase (its ring is then a few stages ahead of the
-    // consumers, who may still be finishing the previous phase or waiting at the barrier), it
-    // first pulls all of the phase's segments toward L2, so HBM streams at full rate beyond the
-    // ring's depth.
+    // take them, running up to the ring's depth ahead of them (into the next phase while they
+    // finish one or wait at a barrier).  No L2 prefetch of a whole phase ahead of the ring: the
+    // copy engine takes requests in order, so such prefetches delay the ring's own copies (with
+    // L2 flushed between scores, 55.5 us per score with them, 51.5 without).
     grid_dependency_wait();
     const Own o0 = own_rows(0, c, G, p.D);
     if (lane == 0) mbar_arrive_expect_tx(&src_bar, (uint32_t)(B * p.D * sizeof(float)));
@@ -750,7 +742,6 @@ __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedPar
     int k = 0;
     for (int ph = 0; ph < 6; ++ph) {
       const Own o = own_rows(ph, c, G, p.D);
-      prefetch_phase(p, o, lane);
       const int ngrp = (o.nseg + kFC - 1) / kFC;
       for (int ch = 0; ch < o.nchunk; ++ch)
         for (int g = 0; g < ngrp; ++g, ++k) {
