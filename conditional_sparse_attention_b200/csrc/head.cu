@@ -455,6 +455,7 @@ struct FusedParams {
   int32_t* cnt;           // [0] grid-barrier arrivals, [1] finished CTAs; both back to 0 at exit
   int32_t* err;
   int B, D, ring;
+  int any_or;             // a later slice of a larger batch: OR into *any_flag instead of setting it
   float theta;
 };
 
@@ -834,7 +835,8 @@ __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedPar
                    &s_any, lane);
   consumer_sync();
   if (tid == 0) {
-    *p.any_flag = s_any;
+    if (!p.any_or) *p.any_flag = s_any;
+    else if (s_any) *p.any_flag = 1;   // the slices run in stream order
     p.cnt[0] = 0;
     p.cnt[1] = 0;
   }
@@ -965,7 +967,12 @@ oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const flo
   for (const void* q : mats)
     if (reinterpret_cast<uintptr_t>(q) & 15)
       return set_error(ODA_ERR_INVALID_ARG, "recall_score: matrices and inputs must be 16-byte aligned");
-  const FusedPlan pl = fused_plan(ctx->cfg.batch, ctx->cfg.head_in_dim, ctx->n_sms);
+  const int B = ctx->cfg.batch, D = ctx->cfg.head_in_dim;
+  // The fused kernel takes up to 8 sequences; a larger batch runs it once per slice of 8 (each
+  // slice streams the weights again, still far fewer round trips than the six phase launches),
+  // when a full slice fits its plan.
+  const int slice = std::min(B, kBTMax);
+  const FusedPlan pl = fused_plan(slice, D, ctx->n_sms);
   int per_sm = 0;
   if (pl.bt) {
     const void* kern = pl.bt == 4 ? reinterpret_cast<const void*>(head_fused_kernel<4>)
@@ -975,38 +982,46 @@ oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const flo
     if (st != ODA_OK) return st;
   }
   if (pl.bt && per_sm >= 1) {
-    // one CTA per SM, all resident at once (cooperative launch): the grid barrier needs that
-    FusedParams f;
-    f.w = *w;
-    f.x[0] = h_prev;
-    f.x[1] = emb;
-    f.x[2] = h_loc;
-    f.sched = sched;
-    f.score = score;
-    f.flag = flag;
-    f.any_flag = any_flag;
-    f.u = ctx->head_u;
-    f.f = ctx->head_f;
-    f.act = ctx->head_act;
-    f.cnt = ctx->head_cnt;
-    f.err = ctx->err;
-    f.B = ctx->cfg.batch;
-    f.D = ctx->cfg.head_in_dim;
-    f.ring = pl.ring;
-    f.theta = ctx->cfg.theta;
-    cudaLaunchConfig_t lc = {};
-    lc.gridDim = dim3(ctx->n_sms);
-    lc.blockDim = dim3(kFThreads);
-    lc.dynamicSmemBytes = pl.smem;
-    lc.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    lc.attrs = attr;
-    lc.numAttrs = 1;
-    return check_cuda(pl.bt == 4 ? cudaLaunchKernelEx(&lc, head_fused_kernel<4>, f)
-                                 : cudaLaunchKernelEx(&lc, head_fused_kernel<8>, f),
-                      "recall head launch");
+    for (int b0 = 0; b0 < B; b0 += kBTMax) {
+      const int nb = std::min(kBTMax, B - b0);
+      const FusedPlan ps = nb == slice ? pl : fused_plan(nb, D, ctx->n_sms);
+      if (!ps.bt) return set_error(ODA_ERR_UNSUPPORTED, "recall_score: no fused plan for a slice of %d", nb);
+      // one CTA per SM, all resident at once (cooperative launch): the grid barrier needs that
+      FusedParams f;
+      f.w = *w;
+      f.x[0] = h_prev + (size_t)b0 * D;
+      f.x[1] = emb + (size_t)b0 * D;
+      f.x[2] = h_loc + (size_t)b0 * D;
+      f.sched = sched ? sched + b0 : nullptr;
+      f.score = score + b0;
+      f.flag = flag + b0;
+      f.any_flag = any_flag;
+      f.any_or = b0 > 0;
+      f.u = ctx->head_u;        // the slices reuse the scratch (stride nb), one after another
+      f.f = ctx->head_f;
+      f.act = ctx->head_act;
+      f.cnt = ctx->head_cnt;
+      f.err = ctx->err;
+      f.B = nb;
+      f.D = D;
+      f.ring = ps.ring;
+      f.theta = ctx->cfg.theta;
+      cudaLaunchConfig_t lc = {};
+      lc.gridDim = dim3(ctx->n_sms);
+      lc.blockDim = dim3(kFThreads);
+      lc.dynamicSmemBytes = ps.smem;
+      lc.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeCooperative;
+      attr[0].val.cooperative = 1;
+      lc.attrs = attr;
+      lc.numAttrs = 1;
+      const oda_status st = check_cuda(ps.bt == 4 ? cudaLaunchKernelEx(&lc, head_fused_kernel<4>, f)
+                                                  : cudaLaunchKernelEx(&lc, head_fused_kernel<8>, f),
+                                       "recall head launch");
+      if (st != ODA_OK) return st;
+    }
+    return ODA_OK;
   }
   HeadParams p;
   p.w = *w;

@@ -38,9 +38,10 @@ def _run(B, D, perturb=True, seed=500, sched=None, theta=0.0, bias=0.0, inputs_o
 
 
 # fused single-launch head for B <= 8 (ring depth from the shared memory the inputs leave:
-# 5 stages at (1, 2048), 4 at (4, 4096), 3 at (8, 2048) and (2, 8192), 2 at (8, 4096)); the six
-# phase launches for B > 8, where the inputs do not fit (8, 8192) and where D is not a multiple of
-# 1024 (512, 1536: the tower phase's per-chunk sums of squares fill their whole scratch at D = 512)
+# 5 stages at (1, 2048), 4 at (4, 4096), 3 at (8, 2048) and (2, 8192), 2 at (8, 4096)), once per
+# slice of 8 sequences for B > 8 (13, 32); the six phase launches where the inputs do not fit
+# (8, 8192) and where D is not a multiple of 1024 (512, 1536: the tower phase's per-chunk sums of
+# squares fill their whole scratch at D = 512)
 @pytest.mark.parametrize("B,D", [(1, 2048), (4, 4096), (8, 2048), (2, 8192), (8, 4096), (8, 8192),
                                  (13, 2048), (32, 2048), (2, 512), (8, 512), (3, 1536)])
 def test_scores_and_gate_match_oracle(B, D):
@@ -96,6 +97,18 @@ def test_theta_and_schedule_override():
     assert np.array_equal(score2, score)  # the head still runs under a schedule (deterministic)
     _, _, _, flag3, any3 = _run(6, 2048, seed=601, sched=[0] * 6)
     assert flag3.tolist() == [0] * 6 and any3 == 0
+
+
+def test_any_flag_over_sequence_slices():
+    """Batches above 8 run the fused head once per slice of 8 sequences; the routing flag must be
+    the OR over all slices (a later slice without a flagged sequence keeps an earlier one's)."""
+    B = 16
+    for hot in (2, 14, None):
+        sched = [0] * B
+        if hot is not None:
+            sched[hot] = 1
+        _, _, score, flag, anyf = _run(B, 2048, seed=611, sched=sched)
+        assert flag.tolist() == sched and anyf == int(hot is not None), hot
 
 
 @pytest.mark.parametrize("bad", [np.nan, np.inf, -np.inf])
