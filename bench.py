@@ -594,7 +594,7 @@ def run_ours(args, wl, rank, world, local_rank):
     wl = replica_workload(wl, rank, world)
     W, K = args.warmup, args.steps
     n_e2e = K if args.e2e else 0
-    cap = W + K + W + n_e2e + 4
+    cap = W + K + W + n_e2e + 24   # + the unflagged / one-flag probes (2 x 9 steps)
     t_setup = time.perf_counter()
     dec = OdaDecoder(wl, device=dev, capacity_steps=cap, kv_format=args.kv)
     n_store = min(cap, W + K)
@@ -735,15 +735,24 @@ def run_ours(args, wl, rank, world, local_rank):
     quiet = dec.make_step_buffer(0)
     dec.layout.views(quiet)["sched"].zero_()
     if dec.routing_scheduled:
-        dec.step(quiet)
-        dec.synchronize()
-        q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        q0.record(dec.stream)
-        for _ in range(2):
-            dec.step(quiet)
-        q1.record(dec.stream)
-        q1.synchronize()
-        quiet_us = q0.elapsed_time(q1) * 1e3 / 2
+        n_probe = 8
+
+        def probe_us(buf):
+            """Device time per step of n_probe steps on one buffer; a sleep kernel ahead of the
+            first event keeps the host's issue of the steps out of the interval."""
+            dec.step(buf)
+            dec.synchronize()
+            p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(dec.stream):
+                torch.cuda._sleep(4_000_000)
+                p0.record(dec.stream)
+                for _ in range(n_probe):
+                    dec.step(buf)
+                p1.record(dec.stream)
+            p1.synchronize()
+            return p0.elapsed_time(p1) * 1e3 / n_probe
+
+        quiet_us = probe_us(quiet)
         # the step-input staging copy alone (device to device, in the step stream); a sleep
         # kernel ahead of the copies keeps the host's issue time out of the interval
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -765,15 +774,7 @@ def run_ours(args, wl, rank, world, local_rank):
         ov = dec.layout.views(one)["sched"]
         ov.zero_()
         ov[0] = 1
-        dec.step(one)
-        dec.synchronize()
-        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        r0.record(dec.stream)
-        for _ in range(2):
-            dec.step(one)
-        r1.record(dec.stream)
-        r1.synchronize()
-        one_us = r0.elapsed_time(r1) * 1e3 / 2
+        one_us = probe_us(one)
         rho = statistics.mean(wl.rates) if wl.rates else 0.0
         retry_us = one_us - quiet_us
         norm_us = quiet_us + rho * wl.B * retry_us
