@@ -11,9 +11,10 @@
 //   q   = w_o . (RMSNorm(f) * gamma_o) + b_o
 //
 // Design: at batch sizes of a few sequences the head is a weight-streaming problem (113 MB of
-// fp32 weights for D = 2048, 2*B flops per 4-byte weight) on CUDA cores.  Up to 8 sequences run
-// in one cooperative launch of all six phases (head_fused_kernel, further down).  Larger batches
-// run six phase launches, each a split-K GEMV: a CTA streams a 32-row x Kc slab of one weight
+// fp32 weights for D = 2048, 2*B flops per 4-byte weight) on CUDA cores.  The whole batch runs in
+// one cooperative launch of all six phases (head_fused_kernel, further down), in groups of up to 8
+// sequences.  Where that kernel's inputs do not fit, six phase launches run instead, each a
+// split-K GEMV: a CTA streams a 32-row x Kc slab of one weight
 // matrix exactly once with 16-byte non-allocating loads and multiplies it against a
 // shared-memory tile of up to 8 sequences' inputs; lanes reduce with a 31-shuffle butterfly.
 // The input transform of a phase (RMSNorm scale, the interaction vector, the gated activation)
@@ -422,9 +423,13 @@ __global__ void __launch_bounds__(kHT) head_phase_kernel(const HeadParams p) {
   }
 }
 
-// ------------------------------------------------------------ fused head (batch <= 8)
-// One cooperative launch, one CTA per SM, runs all six phases.  Warp 8 streams every weight row
-// segment (1024 floats, 4 KiB) the CTA owns through a ring of 32 KiB stages with bulk copies,
+// ------------------------------------------------------------ fused head
+// One cooperative launch, one CTA per SM, runs all six phases.  The batch is cut into groups of
+// up to 8 sequences (the tile width), each on its own share of the grid; every group streams all
+// the weights, and as CTA i of each group reads the same segments in the same order, in step with
+// the other groups through the phase barriers, HBM serves a segment once and L2 the other groups.
+// Warp 8 streams every weight row segment (1024 floats, 4 KiB) the CTA owns through a ring of
+// 32 KiB stages with bulk copies,
 // phase after phase: the weights never depend on a phase's inputs, so HBM keeps streaming while
 // the grid waits between phases.  Warps 0-7 take one segment each per stage and dot it against
 // the phase's input, held whole in shared memory for the sequence tile.  Each CTA owns whole
@@ -438,7 +443,7 @@ constexpr int kSeg = 1024;                          // floats per weight segment
 constexpr int kSegBytes = kSeg * 4;
 constexpr int kFStageBytes = kFC * kSegBytes;       // one segment per consumer warp
 constexpr int kMaxRing = 5;
-constexpr int kMaxOwnSegs = 32;                     // segments per chunk a CTA may own in a phase
+constexpr int kMaxOwnSegs = 32;                     // segments of one batch of a CTA's rows
 constexpr uint64_t kFWaitNs = 2000000000ull;
 constexpr uint64_t kGridWaitNs = 1000000000ull;
 
@@ -455,7 +460,7 @@ struct FusedParams {
   int32_t* cnt;           // [0] grid-barrier arrivals, [1] finished CTAs; both back to 0 at exit
   int32_t* err;
   int B, D, ring;
-  int any_or;             // a later slice of a larger batch: OR into *any_flag instead of setting it
+  int groups, gsize;      // sequence groups of the tile width, and CTAs per group
   float theta;
 };
 
@@ -485,6 +490,19 @@ __device__ __forceinline__ Own own_rows(int ph, int c, int G, int D) {
   o.lo = (int)((long long)rows * cc / gg);
   o.n = (int)((long long)rows * (cc + 1) / gg) - o.lo;
   o.nchunk = o.kind == kTower ? D / kSeg : o.kind == kFuse ? 9 : o.kind == kUp ? 1 : kF / kSeg;
+  o.nseg = o.kind == kUp ? 2 * o.n : o.n;
+  return o;
+}
+
+// A CTA takes its rows of a phase in batches of at most kMaxOwnSegs segments (gate/up rows of the
+// same units stay together), the size of its row-sum area.  With one sequence group every CTA
+// owns few enough rows for one batch; with several groups each CTA owns more rows.
+__device__ __forceinline__ int batch_rows(const Own& o) { return o.kind == kUp ? kMaxOwnSegs / 2 : kMaxOwnSegs; }
+__device__ __forceinline__ int n_batches(const Own& o) { return (o.n + batch_rows(o) - 1) / batch_rows(o); }
+__device__ __forceinline__ Own batch_of(Own o, int j) {
+  const int per = batch_rows(o);
+  o.lo += j * per;
+  o.n = min(per, o.n - j * per);
   o.nseg = o.kind == kUp ? 2 * o.n : o.n;
   return o;
 }
@@ -594,8 +612,8 @@ __device__ __forceinline__ void stage_dot(const uint8_t* stage, int n, int col4,
 // applied to the dot products); down act [BT][F].  These rows were written by other CTAs of
 // this launch (L2 loads).  Ends with a consumer barrier.
 template <int BT>
-__device__ void load_source(const FusedParams& p, const Own& o, float* src, float* red, float* inv,
-                            int tid) {
+__device__ void load_source(const FusedParams& p, const Own& o, int b0, int Bs, float* src, float* red,
+                            float* inv, int tid) {
   const int B = p.B, lane = tid & 31, warp = tid >> 5;
   float4* s4 = reinterpret_cast<float4*>(src);
   const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -605,7 +623,7 @@ __device__ void load_source(const FusedParams& p, const Own& o, float* src, floa
     float4 v[BT];   // kT / 4 == 256 == consumer threads: one float4 of f per sequence each
 #pragma unroll
     for (int bb = 0; bb < BT; ++bb)
-      v[bb] = bb < B ? __ldcg(reinterpret_cast<const float4*>(p.f + ((size_t)o.blk * B + bb) * kT) + tid) : zero;
+      v[bb] = bb < Bs ? __ldcg(reinterpret_cast<const float4*>(p.f + ((size_t)o.blk * B + b0 + bb) * kT) + tid) : zero;
     const float4 g = g4[tid];
 #pragma unroll
     for (int bb = 0; bb < BT; ++bb) {
@@ -632,8 +650,8 @@ __device__ void load_source(const FusedParams& p, const Own& o, float* src, floa
     for (int i = 0; i < 3; ++i)
 #pragma unroll
       for (int bb = 0; bb < BT; ++bb)
-        v[i][bb] = bb < B ? __ldcg(reinterpret_cast<const float4*>(p.u + ((size_t)i * B + bb) * kT) + tid)
-                          : zero;
+        v[i][bb] = bb < Bs ? __ldcg(reinterpret_cast<const float4*>(p.u + ((size_t)i * B + b0 + bb) * kT) + tid)
+                           : zero;
 #pragma unroll
     for (int i = 0; i < 3; ++i)
 #pragma unroll
@@ -644,8 +662,8 @@ __device__ void load_source(const FusedParams& p, const Own& o, float* src, floa
     for (int bb = 0; bb < BT; ++bb)
 #pragma unroll
       for (int j = 0; j < 2; ++j)
-        v[bb][j] = bb < B ? __ldcg(reinterpret_cast<const float4*>(p.act + (size_t)bb * kF) + tid + j * kFC * 32)
-                          : zero;
+        v[bb][j] = bb < Bs ? __ldcg(reinterpret_cast<const float4*>(p.act + (size_t)(b0 + bb) * kF) + tid + j * kFC * 32)
+                           : zero;
 #pragma unroll
     for (int bb = 0; bb < BT; ++bb)
 #pragma unroll
@@ -654,18 +672,17 @@ __device__ void load_source(const FusedParams& p, const Own& o, float* src, floa
   consumer_sync();
 }
 
-// The operand of output item idx (row idx / B, sequence idx % B) of the phase that comes from
-// global memory: the tower or fusion bias, or the residual f_j of a down projection (written two
-// phases earlier).  Each thread loads the one for its own item while the phase's stages stream.
-__device__ __forceinline__ float finish_operand(const FusedParams& p, const Own& o, int idx) {
-  const int B = p.B;
-  if (idx >= o.n * B) return 0.f;
-  const int r = idx / B, b = idx - r * B, n = o.lo + r;
+// The operand of output item idx (row idx / Bs, sequence b0 + idx % Bs) of the phase that comes
+// from global memory: the tower or fusion bias, or the residual f_j of a down projection (written
+// two phases earlier).  Each thread loads the one for its own item while the phase's stages stream.
+__device__ __forceinline__ float finish_operand(const FusedParams& p, const Own& o, int b0, int Bs, int idx) {
+  if (idx >= o.n * Bs) return 0.f;
+  const int r = idx / Bs, b = idx - r * Bs, n = o.lo + r;
   switch (o.kind) {
     case kTower: return p.w.tower_b[o.tower][n];
     case kFuse: return p.w.fuse_b[n];
     case kUp: return 0.f;
-    default: return __ldcg(p.f + ((size_t)o.blk * B + b) * kT + n);
+    default: return __ldcg(p.f + ((size_t)o.blk * p.B + b0 + b) * kT + n);
   }
 }
 
@@ -673,8 +690,8 @@ __device__ __forceinline__ float finish_operand(const FusedParams& p, const Own&
 // sum of the eight warps' column shares accw[w][r][b], taken in warp order.  `pre` is this
 // thread's finish_operand.
 template <int BT>
-__device__ void finish_rows(const FusedParams& p, const Own& o, const float* src, const float* accw,
-                            const float* inv, float pre, int tid) {
+__device__ void finish_rows(const FusedParams& p, const Own& o, int b0, int Bs, const float* src,
+                            const float* accw, const float* inv, float pre, int tid) {
   const int B = p.B;
   auto rowsum = [&](int r, int b) {
     float t = 0.f;
@@ -682,21 +699,21 @@ __device__ void finish_rows(const FusedParams& p, const Own& o, const float* src
     for (int w = 0; w < kFC; ++w) t += accw[(w * kMaxOwnSegs + r) * BT + b];
     return t;
   };
-  for (int idx = tid; idx < o.n * B; idx += kFC * 32) {
-    const int r = idx / B, b = idx - r * B, n = o.lo + r;
+  for (int idx = tid; idx < o.n * Bs; idx += kFC * 32) {
+    const int r = idx / Bs, b = idx - r * Bs, n = o.lo + r;
     const float acc = rowsum(r, b);
-    const float opnd = idx == tid ? pre : finish_operand(p, o, idx);
+    const float opnd = idx == tid ? pre : finish_operand(p, o, b0, Bs, idx);
     if (o.kind == kTower) {
-      p.u[((size_t)o.tower * B + b) * kT + n] = silu(acc * inv[b] + opnd);
+      p.u[((size_t)o.tower * B + b0 + b) * kT + n] = silu(acc * inv[b] + opnd);
     } else if (o.kind == kFuse) {
       const float mean = (src[(0 * BT + b) * kT + n] + src[(1 * BT + b) * kT + n] +
                           src[(2 * BT + b) * kT + n]) / 3.0f;
-      p.f[(size_t)b * kT + n] = acc + opnd + mean;
+      p.f[(size_t)(b0 + b) * kT + n] = acc + opnd + mean;
     } else if (o.kind == kUp) {
       const float ga = acc * inv[b], ua = rowsum(o.n + r, b) * inv[b];
-      p.act[(size_t)b * kF + n] = silu(ga) * ua;
+      p.act[(size_t)(b0 + b) * kF + n] = silu(ga) * ua;
     } else {
-      p.f[((size_t)(o.blk + 1) * B + b) * kT + n] = opnd + acc;
+      p.f[((size_t)(o.blk + 1) * B + b0 + b) * kT + n] = opnd + acc;
     }
   }
 }
@@ -716,6 +733,16 @@ __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedPar
   __shared__ int s_last, s_any;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x, G = gridDim.x, B = p.B;
+  // sequence group of this CTA: sequences [b0, b0 + Bs) on CTAs [grp * gsize, grp * gsize + gsize);
+  // CTAs past the last group own no rows and only take part in the grid barriers
+  const int grp = c / p.gsize, cg = c - grp * p.gsize;
+  const int b0 = grp * BT;
+  const int Bs = grp < p.groups ? min(BT, B - b0) : 0;
+  auto own = [&](int ph) {
+    Own o = own_rows(ph, cg, p.gsize, p.D);
+    if (Bs == 0) o.n = o.nseg = 0;
+    return o;
+  };
   if (tid == 0) {
     for (int i = 0; i < R; ++i) {
       mbar_init(&full[i], 1);
@@ -727,35 +754,40 @@ __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedPar
   __syncthreads();
 
   if (warp == kFC) {
-    // ---- producer.  First the tower input rows x_i[b] of this CTA's tower (they may come from
-    // the previous kernel), then every weight segment of every phase in the order the consumers
-    // take them, running up to the ring's depth ahead of them (into the next phase while they
-    // finish one or wait at a barrier).  No L2 prefetch of a whole phase ahead of the ring: the
-    // copy engine takes requests in order, so such prefetches delay the ring's own copies (with
-    // L2 flushed between scores, 55.5 us per score with them, 51.5 without).
+    // ---- producer.  First the tower input rows x_i[b] of this CTA's tower and sequence group
+    // (they may come from the previous kernel), then every weight segment of every phase in the
+    // order the consumers take them, running up to the ring's depth ahead of them (into the next
+    // phase while they finish one or wait at a barrier).  No L2 prefetch ahead of the ring: the
+    // copy engine takes requests in order, so bulk prefetches delay the ring's own copies (with L2
+    // flushed between scores, 55.5 us per score with them, 51.5 without), and line prefetches
+    // issued at the phase boundaries compete with the copies in flight (61.8 vs 55.7 us).
     grid_dependency_wait();
-    const Own o0 = own_rows(0, c, G, p.D);
-    if (lane == 0) mbar_arrive_expect_tx(&src_bar, (uint32_t)(B * p.D * sizeof(float)));
+    const Own o0 = own(0);
+    if (lane == 0) mbar_arrive_expect_tx(&src_bar, (uint32_t)(Bs * p.D * sizeof(float)));
     __syncwarp();
-    if (lane < B)
-      bulk_load(src + (size_t)lane * p.D, p.x[o0.tower] + (size_t)lane * p.D,
+    if (lane < Bs)
+      bulk_load(src + (size_t)lane * p.D, p.x[o0.tower] + (size_t)(b0 + lane) * p.D,
                 (uint32_t)(p.D * sizeof(float)), &src_bar);
     int k = 0;
     for (int ph = 0; ph < 6; ++ph) {
-      const Own o = own_rows(ph, c, G, p.D);
-      const int ngrp = (o.nseg + kFC - 1) / kFC;
-      for (int ch = 0; ch < o.nchunk; ++ch)
-        for (int g = 0; g < ngrp; ++g, ++k) {
-          const int s = k % R;
-          if (k >= R && !mbar_wait_bounded(&empty[s], (uint32_t)(k / R - 1) & 1u, kFWaitNs) && lane == 0)
-            atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
-          const int n = min(kFC, o.nseg - g * kFC);
-          if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(n * kSegBytes));
-          __syncwarp();
-          if (lane < n)
-            bulk_load(ring + (size_t)s * kFStageBytes + lane * kSegBytes, seg_ptr(p, o, ch, g * kFC + lane),
-                      kSegBytes, &full[s]);
-        }
+      const Own oa = own(ph);
+      const int nbat = n_batches(oa);
+      for (int j = 0; j < nbat; ++j) {
+        const Own o = batch_of(oa, j);
+        const int ngrp = (o.nseg + kFC - 1) / kFC;
+        for (int ch = 0; ch < o.nchunk; ++ch)
+          for (int g = 0; g < ngrp; ++g, ++k) {
+            const int s = k % R;
+            if (k >= R && !mbar_wait_bounded(&empty[s], (uint32_t)(k / R - 1) & 1u, kFWaitNs) && lane == 0)
+              atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
+            const int n = min(kFC, o.nseg - g * kFC);
+            if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)(n * kSegBytes));
+            __syncwarp();
+            if (lane < n)
+              bulk_load(ring + (size_t)s * kFStageBytes + lane * kSegBytes, seg_ptr(p, o, ch, g * kFC + lane),
+                        kSegBytes, &full[s]);
+          }
+      }
     }
     return;
   }
@@ -768,62 +800,68 @@ __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedPar
   const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
   int k = 0;
   for (int ph = 0; ph < 6; ++ph) {
-    const Own o = own_rows(ph, c, G, p.D);
-    for (int i = lane; i < kMaxOwnSegs * BT; i += 32) acc[i] = 0.f;
-    const bool tower = o.kind == kTower;
-    const float4* gam4 = reinterpret_cast<const float4*>(p.w.tower_norm[o.tower]);
-    float4 gnext = tower ? __ldg(gam4 + col4) : zero;
+    const Own oa = own(ph);
+    const bool tower = oa.kind == kTower;
+    const float4* gam4 = reinterpret_cast<const float4*>(p.w.tower_norm[oa.tower]);
     if (tower) {
       if (!mbar_wait_bounded(&src_bar, 0u, kFWaitNs) && lane == 0) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
     } else {
-      load_source<BT>(p, o, src, red, s_inv, tid);
+      load_source<BT>(p, oa, b0, Bs, src, red, s_inv, tid);
     }
-    __syncwarp();
-    const float pre = finish_operand(p, o, tid);
-    float ssl[BT];
+    const int nbat = n_batches(oa);
+    for (int j = 0; j < nbat; ++j) {
+      const Own o = batch_of(oa, j);
+      for (int i = lane; i < kMaxOwnSegs * BT; i += 32) acc[i] = 0.f;
+      float4 gnext = tower ? __ldg(gam4 + col4) : zero;
+      __syncwarp();
+      const float pre = finish_operand(p, o, b0, Bs, tid);
+      float ssl[BT];
 #pragma unroll
-    for (int bb = 0; bb < BT; ++bb) ssl[bb] = 0.f;
-    const int ngrp = (o.nseg + kFC - 1) / kFC;
-    for (int ch = 0; ch < o.nchunk; ++ch) {
-      const float4 gam = gnext;
-      if (tower && ch + 1 < o.nchunk) gnext = __ldg(gam4 + (ch + 1) * (kSeg / 4) + col4);
-      float4 xs[BT];
-      input_slice<BT>(o, B, p.D, src, ch, col4, gam, ssl, xs);
-      for (int g = 0; g < ngrp; ++g, ++k) {
-        const int s = k % R;
-        if (!mbar_wait_bounded(&full[s], (uint32_t)(k / R) & 1u, kFWaitNs) && lane == 0)
-          atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
-        stage_dot<BT>(ring + (size_t)s * kFStageBytes, min(kFC, o.nseg - g * kFC), col4, xs, acc, g, lane);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+      for (int bb = 0; bb < BT; ++bb) ssl[bb] = 0.f;
+      const int ngrp = (o.nseg + kFC - 1) / kFC;
+      for (int ch = 0; ch < o.nchunk; ++ch) {
+        const float4 gam = gnext;
+        if (tower && ch + 1 < o.nchunk) gnext = __ldg(gam4 + (ch + 1) * (kSeg / 4) + col4);
+        float4 xs[BT];
+        input_slice<BT>(o, Bs, p.D, src, ch, col4, gam, ssl, xs);
+        for (int g = 0; g < ngrp; ++g, ++k) {
+          const int s = k % R;
+          if (!mbar_wait_bounded(&full[s], (uint32_t)(k / R) & 1u, kFWaitNs) && lane == 0)
+            atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
+          stage_dot<BT>(ring + (size_t)s * kFStageBytes, min(kFC, o.nseg - g * kFC), col4, xs, acc, g, lane);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[s]);
+        }
       }
-    }
-    if (tower) {
-      // 1 / rms(x_i): the warps' column shares of the sum of squares, summed in warp order
+      if (tower) {
+        // 1 / rms(x_i): the warps' column shares of the sum of squares, summed in warp order (the
+        // same value for every batch of rows)
 #pragma unroll
-      for (int bb = 0; bb < BT; ++bb)
+        for (int bb = 0; bb < BT; ++bb)
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ssl[bb] += __shfl_xor_sync(0xffffffffu, ssl[bb], off);
-      if (lane == 0)
+          for (int off = 16; off > 0; off >>= 1) ssl[bb] += __shfl_xor_sync(0xffffffffu, ssl[bb], off);
+        if (lane == 0)
 #pragma unroll
-        for (int bb = 0; bb < BT; ++bb) red[warp * BT + bb] = ssl[bb];
+          for (int bb = 0; bb < BT; ++bb) red[warp * BT + bb] = ssl[bb];
+        consumer_sync();
+        if (tid < BT) {
+          float t = 0.f;
+          for (int w = 0; w < kFC; ++w) t += red[w * BT + tid];
+          s_inv[tid] = rsqrtf(t / p.D + kEps);
+        }
+      }
       consumer_sync();
-      if (tid < BT) {
-        float t = 0.f;
-        for (int w = 0; w < kFC; ++w) t += red[w * BT + tid];
-        s_inv[tid] = rsqrtf(t / p.D + kEps);
-      }
+      finish_rows<BT>(p, o, b0, Bs, src, accw, s_inv, pre, tid);
+      consumer_sync();
     }
-    consumer_sync();
-    finish_rows<BT>(p, o, src, accw, s_inv, pre, tid);
-    consumer_sync();
     if (ph < 5) {
       if (tid == 0 && !grid_barrier_bounded(p.cnt, (ph + 1) * G, kGridWaitNs)) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
       consumer_sync();
     }
   }
 
-  // ---- the last CTA to finish computes q and the gate, then returns the counters to zero
+  // ---- the last CTA to finish computes q and the gate of every sequence, then returns the
+  // counters to zero
   if (tid == 0) {
     s_last = atom_add_acq_rel_gpu(p.cnt + 1, 1) == G - 1;
     s_any = 0;
@@ -835,8 +873,7 @@ __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedPar
                    &s_any, lane);
   consumer_sync();
   if (tid == 0) {
-    if (!p.any_or) *p.any_flag = s_any;
-    else if (s_any) *p.any_flag = 1;   // the slices run in stream order
+    *p.any_flag = s_any;
     p.cnt[0] = 0;
     p.cnt[1] = 0;
   }
@@ -884,19 +921,22 @@ int g_fused_static[2] = {-1, -1};   // head_fused_kernel<4>, <8>
 int g_smem_optin = 0;
 int g_coop = 0;
 
-// Fused-head plan: sequence tile, ring depth and dynamic shared memory; bt = 0 where the fused
-// kernel does not apply (batch above 8, D not a multiple of 1024, fewer than 128 SMs, no
+// Fused-head plan: sequence tile, sequence groups, ring depth and dynamic shared memory; bt = 0
+// where the fused kernel does not apply (D not a multiple of 1024, fewer than 128 SMs, no
 // cooperative launch, or too little shared memory for a ring of two stages), and the six phase
 // kernels run instead.
 struct FusedPlan {
-  int bt, ring;
+  int bt, groups, gsize, ring;
   size_t smem;
 };
 
 FusedPlan fused_plan(int B, int D, int n_sms) {
-  FusedPlan pl = {0, 0, 0};
-  if (B < 1 || B > kBTMax || D % kSeg != 0 || n_sms < 128 || !g_coop) return pl;
+  FusedPlan pl = {0, 0, 0, 0, 0};
+  if (B < 1 || D % kSeg != 0 || n_sms < 128 || !g_coop) return pl;
   const int bt = B <= 4 ? 4 : 8;
+  const int groups = (B + bt - 1) / bt;
+  const int gsize = n_sms / groups;
+  if (gsize < 3) return pl;   // the tower phase gives each of the three towers a CTA at least
   const int stat = g_fused_static[bt == 4 ? 0 : 1];
   if (stat < 0) return pl;
   const size_t src = (size_t)std::max(D, 3 * kT) * bt * sizeof(float);
@@ -905,6 +945,8 @@ FusedPlan fused_plan(int B, int D, int n_sms) {
   const int ring = (int)std::min<long long>(kMaxRing, room / kFStageBytes);
   if (ring < 2) return pl;
   pl.bt = bt;
+  pl.groups = groups;
+  pl.gsize = gsize;
   pl.ring = ring;
   pl.smem = (size_t)ring * kFStageBytes + src + res;
   return pl;
@@ -968,11 +1010,11 @@ oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const flo
     if (reinterpret_cast<uintptr_t>(q) & 15)
       return set_error(ODA_ERR_INVALID_ARG, "recall_score: matrices and inputs must be 16-byte aligned");
   const int B = ctx->cfg.batch, D = ctx->cfg.head_in_dim;
-  // The fused kernel takes up to 8 sequences; a larger batch runs it once per slice of 8 (each
-  // slice streams the weights again, still far fewer round trips than the six phase launches),
-  // when a full slice fits its plan.
-  const int slice = std::min(B, kBTMax);
-  const FusedPlan pl = fused_plan(slice, D, ctx->n_sms);
+  // One cooperative launch for the whole batch: groups of up to 8 sequences, each on its own
+  // share of the SMs, all groups in step (one grid barrier per phase).  CTA i of every group
+  // streams the same weight segments at about the same time, so HBM serves each segment once and
+  // L2 the other groups.
+  const FusedPlan pl = fused_plan(B, D, ctx->n_sms);
   int per_sm = 0;
   if (pl.bt) {
     const void* kern = pl.bt == 4 ? reinterpret_cast<const void*>(head_fused_kernel<4>)
@@ -982,46 +1024,40 @@ oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const flo
     if (st != ODA_OK) return st;
   }
   if (pl.bt && per_sm >= 1) {
-    for (int b0 = 0; b0 < B; b0 += kBTMax) {
-      const int nb = std::min(kBTMax, B - b0);
-      const FusedPlan ps = nb == slice ? pl : fused_plan(nb, D, ctx->n_sms);
-      if (!ps.bt) return set_error(ODA_ERR_UNSUPPORTED, "recall_score: no fused plan for a slice of %d", nb);
-      // one CTA per SM, all resident at once (cooperative launch): the grid barrier needs that
-      FusedParams f;
-      f.w = *w;
-      f.x[0] = h_prev + (size_t)b0 * D;
-      f.x[1] = emb + (size_t)b0 * D;
-      f.x[2] = h_loc + (size_t)b0 * D;
-      f.sched = sched ? sched + b0 : nullptr;
-      f.score = score + b0;
-      f.flag = flag + b0;
-      f.any_flag = any_flag;
-      f.any_or = b0 > 0;
-      f.u = ctx->head_u;        // the slices reuse the scratch (stride nb), one after another
-      f.f = ctx->head_f;
-      f.act = ctx->head_act;
-      f.cnt = ctx->head_cnt;
-      f.err = ctx->err;
-      f.B = nb;
-      f.D = D;
-      f.ring = ps.ring;
-      f.theta = ctx->cfg.theta;
-      cudaLaunchConfig_t lc = {};
-      lc.gridDim = dim3(ctx->n_sms);
-      lc.blockDim = dim3(kFThreads);
-      lc.dynamicSmemBytes = ps.smem;
-      lc.stream = s;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeCooperative;
-      attr[0].val.cooperative = 1;
-      lc.attrs = attr;
-      lc.numAttrs = 1;
-      const oda_status st = check_cuda(ps.bt == 4 ? cudaLaunchKernelEx(&lc, head_fused_kernel<4>, f)
-                                                  : cudaLaunchKernelEx(&lc, head_fused_kernel<8>, f),
-                                       "recall head launch");
-      if (st != ODA_OK) return st;
-    }
-    return ODA_OK;
+    // one CTA per SM, all resident at once (cooperative launch): the grid barrier needs that
+    FusedParams f;
+    f.w = *w;
+    f.x[0] = h_prev;
+    f.x[1] = emb;
+    f.x[2] = h_loc;
+    f.sched = sched;
+    f.score = score;
+    f.flag = flag;
+    f.any_flag = any_flag;
+    f.u = ctx->head_u;
+    f.f = ctx->head_f;
+    f.act = ctx->head_act;
+    f.cnt = ctx->head_cnt;
+    f.err = ctx->err;
+    f.B = B;
+    f.D = D;
+    f.ring = pl.ring;
+    f.groups = pl.groups;
+    f.gsize = pl.gsize;
+    f.theta = ctx->cfg.theta;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(ctx->n_sms);
+    lc.blockDim = dim3(kFThreads);
+    lc.dynamicSmemBytes = pl.smem;
+    lc.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    return check_cuda(pl.bt == 4 ? cudaLaunchKernelEx(&lc, head_fused_kernel<4>, f)
+                                 : cudaLaunchKernelEx(&lc, head_fused_kernel<8>, f),
+                      "recall head launch");
   }
   HeadParams p;
   p.w = *w;

@@ -38,12 +38,16 @@ def _run(B, D, perturb=True, seed=500, sched=None, theta=0.0, bias=0.0, inputs_o
 
 
 # fused single-launch head for B <= 8 (ring depth from the shared memory the inputs leave:
-# 5 stages at (1, 2048), 4 at (4, 4096), 3 at (8, 2048) and (2, 8192), 2 at (8, 4096)), once per
-# slice of 8 sequences for B > 8 (13, 32); the six phase launches where the inputs do not fit
-# (8, 8192) and where D is not a multiple of 1024 (512, 1536: the tower phase's per-chunk sums of
-# squares fill their whole scratch at D = 512)
+# 5 stages at (1, 2048), 4 at (4, 4096), 3 at (8, 2048) and (2, 8192), 2 at (8, 4096)); for
+# B > 8 the same launch in groups of 8 sequences on shares of the grid (13: 2 groups, the last
+# ragged; 32: 4; 20 at D = 4096: 3, 2-stage ring; 67: 9 groups of 16 CTAs, 4 CTAs idle, each CTA
+# taking its tower and up rows in several batches; 256: 32 groups of 4 CTAs, one tower row range
+# of 1024 rows per CTA); the six phase launches where the inputs do not fit (8, 8192) and where
+# D is not a multiple of 1024 (512, 1536: the tower phase's per-chunk sums of squares fill their
+# whole scratch at D = 512)
 @pytest.mark.parametrize("B,D", [(1, 2048), (4, 4096), (8, 2048), (2, 8192), (8, 4096), (8, 8192),
-                                 (13, 2048), (32, 2048), (2, 512), (8, 512), (3, 1536)])
+                                 (13, 2048), (32, 2048), (20, 4096), (67, 1024), (256, 1024),
+                                 (2, 512), (8, 512), (3, 1536)])
 def test_scores_and_gate_match_oracle(B, D):
     P, xs, score, flag, anyf = _run(B, D, perturb=True, seed=500 + B + D)
     ref = np.array([recall_head(P, xs[0][b], xs[1][b], xs[2][b]) for b in range(B)])
@@ -99,9 +103,9 @@ def test_theta_and_schedule_override():
     assert flag3.tolist() == [0] * 6 and any3 == 0
 
 
-def test_any_flag_over_sequence_slices():
-    """Batches above 8 run the fused head once per slice of 8 sequences; the routing flag must be
-    the OR over all slices (a later slice without a flagged sequence keeps an earlier one's)."""
+def test_any_flag_over_sequence_groups():
+    """Batches above 8 run the fused head in groups of 8 sequences; the routing flag must be the
+    OR over all groups (a flagged sequence in any group sets it)."""
     B = 16
     for hot in (2, 14, None):
         sched = [0] * B
@@ -109,6 +113,19 @@ def test_any_flag_over_sequence_slices():
             sched[hot] = 1
         _, _, score, flag, anyf = _run(B, 2048, seed=611, sched=sched)
         assert flag.tolist() == sched and anyf == int(hot is not None), hot
+
+
+def test_sequence_groups_do_not_change_the_arithmetic():
+    """A sequence's score does not depend on which group of the grid computes it: a batch of 24
+    (3 groups of 8 on 49 CTAs each, rows taken in batches) gives the bits of three batches of 8
+    (one group on the whole grid) on the same inputs."""
+    B, D = 24, 2048
+    xs = [gen.normal_f32(gen.key(612, 90, i), B * D).reshape(B, D) for i in range(3)]
+    _, _, whole, _, _ = _run(B, D, seed=612, inputs_override=xs)
+    for g in range(3):
+        part = [x[8 * g:8 * g + 8] for x in xs]
+        _, _, sc, _, _ = _run(8, D, seed=612, inputs_override=part)
+        assert np.array_equal(sc, whole[8 * g:8 * g + 8]), g
 
 
 @pytest.mark.parametrize("bad", [np.nan, np.inf, -np.inf])
