@@ -980,6 +980,12 @@ oda_status prepare_head_kernel() {
     cudaFuncAttributes fa;
     st = check_cuda(cudaFuncGetAttributes(&fa, kernels[i]), "cudaFuncGetAttributes(head)");
     if (st != ODA_OK) return st;
+    // 288 threads (9 warps, three on one SM sub-partition) allow at most 168 registers per thread;
+    // a kernel built with more could never launch, every plan would fail and the phase kernels
+    // would run in silence: refuse it here instead
+    if (fa.maxThreadsPerBlock < kFThreads)
+      return set_error(ODA_ERR_UNSUPPORTED, "fused recall head: %d registers per thread leave %d threads per block",
+                       fa.numRegs, fa.maxThreadsPerBlock);
     g_fused_static[i] = (int)fa.sharedSizeBytes;
     st = check_cuda(cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          g_smem_optin - g_fused_static[i]),

@@ -129,11 +129,13 @@ def test_sequence_groups_do_not_change_the_arithmetic():
 
 
 @pytest.mark.parametrize("bad", [np.nan, np.inf, -np.inf])
-def test_non_finite_score_routes_full(bad):
-    B, D = 3, 2048
+@pytest.mark.parametrize("B", [3, 8])   # 4-wide tile on CUDA cores, 8-wide tile on tensor cores
+def test_non_finite_score_routes_full(bad, B):
+    D = 2048
     xs = [gen.normal_f32(gen.key(602, 90, i), B * D).reshape(B, D) for i in range(3)]
     xs[2] = xs[2].copy()
     xs[2][1, 5] = bad           # poisons sequence 1's score only
     P, _, score, flag, anyf = _run(B, D, seed=602, inputs_override=xs, bias=-50.0)
     assert not np.isfinite(score[1]) and flag[1] == 1 and anyf == 1
-    assert np.isfinite(score[0]) and flag[0] == 0 and flag[2] == 0
+    others = [b for b in range(B) if b != 1]
+    assert all(np.isfinite(score[b]) and flag[b] == 0 for b in others)

@@ -166,6 +166,13 @@ def cfg2_ctx32k_l2() -> Workload:
                           ctx=(32768,) * 4, steps=8)
 
 
+def cfg3_ctx8k_l2() -> Workload:
+    """Profiling case of the divergent batch's kernels: the same 32 sequences and heads, 2 layers,
+    context 8192 (2.1 GB of cache: larger than L2, small enough for a many-pass profiler capture)."""
+    return cfg3().replace(name="cfg3_profile_ctx8k_l2", n_layers=2, attn_layers=(0, 1),
+                          ctx=(8192,) * 32, steps=8)
+
+
 def bb_qwen3_1p7b_l2() -> Workload:
     """Profiling case of the synthetic-backbone step: the same layer shapes, 2 layers, 4K
     context (under 1 GB on the device, so a many-pass profiler capture stays small)."""
@@ -173,7 +180,7 @@ def bb_qwen3_1p7b_l2() -> Workload:
 
 
 ALL = {"cfg0": cfg0, "cfg1": cfg1, "cfg2": cfg2, "cfg3": cfg3, "cfg4": cfg4,
-       "cfg2_ctx32k_l2": cfg2_ctx32k_l2, "bb": bb_qwen3_1p7b, "bb_l2": bb_qwen3_1p7b_l2}
+       "cfg2_ctx32k_l2": cfg2_ctx32k_l2, "cfg3_ctx8k_l2": cfg3_ctx8k_l2, "bb": bb_qwen3_1p7b, "bb_l2": bb_qwen3_1p7b_l2}
 
 
 def get(name: str) -> Workload:
