@@ -258,8 +258,17 @@ oda_status oda_index_positions(oda_ctx* ctx, int32_t mode, const int32_t* pos, c
  * E(x_t), h^L_t) with inputs h_prev, emb, h_loc (fp32 [B][D]); [notes §2.3]:
  * flag[b] = (score[b] > theta) || !isfinite(score[b]).  If sched is non-NULL the head still
  * runs but flag[b] = (sched[b] != 0) (hand-scheduled full calls, [notes §3.3]).
- * *any_flag = OR of flag[b] (int32, device).  Layer arrangement: see the notes' reading in
- * the design notes; all arithmetic fp32 with fixed reduction order (deterministic). */
+ * *any_flag = OR of flag[b] (int32, device).  Layer arrangement (the notes fix the three
+ * inputs, the 1024-wide towers, the 9216-d interaction, two gated blocks of 2048 and the scalar
+ * output; this library reads them as):
+ *   u_i = SiLU(W_i (RMSNorm(x_i) * gamma_i) + b_i),  x = (h_prev, emb, h_loc)
+ *   z   = [u_0, u_1, u_2, u_0*u_1, u_0*u_2, u_1*u_2, |u_0-u_1|, |u_0-u_2|, |u_1-u_2|]
+ *   f   = W_f z + b_f + (u_0 + u_1 + u_2) / 3
+ *   f  += W_d (SiLU(W_g m) * (W_u m)),  m = RMSNorm(f) * gamma_j      (two blocks)
+ *   q   = w_o . (RMSNorm(f) * gamma_o) + b_o
+ * All arithmetic fp32 with a fixed reduction order (deterministic).  The whole batch runs in
+ * one cooperative launch (groups of up to 8 sequences on shares of the SMs) where D is a
+ * multiple of 1024 and the inputs fit shared memory, else in six phase launches. */
 oda_status oda_recall_score(oda_ctx* ctx, const oda_head_weights* w, const float* h_prev,
                             const float* emb, const float* h_loc, const int32_t* sched,
                             float* score, int32_t* flag, int32_t* any_flag, cudaStream_t stream);
