@@ -96,6 +96,7 @@ _SIGS = {
                              c_void_p], c_int32),
     "oda_recall_score": ([c_void_p, _P(OdaHeadWeights), c_void_p, c_void_p, c_void_p, c_void_p,
                           c_void_p, c_void_p, c_void_p, c_void_p], c_int32),
+    "oda_recall_plan": ([c_void_p, _P(c_int32), _P(c_int32), _P(c_int32)], c_int32),
     "oda_recall_grad_workspace_bytes": ([c_int32, c_int32], ctypes.c_size_t),
     "oda_recall_grad": ([_P(OdaHeadWeights), _P(OdaHeadGrads), c_int32, c_int32, c_void_p, c_void_p,
                          c_void_p, c_void_p, c_void_p, c_void_p, ctypes.c_float, c_void_p, c_void_p,

@@ -278,6 +278,11 @@ oda_status oda_recall_score(oda_ctx* ctx, const oda_head_weights* w, const float
   return oda::launch_recall_head(ctx, w, h_prev, emb, h_loc, sched, score, flag, any_flag, stream);
 }
 
+oda_status oda_recall_plan(oda_ctx* ctx, int32_t* tile, int32_t* groups, int32_t* ring) {
+  if (!ctx || !tile || !groups || !ring) return set_error(ODA_ERR_INVALID_ARG, "recall_plan: null argument");
+  return oda::recall_head_plan(ctx, tile, groups, ring);
+}
+
 size_t oda_recall_grad_workspace_bytes(int32_t batch, int32_t head_in_dim) {
   if (batch < 1 || head_in_dim < 1) return 0;
   return oda::recall_grad_workspace_bytes(batch, head_in_dim);

@@ -995,6 +995,26 @@ oda_status prepare_head_kernel() {
   return ODA_OK;
 }
 
+// The path oda_recall_score takes for this context: the fused launch's tile width, sequence
+// groups and ring depth, or zeros where the six phase kernels run.  Same plan and occupancy test
+// as the launch below.
+oda_status recall_head_plan(oda_ctx* ctx, int32_t* tile, int32_t* groups, int32_t* ring) {
+  const FusedPlan pl = fused_plan(ctx->cfg.batch, ctx->cfg.head_in_dim, ctx->n_sms);
+  int per_sm = 0;
+  if (pl.bt) {
+    const void* kern = pl.bt == 4 ? reinterpret_cast<const void*>(head_fused_kernel<4>)
+                                  : reinterpret_cast<const void*>(head_fused_kernel<8>);
+    const oda_status st = check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFThreads, pl.smem),
+                                     "cudaOccupancyMaxActiveBlocksPerMultiprocessor(head)");
+    if (st != ODA_OK) return st;
+  }
+  const bool fused = pl.bt && per_sm >= 1;
+  *tile = fused ? pl.bt : 0;
+  *groups = fused ? pl.groups : 0;
+  *ring = fused ? pl.ring : 0;
+  return ODA_OK;
+}
+
 oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const float* h_prev,
                               const float* emb, const float* h_loc, const int32_t* sched,
                               float* score, int32_t* flag, int32_t* any_flag, cudaStream_t s) {

@@ -83,6 +83,7 @@ oda_status launch_attention_noalloc(const oda_config* cfg, const oda_kv_layer* l
 oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const float* h_prev,
                               const float* emb, const float* h_loc, const int32_t* sched,
                               float* score, int32_t* flag, int32_t* any_flag, cudaStream_t s);
+oda_status recall_head_plan(oda_ctx* ctx, int32_t* tile, int32_t* groups, int32_t* ring);
 size_t head_part_floats(int B, int D);
 size_t head_ss_floats(int B, int D);
 int head_counter_count(int D);

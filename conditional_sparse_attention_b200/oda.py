@@ -175,6 +175,14 @@ def oda_recall_score(ctx, w: OdaHeadWeights, h_prev, emb, h_loc, sched, score, f
                                        _p(sched), _p(score), _p(flag), _p(any_flag), _s(stream)))
 
 
+def oda_recall_plan(ctx) -> tuple:
+    """(tile, groups, ring) of the fused head launch for this context, or (0, 0, 0) where the
+    six phase launches run."""
+    t, g, r = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int32(0)
+    check(_lib.load().oda_recall_plan(ctx.handle, ctypes.byref(t), ctypes.byref(g), ctypes.byref(r)))
+    return t.value, g.value, r.value
+
+
 def oda_recall_grad_workspace_bytes(batch: int, head_in_dim: int) -> int:
     return int(_lib.load().oda_recall_grad_workspace_bytes(batch, head_in_dim))
 

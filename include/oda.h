@@ -273,6 +273,12 @@ oda_status oda_recall_score(oda_ctx* ctx, const oda_head_weights* w, const float
                             const float* emb, const float* h_loc, const int32_t* sched,
                             float* score, int32_t* flag, int32_t* any_flag, cudaStream_t stream);
 
+/* Which path oda_recall_score takes for this context's batch and head_in_dim (host only, no
+ * launch): *tile = sequences per tile of the single cooperative launch (4 or 8), *groups = its
+ * sequence groups, *ring = its weight-ring depth in 32 KiB stages; all three 0 where the six
+ * phase launches run.  ODA_ERR_INVALID_ARG on a NULL argument. */
+oda_status oda_recall_plan(oda_ctx* ctx, int32_t* tile, int32_t* groups, int32_t* ring);
+
 /* Training-side arithmetic of the recall head (the head is the only trained part).
  * [notes §2.1, eq. g_t]: gain g = ln p_full - ln p_local (nats), where p_full and p_local are
  * the probabilities of the next token under the full and the local pass; [notes §2.2, eqs.

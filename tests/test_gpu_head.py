@@ -49,6 +49,16 @@ def _run(B, D, perturb=True, seed=500, sched=None, theta=0.0, bias=0.0, inputs_o
                                  (13, 2048), (32, 2048), (20, 4096), (67, 1024), (256, 1024),
                                  (2, 512), (8, 512), (3, 1536)])
 def test_scores_and_gate_match_oracle(B, D):
+    # the path these shapes must take: a fallback to the phase launches would still pass parity
+    # and hide a fused kernel that never runs
+    from conditional_sparse_attention_b200 import oda
+    c = oda.oda_create(oda.make_config(B, D // 128, max(1, D // 256), 4, D))
+    tile, groups, ring = oda.oda_recall_plan(c)
+    c.close()
+    if D % 1024 == 0 and (B, D) != (8, 8192):
+        assert (tile, groups) == ((4, 1) if B <= 4 else (8, (B + 7) // 8)) and ring >= 2, (tile, groups, ring)
+    else:
+        assert (tile, groups, ring) == (0, 0, 0)
     P, xs, score, flag, anyf = _run(B, D, perturb=True, seed=500 + B + D)
     ref = np.array([recall_head(P, xs[0][b], xs[1][b], xs[2][b]) for b in range(B)])
     for b in range(B):
