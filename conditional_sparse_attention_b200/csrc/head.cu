@@ -718,7 +718,10 @@ __device__ void finish_rows(const FusedParams& p, const Own& o, int b0, int Bs, 
   }
 }
 
-template <int BT>
+// kGroups: the batch is cut into sequence groups on shares of the grid (batches above the tile
+// width); without it one group spans the grid and every CTA's rows of a phase fit one batch
+// (at least 128 SMs), so that instantiation carries neither the group offsets nor the batch loop.
+template <int BT, bool kGroups>
 __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedParams p) {
   extern __shared__ __align__(16) uint8_t fsm[];
   const int R = p.ring;
@@ -735,14 +738,17 @@ __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedPar
   const int c = blockIdx.x, G = gridDim.x, B = p.B;
   // sequence group of this CTA: sequences [b0, b0 + Bs) on CTAs [grp * gsize, grp * gsize + gsize);
   // CTAs past the last group own no rows and only take part in the grid barriers
-  const int grp = c / p.gsize, cg = c - grp * p.gsize;
-  const int b0 = grp * BT;
-  const int Bs = grp < p.groups ? min(BT, B - b0) : 0;
+  const int grp = kGroups ? c / p.gsize : 0;
+  const int cg = kGroups ? c - grp * p.gsize : c;
+  const int b0 = kGroups ? grp * BT : 0;
+  const int Bs = kGroups ? (grp < p.groups ? min(BT, B - b0) : 0) : B;
   auto own = [&](int ph) {
-    Own o = own_rows(ph, cg, p.gsize, p.D);
-    if (Bs == 0) o.n = o.nseg = 0;
+    Own o = own_rows(ph, cg, kGroups ? p.gsize : G, p.D);
+    if (kGroups && Bs == 0) o.n = o.nseg = 0;
     return o;
   };
+  auto nbatches = [&](const Own& o) { return kGroups ? n_batches(o) : 1; };
+  auto batch = [&](const Own& o, int j) { return kGroups ? batch_of(o, j) : o; };
   if (tid == 0) {
     for (int i = 0; i < R; ++i) {
       mbar_init(&full[i], 1);
@@ -771,9 +777,9 @@ __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedPar
     int k = 0;
     for (int ph = 0; ph < 6; ++ph) {
       const Own oa = own(ph);
-      const int nbat = n_batches(oa);
+      const int nbat = nbatches(oa);
       for (int j = 0; j < nbat; ++j) {
-        const Own o = batch_of(oa, j);
+        const Own o = batch(oa, j);
         const int ngrp = (o.nseg + kFC - 1) / kFC;
         for (int ch = 0; ch < o.nchunk; ++ch)
           for (int g = 0; g < ngrp; ++g, ++k) {
@@ -803,16 +809,18 @@ __global__ void __launch_bounds__(kFThreads, 1) head_fused_kernel(const FusedPar
     const Own oa = own(ph);
     const bool tower = oa.kind == kTower;
     const float4* gam4 = reinterpret_cast<const float4*>(p.w.tower_norm[oa.tower]);
+    // one group: the tower norm weights of the first chunk, loaded before the input wait
+    const float4 gfirst = !kGroups && tower ? __ldg(gam4 + col4) : zero;
     if (tower) {
       if (!mbar_wait_bounded(&src_bar, 0u, kFWaitNs) && lane == 0) atomicOr(p.err, ODA_DEVERR_WAIT_TIMEOUT);
     } else {
       load_source<BT>(p, oa, b0, Bs, src, red, s_inv, tid);
     }
-    const int nbat = n_batches(oa);
+    const int nbat = nbatches(oa);
     for (int j = 0; j < nbat; ++j) {
-      const Own o = batch_of(oa, j);
+      const Own o = batch(oa, j);
       for (int i = lane; i < kMaxOwnSegs * BT; i += 32) acc[i] = 0.f;
-      float4 gnext = tower ? __ldg(gam4 + col4) : zero;
+      float4 gnext = kGroups ? (tower ? __ldg(gam4 + col4) : zero) : gfirst;
       __syncwarp();
       const float pre = finish_operand(p, o, b0, Bs, tid);
       float ssl[BT];
@@ -917,7 +925,15 @@ int head_counter_count(int D) {
 
 namespace {
 // device properties and the fused kernels' static shared memory, read by prepare_head_kernel
-int g_fused_static[2] = {-1, -1};   // head_fused_kernel<4>, <8>
+int g_fused_static[3] = {-1, -1, -1};   // head_fused_kernel<4, false>, <8, false>, <8, true>
+
+// The fused kernel for a plan's tile width and grouping, and its index above.
+using FusedKernel = void (*)(FusedParams);
+int fused_index(int bt, bool grouped) { return bt == 4 ? 0 : grouped ? 2 : 1; }
+FusedKernel fused_kernel(int index) {
+  return index == 0 ? head_fused_kernel<4, false> : index == 1 ? head_fused_kernel<8, false>
+                                                                : head_fused_kernel<8, true>;
+}
 int g_smem_optin = 0;
 int g_coop = 0;
 
@@ -927,17 +943,24 @@ int g_coop = 0;
 // kernels run instead.
 struct FusedPlan {
   int bt, groups, gsize, ring;
+  bool grouped;   // the kernel with sequence groups and row batches
   size_t smem;
 };
 
 FusedPlan fused_plan(int B, int D, int n_sms) {
-  FusedPlan pl = {0, 0, 0, 0, 0};
+  FusedPlan pl = {0, 0, 0, 0, false, 0};
   if (B < 1 || D % kSeg != 0 || n_sms < 128 || !g_coop) return pl;
   const int bt = B <= 4 ? 4 : 8;
   const int groups = (B + bt - 1) / bt;
   const int gsize = n_sms / groups;
   if (gsize < 3) return pl;   // the tower phase gives each of the three towers a CTA at least
-  const int stat = g_fused_static[bt == 4 ? 0 : 1];
+  // one group whose CTAs each own few enough rows of every phase for one batch (true from about
+  // 96 SMs) runs the kernel without groups and batches; a 4-wide tile never needs them
+  const int g3 = gsize / 3;
+  const bool one_batch = (kT + g3 - 1) / g3 <= kMaxOwnSegs && (kF + gsize - 1) / gsize <= kMaxOwnSegs / 2;
+  const bool grouped = groups > 1 || !one_batch;
+  if (grouped && bt == 4) return pl;
+  const int stat = g_fused_static[fused_index(bt, grouped)];
   if (stat < 0) return pl;
   const size_t src = (size_t)std::max(D, 3 * kT) * bt * sizeof(float);
   const size_t res = (size_t)kFC * kMaxOwnSegs * bt * sizeof(float);   // per-warp row sums
@@ -947,6 +970,7 @@ FusedPlan fused_plan(int B, int D, int n_sms) {
   pl.bt = bt;
   pl.groups = groups;
   pl.gsize = gsize;
+  pl.grouped = grouped;
   pl.ring = ring;
   pl.smem = (size_t)ring * kFStageBytes + src + res;
   return pl;
@@ -974,11 +998,10 @@ oda_status prepare_head_kernel() {
     st = check_cuda(cudaDeviceGetAttribute(&g_coop, cudaDevAttrCooperativeLaunch, dev),
                     "cudaDeviceGetAttribute");
   if (st != ODA_OK) return st;
-  const void* kernels[2] = {reinterpret_cast<const void*>(head_fused_kernel<4>),
-                            reinterpret_cast<const void*>(head_fused_kernel<8>)};
-  for (int i = 0; i < 2; ++i) {
+  for (int i = 0; i < 3; ++i) {
+    const void* kern = reinterpret_cast<const void*>(fused_kernel(i));
     cudaFuncAttributes fa;
-    st = check_cuda(cudaFuncGetAttributes(&fa, kernels[i]), "cudaFuncGetAttributes(head)");
+    st = check_cuda(cudaFuncGetAttributes(&fa, kern), "cudaFuncGetAttributes(head)");
     if (st != ODA_OK) return st;
     // 288 threads (9 warps, three on one SM sub-partition) allow at most 168 registers per thread;
     // a kernel built with more could never launch, every plan would fail and the phase kernels
@@ -987,7 +1010,7 @@ oda_status prepare_head_kernel() {
       return set_error(ODA_ERR_UNSUPPORTED, "fused recall head: %d registers per thread leave %d threads per block",
                        fa.numRegs, fa.maxThreadsPerBlock);
     g_fused_static[i] = (int)fa.sharedSizeBytes;
-    st = check_cuda(cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
+    st = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          g_smem_optin - g_fused_static[i]),
                     "cudaFuncSetAttribute(head)");
     if (st != ODA_OK) return st;
@@ -1002,8 +1025,7 @@ oda_status recall_head_plan(oda_ctx* ctx, int32_t* tile, int32_t* groups, int32_
   const FusedPlan pl = fused_plan(ctx->cfg.batch, ctx->cfg.head_in_dim, ctx->n_sms);
   int per_sm = 0;
   if (pl.bt) {
-    const void* kern = pl.bt == 4 ? reinterpret_cast<const void*>(head_fused_kernel<4>)
-                                  : reinterpret_cast<const void*>(head_fused_kernel<8>);
+    const void* kern = reinterpret_cast<const void*>(fused_kernel(fused_index(pl.bt, pl.grouped)));
     const oda_status st = check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFThreads, pl.smem),
                                      "cudaOccupancyMaxActiveBlocksPerMultiprocessor(head)");
     if (st != ODA_OK) return st;
@@ -1043,8 +1065,7 @@ oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const flo
   const FusedPlan pl = fused_plan(B, D, ctx->n_sms);
   int per_sm = 0;
   if (pl.bt) {
-    const void* kern = pl.bt == 4 ? reinterpret_cast<const void*>(head_fused_kernel<4>)
-                                  : reinterpret_cast<const void*>(head_fused_kernel<8>);
+    const void* kern = reinterpret_cast<const void*>(fused_kernel(fused_index(pl.bt, pl.grouped)));
     oda_status st = check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFThreads, pl.smem),
                                "cudaOccupancyMaxActiveBlocksPerMultiprocessor(head)");
     if (st != ODA_OK) return st;
@@ -1081,8 +1102,7 @@ oda_status launch_recall_head(oda_ctx* ctx, const oda_head_weights* w, const flo
     attr[0].val.cooperative = 1;
     lc.attrs = attr;
     lc.numAttrs = 1;
-    return check_cuda(pl.bt == 4 ? cudaLaunchKernelEx(&lc, head_fused_kernel<4>, f)
-                                 : cudaLaunchKernelEx(&lc, head_fused_kernel<8>, f),
+    return check_cuda(cudaLaunchKernelEx(&lc, fused_kernel(fused_index(pl.bt, pl.grouped)), f),
                       "recall head launch");
   }
   HeadParams p;
