@@ -33,7 +33,7 @@ METRIC = "ODA decode-attn steps/s + % of HBM peak, 128K ctx, 12.5% recall, 1 B20
 # 32K-context, 2-layer profiling workload (4 flagged sequences x 32768 cached tokens); the bench
 # scales it to its own launches by cached tokens processed.  Valid only for the kernel source it
 # was taken from (first 16 hex digits of the file's SHA-256).
-NCU_FULL_KERNEL_TRAFFIC = {"attention_cu_sha256": "0529ba2eae03a27d", "bytes": 540988416,
+NCU_FULL_KERNEL_TRAFFIC = {"attention_cu_sha256": "00d69c2bf934804c", "bytes": 540707072,
                            "cached_tokens": 4 * 32768}
 UNIT = "steps/s"
 FALLBACK_HBM_GBS = 6650.0

@@ -1113,8 +1113,11 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   // pages.  Every warp of a CTA whose range starts in (b, h) owns one fixed chunk (rank-major,
   // so it can be fetched before the dependency wait); the remaining chunks are claimed from the
   // (b, h)'s counter by the warps of all CTAs covering it, so that CTAs on faster SMs take more
-  // of them.  Claimed pages wait in a per-warp queue held one entry per lane (entry i in lane
-  // i % 32); copies run kR pages ahead of the arithmetic and may cross into the next segment.
+  // of them.  A CTA whose first (b, h) began before its range and that has more (b, h) after it
+  // claims there no more than its own share: the CTAs for which that (b, h) is the last one
+  // claim the rest, so a CTA covering several short (b, h) does not fall behind on the ones
+  // only it covers.  Claimed pages wait in a per-warp queue held one entry per lane (entry i in
+  // lane i % 32); copies run kR pages ahead of the arithmetic and may cross into the next segment.
   uint32_t issued = 0, consumed = 0, vbits = 0;
   uint32_t f_head = 0, f_tail = 0;            // queue entries [f_head, f_tail)
   int f_phys = -1, f_h = 0, f_lp = 0, f_seg = 0;
@@ -1124,6 +1127,7 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   int is_seg = 0, is_u = u0, is_b = 0, is_h = 0, is_bh = 0, is_nv = 0, is_ncache = 0;
   int is_nch = 0, is_base = 0, is_fixed = -1, pend = 0;
   int is_rank = 0, is_nc = 1, is_next = 0;   // fixed pattern: rank among covering CTAs, count, cursor
+  int is_cap = 0x7fffffff, is_taken = 0;      // this warp's claim limit in the segment, claims taken
   bool is_done = u0 >= u1, claims_ok = false, has_pend = false;
   auto enter_seg = [&](bool first) {
     const Seg cs_ = decode_seg(is_u, u1, s_us, s_nv, B, Hkv);
@@ -1141,6 +1145,13 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     is_base = (int)(cfe - cfs) * kW;
     is_fixed = first ? (int)((long long)vc - cfs) * kW + warp : -1;
     has_pend = false;
+    is_taken = 0;
+    is_cap = 0x7fffffff;
+    if (first && s0 < u0 && s1 < u1) {
+      // the CTA's share [u0, s1) in chunks, less the warps' fixed chunks, split over the warps
+      const int share = (int)((s1 - u0 + kChunk - 1) / kChunk);
+      is_cap = max(0, (share - kW + kW - 1) / kW);
+    }
     if (p.deterministic) {
       // fixed pattern: chunk j goes to covering CTA j % nc, and within it to warp (j / nc) % kW
       const int c0 = cta_of(cs_.s0, U, G), c1 = cta_of(s1 - 1, U, G);
@@ -1150,9 +1161,10 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       is_fixed = -1;
       return;
     }
-    if (claims_ok) {
+    if (claims_ok && is_taken < is_cap) {
       if (lane == 0) pend = atomicAdd(p.claims + is_bh, 1);
       has_pend = true;
+      ++is_taken;
     }
   };
   // lanes look up the physical pages of chunk c of the claim segment into queue entries
@@ -1204,15 +1216,24 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     }
     if (!claims_ok) return;
     if (!has_pend) {
+      if (is_taken >= is_cap) {   // this warp's share of the segment is taken
+        next_segment();
+        return;
+      }
       if (lane == 0) pend = atomicAdd(p.claims + is_bh, 1);
       has_pend = true;
+      ++is_taken;
     }
     const int c = is_base + __shfl_sync(0xffffffffu, pend, 0);
     has_pend = false;
     if (c < is_nch) {
       push_chunk(c);
-      if (lane == 0) pend = atomicAdd(p.claims + is_bh, 1);
-      has_pend = true;
+      // the next claim is taken ahead (it is always used: a claim is never dropped)
+      if (is_taken < is_cap) {
+        if (lane == 0) pend = atomicAdd(p.claims + is_bh, 1);
+        has_pend = true;
+        ++is_taken;
+      }
     } else {
       next_segment();
     }
@@ -1260,9 +1281,10 @@ attn_full_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   grid_dependency_wait();
   grid_dependents_launch();
   claims_ok = true;
-  if (!is_done && is_fixed < 0 && !p.deterministic) {
+  if (!is_done && is_fixed < 0 && !p.deterministic && is_taken < is_cap) {
     if (lane == 0) pend = atomicAdd(p.claims + is_bh, 1);
     has_pend = true;
+    ++is_taken;
   }
 
   // ---- segments of this CTA, in order
